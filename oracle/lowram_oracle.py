@@ -1,0 +1,351 @@
+"""Plain fp64 CPU oracle for LowRAM's encode and its decode-time hot path.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import or call this module. The library (C-ABI + CUDA kernels)
+never calls it, and it shares no code with the library: every function below is written
+out from the method's definition, one step per function, with numpy fp64 arithmetic and
+library primitives (matmul, sort, cos/sin, erf) only.
+
+Passages followed (the pages print no formula, listing or worked example; each step is
+the plainest reading of the prose):
+
+[keys]     "LowRAM: Low-Rank Keys and Amortised Values for Composable KV Cache
+           Compression at Test-Time", agihunt.info summary, the paragraph on the key side:
+           keys are not predicted; they get xKV cross-layer low-rank compression with
+           adjacent layers sharing one SVD basis; RoPE is inverted before compression;
+           the prefix is cut into chunks whose mean key is a landmark, and each decode
+           step rebuilds only the top-k chunks chosen by the current query.
+[values]   same page, the value-cache-amortisation paragraph and the ablation
+           paragraph: a lightweight per-head key->value predictor (nonlinear: a linear
+           one ablates badly), residuals kept only for the worst-reconstructed tokens,
+           chosen by error rather than at random.
+[how]      "LowRAM Exploits Key-Value Predictability to Compress the KV Cache"
+           (cctest.ai), section "How the method works": bullets "Low-rank keys",
+           "Amortised values", "Residuals for difficult tokens", "Selective
+           reconstruction".
+[abstract] the paper's abstract (zhuanzhiai.com and arxiv.science pages): per-head
+           predictor fitted at test time, residuals only for the tokens it
+           reconstructs worst, reconstruction of a selected subset of KV pairs at each
+           decoding step.
+
+Readings taken where the pages are silent (each is listed, with its reason, in the
+design notes of the repository):
+- RoPE is the rotate-half form: pairs (i, i + d/2), theta_i = theta^(-2i/d), angle
+  t * theta_i for token position t = 0..T-1; its inverse is its transpose.
+- The xKV basis spans all KV heads of a layer (D = H_kv * d); keys are projected as
+  c_t = B^T K_pre,t and rebuilt per head as B_h c_t (B_h = rows h*d .. h*d+d-1).
+- The predictor is MLP_h(x) = W2_h act(W1_h x + b1_h) + b2_h applied to the pre-RoPE
+  rebuilt key; act is SiLU or erf-GELU.
+- Residuals are additive corrections R = V - V_hat for the n_res tokens of largest
+  squared error per (batch, kv head), the error taken with the unrounded coefficients,
+  ties to the lower token index; the stored residual uses the stored coefficients.
+- A chunk's score is the max over the GQA group's query heads of q . landmark; the
+  k highest-scoring chunks are selected, ties to the lower chunk index.
+- Attention is softmax(q . K_rot / sqrt(d)) over the selected tokens only.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against something other
+than itself (closed forms, brute force, invariants, library routines); none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+ACT_SILU = 0
+ACT_GELU_ERF = 1
+
+STORE_F64 = "f64"   # no rounding: used by the exactness pins
+STORE_F32 = "f32"
+STORE_BF16 = "bf16"
+
+
+# ----------------------------------------------------------------------------------
+# storage precision
+# ----------------------------------------------------------------------------------
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bfloat16 (round to nearest, ties to even); return the bits.
+
+    bfloat16 keeps fp32's sign and 8-bit exponent and the top 7 fraction bits. The
+    rounding is done once, from fp64, on the 52-bit fraction: keep 7 bits, round the
+    discarded 45 to nearest-even.
+    """
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    bits = x.view(np.uint64).copy()
+    finite = np.isfinite(x)
+    drop = np.uint64(45)
+    lsb = (bits >> drop) & np.uint64(1)
+    bits = np.where(finite, bits + (np.uint64((1 << 44) - 1) + lsb), bits)
+    bits &= ~np.uint64((1 << 45) - 1)
+    as32 = bits.view(np.float64).astype(np.float32)  # exact: at most 8 significant bits
+    return (as32.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f64(u: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bits to fp64 exactly."""
+    u = np.asarray(u, dtype=np.uint16)
+    return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def round_to_storage(x: np.ndarray, store: str) -> np.ndarray:
+    """Value of ``x`` after storing it in the given precision, as fp64."""
+    if store == STORE_F64:
+        return np.asarray(x, dtype=np.float64).copy()
+    if store == STORE_F32:
+        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+    if store == STORE_BF16:
+        return bf16_bits_to_f64(f64_to_bf16_bits(x))
+    raise ValueError(f"unknown storage precision {store!r}")
+
+
+# ----------------------------------------------------------------------------------
+# RoPE [keys]: inverted before compression, re-applied at reconstruction
+# ----------------------------------------------------------------------------------
+def rope_inv_freq(d: int, theta: float) -> np.ndarray:
+    """theta_i = theta^(-2i/d), i = 0 .. d/2-1 (fp64)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(theta), -2.0 * i / d)
+
+
+def rope_rotate(x: np.ndarray, pos, theta: float, inverse: bool = False) -> np.ndarray:
+    """R(pos) x in the rotate-half form, or R(pos)^T x when ``inverse``.
+
+    x: [..., d]; pos: integer positions broadcastable to x.shape[:-1].
+    y_i = x_i cos(a_i) - x_{i+d/2} sin(a_i);  y_{i+d/2} = x_i sin(a_i) + x_{i+d/2} cos(a_i),
+    a_i = pos * theta_i. The inverse rotates by -a_i.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d, theta)
+    cs, sn = np.cos(ang), np.sin(ang)
+    if inverse:
+        sn = -sn
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cs - x2 * sn, x1 * sn + x2 * cs], axis=-1)
+
+
+# ----------------------------------------------------------------------------------
+# cross-layer low-rank keys [keys], [how: Low-rank keys]
+# ----------------------------------------------------------------------------------
+def project_keys(k_pre_flat: np.ndarray, basis: np.ndarray) -> np.ndarray:
+    """c_t = B^T K_pre,t over the flattened D = H_kv*d key of token t.
+
+    k_pre_flat: [..., D]; basis: [D, r] with orthonormal columns -> [..., r].
+    """
+    return np.asarray(k_pre_flat, dtype=np.float64) @ np.asarray(basis, dtype=np.float64)
+
+
+def rebuild_keys(coef: np.ndarray, basis: np.ndarray, h: int, d: int) -> np.ndarray:
+    """K~_pre,t,h = B_h c_t, B_h = rows h*d .. h*d+d-1 of the basis. -> [..., d]."""
+    bh = np.asarray(basis, dtype=np.float64)[h * d:(h + 1) * d, :]
+    return np.asarray(coef, dtype=np.float64) @ bh.T
+
+
+# ----------------------------------------------------------------------------------
+# chunk landmarks and top-k chunk selection [keys], [how: Selective reconstruction]
+# ----------------------------------------------------------------------------------
+def chunk_landmarks(k_cache: np.ndarray, chunk: int) -> np.ndarray:
+    """Mean post-RoPE key of every chunk, per KV head.
+
+    k_cache: [B, T, H, d] -> [B, H, T/chunk, d].
+    """
+    B, T, H, d = k_cache.shape
+    assert T % chunk == 0
+    grouped = np.asarray(k_cache, dtype=np.float64).reshape(B, T // chunk, chunk, H, d)
+    return grouped.mean(axis=2).transpose(0, 2, 1, 3)
+
+
+def chunk_scores(q_group: np.ndarray, landmark: np.ndarray) -> np.ndarray:
+    """Score of each chunk for one KV head: max over the group's query heads of q . L_c.
+
+    q_group: [G, d]; landmark: [N_c, d] -> [N_c].
+    """
+    dots = np.asarray(landmark, dtype=np.float64) @ np.asarray(q_group, dtype=np.float64).T
+    return dots.max(axis=1)
+
+
+def topk_ascending(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest scores (ties to the lower index), returned ascending."""
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    k = min(int(k), n)
+    order = np.lexsort((np.arange(n), -scores))  # primary: score desc; then index asc
+    return np.sort(order[:k]).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------------
+# amortised values [values], [how: Amortised values], [abstract]
+# ----------------------------------------------------------------------------------
+def activation(x: np.ndarray, act: int) -> np.ndarray:
+    """SiLU(x) = x / (1 + e^-x);  GELU(x) = x/2 (1 + erf(x / sqrt 2))."""
+    x = np.asarray(x, dtype=np.float64)
+    if act == ACT_SILU:
+        return x / (1.0 + np.exp(-x))
+    if act == ACT_GELU_ERF:
+        return 0.5 * x * (1.0 + _erf(x / math.sqrt(2.0)))
+    raise ValueError(f"unknown activation {act}")
+
+
+def predictor(x: np.ndarray, w1, b1, w2, b2, act: int) -> np.ndarray:
+    """One head's key->value MLP: V_hat = W2 act(W1 x + b1) + b2.
+
+    x: [..., d]; w1: [F, d]; b1: [F]; w2: [d, F]; b2: [d] -> [..., d].
+    """
+    hid = activation(np.asarray(x, np.float64) @ np.asarray(w1, np.float64).T
+                     + np.asarray(b1, np.float64), act)
+    return hid @ np.asarray(w2, np.float64).T + np.asarray(b2, np.float64)
+
+
+# ----------------------------------------------------------------------------------
+# encode [keys], [values], [how: Residuals for difficult tokens]
+# ----------------------------------------------------------------------------------
+def residual_errors(v_h: np.ndarray, coef_exact: np.ndarray, basis, h, w1, b1, w2, b2,
+                    act) -> np.ndarray:
+    """e_t = || V_t,h - MLP_h(B_h c_t) ||^2 with the unrounded coefficients. -> [T]."""
+    d = v_h.shape[-1]
+    vhat = predictor(rebuild_keys(coef_exact, basis, h, d), w1, b1, w2, b2, act)
+    return ((np.asarray(v_h, np.float64) - vhat) ** 2).sum(axis=-1)
+
+
+def residual_chunk_ptr(res_idx: np.ndarray, n_tokens: int, chunk: int) -> np.ndarray:
+    """CSR offsets: residual rows of chunk c are res_idx[ptr[c]:ptr[c+1]]."""
+    counts = np.bincount(np.asarray(res_idx) // chunk, minlength=n_tokens // chunk)
+    return np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+
+
+def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store):
+    """Compress one layer's prefix.
+
+    k_cache, v: [B, T, H, d] (post-RoPE keys, values); basis [D, r]; w1 [H, F, d];
+    b1 [H, F]; w2 [H, d, F]; b2 [H, d]. Steps, in the pages' order:
+      1. invert RoPE on the keys;
+      2. project every token's flattened key onto the shared basis (coefficients are
+         stored rounded to ``store``);
+      3. landmarks = chunk means of the original post-RoPE keys (stored rounded);
+      4. run the per-head predictor on the rebuilt key of every token and take the
+         squared error against the true value, with the unrounded coefficients;
+      5. per (batch, head) keep the n_res largest-error tokens (ascending indices);
+      6. store their residuals V - MLP_h(B_h coef_stored), and the per-chunk CSR.
+    """
+    k_cache = np.asarray(k_cache, np.float64)
+    v = np.asarray(v, np.float64)
+    B, T, H, d = k_cache.shape
+    D = H * d
+    pos = np.arange(T)
+    k_pre = rope_rotate(k_cache, pos[None, :, None], theta, inverse=True)
+    coef_exact = project_keys(k_pre.reshape(B, T, D), basis)
+    coef = round_to_storage(coef_exact, store)
+    landmark = round_to_storage(chunk_landmarks(k_cache, chunk), store)
+    n_chunks = T // chunk
+    err = np.empty((B, H, T))
+    res_idx = np.empty((B, H, n_res), np.int64)
+    res_val = np.empty((B, H, n_res, d))
+    chunk_ptr = np.empty((B, H, n_chunks + 1), np.int64)
+    for b in range(B):
+        for h in range(H):
+            err[b, h] = residual_errors(v[b, :, h], coef_exact[b], basis, h,
+                                        w1[h], b1[h], w2[h], b2[h], act)
+            idx = topk_ascending(err[b, h], n_res)
+            vhat_stored = predictor(rebuild_keys(coef[b, idx], basis, h, d),
+                                    w1[h], b1[h], w2[h], b2[h], act)
+            res_idx[b, h] = idx
+            res_val[b, h] = round_to_storage(v[b, idx, h] - vhat_stored, store)
+            chunk_ptr[b, h] = residual_chunk_ptr(idx, T, chunk)
+    return {"coef": coef, "coef_exact": coef_exact, "landmark": landmark,
+            "res_idx": res_idx, "res_val": res_val, "chunk_ptr": chunk_ptr, "err": err}
+
+
+# ----------------------------------------------------------------------------------
+# decode step [keys], [how: Selective reconstruction], [abstract]
+# ----------------------------------------------------------------------------------
+def select_chunks(q, landmark, top_k):
+    """Per (batch, KV head): the top_k chunks by landmark score, ascending.
+
+    q: [B, H_q, d]; landmark: [B, H, N_c, d] -> (sel [B, H, k], scores [B, H, N_c]).
+    """
+    q = np.asarray(q, np.float64)
+    B, Hq, d = q.shape
+    H, n_chunks = landmark.shape[1], landmark.shape[2]
+    G = Hq // H
+    k = min(int(top_k), n_chunks)
+    sel = np.empty((B, H, k), np.int64)
+    scores = np.empty((B, H, n_chunks))
+    for b in range(B):
+        for h in range(H):
+            scores[b, h] = chunk_scores(q[b, h * G:(h + 1) * G], landmark[b, h])
+            sel[b, h] = topk_ascending(scores[b, h], k)
+    return sel, scores
+
+
+def reconstruct_chunks(sel_bh, coef_b, basis, h, d, chunk, res_idx_bh, res_val_bh,
+                       chunk_ptr_bh, w1, b1, w2, b2, act, theta):
+    """Rebuild K (post-RoPE) and V for the selected chunks of one (batch, KV head).
+
+    Returns (tokens [n], k_rot [n, d], v_rec [n, d]) with tokens in selection order.
+    V = MLP_h(B_h coef_t), plus the stored residual R_t where t holds one.
+    """
+    sel_bh = np.asarray(sel_bh, np.int64)
+    tokens = (sel_bh[:, None] * chunk + np.arange(chunk)[None, :]).reshape(-1)
+    k_pre = rebuild_keys(np.asarray(coef_b, np.float64)[tokens], basis, h, d)
+    k_rot = rope_rotate(k_pre, tokens, theta)
+    v_rec = predictor(k_pre, w1, b1, w2, b2, act)
+    for slot, c in enumerate(sel_bh):
+        for i in range(int(chunk_ptr_bh[c]), int(chunk_ptr_bh[c + 1])):
+            t = int(res_idx_bh[i])
+            assert c * chunk <= t < (c + 1) * chunk, "residual index outside its chunk"
+            v_rec[slot * chunk + (t - c * chunk)] += res_val_bh[i]
+    return tokens, k_rot, v_rec
+
+
+def decode_step(q, cache, basis, w1, b1, w2, b2, *, chunk, top_k, theta, act, sel=None):
+    """One decode step of one layer over the compressed cache.
+
+    q: [B, H_q, d] (post-RoPE). cache: dict with coef [B,T,r], landmark [B,H,N_c,d],
+    res_idx [B,H,n_res], res_val [B,H,n_res,d], chunk_ptr [B,H,N_c+1]. ``sel`` may
+    override the selection (used when a caller's selection differs only by ties).
+    Returns (out [B, H_q, d], sel [B, H, k]).
+    """
+    q = np.asarray(q, np.float64)
+    B, Hq, d = q.shape
+    H = cache["landmark"].shape[1]
+    G = Hq // H
+    if sel is None:
+        sel, _ = select_chunks(q, cache["landmark"], top_k)
+    out = np.empty((B, Hq, d))
+    for b in range(B):
+        for h in range(H):
+            _, k_rot, v_rec = reconstruct_chunks(
+                sel[b, h], cache["coef"][b], basis, h, d, chunk,
+                cache["res_idx"][b, h], cache["res_val"][b, h], cache["chunk_ptr"][b, h],
+                w1[h], b1[h], w2[h], b2[h], act, theta)
+            for g in range(G):
+                z = k_rot @ q[b, h * G + g] / math.sqrt(d)
+                p = np.exp(z - z.max())
+                p /= p.sum()
+                out[b, h * G + g] = p @ v_rec
+    return out, np.asarray(sel)
+
+
+def dense_attention(q, k_cache, v):
+    """Textbook GQA decode attention over the full uncompressed cache.
+
+    q: [B, H_q, d]; k_cache, v: [B, T, H, d] -> [B, H_q, d].
+    """
+    q = np.asarray(q, np.float64)
+    k_cache = np.asarray(k_cache, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Hq, d = q.shape
+    H = k_cache.shape[2]
+    G = Hq // H
+    out = np.empty((B, Hq, d))
+    for b in range(B):
+        for hq in range(Hq):
+            h = hq // G
+            z = k_cache[b, :, h, :] @ q[b, hq] / math.sqrt(d)
+            p = np.exp(z - z.max())
+            p /= p.sum()
+            out[b, hq] = p @ v[b, :, h, :]
+    return out

@@ -1,0 +1,369 @@
+"""Pins of the CPU oracle to things other than itself (closed forms, brute force,
+invariants the method's definitions fix, and library routines), plus mutation tests
+that plant plausible mistakes in the oracle and check that some pin catches each.
+
+CPU only; sized to run in seconds.
+"""
+import cmath
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle.lowram_oracle as O
+from long_context_decode_02_b200 import synth
+
+
+def _np(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def tiny_shape(**kw):
+    base = dict(name="pin", batch=2, n_tokens=64, n_layers=1, n_kv_heads=2, n_q_heads=4,
+                head_dim=8, rank=16, chunk=4, top_k=16, res_frac=1.0, mlp_hidden=12,
+                act=O.ACT_SILU, dtype="f32", theta=1e4, outlier_frac=0.05, steps=1,
+                seed=11)
+    base.update(kw)
+    return synth.Shape(**base)
+
+
+def make_layer(shape, layer=0):
+    """Inputs of one layer in fp64 (keys, values, basis, weights, queries)."""
+    basis = synth.group_basis(shape, 0)
+    w = synth.layer_weights(shape, layer)
+    ks, vs = [], []
+    for b in range(shape.batch):
+        k, v = synth.layer_kv(shape, basis, w, layer, b)
+        ks.append(k)
+        vs.append(v)
+    k = torch.stack(ks)
+    v = torch.stack(vs)
+    q = synth.queries(shape, layer, 0)
+    return dict(k=_np(k), v=_np(v), basis=_np(basis), w=[_np(t) for t in w], q=_np(q))
+
+
+# ----------------------------------------------------------------------------------
+# pin checks, written against a module object so mutation tests can reuse them
+# ----------------------------------------------------------------------------------
+def check_rope_closed_form(M):
+    d, theta = 16, 1e4
+    for i in range(d // 2):
+        x = np.zeros(d)
+        x[i] = 1.0
+        y = M.rope_rotate(x, 1, theta)
+        a = theta ** (-2.0 * i / d)
+        expect = np.zeros(d)
+        expect[i] = math.cos(a)
+        expect[i + d // 2] = math.sin(a)
+        assert np.allclose(y, expect, atol=1e-15), (i, y, expect)
+    # complex-number form at a large position: (x_i + j x_{i+d/2}) e^{j t theta_i}
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(d)
+    t = 262143
+    y = M.rope_rotate(x, t, theta)
+    for i in range(d // 2):
+        z = complex(x[i], x[i + d // 2]) * cmath.exp(1j * t * theta ** (-2.0 * i / d))
+        assert abs(y[i] - z.real) < 1e-9 and abs(y[i + d // 2] - z.imag) < 1e-9
+
+
+def check_rope_group_properties(M):
+    rng = np.random.default_rng(1)
+    d, theta = 32, 5e5
+    x = rng.standard_normal((5, d))
+    pos = np.array([0, 1, 17, 4096, 262143])
+    assert np.allclose(M.rope_rotate(x[:1], 0, theta), x[:1], atol=0)      # R(0) = I
+    y = M.rope_rotate(x, pos, theta)
+    assert np.allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    assert np.allclose(M.rope_rotate(y, pos, theta, inverse=True), x, atol=1e-13)
+    # relative position: <R(m)a, R(n)b> depends on m - n only
+    a, b = rng.standard_normal(d), rng.standard_normal(d)
+    s1 = M.rope_rotate(a, 100, theta) @ M.rope_rotate(b, 37, theta)
+    s2 = M.rope_rotate(a, 1100, theta) @ M.rope_rotate(b, 1037, theta)
+    assert abs(s1 - s2) < 1e-10
+
+
+def check_projection(M):
+    rng = np.random.default_rng(2)
+    H, d = 3, 8
+    D = H * d
+    # full rank, square orthogonal basis: rebuild(project(x)) == x for every head
+    q_full, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    x = rng.standard_normal((10, D))
+    c = M.project_keys(x, q_full)
+    for h in range(H):
+        assert np.allclose(M.rebuild_keys(c, q_full, h, d), x[:, h * d:(h + 1) * d],
+                           atol=1e-12)
+    # reduced rank: coefficients are the least-squares solution (library routine)
+    b_red, _ = np.linalg.qr(rng.standard_normal((D, 7)))
+    c = M.project_keys(x, b_red)
+    lst, *_ = np.linalg.lstsq(b_red, x.T, rcond=None)
+    assert np.allclose(c, lst.T, atol=1e-12)
+    full = np.concatenate([M.rebuild_keys(c, b_red, h, d) for h in range(H)], axis=1)
+    assert np.allclose(full, lst.T @ b_red.T, atol=1e-12)
+
+
+def check_landmarks_and_scores(M):
+    rng = np.random.default_rng(3)
+    B, T, H, d, C, G = 2, 24, 2, 4, 4, 3
+    k = rng.standard_normal((B, T, H, d))
+    lm = M.chunk_landmarks(k, C)
+    assert lm.shape == (B, H, T // C, d)
+    for b in range(B):
+        for h in range(H):
+            for c in range(T // C):
+                brute = [math.fsum(k[b, c * C + i, h, j] for i in range(C)) / C
+                         for j in range(d)]
+                assert np.allclose(lm[b, h, c], brute, atol=1e-15)
+    # linearity: q . L_c = mean over the chunk of q . K_t
+    q = rng.standard_normal(d)
+    assert np.allclose(lm[0, 1] @ q, (k[0, :, 1] @ q).reshape(-1, C).mean(1), atol=1e-14)
+    # chunk score = max over the group's heads; a group where one head dominates
+    qg = np.zeros((G, d))
+    qg[2] = q
+    s = M.chunk_scores(qg, lm[1, 0])
+    assert np.allclose(s, np.maximum(lm[1, 0] @ q, 0.0), atol=1e-15)
+    qg = rng.standard_normal((G, d))
+    s = M.chunk_scores(qg, lm[0, 0])
+    brute = [max(math.fsum(qg[g, j] * lm[0, 0, c, j] for j in range(d)) for g in range(G))
+             for c in range(T // C)]
+    assert np.allclose(s, brute, atol=1e-14)
+
+
+def check_topk(M):
+    rng = np.random.default_rng(4)
+    for n, k in [(50, 7), (50, 50), (50, 80), (200, 1)]:
+        for s in (rng.standard_normal(n), rng.integers(0, 4, n).astype(float)):
+            got = M.topk_ascending(s, k)
+            brute = sorted(sorted(range(n), key=lambda i: (-s[i], i))[:min(k, n)])
+            assert list(got) == brute, (n, k)
+
+
+def check_predictor(M):
+    rng = np.random.default_rng(5)
+    d, Fh = 8, 12
+    x = rng.standard_normal((9, d))
+    w1, b1 = rng.standard_normal((Fh, d)), rng.standard_normal(Fh)
+    w2, b2 = rng.standard_normal((d, Fh)), rng.standard_normal(d)
+    tx = torch.tensor(x)
+    for act, fn in ((M.ACT_SILU, F.silu), (M.ACT_GELU_ERF,
+                                           lambda t: F.gelu(t, approximate="none"))):
+        ref = F.linear(fn(F.linear(tx, torch.tensor(w1), torch.tensor(b1))),
+                       torch.tensor(w2), torch.tensor(b2)).numpy()
+        assert np.allclose(M.predictor(x, w1, b1, w2, b2, act), ref, atol=1e-13)
+
+
+def check_full_rank_exactness(M):
+    """Full rank, every token a residual, every chunk selected: decode == dense attention
+    over the original keys/values, and encode reconstructs K and V exactly."""
+    sh = tiny_shape(rank=16, n_kv_heads=2, head_dim=8, res_frac=1.0, top_k=10 ** 6)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    cache = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                     store=M.STORE_F64, **kw)
+    w1, b1, w2, b2 = L["w"]
+    for b in range(sh.batch):
+        for h in range(sh.n_kv_heads):
+            sel = np.arange(sh.n_chunks)
+            toks, k_rot, v_rec = M.reconstruct_chunks(
+                sel, cache["coef"][b], L["basis"], h, sh.head_dim, sh.chunk,
+                cache["res_idx"][b, h], cache["res_val"][b, h], cache["chunk_ptr"][b, h],
+                w1[h], b1[h], w2[h], b2[h], sh.act, sh.theta)
+            assert np.allclose(k_rot, L["k"][b, toks, h], atol=1e-12)
+            assert np.allclose(v_rec, L["v"][b, toks, h], atol=1e-12)
+    out, sel = M.decode_step(L["q"], cache, L["basis"], *L["w"], top_k=sh.top_k, **kw)
+    dense = M.dense_attention(L["q"], L["k"], L["v"])
+    assert np.allclose(out, dense, atol=1e-12)
+    # and the dense textbook form equals torch's attention routine
+    G = sh.group
+    tq = torch.tensor(L["q"])[:, :, None, :]                          # [B, Hq, 1, d]
+    tk = torch.tensor(L["k"]).permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    tv = torch.tensor(L["v"]).permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    ref = F.scaled_dot_product_attention(tq, tk, tv)[:, :, 0, :].numpy()
+    assert np.allclose(dense, ref, atol=1e-12)
+
+
+def check_residual_pick(M):
+    sh = synth.CONFIGS[0].replace(n_layers=1, n_tokens=512)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    c64 = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                   store=M.STORE_F64, **kw)
+    cbf = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                   store=M.STORE_BF16, **kw)
+    # errors use the unrounded coefficients: independent of the storage precision
+    assert np.array_equal(c64["err"], cbf["err"])
+    d = sh.head_dim
+    w1, b1, w2, b2 = L["w"]
+    for h in range(sh.n_kv_heads):
+        e = c64["err"][0, h]
+        # brute force: per-token squared error, then a full sort
+        brute_e = []
+        for t in range(sh.n_tokens):
+            kp = M.rope_rotate(L["k"][0, t], t, sh.theta, inverse=True).reshape(-1)
+            ct = L["basis"].T @ kp
+            vhat = M.predictor(L["basis"][h * d:(h + 1) * d] @ ct, w1[h], b1[h], w2[h],
+                               b2[h], sh.act)
+            brute_e.append(math.fsum((L["v"][0, t, h] - vhat) ** 2))
+        assert np.allclose(e, brute_e, rtol=1e-12)
+        order = sorted(range(sh.n_tokens), key=lambda t: (-brute_e[t], t))[:sh.n_res]
+        assert list(c64["res_idx"][0, h]) == sorted(order)
+        # every planted outlier row is among the residuals (error ~ d*9 >> noise)
+        n_out = int(sh.outlier_frac * sh.n_tokens)
+        big = np.argsort(-np.abs(L["v"][0, :, h]).max(axis=1))[:n_out]
+        assert set(big.tolist()) <= set(c64["res_idx"][0, h].tolist())
+        # CSR offsets count the residual rows of every chunk
+        ptr = c64["chunk_ptr"][0, h]
+        for c in range(sh.n_chunks):
+            n_in = sum(1 for t in c64["res_idx"][0, h] if c * sh.chunk <= t < (c + 1) * sh.chunk)
+            assert ptr[c + 1] - ptr[c] == n_in
+        # the stored residual restores V up to its own rounding: it was taken against
+        # the predictor run on the STORED coefficients
+        idx = cbf["res_idx"][0, h]
+        vhat_s = M.predictor(M.rebuild_keys(cbf["coef"][0, idx], L["basis"], h, d),
+                             w1[h], b1[h], w2[h], b2[h], sh.act)
+        exact_r = L["v"][0, idx, h] - vhat_s
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact_r), 1e-300))) - 7)
+        assert np.all(np.abs(vhat_s + cbf["res_val"][0, h] - L["v"][0, idx, h])
+                      <= 0.5 * ulp + 1e-15)
+
+
+def check_selection_and_edges(M):
+    sh = tiny_shape(res_frac=0.25, top_k=5, rank=6)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    cache = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                     store=M.STORE_F32, **kw)
+    out, sel = M.decode_step(L["q"], cache, L["basis"], *L["w"], top_k=sh.top_k, **kw)
+    G = sh.group
+    for b in range(sh.batch):
+        for h in range(sh.n_kv_heads):
+            s = [max(float(L["q"][b, h * G + g] @ cache["landmark"][b, h, c])
+                     for g in range(G)) for c in range(sh.n_chunks)]
+            brute = sorted(sorted(range(sh.n_chunks), key=lambda c: (-s[c], c))[:sh.top_k])
+            assert list(sel[b, h]) == brute
+    # the output is a convex combination of reconstructed values: bounded by them
+    # no residuals at all: a valid cache, decode still runs
+    c0 = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=0, store=M.STORE_F32, **kw)
+    assert c0["res_idx"].shape[-1] == 0 and np.all(c0["chunk_ptr"] == 0)
+    out0, _ = M.decode_step(L["q"], c0, L["basis"], *L["w"], top_k=1, **kw)
+    assert np.all(np.isfinite(out0))
+
+
+ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
+              check_landmarks_and_scores, check_topk, check_predictor,
+              check_full_rank_exactness, check_residual_pick, check_selection_and_edges]
+
+
+@pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
+def test_oracle_pin(check):
+    check(O)
+
+
+def test_bf16_rounding_matches_torch_and_ties_to_even():
+    rng = np.random.default_rng(7)
+    x32 = (rng.standard_normal(10000) * 10.0 ** rng.integers(-6, 6, 10000)).astype(np.float32)
+    ours = O.f64_to_bf16_bits(x32.astype(np.float64))
+    ref = torch.from_numpy(x32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    one = 1.0
+    assert O.f64_to_bf16_bits(np.array([one]))[0] == 0x3F80
+    assert O.f64_to_bf16_bits(np.array([one + 2.0 ** -8]))[0] == 0x3F80       # tie -> even
+    assert O.f64_to_bf16_bits(np.array([one + 3 * 2.0 ** -8]))[0] == 0x3F82   # tie -> even
+    assert O.f64_to_bf16_bits(np.array([one + 2.0 ** -8 + 2.0 ** -30]))[0] == 0x3F81
+
+
+def test_reorder_identity_fp64():
+    """The library applies W2 after the attention sum; in exact arithmetic this equals
+    attending over the predicted values (softmax weights sum to one)."""
+    rng = np.random.default_rng(8)
+    n, d, Fh = 40, 8, 12
+    kp = rng.standard_normal((n, d))
+    w1, b1 = rng.standard_normal((Fh, d)), rng.standard_normal(Fh)
+    w2, b2 = rng.standard_normal((d, Fh)), rng.standard_normal(d)
+    r = np.zeros((n, d))
+    r[::3] = rng.standard_normal((len(range(0, n, 3)), d))
+    z = rng.standard_normal(n)
+    p = np.exp(z - z.max())
+    plain = (p / p.sum()) @ (O.predictor(kp, w1, b1, w2, b2, O.ACT_SILU) + r)
+    hid = O.activation(kp @ w1.T + b1, O.ACT_SILU)
+    reorder = (w2 @ (p @ hid) + p @ r) / p.sum() + b2
+    assert np.allclose(plain, reorder, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------
+# mutation tests: plant a plausible mistake in the oracle; some pin must fail
+# ----------------------------------------------------------------------------------
+def _fails(check, monkeypatch, name, bad):
+    monkeypatch.setattr(O, name, bad)
+    with pytest.raises(AssertionError):
+        check(O)
+
+
+def test_mutation_rope_wrong_sign(monkeypatch):
+    orig = O.rope_rotate
+    _fails(lambda M: (check_rope_closed_form(M)), monkeypatch, "rope_rotate",
+           lambda x, pos, theta, inverse=False: orig(x, pos, theta, not inverse))
+
+
+def test_mutation_rope_not_reapplied(monkeypatch):
+    orig = O.rope_rotate
+
+    def bad(x, pos, theta, inverse=False):
+        return orig(x, pos, theta, True) if inverse else np.asarray(x, np.float64)
+    _fails(check_full_rank_exactness, monkeypatch, "rope_rotate", bad)
+
+
+def test_mutation_transposed_basis_head(monkeypatch):
+    def bad(coef, basis, h, d):
+        bh = np.asarray(basis)[h::basis.shape[0] // d][:d]
+        return np.asarray(coef) @ bh.T
+    _fails(check_projection, monkeypatch, "rebuild_keys", bad)
+
+
+def test_mutation_residual_not_added(monkeypatch):
+    orig = O.reconstruct_chunks
+
+    def bad(sel_bh, coef_b, basis, h, d, chunk, res_idx_bh, res_val_bh, chunk_ptr_bh,
+            *rest):
+        zero_ptr = np.zeros_like(np.asarray(chunk_ptr_bh))
+        return orig(sel_bh, coef_b, basis, h, d, chunk, res_idx_bh, res_val_bh, zero_ptr,
+                    *rest)
+    _fails(check_full_rank_exactness, monkeypatch, "reconstruct_chunks", bad)
+
+
+def test_mutation_scores_sum_not_max(monkeypatch):
+    _fails(check_landmarks_and_scores, monkeypatch, "chunk_scores",
+           lambda qg, lm: (np.asarray(lm) @ np.asarray(qg).T).sum(axis=1))
+
+
+def test_mutation_topk_ties_to_higher(monkeypatch):
+    def bad(scores, k):
+        s = np.asarray(scores, np.float64)
+        n = s.shape[0]
+        order = np.lexsort((-np.arange(n), -s))
+        return np.sort(order[:min(k, n)])
+    _fails(check_topk, monkeypatch, "topk_ascending", bad)
+
+
+def test_mutation_predictor_drops_bias(monkeypatch):
+    orig = O.predictor
+    _fails(check_predictor, monkeypatch, "predictor",
+           lambda x, w1, b1, w2, b2, act: orig(x, w1, 0 * np.asarray(b1), w2, b2, act))
+
+
+def test_mutation_errors_from_rounded_coef(monkeypatch):
+    orig = O.residual_errors
+
+    def bad(v_h, coef_exact, *rest):
+        return orig(v_h, O.round_to_storage(coef_exact, O.STORE_BF16), *rest)
+    _fails(check_residual_pick, monkeypatch, "residual_errors", bad)
+
+
+def test_mutation_landmark_of_prerope_keys(monkeypatch):
+    orig = O.chunk_landmarks
+
+    def bad(k_cache, chunk):
+        return orig(k_cache, chunk) * 1.0001
+    _fails(check_landmarks_and_scores, monkeypatch, "chunk_landmarks", bad)
