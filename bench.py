@@ -1,0 +1,551 @@
+#!/usr/bin/env python
+"""Decode throughput of the LowRAM hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the 32-layer Llama-3-8B-shaped decode at 128K context, batch 8 per GPU
+(16 two-layer xKV groups, rank 160, chunk 8, top-256 chunks, 20% residuals, SiLU
+128-256-128 predictor, bf16), seeded synthetic keys/values encoded on the device by
+lowram_encode. A step = one decode step of all 32 layers (landmark scoring + top-k,
+fused reconstruct-and-attend, combine) for the whole batch; the step's queries change
+every step. The compressed caches stay resident in HBM; per-step inputs (10.2 GB of
+algorithmic reads) are far larger than the 126 MB L2, so no flush is needed.
+
+Multi-GPU (torchrun): every rank decodes its own batch of 8 (independent seeds): weak
+scaling, no collective on the data path; time = max over ranks.
+
+--impl reference times the CPU oracle (oracle/) on the host cores on a bounded sample
+of the same workload (one batch element, one layer per step).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s + achieved HBM GB/s (% of ~8 TB/s) at 128K context"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode only the first L layers (profiling runs)")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------------
+# host-side sharding and cross-rank reduction (covered by gloo tests on CPU)
+# ----------------------------------------------------------------------------------
+def rank_shape(shape, rank: int):
+    """Weak scaling: each rank decodes its own batch with its own seeds."""
+    return shape.replace(seed=shape.seed + 100_000 * rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------------
+# algorithmic bytes / flops (per decode step of one layer)
+# ----------------------------------------------------------------------------------
+def select_bytes(sh) -> int:
+    """Kernel (a): every landmark once, the queries, the selection written."""
+    B, H, d, k = sh.batch, sh.n_kv_heads, sh.head_dim, min(sh.top_k, sh.n_chunks)
+    return B * H * sh.n_chunks * d * 2 + B * sh.n_q_heads * d * 2 + B * H * k * 4
+
+
+def attend_bytes(sh, n_res_rows_selected: int) -> int:
+    """Kernel (b) + combine: gathered coefficients and CSR offsets of the selected chunks,
+    the residual rows they hold (value + index), weights once per KV head, q and out."""
+    B, H, d, r, F = sh.batch, sh.n_kv_heads, sh.head_dim, sh.rank, sh.mlp_hidden
+    k = min(sh.top_k, sh.n_chunks)
+    coef = B * H * k * sh.chunk * r * 2
+    csr = B * H * k * 8 + B * H * k * 4
+    res = n_res_rows_selected * (d * 2 + 4)
+    weights = H * (d * r + F * d + F + d * F + d) * 2
+    io = 2 * B * sh.n_q_heads * d * 2
+    return coef + csr + res + weights + io
+
+
+def attend_tensor_flops(sh) -> int:
+    """Dense tensor-core work of kernel (b): K rebuild (2 d r) and layer 1 (2 d F) per
+    selected token and KV head."""
+    k = min(sh.top_k, sh.n_chunks)
+    per = 2 * sh.head_dim * sh.rank + 2 * sh.head_dim * sh.mlp_hidden
+    return sh.batch * sh.n_kv_heads * k * sh.chunk * per
+
+
+# ----------------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.path = None
+        self.uuid = uuid
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["sampler unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3],
+                             parts[4], parts[5], parts[6], parts[7]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in busy for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(busy), "power_w_max": max(r[2] for r in rows)}
+
+
+# ----------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decode_02_b200 import lowram as L
+    from long_context_decode_02_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    base = synth.CONFIGS[2]
+    n_layers = args.layers or base.n_layers
+    sh = rank_shape(base, rank)
+    cfg = L.make_config(sh)
+    ctx = L.Context(cfg, local)
+    st = sh.torch_dtype
+    B, T, Hk, d = sh.batch, sh.n_tokens, sh.n_kv_heads, sh.head_dim
+
+    # ---- compressed caches of every layer, encoded on the device
+    layers = []
+    enc_ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=dev)
+    enc_ms = []
+    basis64 = basis_dev = None
+    for layer in range(n_layers):
+        if layer % 2 == 0:
+            basis64 = synth.group_basis(sh, layer // 2)
+            basis_dev = basis64.to(st).to(dev)
+        w = synth.layer_weights(sh, layer)
+        wd = [x.to(st).to(dev) for x in w]
+        k = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        v = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        for b in range(B):
+            kb, vb = synth.layer_kv(sh, basis64, w, layer, b, device=dev,
+                                    compute_dtype=torch.float32)
+            k[b], v[b] = kb, vb
+            del kb, vb
+        cache = L.alloc_cache(cfg, dev)
+        params = L.layer_params(basis_dev, *wd)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        L.encode(ctx, k, v, params, cache, enc_ws)
+        e1.record()
+        torch.cuda.synchronize()
+        enc_ms.append(e0.elapsed_time(e1))
+        layers.append({"cache": cache, "params": params, "keep": (basis_dev, wd)})
+        del k, v
+    del enc_ws
+    torch.cuda.empty_cache()
+    assert ctx.last_error() == L.OK, "encode reported a device status"
+
+    # ---- per-step queries (distinct every step) and decode buffers
+    W, K = args.warmup, args.steps
+    n_q = W + K
+    q_all = torch.empty(n_q, n_layers, B, sh.n_q_heads, d, dtype=st, device=dev)
+    for i in range(n_q):
+        for layer in range(n_layers):
+            q_all[i, layer] = synth.queries(sh, layer, i, device=dev)
+    q_buf = torch.empty(n_layers, B, sh.n_q_heads, d, dtype=st, device=dev)
+    out_buf = torch.empty_like(q_buf)
+    kk = min(sh.top_k, sh.n_chunks)
+    sel_buf = torch.empty(n_layers, B, Hk, kk, dtype=torch.int32, device=dev)
+    dec_ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_calls():
+        for layer in range(n_layers):
+            Ld = layers[layer]
+            L.decode_step(ctx, Ld["cache"], Ld["params"], q_buf[layer], out_buf[layer], dec_ws,
+                          sel_out=sel_buf[layer])
+
+    def select_calls():
+        for layer in range(n_layers):
+            L.select_chunks(ctx, layers[layer]["cache"]["landmark"], q_buf[layer],
+                            sel_buf[layer], dec_ws)
+
+    def attend_calls():
+        for layer in range(n_layers):
+            Ld = layers[layer]
+            L.attend_selected(ctx, Ld["cache"], Ld["params"], q_buf[layer], sel_buf[layer],
+                              out_buf[layer], dec_ws)
+
+    with torch.cuda.stream(stream):
+        q_buf.copy_(q_all[0])
+        step_calls()
+        select_calls()
+        attend_calls()
+    torch.cuda.synchronize()
+    assert ctx.last_error() == L.OK
+
+    graphs = {}
+    for name, fn in (("step", step_calls), ("select", select_calls), ("attend", attend_calls)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        graphs[name] = g
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+
+    # ---- main timed region: K graph-replayed steps
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            q_buf.copy_(q_all[i])
+            graphs["step"].replay()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    barrier(dev)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(K):
+            q_buf.copy_(q_all[W + i])
+            graphs["step"].replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dev)
+    ms_step = t0.elapsed_time(t1) / K
+    status = ctx.last_error()
+    assert status == L.OK, f"decode reported device status {status}"
+
+    # ---- per-kernel timing: the same steps as two sub-step graphs, events between them
+    n_kt = min(K, 50)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_kt)]
+    with torch.cuda.stream(stream):
+        for i in range(n_kt):
+            q_buf.copy_(q_all[W + i])
+            ev[i][0].record(stream)
+            graphs["select"].replay()
+            ev[i][1].record(stream)
+            graphs["attend"].replay()
+            ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    ms_a = sum(e[0].elapsed_time(e[1]) for e in ev) / (n_kt * n_layers)
+    ms_b = sum(e[1].elapsed_time(e[2]) for e in ev) / (n_kt * n_layers)
+
+    # residual rows inside the selected chunks (for the attend kernel's algorithmic bytes)
+    n_res_sel = 0
+    for layer in range(n_layers):
+        ptr = layers[layer]["cache"]["chunk_ptr"].long()
+        s = sel_buf[layer].long()
+        n_res_sel += int((ptr.gather(2, s + 1) - ptr.gather(2, s)).sum().item())
+    n_res_sel_per_layer = n_res_sel / n_layers
+
+    # ---- e2e: the public C-ABI call with host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        q_host = q_all[W:W + K].cpu().pin_memory()
+        out_host = torch.empty(out_buf.shape, dtype=st).pin_memory()
+        with torch.cuda.stream(stream):
+            for i in range(min(W, 2)):
+                q_buf.copy_(q_host[i], non_blocking=True)
+                step_calls()
+                out_host.copy_(out_buf, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(dev)
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            u0.record(stream)
+            for i in range(K):
+                q_buf.copy_(q_host[i], non_blocking=True)
+                step_calls()
+                out_host.copy_(out_buf, non_blocking=True)
+            u1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(u0.elapsed_time(u1) / K, dev)
+        e2e = {"value": B * world / (ms_e2e / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(q_buf.numel() * q_buf.element_size()),
+               "d2h_bytes_per_step": int(out_buf.numel() * out_buf.element_size()),
+               "path": "lowram_decode_step per layer (eager), pinned host queries/outputs"}
+    clocks = sampler.stop()
+
+    ms_step_max = max_over_ranks(ms_step, dev)
+    ms_a_max = max_over_ranks(ms_a, dev)
+    ms_b_max = max_over_ranks(ms_b, dev)
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    tc_peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+
+    bytes_a = select_bytes(sh)
+    bytes_b = attend_bytes(sh, int(round(n_res_sel_per_layer)))
+    step_bytes = n_layers * (bytes_a + bytes_b)
+    tokens_per_s = B * world / (ms_step_max / 1e3)
+    hbm_gbs = step_bytes / (ms_step_max / 1e3) / 1e9
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get("score_select_kernel")
+        except Exception:
+            traffic = None
+
+    ach_a = bytes_a / (ms_a_max / 1e3) / 1e9
+    ach_b = bytes_b / (ms_b_max / 1e3) / 1e9
+    tflops_b = attend_tensor_flops(sh) / (ms_b_max / 1e3) / 1e12
+    roofline = {"kernel": "score_select_kernel (landmark scoring + top-k)", "bound": "hbm",
+                "achieved": round(ach_a, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(ach_a / hbm_peak, 4), "traffic": traffic,
+                "peak_source": hbm_src + " (burst copy)",
+                "algorithmic_bytes_per_launch": bytes_a, "us_per_launch": round(ms_a_max * 1e3, 2)}
+    roof_b = {"kernel": "attend_tc_kernel + combine (reconstruct-and-attend)",
+              "bound": "tensor", "achieved_tflops": round(tflops_b, 1), "peak_tflops": tc_peak,
+              "tensor_frac": round(tflops_b / tc_peak, 4), "achieved_gbs": round(ach_b, 1),
+              "hbm_frac": round(ach_b / hbm_peak, 4), "hbm_frac_of_8tbs": round(ach_b / NOMINAL_HBM_GBS, 4),
+              "algorithmic_bytes_per_launch": bytes_b,
+              "tensor_flops_per_launch": attend_tensor_flops(sh),
+              "us_per_launch": round(ms_b_max * 1e3, 2)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_from_device(sh, layers, q_all, W, n_layers, args.cpu_baseline_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, encoded on device",
+        "config": {"workload": f"{base.name}" + ("" if n_layers == base.n_layers else f"-{n_layers}layers"),
+                   "batch_per_gpu": B, "context": T, "layers": n_layers, "kv_heads": Hk,
+                   "q_heads": sh.n_q_heads, "head_dim": d, "rank": sh.rank, "chunk": sh.chunk,
+                   "top_k_chunks": sh.top_k, "residual_frac": sh.res_frac,
+                   "predictor": "SiLU 128-256-128", "parallelism": f"batch replicas x{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "hbm_gbs": round(hbm_gbs, 1), "hbm_frac_of_8tbs": round(hbm_gbs / NOMINAL_HBM_GBS, 4),
+        "hbm_frac_of_measured": round(hbm_gbs / hbm_peak, 4),
+        "algorithmic_bytes_per_step": step_bytes,
+        "roofline": roofline,
+        "roofline_reconstruct_attend": roof_b,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * n_layers * K,
+        "clocks": clocks,
+        "encode": {"ms_per_layer": round(statistics.mean(enc_ms), 2),
+                   "tokens_per_s": round(B * T / (statistics.mean(enc_ms) / 1e3), 1)},
+    }
+    for g in graphs.values():
+        g.reset()
+    del graphs
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def _oracle_unit(O, sh, q, cache_np, p):
+    """Oracle decode of one (batch element, layer) unit."""
+    return O.decode_step(q, cache_np, p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
+                         chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta, act=sh.act)
+
+
+def cpu_baseline_from_device(sh, layers, q_all, W, n_layers, seconds):
+    """The oracle, as it stands, on host cores: decode units of (batch element 0, layer l)
+    with the same stored caches and queries, until ~`seconds` of CPU work."""
+    import numpy as np
+    import torch
+
+    import oracle.lowram_oracle as O
+
+    def f64(t):
+        return t.detach().to("cpu", torch.float64).numpy()
+
+    units, t_total = 0, 0.0
+    layer = 0
+    while t_total < seconds and units < 4 * n_layers:
+        Ld = layers[layer % n_layers]
+        c = Ld["cache"]
+        basis_dev, wd = Ld["keep"]
+        cache_np = {"coef": f64(c["coef"][0:1]), "landmark": f64(c["landmark"][0:1]),
+                    "res_idx": c["res_idx"][0:1].cpu().numpy().astype(np.int64),
+                    "res_val": f64(c["res_val"][0:1]),
+                    "chunk_ptr": c["chunk_ptr"][0:1].cpu().numpy().astype(np.int64)}
+        p = {"basis": f64(basis_dev), "w1": f64(wd[0]), "b1": f64(wd[1]), "w2": f64(wd[2]),
+             "b2": f64(wd[3])}
+        q = f64(q_all[W, layer % n_layers, 0:1])
+        t0 = time.perf_counter()
+        _oracle_unit(O, sh, q, cache_np, p)
+        t_total += time.perf_counter() - t0
+        units += 1
+        layer += 1
+    per_unit = t_total / units
+    return {"value": round(1.0 / (per_unit * n_layers), 4), "unit": "tokens/s",
+            "cores": _threads(), "host_cpus": os.cpu_count(), "kind": "oracle",
+            "sample": f"{units} (batch element 0, layer) decode units of the same workload "
+                      f"({t_total:.1f} s); tokens/s = units/s / {n_layers} layers"}
+
+
+# ----------------------------------------------------------------------------------
+# reference arm: the CPU oracle on the host cores
+# ----------------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle.lowram_oracle as O
+    from long_context_decode_02_b200 import synth
+
+    base = synth.CONFIGS[2]
+    sh = base.replace(batch=1)
+    n_layers = args.layers or base.n_layers
+    # one batch element of layer 0, generated and encoded on the CPU by the oracle
+    basis = synth.group_basis(sh, 0)
+    w = synth.layer_weights(sh, 0)
+    k, v = synth.layer_kv(sh, basis, w, 0, 0, compute_dtype=torch.float32)
+    st = sh.torch_dtype
+    f = lambda t: t.to(st).to(torch.float64).numpy()
+    p = {"basis": f(basis), "w1": f(w[0]), "b1": f(w[1]), "w2": f(w[2]), "b2": f(w[3])}
+    cache = O.encode(f(k)[None], f(v)[None], p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
+                     chunk=sh.chunk, n_res=sh.n_res, theta=sh.theta, act=sh.act,
+                     store=O.STORE_BF16)
+    del k, v
+    W, K = args.warmup, args.steps
+    qs = [synth.queries(sh, 0, i).to(torch.float64).numpy() for i in range(W + K)]
+    for i in range(W):
+        _oracle_unit(O, sh, qs[i], cache, p)
+    t0 = time.perf_counter()
+    for i in range(K):
+        _oracle_unit(O, sh, qs[W + i], cache, p)
+    per_unit = (time.perf_counter() - t0) / K
+    value = 1.0 / (per_unit * n_layers)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K, "warmup": W,
+        "ms_per_step": round(per_unit * n_layers * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, encoded by the oracle",
+        "config": {"workload": base.name, "batch_per_gpu": base.batch, "context": base.n_tokens,
+                   "layers": n_layers, "sampled": "one batch element of layer 0 per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": _threads(),
+                         "host_cpus": os.cpu_count(), "kind": "oracle",
+                         "sample": f"each step = oracle decode of 1 (batch element, layer) "
+                                   f"unit; tokens/s = units/s / {n_layers} layers"},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * lowram.h -- C ABI of liblowram.so: LowRAM's encode and decode-time hot path on one
+ * B200 (sm_100a).
+ *
+ * The method ("LowRAM: Low-Rank Keys and Amortised Values for Composable KV Cache
+ * Compression at Test-Time"; summary on agihunt.info, overview "LowRAM Exploits
+ * Key-Value Predictability to Compress the KV Cache" on cctest.ai, and the abstract):
+ *   - keys: RoPE is inverted, then every token's key (all KV heads of a layer, flattened
+ *     to D = H_kv*d) is projected onto a low-rank basis shared by two adjacent layers
+ *     (xKV); the prefix is cut into chunks whose mean key is kept as a landmark;
+ *   - values: a small per-head key->value MLP predicts V from the rebuilt key; residual
+ *     corrections are stored only for the tokens it predicts worst;
+ *   - decode: the query scores the chunk landmarks, the top-k chunks are selected, only
+ *     their keys (low rank, RoPE re-applied) and values (MLP + residuals) are rebuilt,
+ *     and GQA attention runs over that subset.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers on the context's device unless stated.
+ *     Arrays are dense, row-major, in the order of the brackets given.
+ *   - Element type: every cache, weight, query and output array is stored in
+ *     cfg->dtype (fp32 or bf16); index arrays are int32. Arithmetic is fp32 with fp64
+ *     used to settle selections near their threshold.
+ *   - The caller owns every buffer (inputs, cache, outputs, workspace). The context owns
+ *     only small tables (RoPE cos/sin, a status word, completion counters). Calls
+ *     allocate nothing.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t passed as void*; NULL =
+ *     the legacy default stream). Arguments are validated on the host first; on any
+ *     error nothing is launched and the status says why.
+ *   - Alignment: every pointer must be 16-byte aligned (LOWRAM_ERR_ALIGN otherwise).
+ *   - One context serves one stream at a time: concurrent calls with the same context
+ *     on different streams race on its counters. Use one context per stream.
+ *   - The ABI is per layer. Two layers of one xKV group pass the same basis pointer.
+ */
+#ifndef LOWRAM_H
+#define LOWRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lowram_status {
+  LOWRAM_OK = 0,
+  LOWRAM_ERR_INVALID_ARG = 1,  /* null pointer, unknown enum value                    */
+  LOWRAM_ERR_SHAPE = 2,        /* sizes inconsistent with each other                  */
+  LOWRAM_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned                    */
+  LOWRAM_ERR_UNSUPPORTED = 4,  /* valid sizes this build does not implement           */
+  LOWRAM_ERR_WORKSPACE = 5,    /* workspace smaller than lowram_workspace_size()      */
+  LOWRAM_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed                */
+  LOWRAM_ERR_DEVICE_CHECK = 7, /* a kernel found malformed cache contents (reported by
+                                  lowram_last_error)                                   */
+  LOWRAM_ERR_TIMEOUT = 8       /* a kernel's bounded wait gave up (lowram_last_error)  */
+} lowram_status;
+
+enum { LOWRAM_DTYPE_F32 = 0, LOWRAM_DTYPE_BF16 = 1 };
+enum { LOWRAM_ACT_SILU = 0, LOWRAM_ACT_GELU_ERF = 1 };
+/* Which reconstruct-and-attend kernel decode uses. AUTO picks the tcgen05 tensor-core
+ * kernel where it applies (bf16, d = 128, F = 256, r % 32 == 0, r <= 160, G = 4) and the
+ * CUDA-core kernel otherwise (always for fp32, whose 1e-4 tolerance tensor cores cannot
+ * meet). */
+enum { LOWRAM_DECODE_AUTO = 0, LOWRAM_DECODE_SIMT = 1, LOWRAM_DECODE_TCGEN05 = 2 };
+enum { LOWRAM_OP_ENCODE = 0, LOWRAM_OP_DECODE = 1 };
+
+/* Sizes of one layer call. T % chunk == 0; n_q_heads % n_kv_heads == 0. */
+typedef struct lowram_config {
+  int32_t batch;          /* B                                                          */
+  int32_t n_tokens;       /* T, prefix length (token positions 0 .. T-1)               */
+  int32_t n_kv_heads;     /* H_kv                                                       */
+  int32_t n_q_heads;      /* H_q; G = H_q / H_kv query heads share a KV head (GQA)      */
+  int32_t head_dim;       /* d: 64 or 128                                               */
+  int32_t rank;           /* r: xKV rank, multiple of 16, 16 .. 256                      */
+  int32_t chunk;          /* C: tokens per chunk, one of 1, 2, 4, 8, 16, 32             */
+  int32_t mlp_hidden;     /* F: predictor hidden width, 128 or 256                      */
+  int32_t top_k;          /* chunks selected per step, >= 1; >= T/C selects all         */
+  int32_t n_res;          /* residual rows per (batch, KV head), 0 .. T                 */
+  int32_t act;            /* LOWRAM_ACT_*                                               */
+  int32_t dtype;          /* LOWRAM_DTYPE_*                                             */
+  int32_t decode_variant; /* LOWRAM_DECODE_*                                            */
+  int32_t reserved;       /* must be 0                                                  */
+  double rope_theta;      /* RoPE base; theta_i = rope_theta^(-2i/d)                    */
+} lowram_config;
+
+/* One layer's parameters (inputs; never written).
+ *   basis [H_kv*d][r]   columns orthonormal (precondition, not checked); shared by the two
+ *                       layers of an xKV group ("adjacent layers share the SVD basis")
+ *   w1 [H_kv][F][d], b1 [H_kv][F], w2 [H_kv][d][F], b2 [H_kv][d]:
+ *                       per-head predictor V_hat = w2 act(w1 x + b1) + b2 (x = pre-RoPE key)
+ */
+typedef struct lowram_layer_params {
+  const void* basis;
+  const void* w1;
+  const void* b1;
+  const void* w2;
+  const void* b2;
+} lowram_layer_params;
+
+/* One layer's compressed cache (written by lowram_encode, read by lowram_decode_step).
+ *   coef      [B][T][r]          low-rank key coefficients c_t = basis^T RoPE^-1(K_t)
+ *   landmark  [B][H_kv][T/C][d]  mean post-RoPE key of each chunk
+ *   res_idx   [B][H_kv][n_res]   int32 token indices of the residual rows, ascending
+ *   res_val   [B][H_kv][n_res][d] residual corrections V_t - V_hat_t
+ *   chunk_ptr [B][H_kv][T/C + 1] int32 CSR: rows of chunk c are ptr[c] .. ptr[c+1]-1
+ * The layout is fixed by these shapes, so a cache can be saved and restored byte for
+ * byte (lowram_cache_layout gives the five sizes). res_idx and res_val may be NULL when
+ * n_res == 0. */
+typedef struct lowram_cache {
+  void* coef;
+  void* landmark;
+  int32_t* res_idx;
+  void* res_val;
+  int32_t* chunk_ptr;
+} lowram_cache;
+
+typedef struct lowram_ctx lowram_ctx;
+
+/* Validate a configuration on the host only (no CUDA call). Returns LOWRAM_OK or the
+ * first failing check's status. */
+lowram_status lowram_check_config(const lowram_config* cfg);
+
+/* Create a context on `device`: checks cfg, builds the RoPE tables (two-level cos/sin of
+ * t*theta_i computed in fp64 on the host, stored fp32 and fp64 on the device) and the
+ * counters. *out is set only on success. Destroy with lowram_destroy. */
+lowram_status lowram_create(const lowram_config* cfg, int device, lowram_ctx** out);
+
+/* Free the context's tables. Waits for nothing: the caller must have synchronised any
+ * stream still using the context. NULL is accepted. */
+void lowram_destroy(lowram_ctx* ctx);
+
+/* Host only. bytes_out[0..4] = sizes of coef, landmark, res_idx, res_val, chunk_ptr. */
+lowram_status lowram_cache_layout(const lowram_config* cfg, size_t bytes_out[5]);
+
+/* Host only. Workspace bytes needed by op (LOWRAM_OP_ENCODE or LOWRAM_OP_DECODE). The
+ * workspace needs no initialisation and holds nothing between calls. */
+lowram_status lowram_workspace_size(const lowram_config* cfg, int op, size_t* bytes);
+
+/* Encode one layer's prefix into `out` (all five arrays written).
+ *   k_cache [B][T][H_kv][d]  post-RoPE keys;  v [B][T][H_kv][d] values.
+ * Steps (agihunt summary, key paragraph and value-amortisation paragraph; cctest "How
+ * the method works": Low-rank keys, Amortised values, Residuals for difficult tokens):
+ * invert RoPE, project onto the basis (coef stored rounded), landmarks = chunk means of
+ * the original keys, squared predictor error of every token with the unrounded
+ * coefficients, per (batch, KV head) the n_res largest errors (ties to the lower token;
+ * candidates near the threshold re-scored in fp64), residual rows against the stored
+ * coefficients, chunk CSR. */
+lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
+                            const lowram_layer_params* params, const lowram_cache* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* One decode step of one layer.
+ *   q   [B][H_q][d]  post-RoPE queries (input)
+ *   out [B][H_q][d]  attention output (written)
+ *   sel_out [B][H_kv][k] int32, k = min(top_k, T/C): the selected chunks, ascending
+ *           (written when not NULL)
+ * Steps (agihunt summary, key paragraph; cctest "Selective reconstruction"; abstract):
+ * score every chunk by max over the GQA group of q . landmark, select the top-k (ties to
+ * the lower chunk; candidates near the threshold re-scored in fp64), rebuild the selected
+ * chunks' keys from coef and basis and re-apply RoPE, predict their values with the
+ * per-head MLP plus the stored residuals, and attend over them with scale 1/sqrt(d).
+ * Rebuilt keys and values never reach global memory. */
+lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
+                                 const lowram_layer_params* params, const void* q,
+                                 void* out, int32_t* sel_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Decode sub-step 1 (kernel (a) alone): score every chunk by max over the GQA group of
+ * q . landmark and write the top-k chunks per (batch, KV head), ascending, ties to the
+ * lower chunk (agihunt summary, key paragraph; cctest "Selective reconstruction").
+ *   landmark [B][H_kv][T/C][d]; q [B][H_q][d]; sel_out [B][H_kv][k] int32 (written).
+ * Uses the decode workspace. lowram_decode_step = this + lowram_attend_selected. */
+lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark, const void* q,
+                                   int32_t* sel_out, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/* Decode sub-step 2 (kernel (b) + split-K combine): rebuild the chunks listed in sel
+ * ([B][H_kv][k] int32, k = min(top_k, T/C), each entry in 0 .. T/C-1; out-of-range
+ * entries are skipped and reported through lowram_last_error) and attend over them.
+ *   q [B][H_q][d] (input); out [B][H_q][d] (written). Uses the decode workspace. */
+lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
+                                     const lowram_layer_params* params, const void* q,
+                                     const int32_t* sel, void* out, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Synchronise the device, then return and clear the context's status word: LOWRAM_OK,
+ * LOWRAM_ERR_DEVICE_CHECK (a kernel met a residual index outside its chunk or a CSR
+ * offset out of range, and skipped it) or LOWRAM_ERR_TIMEOUT (a bounded wait expired;
+ * the kernel returned early and its outputs are not valid). */
+lowram_status lowram_last_error(lowram_ctx* ctx);
+
+/* Static string naming a status. */
+const char* lowram_status_string(lowram_status status);
+
+/* Test only (no counterpart in the method): one 128 x 128 tcgen05 tile product
+ * d[m][n] = sum_k a[m][k] * b[n][k] with a [128][K], b [128][K] bf16 row-major (device)
+ * and d [128][128] fp32 (device), staged through the same shared-memory layouts and
+ * descriptors as the tensor-core decode kernel.
+ *   mode 0: K % 32 == 0, 32 <= K <= 256; a and b TMA-loaded with the 64-byte swizzle
+ *           (a in 8-row boxes like the gathered coefficients, b like the basis);
+ *   mode 1: K == 128; a TMA-loaded with the 128-byte swizzle (like W1), b stored by
+ *           threads in the 128-byte-swizzled layout (like the rebuilt keys).
+ * Synchronous: returns after the kernel finished. */
+lowram_status lowram_debug_tc_tile(const void* a, const void* b, float* d, int32_t k,
+                                   int32_t mode, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LOWRAM_H */

@@ -1,0 +1,641 @@
+// Kernel (b), tensor-core form: fused reconstruct-and-attend split-K flash-decode on
+// tcgen05 / TMEM (bf16 storage, d = 128, F = 256, G = 4, C = 8, r % 32 == 0, r <= 160).
+//
+// Method (LowRAM summary on agihunt.info, key paragraph and value-amortisation
+// paragraph; cctest "How the method works": Low-rank keys, Amortised values, Residuals
+// for difficult tokens, Selective reconstruction): rebuild the selected chunks' keys
+// from the xKV coefficients and basis, re-apply RoPE, predict their values with the
+// per-head MLP plus the stored residuals, and attend over them.
+//
+// Exact reordering used here: softmax weights sum to one, so
+//   sum_t p_t (W2 h_t + b2 + R_t) / sum_t p_t = (W2 (sum_t p_t h_t) + sum_t p_t R_t)/l + b2
+// with h_t = act(W1 K~_pre,t + b1): W2 is applied once per query head in the combine
+// kernel instead of once per token, removing a third of the tensor work.
+//
+// Per persistent CTA (one KV head h; weights B_h and W1_h stay in shared memory), per
+// tile of 128 selected tokens (16 chunks of 8):
+//   producer warp : TMA-gathers the 16 chunks' coefficient rows (each chunk is a
+//                   contiguous 8 x r block) into a 64B-swizzled K-major tile.
+//   MMA warp      : K~_pre^T... as D[tok][d] = coef[tok][r] . B_h[d][r]^T   -> TMEM
+//                   H^T  as D[f][tok] = W1[f][d] . K~bf16[tok][d]^T (2 x M=128) -> TMEM
+//   8 epilogue warps (two per TMEM lane quadrant):
+//     A: K~_pre rows from TMEM -> bf16 into shared memory (operand of the H GEMM);
+//        RoPE from host-fp64 tables; logits for the 4 query heads; tile max and
+//        p = 2^(z - m) in fp32 -> shared memory.
+//     B: H^T rows from TMEM (lane = hidden unit f, columns = tokens): act(h + b1) and
+//        Hacc_g[f] += p_g(t) act  (a reduction along each thread's own row);
+//        residual rows of the tile's chunks (CSR spans): Racc_g[j] += p_g(t) R_t[j].
+//     The tile's (m, l, Hacc, Racc) go to a split-K partial; the combine kernel merges
+//     the tiles and applies W2 and b2.
+// The epilogue interleaves A(i+1) before B(i) so the H GEMM of tile i runs under the
+// CUDA-core work of tile i+1; TMEM holds two K~ buffers (2 x 128 columns) and H^T
+// (256 columns). Rebuilt keys and values never leave the SM.
+// Every wait is bounded (~2 s); on expiry the kernel raises a timeout status, drains its
+// own outstanding copies and MMAs (again bounded), frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "device_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace lowram {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128, kF = 256, kG = 4, kTile = 128, kChunk = 8, kChunksPerTile = 16;
+constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2..9 epilogue
+constexpr int kEpiThreads = 256;
+constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
+constexpr int kPartFloats = 2 * kG + kG * kF + 2 * kG * kD;
+
+struct TcMaps {
+  CUtensorMap coef;   // [B*T][r] bf16, box 32 x 8,   64B swizzle
+  CUtensorMap basis;  // [H*d][r] bf16, box 32 x 128, 64B swizzle
+  CUtensorMap w1;     // [H*F][d] bf16, box 64 x 128, 128B swizzle
+};
+
+struct Layout {
+  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, bar, total;
+};
+__host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) {
+  return (x + a - 1) / a * a;
+}
+__host__ __device__ inline Layout make_layout(int r) {
+  Layout L{};
+  const uint32_t kb = (uint32_t)r / 32;
+  L.basis = 0;
+  L.w1 = align_up(L.basis + kb * 8192, 1024);
+  L.coef = L.w1 + 65536;
+  L.kbf = align_up(L.coef + kb * 8192, 1024);
+  L.p = L.kbf + 65536;          // [2][128][4] fp32
+  L.q = L.p + 4096;             // [4][128] fp32
+  L.b1 = L.q + 2048;            // [256] fp32
+  L.zx = L.b1 + 1024;           // [128][4] fp32
+  L.red = L.zx + 2048;          // 512 B of reduction scratch
+  L.bar = L.red + 512;          // barriers + TMEM address holder
+  L.total = L.bar + 256 + 1024; // + alignment slack of the dynamic base
+  return L;
+}
+
+// barrier slots (8 bytes each) inside L.bar
+enum {
+  BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
+  BAR_KT_EMPTY1, BAR_KBF_FULL0, BAR_KBF_FULL1, BAR_KBF_EMPTY0, BAR_KBF_EMPTY1, BAR_H_FULL,
+  BAR_H_EMPTY, BAR_DRAIN, BAR_COUNT
+};
+
+template <int ACT>
+__device__ __forceinline__ float act_fast(float x) {
+  if (ACT == LOWRAM_ACT_SILU) {
+    const float hx = 0.5f * x;
+    return fmaf(hx, tanh_approx(hx), hx);   // x * sigmoid(x) = x/2 (1 + tanh(x/2))
+  }
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+template <int ACT>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int cta_per_head) {
+  const Dims& dm = a.dm;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = align_up(raw, 1024);
+  uint8_t* gbase = smem_raw + (base - raw);
+  const Layout L = make_layout(dm.r);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x / cta_per_head;
+  const int cta_in_head = blockIdx.x % cta_per_head;
+  const int n_items = dm.B * a.n_tiles;
+  const int kb_r = dm.r / 32;
+  const int ksteps_r = dm.r / 16;
+
+  auto bar = [&](int i) { return base + L.bar + 8u * (uint32_t)i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + L.bar + 8 * BAR_COUNT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.bar + 8 * BAR_COUNT + 4);
+  float* sP = reinterpret_cast<float*>(gbase + L.p);
+  float* sQ = reinterpret_cast<float*>(gbase + L.q);
+  float* sB1 = reinterpret_cast<float*>(gbase + L.b1);
+  float* sZx = reinterpret_cast<float*>(gbase + L.zx);
+  float* sRed = reinterpret_cast<float*>(gbase + L.red);  // [4 quadrants][4 g] x 2, ml[2][4][2]
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(BAR_W), 1);
+    mbar_init(bar(BAR_COEF_FULL), 1);
+    mbar_init(bar(BAR_COEF_EMPTY), 1);
+    mbar_init(bar(BAR_KT_FULL0), 1);
+    mbar_init(bar(BAR_KT_FULL1), 1);
+    mbar_init(bar(BAR_KT_EMPTY0), 8);
+    mbar_init(bar(BAR_KT_EMPTY1), 8);
+    mbar_init(bar(BAR_KBF_FULL0), 8);
+    mbar_init(bar(BAR_KBF_FULL1), 8);
+    mbar_init(bar(BAR_KBF_EMPTY0), 1);
+    mbar_init(bar(BAR_KBF_EMPTY1), 1);
+    mbar_init(bar(BAR_H_FULL), 1);
+    mbar_init(bar(BAR_H_EMPTY), 8);
+    mbar_init(bar(BAR_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const int32_t* sel_all = a.sel;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int issued_phase = -1;  // parity of the last coef load issued (for the drain)
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192 + 65536));
+      for (int kb = 0; kb < kb_r; ++kb)
+        tma_load_2d(base + L.basis + kb * 8192, &maps.basis, kb * 32, h * kD, bar(BAR_W));
+      for (int hf = 0; hf < 2; ++hf)
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
+                      h * kF + hf * 128, bar(BAR_W));
+    }
+    int i = 0;
+    for (int it = cta_in_head; it < n_items; it += cta_per_head, ++i) {
+      const int b = it / a.n_tiles, tile = it % a.n_tiles;
+      int got = 0;
+      if (lane == 0) got = mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      int cid = 0;
+      if (lane < kChunksPerTile) {
+        const int slot = tile * kChunksPerTile + lane;
+        if (slot < dm.k) cid = sel_all[((size_t)b * dm.H + h) * dm.k + slot];
+        if (cid < 0 || cid >= dm.Nc) cid = 0;
+      }
+      if (lane == 0)
+        mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
+      __syncwarp();
+      if (lane < kChunksPerTile) {
+        const int row = b * dm.T + cid * kChunk;
+        for (int kb = 0; kb < kb_r; ++kb)
+          tma_load_2d(base + L.coef + kb * 8192 + lane * 512, &maps.coef, kb * 32, row,
+                      bar(BAR_COEF_FULL));
+      }
+      issued_phase = i & 1;
+    }
+    // drain: a load still in flight (only possible after an abort) must land before exit
+    if (lane == 0 && *abort_flag && issued_phase >= 0) {
+      int dummy = 0;
+      mbar_wait_bounded(bar(BAR_COEF_FULL), (uint32_t)issued_phase, (volatile int*)&dummy);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(bar(BAR_W), 0, abort_flag);
+      const uint32_t sb = base + L.basis, sw1 = base + L.w1, sc = base + L.coef;
+      auto issue_k = [&](int i) -> bool {
+        const int u = i & 1;
+        if (!mbar_wait_bounded(bar(BAR_COEF_FULL), i & 1, abort_flag)) return false;
+        if (!mbar_wait_bounded(bar(BAR_KT_EMPTY0 + u), ((i >> 1) & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d_t = tmem + (uint32_t)(u * 128);
+        for (int s = 0; s < ksteps_r; ++s) {
+          const uint32_t off = (uint32_t)((s >> 1) * 8192 + (s & 1) * 32);
+          mma_bf16(d_t, smem_desc_kmajor(sc + off, 512, kSwizzle64B),
+                   smem_desc_kmajor(sb + off, 512, kSwizzle64B), kIdesc, s > 0);
+        }
+        mma_commit(bar(BAR_KT_FULL0 + u));
+        mma_commit(bar(BAR_COEF_EMPTY));
+        return true;
+      };
+      auto issue_h = [&](int i) -> bool {
+        const int u = i & 1;
+        if (!mbar_wait_bounded(bar(BAR_KBF_FULL0 + u), (i >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_bounded(bar(BAR_H_EMPTY), (i & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t skb = base + L.kbf + (uint32_t)u * 32768;
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t d_t = tmem + 256u + (uint32_t)hf * 128u;
+          for (int s = 0; s < 8; ++s) {
+            const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+            mma_bf16(d_t, smem_desc_kmajor(sw1 + hf * 32768 + off, 1024, kSwizzle128B),
+                     smem_desc_kmajor(skb + off, 1024, kSwizzle128B), kIdesc, s > 0);
+          }
+        }
+        mma_commit(bar(BAR_H_FULL));
+        mma_commit(bar(BAR_KBF_EMPTY0 + u));
+        return true;
+      };
+      int n_mine = 0;
+      for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
+      if (ok && n_mine > 0) ok = issue_k(0);
+      for (int i = 0; ok && i < n_mine; ++i) {
+        if (i + 1 < n_mine) ok = issue_k(i + 1);
+        if (ok) ok = issue_h(i);
+      }
+      // drain every MMA this thread issued before TMEM is released
+      mma_commit(bar(BAR_DRAIN));
+      int dummy = 0;
+      mbar_wait_bounded(bar(BAR_DRAIN), 0, (volatile int*)&dummy);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;             // 0..7
+    const int qd = warp & 3;             // TMEM lane quadrant this warp may access
+    const int hf = ew >> 2;              // column half
+    const int et = threadIdx.x - 64;     // 0..255
+    const int trow = 32 * qd + lane;     // token row (A) / hidden-unit row within a half (B)
+    const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
+    const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
+    const int32_t* ptr_all = a.chunk_ptr;
+    const int32_t* ridx_all = a.res_idx;
+    const __nv_bfloat16* rval_all = (const __nv_bfloat16*)a.res_val;
+    const __nv_bfloat16* q_all = (const __nv_bfloat16*)a.q;
+    float* s_ml = sRed + 64;  // [2][4][2]
+
+    for (int i = et; i < kF; i += kEpiThreads)
+      sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
+
+    int n_mine = 0;
+    for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
+    bool ok = true;
+
+    auto item_of = [&](int i, int& b, int& tile) {
+      const int it = cta_in_head + i * cta_per_head;
+      b = it / a.n_tiles;
+      tile = it % a.n_tiles;
+    };
+
+    // ---- part A of tile i
+    // A failed (timed-out) wait never changes the sequence of named barriers: the
+    // thread carries on with `good` false so every barrier is still reached.
+    auto part_a = [&](int i) -> bool {
+      bool good = true;
+      int b, tile;
+      item_of(i, b, tile);
+      const int u = i & 1;
+      named_bar_sync(1, kEpiThreads);  // previous readers of sQ / sZx are done
+      for (int e = et; e < kG * kD; e += kEpiThreads)
+        sQ[e] = __bfloat162float(q_all[((size_t)b * dm.Hq + (size_t)h * kG) * kD + e]);
+      const int slot = tile * kChunksPerTile + (trow >> 3);
+      int cid = slot < dm.k ? sel_all[((size_t)b * dm.H + h) * dm.k + slot] : -1;
+      if (cid >= dm.Nc) cid = -1;
+      const bool valid = cid >= 0;
+      const int pos = valid ? cid * kChunk + (trow & 7) : 0;
+
+      good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag);
+      tc_fence_after();
+      float x[32], y[32];
+      const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + 32 * hf);
+      tmem_ld_x32(tcol, x);
+      tmem_ld_x32(tcol + 64, y);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY0 + u));
+
+      // K~_pre in bf16 -> shared memory, 128B-swizzled K-major [tok][d]
+      good = mbar_wait_bounded(bar(BAR_KBF_EMPTY0 + u), ((i >> 1) & 1) ^ 1, abort_flag) && good;
+      const uint32_t skb = base + L.kbf + (uint32_t)u * 32768;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        st_shared_v4(skb + sw128_offset(trow, 4 * hf + cc),
+                     pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]), pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]),
+                     pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]), pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]));
+        st_shared_v4(skb + 16384 + sw128_offset(trow, 4 * hf + cc),
+                     pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]), pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]),
+                     pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]), pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL0 + u));
+
+      named_bar_sync(1, kEpiThreads);  // sQ ready
+      // RoPE on pairs (32hf + i, 64 + 32hf + i) and partial logits
+      float z[kG] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int pi = 32 * hf + e;
+        const float2 cs = rope_cs32(a.rope, pi, pos);
+        const float xr = x[e] * cs.x - y[e] * cs.y;
+        const float yr = x[e] * cs.y + y[e] * cs.x;
+#pragma unroll
+        for (int g = 0; g < kG; ++g)
+          z[g] = fmaf(sQ[g * kD + pi], xr, fmaf(sQ[g * kD + 64 + pi], yr, z[g]));
+      }
+      if (hf == 1) *reinterpret_cast<float4*>(sZx + 4 * trow) = make_float4(z[0], z[1], z[2], z[3]);
+      named_bar_sync(1, kEpiThreads);
+      if (hf == 0) {
+        const float4 o = *reinterpret_cast<const float4*>(sZx + 4 * trow);
+        z[0] = valid ? (z[0] + o.x) * zscale : -INFINITY;
+        z[1] = valid ? (z[1] + o.y) * zscale : -INFINITY;
+        z[2] = valid ? (z[2] + o.z) * zscale : -INFINITY;
+        z[3] = valid ? (z[3] + o.w) * zscale : -INFINITY;
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          const float m = warp_max(z[g]);
+          if (lane == 0) sRed[qd * 4 + g] = m;
+        }
+        named_bar_sync(2, 128);
+        float m[kG], pv[kG];
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          m[g] = fmaxf(fmaxf(sRed[g], sRed[4 + g]), fmaxf(sRed[8 + g], sRed[12 + g]));
+          pv[g] = valid ? ex2_approx(z[g] - m[g]) : 0.f;
+        }
+        *reinterpret_cast<float4*>(sP + u * 512 + 4 * trow) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          const float l = warp_sum(pv[g]);
+          if (lane == 0) sRed[16 + qd * 4 + g] = l;
+        }
+        named_bar_sync(2, 128);
+        if (ew == 0 && lane < kG) {
+          const int g = lane;
+          s_ml[u * 8 + g * 2 + 0] = m[g];
+          s_ml[u * 8 + g * 2 + 1] = sRed[16 + g] + sRed[20 + g] + sRed[24 + g] + sRed[28 + g];
+        }
+      }
+      named_bar_sync(1, kEpiThreads);  // P and (m, l) of tile i visible to all
+      return good;
+    };
+
+    // ---- part B of tile i
+    auto part_b = [&](int i) -> bool {
+      int b, tile;
+      item_of(i, b, tile);
+      const int u = i & 1;
+      const int p = b * dm.H + h;
+      float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
+      const bool good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag);
+      tc_fence_after();
+      const int f = 128 * hf + trow;
+      const float bias = sB1[f];
+      float hacc[kG] = {0.f, 0.f, 0.f, 0.f};
+      const float4* P4 = reinterpret_cast<const float4*>(sP + u * 512);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float hv[32];
+        tmem_ld_x32(tmem + lane_addr + 256u + (uint32_t)(hf * 128 + 32 * c), hv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float av = act_fast<ACT>(hv[e] + bias);
+          const float4 pv = P4[32 * c + e];
+          hacc[0] = fmaf(pv.x, av, hacc[0]);
+          hacc[1] = fmaf(pv.y, av, hacc[1]);
+          hacc[2] = fmaf(pv.z, av, hacc[2]);
+          hacc[3] = fmaf(pv.w, av, hacc[3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
+#pragma unroll
+      for (int g = 0; g < kG; ++g) part[2 * kG + g * kF + f] = hacc[g];
+
+      // residual rows of the tile's chunks; thread = column j, rows split by half
+      const int j = trow;
+      float racc[kG] = {0.f, 0.f, 0.f, 0.f};
+      const int32_t* ptr = ptr_all + (size_t)p * (dm.Nc + 1);
+      const int32_t* ridx = ridx_all + (size_t)p * dm.n_res;
+      const __nv_bfloat16* rval = rval_all + (size_t)p * dm.n_res * kD;
+      for (int slot = 0; slot < kChunksPerTile; ++slot) {
+        const int gs = tile * kChunksPerTile + slot;
+        if (gs >= dm.k) break;
+        const int cid = sel_all[(size_t)p * dm.k + gs];
+        if (cid < 0 || cid >= dm.Nc) continue;
+        const int e0 = ptr[cid], e1 = ptr[cid + 1];
+        if (e0 < 0 || e1 < e0 || e1 > dm.n_res || e1 - e0 > kChunk) {
+          if (j == 0) raise_status(a.status, kStatusDeviceCheck);
+          continue;
+        }
+        for (int e = e0 + hf; e < e1; e += 2) {
+          const int tt = ridx[e] - cid * kChunk;
+          if (tt < 0 || tt >= kChunk) {
+            if (j == 0) raise_status(a.status, kStatusDeviceCheck);
+            continue;
+          }
+          const float4 pv = P4[slot * kChunk + tt];
+          const float rv = __bfloat162float(rval[(size_t)e * kD + j]);
+          racc[0] = fmaf(pv.x, rv, racc[0]);
+          racc[1] = fmaf(pv.y, rv, racc[1]);
+          racc[2] = fmaf(pv.z, rv, racc[2]);
+          racc[3] = fmaf(pv.w, rv, racc[3]);
+        }
+      }
+      float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
+#pragma unroll
+      for (int g = 0; g < kG; ++g) pr[g * kD + j] = racc[g];
+      if (ew == 0 && lane < 2 * kG) part[lane] = s_ml[u * 8 + lane];
+      return good;
+    };
+
+    // Every epilogue thread runs the full sequence; once the abort flag is set, the
+    // remaining waits return at once and the results are discarded by the caller.
+    if (n_mine > 0) ok = part_a(0) && ok;
+    for (int i = 0; i < n_mine; ++i) {
+      if (i + 1 < n_mine) ok = part_a(i + 1) && ok;
+      ok = part_b(i) && ok;
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) raise_status(a.status, kStatusTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// --------------------------------------------------------------------- debug tile
+// d[m][n] = sum_k a[m][k] b[n][k]. mode 0: both operands TMA-loaded with the 64B swizzle
+// exactly as coef (8-row boxes) and basis (128-row boxes) in the decode kernel; mode 1:
+// a TMA-loaded with the 128B swizzle like W1, b written by threads with the 128B swizzle
+// like K~bf16 (K = 128).
+__global__ void __launch_bounds__(128, 1)
+debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_constant__ CUtensorMap mb,
+                     const __nv_bfloat16* bsrc, float* d, int K, int mode, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = align_up(raw, 1024);
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sa = base, sb = base + 65536;
+  const uint32_t barf = base + 131072, bard = barf + 8;
+  uint32_t* holder = reinterpret_cast<uint32_t*>(gbase + 131072 + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + 131072 + 20);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(barf, 1);
+    mbar_init(bard, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(holder), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *holder;
+  const int kb32 = K / 32;
+  if (mode == 1) {
+    // b by threads: row n = threadIdx.x, 128B-swizzled K-major, two 64-wide K blocks
+    const int n = threadIdx.x;
+    for (int c = 0; c < 16; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(bsrc + (size_t)n * 128 + 8 * c);
+      st_shared_v4(sb + (c >> 3) * 16384 + sw128_offset(n, c & 7), v.x, v.y, v.z, v.w);
+    }
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok;
+    if (mode == 0) {
+      mbar_arrive_expect_tx(barf, (uint32_t)(2 * kb32 * 8192));
+      for (int kb = 0; kb < kb32; ++kb) {
+        for (int c = 0; c < 16; ++c) tma_load_2d(sa + kb * 8192 + c * 512, &ma, kb * 32, c * 8, barf);
+        tma_load_2d(sb + kb * 8192, &mb, kb * 32, 0, barf);
+      }
+    } else {
+      mbar_arrive_expect_tx(barf, 2u * 16384u);
+      for (int kb = 0; kb < 2; ++kb) tma_load_2d(sa + kb * 16384, &ma, kb * 64, 0, barf);
+    }
+    ok = mbar_wait_bounded(barf, 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      if (mode == 0) {
+        for (int s = 0; s < K / 16; ++s) {
+          const uint32_t off = (uint32_t)((s >> 1) * 8192 + (s & 1) * 32);
+          mma_bf16(tmem, smem_desc_kmajor(sa + off, 512, kSwizzle64B),
+                   smem_desc_kmajor(sb + off, 512, kSwizzle64B), kIdesc, s > 0);
+        }
+      } else {
+        for (int s = 0; s < 8; ++s) {
+          const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
+          mma_bf16(tmem, smem_desc_kmajor(sa + off, 1024, kSwizzle128B),
+                   smem_desc_kmajor(sb + off, 1024, kSwizzle128B), kIdesc, s > 0);
+        }
+      }
+    }
+    mma_commit(bard);
+    if (!mbar_wait_bounded(bard, 0, abort_flag)) ok = false;
+    if (!ok) raise_status(status, kStatusTimeout);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (!*abort_flag) {
+    const int m = threadIdx.x;  // warp w reads lanes 32w..32w+31
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      tmem_ld_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(32 * c), v);
+      tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) d[(size_t)m * 128 + 32 * c + e] = v[e];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// --------------------------------------------------------------------- host helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor map over a row-major [rows][cols] array.
+bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Dims& dm) {
+  return dm.dtype == LOWRAM_DTYPE_BF16 && dm.d == kD && dm.F == kF && dm.G == kG &&
+         dm.C == kChunk && dm.r % 32 == 0 && dm.r >= 32 && dm.r <= 160 &&
+         (dm.act == LOWRAM_ACT_SILU || dm.act == LOWRAM_ACT_GELU_ERF) &&
+         (dm.k * kChunk + kTile - 1) / kTile <= 64;
+}
+
+size_t attend_tc_part_floats(const Dims& dm, int n_tiles) {
+  return (size_t)dm.B * dm.H * n_tiles * kPartFloats;
+}
+
+cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
+  const Dims& dm = a.dm;
+  TcMaps maps;
+  if (!make_map_2d(&maps.coef, a.coef, dm.r, (uint64_t)dm.B * dm.T, 32, 8,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_2d(&maps.basis, a.basis, dm.r, (uint64_t)dm.H * kD, 32, 128,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_2d(&maps.w1, a.w1, kD, (uint64_t)dm.H * kF, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const Layout L = make_layout(dm.r);
+  const int n_items = dm.B * a.n_tiles;
+  int cph = num_sms / dm.H;
+  if (cph < 1) cph = 1;
+  if (cph > n_items) cph = n_items;
+  cudaError_t e;
+  if (dm.act == LOWRAM_ACT_SILU) {
+    auto kern = attend_tc_kernel<LOWRAM_ACT_SILU>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)L.total)) != cudaSuccess) return e;
+    kern<<<dm.H * cph, kThreads, L.total, s>>>(a, maps, cph);
+  } else {
+    auto kern = attend_tc_kernel<LOWRAM_ACT_GELU_ERF>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)L.total)) != cudaSuccess) return e;
+    kern<<<dm.H * cph, kThreads, L.total, s>>>(a, maps, cph);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, int mode,
+                                 int* status, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (mode == 0) {
+    if (!make_map_2d(&ma, a, (uint64_t)k, 128, 32, 8, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_2d(&mb, b, (uint64_t)k, 128, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map_2d(&ma, a, 128, 128, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    mb = ma;
+  }
+  const int smem = 131072 + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(debug_tc_tile_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  debug_tc_tile_kernel<<<1, 128, smem, s>>>(ma, mb, (const __nv_bfloat16*)b, d, k, mode, status);
+  return cudaGetLastError();
+}
+
+}  // namespace lowram

@@ -1,0 +1,414 @@
+// Kernel (c): encode one layer's prefix into the compressed cache.
+//
+// Method (LowRAM summary on agihunt.info, key paragraph: RoPE is inverted before the
+// keys are projected onto the xKV basis shared by two adjacent layers, chunk mean keys
+// are the landmarks; value-cache-amortisation and ablation paragraphs, cctest "How the
+// method works": a per-head key->value predictor, residuals kept only for the
+// worst-reconstructed tokens, chosen by error):
+//   E1 K_pre = R(t)^T K_cache                      (fp32, host-fp64 RoPE tables)
+//   E2 c_t = B^T K_pre,t over D = H_kv*d            -> coef (stored rounded)
+//   E3 L_c = mean of the chunk's post-RoPE keys      -> landmark
+//   E4 e_t,h = ||V_t,h - MLP_h(B_h c_t)||^2 with the unrounded c (fp32)
+//   E5 per (b, h): the n_res largest e (ties -> lower t). fp32 radix select finds the
+//      threshold; tokens within 2e-3 relative of it are re-scored with the whole chain
+//      recomputed in fp64 and ranked exactly; ascending res_idx and the chunk CSR.
+//   E6 R_t = V_t,h - MLP_h(B_h coef_stored,t) for the picked tokens -> res_val
+// Encode runs once per prefix; it is not on the per-token decode path.
+#include <cuda_bf16.h>
+
+#include "device_common.cuh"
+
+namespace lowram {
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kTE = 16;          // tokens per CTA in the projection / residual kernels
+constexpr int kSelEncThreads = 1024;
+constexpr int kRescoreCtas = 96; // CTAs per (b, h) looping over the fp64 candidates
+
+// E3: landmarks, one thread per output element.
+template <typename T>
+__global__ void landmark_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const size_t n = (size_t)dm.B * dm.H * dm.Nc * dm.d;
+  for (size_t o = (size_t)blockIdx.x * blockDim.x + threadIdx.x; o < n;
+       o += (size_t)gridDim.x * blockDim.x) {
+    const int j = (int)(o % dm.d);
+    size_t rest = o / dm.d;
+    const int c = (int)(rest % dm.Nc);
+    rest /= dm.Nc;
+    const int h = (int)(rest % dm.H);
+    const int b = (int)(rest / dm.H);
+    float acc = 0.f;
+    for (int i = 0; i < dm.C; ++i)
+      acc += ldf((const T*)a.k_cache, (((size_t)b * dm.T + (size_t)c * dm.C + i) * dm.H + h) * dm.d + j);
+    ((T*)a.landmark)[o] = from_f<T>(acc / (float)dm.C);
+  }
+}
+
+// Rebuild keys for kTE tokens and run head h's predictor. cs [kTE][r] holds the
+// coefficients; on return vh [kTE][D] holds V_hat. hid is [kTE][FH] scratch.
+template <typename T, int D, int FH>
+__device__ void predict_tile(const EncodeArgs& a, int h, const float* cs, float* vh,
+                             float* hid) {
+  const int r = a.dm.r, tid = threadIdx.x;
+  {
+    constexpr int NG = kEncThreads / D, R = kTE / NG;
+    const int j = tid % D, tg = tid / D;
+    const T* brow = (const T*)a.basis + ((size_t)h * D + j) * r;
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.f;
+    for (int kk = 0; kk < r; ++kk) {
+      const float bj = ldf(brow, kk);
+#pragma unroll
+      for (int i = 0; i < R; ++i) acc[i] = fmaf(bj, cs[(tg + NG * i) * r + kk], acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) vh[(tg + NG * i) * D + j] = acc[i];   // K~_pre for now
+  }
+  __syncthreads();
+  {
+    constexpr int NG = kEncThreads / FH, R = kTE / NG;
+    const int f = tid % FH, tg = tid / FH;
+    const T* wrow = (const T*)a.w1 + ((size_t)h * FH + f) * D;
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.f;
+    for (int j = 0; j < D; ++j) {
+      const float w = ldf(wrow, j);
+#pragma unroll
+      for (int i = 0; i < R; ++i) acc[i] = fmaf(w, vh[(tg + NG * i) * D + j], acc[i]);
+    }
+    const float bias = ldf((const T*)a.b1, (size_t)h * FH + f);
+#pragma unroll
+    for (int i = 0; i < R; ++i) hid[(tg + NG * i) * FH + f] = act_f(acc[i] + bias, a.dm.act);
+  }
+  __syncthreads();
+  {
+    constexpr int NG = kEncThreads / D, R = kTE / NG;
+    const int j = tid % D, tg = tid / D;
+    const T* wrow = (const T*)a.w2 + ((size_t)h * D + j) * FH;
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.f;
+    for (int f = 0; f < FH; ++f) {
+      const float w = ldf(wrow, f);
+#pragma unroll
+      for (int i = 0; i < R; ++i) acc[i] = fmaf(w, hid[(tg + NG * i) * FH + f], acc[i]);
+    }
+    const float bias = ldf((const T*)a.b2, (size_t)h * D + j);
+#pragma unroll
+    for (int i = 0; i < R; ++i) vh[(tg + NG * i) * D + j] = acc[i] + bias;
+  }
+  __syncthreads();
+}
+
+// E1 + E2 + E4 for kTE tokens of one batch element.
+template <typename T, int D, int FH>
+__global__ void __launch_bounds__(kEncThreads) project_error_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const int b = blockIdx.y, t0 = blockIdx.x * kTE, tid = threadIdx.x;
+  const int H = dm.H, r = dm.r, Dt = H * D;
+  extern __shared__ float sm[];
+  float* kp = sm;                 // [kTE][Dt]
+  float* cs = kp + kTE * Dt;      // [kTE][r]
+  float* vh = cs + kTE * r;       // [kTE][D]
+  float* hid = vh + kTE * D;      // [kTE][FH]
+  const T* kc = (const T*)a.k_cache;
+
+  // E1: inverse rotation, pairs (i, i + D/2) of every head
+  for (int o = tid; o < kTE * H * (D / 2); o += blockDim.x) {
+    const int i = o % (D / 2);
+    const int h = (o / (D / 2)) % H;
+    const int t = o / ((D / 2) * H);
+    const int pos = t0 + t;
+    const size_t base = (((size_t)b * dm.T + pos) * H + h) * D;
+    const float x = ldf(kc, base + i), y = ldf(kc, base + i + D / 2);
+    const float2 c2 = rope_cs32(a.rope, i, pos);
+    kp[t * Dt + h * D + i] = x * c2.x + y * c2.y;
+    kp[t * Dt + h * D + i + D / 2] = y * c2.x - x * c2.y;
+  }
+  __syncthreads();
+  // E2: projection onto the basis
+  if (tid < r) {
+    float acc[kTE];
+#pragma unroll
+    for (int t = 0; t < kTE; ++t) acc[t] = 0.f;
+    const T* bcol = (const T*)a.basis + tid;
+    for (int i = 0; i < Dt; ++i) {
+      const float bv = ldf(bcol, (size_t)i * r);
+#pragma unroll
+      for (int t = 0; t < kTE; ++t) acc[t] = fmaf(bv, kp[t * Dt + i], acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kTE; ++t) {
+      cs[t * r + tid] = acc[t];
+      ((T*)a.coef)[((size_t)b * dm.T + t0 + t) * r + tid] = from_f<T>(acc[t]);
+    }
+  }
+  __syncthreads();
+  // E4: per head, predictor on the rebuilt key and squared error against V
+  const T* vin = (const T*)a.v;
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int h = 0; h < H; ++h) {
+    predict_tile<T, D, FH>(a, h, cs, vh, hid);
+    for (int o = tid; o < kTE * D; o += blockDim.x) {
+      const int t = o / D, j = o - t * D;
+      const float dv = ldf(vin, (((size_t)b * dm.T + t0 + t) * H + h) * D + j) - vh[o];
+      vh[o] = dv * dv;
+    }
+    __syncthreads();
+    for (int t = warp; t < kTE; t += kEncThreads / 32) {
+      float s = 0.f;
+      for (int j = lane; j < D; j += 32) s += vh[t * D + j];
+      s = warp_sum(s);
+      if (lane == 0) a.err[((size_t)b * H + h) * dm.T + t0 + t] = s;
+    }
+    __syncthreads();
+  }
+}
+
+// E5a: per (b, h) threshold and classification. flags: 1 = in, 2 = fp64 candidate.
+__global__ void __launch_bounds__(kSelEncThreads) residual_threshold_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const int p = blockIdx.x, T = dm.T, tid = threadIdx.x;
+  const float* e = a.err + (size_t)p * T;
+  uint8_t* flags = a.flags + (size_t)p * T;
+  int* cidx = a.cand_idx + (size_t)p * T;
+  __shared__ unsigned hist[256];
+  __shared__ unsigned bc[4];
+  __shared__ float fscr[33];
+  __shared__ int iscr[33];
+  __shared__ int cnt;
+  if (dm.n_res == 0 || dm.n_res >= T) {
+    const uint8_t f = dm.n_res == 0 ? 0 : 1;
+    for (int i = tid; i < T; i += blockDim.x) flags[i] = f;
+    if (tid == 0) { a.cand_count[p] = 0; a.in_count[p] = dm.n_res == 0 ? 0 : T; }
+    return;
+  }
+  float mx = 0.f;
+  for (int i = tid; i < T; i += blockDim.x) mx = fmaxf(mx, fabsf(e[i]));
+  mx = block_max(mx, fscr);
+  const uint32_t tk = block_kth_largest(T, dm.n_res, [&](int i) { return f2key(e[i]); },
+                                        hist, bc);
+  const double tau = (double)key2f(tk);
+  const double delta = 2e-3 * fabs(tau) + 1e-6 * (double)mx + 1e-30;
+  const double hi = tau + delta, lo = tau - delta;
+  if (tid == 0) cnt = 0;
+  __syncthreads();
+  int n_in = 0;
+  for (int i = tid; i < T; i += blockDim.x) {
+    const double x = (double)e[i];
+    uint8_t f = 0;
+    if (x > hi) {
+      f = 1;
+      ++n_in;
+    } else if (x >= lo) {
+      f = 2;
+      cidx[atomicAdd(&cnt, 1)] = i;
+    }
+    flags[i] = f;
+  }
+  int total;
+  (void)block_exclusive_scan(n_in, iscr, &total);
+  if (tid == 0) { a.in_count[p] = total; a.cand_count[p] = cnt; }
+}
+
+// E5b: fp64 error of every candidate: the whole chain recomputed in fp64 from the
+// stored inputs (inputs widen exactly; fp64 RoPE tables; fp64 exp / erf).
+template <typename T, int D, int FH>
+__global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const int p = blockIdx.y, b = p / dm.H, h = p % dm.H, tid = threadIdx.x;
+  const int H = dm.H, r = dm.r, Dt = H * D;
+  extern __shared__ double smd[];
+  double* kp = smd;            // [Dt]
+  double* c64 = kp + Dt;       // [r]
+  double* kt = c64 + r;        // [D]
+  double* hid = kt + D;        // [FH]
+  double* red = hid + FH;      // [kEncThreads / 32]
+  const int n = a.cand_count[p];
+  const T* kc = (const T*)a.k_cache;
+  for (int j = blockIdx.x; j < n; j += gridDim.x) {
+    const int t = a.cand_idx[(size_t)p * dm.T + j];
+    for (int o = tid; o < H * (D / 2); o += blockDim.x) {
+      const int i = o % (D / 2), hh = o / (D / 2);
+      const size_t base = (((size_t)b * dm.T + t) * H + hh) * D;
+      const double x = ldd(kc, base + i), y = ldd(kc, base + i + D / 2);
+      const double2 c2 = rope_cs64(a.rope, i, t);
+      kp[hh * D + i] = x * c2.x + y * c2.y;
+      kp[hh * D + i + D / 2] = y * c2.x - x * c2.y;
+    }
+    __syncthreads();
+    for (int kk = tid; kk < r; kk += blockDim.x) {
+      double acc = 0.0;
+      for (int i = 0; i < Dt; ++i) acc += ldd((const T*)a.basis, (size_t)i * r + kk) * kp[i];
+      c64[kk] = acc;
+    }
+    __syncthreads();
+    for (int jj = tid; jj < D; jj += blockDim.x) {
+      double acc = 0.0;
+      for (int kk = 0; kk < r; ++kk)
+        acc += ldd((const T*)a.basis, ((size_t)h * D + jj) * r + kk) * c64[kk];
+      kt[jj] = acc;
+    }
+    __syncthreads();
+    for (int f = tid; f < FH; f += blockDim.x) {
+      double acc = ldd((const T*)a.b1, (size_t)h * FH + f);
+      for (int jj = 0; jj < D; ++jj) acc += ldd((const T*)a.w1, ((size_t)h * FH + f) * D + jj) * kt[jj];
+      hid[f] = act_d(acc, dm.act);
+    }
+    __syncthreads();
+    double sq = 0.0;
+    for (int jj = tid; jj < D; jj += blockDim.x) {
+      double acc = ldd((const T*)a.b2, (size_t)h * D + jj);
+      for (int f = 0; f < FH; ++f) acc += ldd((const T*)a.w2, ((size_t)h * D + jj) * FH + f) * hid[f];
+      const double dv = ldd((const T*)a.v, (((size_t)b * dm.T + t) * H + h) * D + jj) - acc;
+      sq += dv * dv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if ((tid & 31) == 0) red[tid >> 5] = sq;
+    __syncthreads();
+    if (tid == 0) {
+      double s = 0.0;
+      for (int w = 0; w < kEncThreads / 32; ++w) s += red[w];
+      a.cand_e64[(size_t)p * dm.T + j] = s;
+    }
+    __syncthreads();
+  }
+}
+
+// E5c: exact ranking of the candidates, ascending compaction, chunk CSR.
+__global__ void __launch_bounds__(kSelEncThreads) residual_finalize_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const int p = blockIdx.x, T = dm.T, tid = threadIdx.x;
+  uint8_t* flags = a.flags + (size_t)p * T;
+  const int* cidx = a.cand_idx + (size_t)p * T;
+  const double* ce = a.cand_e64 + (size_t)p * T;
+  int32_t* ridx = a.res_idx + (size_t)p * dm.n_res;
+  int32_t* ptr = a.chunk_ptr + (size_t)p * (dm.Nc + 1);
+  __shared__ int iscr[33];
+  const int n_w = a.cand_count[p];
+  const int need = dm.n_res - a.in_count[p];
+  for (int j = tid; j < n_w; j += blockDim.x) {
+    const double sj = ce[j];
+    const int ij = cidx[j];
+    int rank = 0;
+    for (int m = 0; m < n_w; ++m) {
+      const double sm = ce[m];
+      rank += (sm > sj) || (sm == sj && cidx[m] < ij);
+    }
+    flags[ij] = rank < need ? 1 : 0;
+  }
+  __syncthreads();
+  int base = 0;
+  for (int c0 = 0; c0 < T; c0 += blockDim.x) {
+    const int i = c0 + tid;
+    const int f = (i < T && flags[i] == 1) ? 1 : 0;
+    int total;
+    const int ex = block_exclusive_scan(f, iscr, &total);
+    if (f && base + ex < dm.n_res) ridx[base + ex] = i;
+    base += total;
+  }
+  __syncthreads();
+  // ptr[c] = number of residual tokens below c*C (binary search in the ascending list)
+  for (int c = tid; c <= dm.Nc; c += blockDim.x) {
+    const int key = c * dm.C;
+    int lo = 0, hi = dm.n_res;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (ridx[mid] < key) lo = mid + 1; else hi = mid;
+    }
+    ptr[c] = lo;
+  }
+}
+
+// E6: residual rows against the STORED coefficients.
+template <typename T, int D, int FH>
+__global__ void __launch_bounds__(kEncThreads) residual_rows_kernel(const EncodeArgs a) {
+  const Dims& dm = a.dm;
+  const int p = blockIdx.y, b = p / dm.H, h = p % dm.H, tid = threadIdx.x;
+  const int r = dm.r, s0 = blockIdx.x * kTE;
+  extern __shared__ float sm[];
+  float* cs = sm;                 // [kTE][r]
+  float* vh = cs + kTE * r;       // [kTE][D]
+  float* hid = vh + kTE * D;      // [kTE][FH]
+  __shared__ int s_tok[kTE];
+  const int32_t* ridx = a.res_idx + (size_t)p * dm.n_res;
+  if (tid < kTE) s_tok[tid] = (s0 + tid < dm.n_res) ? ridx[s0 + tid] : -1;
+  __syncthreads();
+  for (int o = tid; o < kTE * r; o += blockDim.x) {
+    const int t = o / r, kk = o - t * r;
+    const int tok = s_tok[t];
+    cs[o] = tok >= 0 ? ldf((const T*)a.coef, ((size_t)b * dm.T + tok) * r + kk) : 0.f;
+  }
+  __syncthreads();
+  predict_tile<T, D, FH>(a, h, cs, vh, hid);
+  for (int o = tid; o < kTE * D; o += blockDim.x) {
+    const int t = o / D, j = o - t * D;
+    const int tok = s_tok[t];
+    if (tok < 0) continue;
+    const float v = ldf((const T*)a.v, (((size_t)b * dm.T + tok) * dm.H + h) * D + j);
+    ((T*)a.res_val)[((size_t)p * dm.n_res + s0 + t) * D + j] = from_f<T>(v - vh[o]);
+  }
+}
+
+template <typename T, int D, int FH>
+cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
+  const Dims& dm = a.dm;
+  cudaError_t e;
+  {
+    const size_t n = (size_t)dm.B * dm.H * dm.Nc * dm.d;
+    const int blocks = (int)((n + 255) / 256 < 65535 * 8 ? (n + 255) / 256 : 65535 * 8);
+    landmark_kernel<T><<<blocks, 256, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  {
+    const size_t smem = sizeof(float) * ((size_t)kTE * dm.H * D + (size_t)kTE * dm.r +
+                                         kTE * D + kTE * FH);
+    auto kern = project_error_kernel<T, D, FH>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess) return e;
+    kern<<<dim3(dm.T / kTE, dm.B), kEncThreads, smem, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  residual_threshold_kernel<<<dm.B * dm.H, kSelEncThreads, 0, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    const size_t smem = sizeof(double) * ((size_t)dm.H * D + dm.r + D + FH + kEncThreads / 32);
+    auto kern = residual_rescore_kernel<T, D, FH>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess) return e;
+    kern<<<dim3(kRescoreCtas, dm.B * dm.H), kEncThreads, smem, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  residual_finalize_kernel<<<dm.B * dm.H, kSelEncThreads, 0, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (dm.n_res > 0) {
+    const size_t smem = sizeof(float) * ((size_t)kTE * dm.r + kTE * D + kTE * FH);
+    auto kern = residual_rows_kernel<T, D, FH>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess) return e;
+    kern<<<dim3((dm.n_res + kTE - 1) / kTE, dm.B * dm.H), kEncThreads, smem, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s) {
+  const bool bf = a.dm.dtype == LOWRAM_DTYPE_BF16;
+  const int D = a.dm.d, FH = a.dm.F;
+#define LR_CASE(DD, FF)                                                    \
+  if (D == DD && FH == FF)                                                 \
+    return bf ? launch_encode_typed<__nv_bfloat16, DD, FF>(a, s)           \
+              : launch_encode_typed<float, DD, FF>(a, s);
+  LR_CASE(64, 128) LR_CASE(64, 256) LR_CASE(128, 128) LR_CASE(128, 256)
+#undef LR_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lowram

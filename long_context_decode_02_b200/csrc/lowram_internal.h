@@ -1,0 +1,105 @@
+// Internal declarations of liblowram: launch argument blocks and launchers.
+// Not part of the public ABI (include/lowram.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/lowram.h"
+
+namespace lowram {
+
+// Status-word bits set by kernels (read back by lowram_last_error).
+constexpr int kStatusDeviceCheck = 1;
+constexpr int kStatusTimeout = 2;
+
+// Two-level RoPE tables. For pair i and position t:
+//   lo[i * kRopeLo + (t & (kRopeLo-1))] = (cos, sin)((t mod kRopeLo) * theta_i)
+//   hi[i * n_hi   + (t >> kRopeLoBits)] = (cos, sin)((t - t mod kRopeLo) * theta_i)
+// and the angle of t is recovered by the angle-addition formulas. Entries are computed
+// in fp64 on the host, so the fp32 copy carries only its own rounding.
+constexpr int kRopeLoBits = 9;
+constexpr int kRopeLo = 1 << kRopeLoBits;
+
+struct RopeTables {
+  const float2* lo32;
+  const float2* hi32;
+  const double2* lo64;
+  const double2* hi64;
+  int n_hi;
+};
+
+struct Dims {
+  int B, T, H, Hq, G, d, r, C, F, Nc, k, n_res, act, dtype;
+};
+
+// ---------------- decode: landmark scoring + top-k selection ----------------
+struct SelectArgs {
+  Dims dm;
+  const void* landmark;   // [B][H][Nc][d]
+  const void* q;          // [B][Hq][d]
+  float* scores;          // ws [B*H][Nc]
+  double* cand_s64;       // ws [B*H][Nc]
+  int* cand_idx;          // ws [B*H][Nc]
+  uint8_t* flags;         // ws [B*H][Nc]
+  int* counters;          // ctx [B*H], zero between launches
+  int32_t* sel;           // [B*H][k]
+  int* status;
+  int slice_len;          // chunks scored per CTA
+  int n_slices;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+
+// ---------------- decode: reconstruct + attend ----------------
+struct AttendArgs {
+  Dims dm;
+  const void* coef;       // [B][T][r]
+  const int32_t* res_idx; // [B][H][n_res]
+  const void* res_val;    // [B][H][n_res][d]
+  const int32_t* chunk_ptr; // [B][H][Nc+1]
+  const void* basis;      // [H*d][r]
+  const void* w1; const void* b1; const void* w2; const void* b2;
+  const void* q;          // [B][Hq][d]
+  void* out;              // [B][Hq][d]
+  const int32_t* sel;     // [B*H][k]
+  float* part;            // ws partials
+  RopeTables rope;
+  int* status;
+  int n_tiles;            // tiles per (b, h)
+  int tile_tokens;
+};
+size_t attend_simt_part_floats(const Dims& dm, int n_tiles);
+int attend_simt_tile_tokens(const Dims& dm);
+cudaError_t launch_attend_simt(const AttendArgs& a, cudaStream_t s);
+
+bool attend_tc_supported(const Dims& dm);
+size_t attend_tc_part_floats(const Dims& dm, int n_tiles);
+constexpr int kTcTileTokens = 128;
+cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s);
+
+cudaError_t launch_combine(const AttendArgs& a, bool reorder_form, cudaStream_t s);
+
+// ---------------- encode ----------------
+struct EncodeArgs {
+  Dims dm;
+  const void* k_cache;    // [B][T][H][d]
+  const void* v;          // [B][T][H][d]
+  const void* basis; const void* w1; const void* b1; const void* w2; const void* b2;
+  void* coef; void* landmark; int32_t* res_idx; void* res_val; int32_t* chunk_ptr;
+  float* err;             // ws [B*H][T]
+  double* cand_e64;       // ws [B*H][T]
+  int* cand_idx;          // ws [B*H][T]
+  uint8_t* flags;         // ws [B*H][T]
+  int* cand_count;        // ws [B*H]
+  int* in_count;          // ws [B*H]
+  RopeTables rope;
+  int* status;
+};
+cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
+
+// ---------------- test-only ----------------
+cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, int mode,
+                                 int* status, cudaStream_t s);
+
+}  // namespace lowram

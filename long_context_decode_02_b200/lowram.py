@@ -1,0 +1,237 @@
+"""ctypes binding of liblowram.so (include/lowram.h). Argument marshalling only: every
+step of encode and decode runs in the library's CUDA kernels.
+
+Importing this module loads the library and raises if it is missing; there is no
+fallback path. Build it with ``python -m long_context_decode_02_b200.build``.
+
+Functions with the C names take raw integers/pointers; the helpers below them take
+torch tensors (device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblowram.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lowram.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m long_context_decode_02_b200.build`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_SHAPE = 2
+ERR_ALIGN = 3
+ERR_UNSUPPORTED = 4
+ERR_WORKSPACE = 5
+ERR_CUDA = 6
+ERR_DEVICE_CHECK = 7
+ERR_TIMEOUT = 8
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+ACT_SILU = 0
+ACT_GELU_ERF = 1
+DECODE_AUTO = 0
+DECODE_SIMT = 1
+DECODE_TCGEN05 = 2
+OP_ENCODE = 0
+OP_DECODE = 1
+
+
+class lowram_config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_tokens", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("chunk", ctypes.c_int32), ("mlp_hidden", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_res", ctypes.c_int32),
+                ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("decode_variant", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("rope_theta", ctypes.c_double)]
+
+
+class lowram_layer_params(ctypes.Structure):
+    _fields_ = [("basis", ctypes.c_void_p), ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
+class lowram_cache(ctypes.Structure):
+    _fields_ = [("coef", ctypes.c_void_p), ("landmark", ctypes.c_void_p),
+                ("res_idx", ctypes.c_void_p), ("res_val", ctypes.c_void_p),
+                ("chunk_ptr", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_S = ctypes.c_int
+_sig = {
+    "lowram_check_config": (_S, [ctypes.POINTER(lowram_config)]),
+    "lowram_create": (_S, [ctypes.POINTER(lowram_config), ctypes.c_int, ctypes.POINTER(_P)]),
+    "lowram_destroy": (None, [_P]),
+    "lowram_cache_layout": (_S, [ctypes.POINTER(lowram_config), ctypes.POINTER(ctypes.c_size_t)]),
+    "lowram_workspace_size": (_S, [ctypes.POINTER(lowram_config), ctypes.c_int,
+                                   ctypes.POINTER(ctypes.c_size_t)]),
+    "lowram_encode": (_S, [_P, _P, _P, ctypes.POINTER(lowram_layer_params),
+                           ctypes.POINTER(lowram_cache), _P, ctypes.c_size_t, _P]),
+    "lowram_decode_step": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P,
+                                ctypes.c_size_t, _P]),
+    "lowram_select_chunks": (_S, [_P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_attend_selected": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                    ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P,
+                                    ctypes.c_size_t, _P]),
+    "lowram_last_error": (_S, [_P]),
+    "lowram_status_string": (ctypes.c_char_p, [_S]),
+    "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+    globals()[_name] = _f
+EXPORTED = tuple(_sig)
+
+
+class LowRAMError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = lowram_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+def check(status: int, where: str) -> None:
+    if status != OK:
+        raise LowRAMError(status, where)
+
+
+# ------------------------------------------------------------------ torch helpers
+def make_config(shape, decode_variant: int = DECODE_AUTO, **over) -> lowram_config:
+    """lowram_config from a workload shape (long_context_decode_02_b200.synth.Shape)."""
+    c = lowram_config(batch=shape.batch, n_tokens=shape.n_tokens, n_kv_heads=shape.n_kv_heads,
+                      n_q_heads=shape.n_q_heads, head_dim=shape.head_dim, rank=shape.rank,
+                      chunk=shape.chunk, mlp_hidden=shape.mlp_hidden, top_k=shape.top_k,
+                      n_res=shape.n_res, act=shape.act,
+                      dtype=DTYPE_BF16 if shape.dtype == "bf16" else DTYPE_F32,
+                      decode_variant=decode_variant, reserved=0, rope_theta=shape.theta)
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def _ptr(t):
+    """Device address of a dense row-major tensor (strided views are refused: the C ABI
+    takes plain pointers and reads every array densely)."""
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError(f"tensor of shape {tuple(t.shape)} is not contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def cache_layout(cfg: lowram_config):
+    out = (ctypes.c_size_t * 5)()
+    check(lowram_cache_layout(ctypes.byref(cfg), out), "lowram_cache_layout")
+    return list(out)
+
+
+def workspace_size(cfg: lowram_config, op: int) -> int:
+    n = ctypes.c_size_t()
+    check(lowram_workspace_size(ctypes.byref(cfg), op, ctypes.byref(n)), "lowram_workspace_size")
+    return n.value
+
+
+class Context:
+    """Owns a lowram_ctx (RoPE tables, status word, counters) on one device."""
+
+    def __init__(self, cfg: lowram_config, device: int = 0):
+        self.cfg = cfg
+        self._h = ctypes.c_void_p()
+        check(lowram_create(ctypes.byref(cfg), device, ctypes.byref(self._h)), "lowram_create")
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if self._h:
+            lowram_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def last_error(self) -> int:
+        return lowram_last_error(self._h)
+
+
+def layer_params(basis, w1, b1, w2, b2) -> lowram_layer_params:
+    return lowram_layer_params(_ptr(basis), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
+
+
+def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr) -> lowram_cache:
+    return lowram_cache(_ptr(coef), _ptr(landmark), _ptr(res_idx), _ptr(res_val),
+                        _ptr(chunk_ptr))
+
+
+def alloc_cache(cfg: lowram_config, device):
+    """Device tensors of one layer's compressed cache (shapes of include/lowram.h)."""
+    import torch
+    dt = torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
+    B, T, H, d = cfg.batch, cfg.n_tokens, cfg.n_kv_heads, cfg.head_dim
+    nc = T // cfg.chunk
+    return {
+        "coef": torch.empty(B, T, cfg.rank, dtype=dt, device=device),
+        "landmark": torch.empty(B, H, nc, d, dtype=dt, device=device),
+        "res_idx": torch.empty(B, H, cfg.n_res, dtype=torch.int32, device=device),
+        "res_val": torch.empty(B, H, cfg.n_res, d, dtype=dt, device=device),
+        "chunk_ptr": torch.empty(B, H, nc + 1, dtype=torch.int32, device=device),
+    }
+
+
+def encode(ctx: Context, k_cache, v, params: lowram_layer_params, cache: dict, workspace,
+           stream=None) -> None:
+    cs = cache_struct(**cache)
+    check(lowram_encode(ctx.handle, _ptr(k_cache), _ptr(v), ctypes.byref(params),
+                        ctypes.byref(cs), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                        _stream(stream)), "lowram_encode")
+
+
+def decode_step(ctx: Context, cache: dict, params: lowram_layer_params, q, out, workspace,
+                sel_out=None, stream=None) -> None:
+    cs = cache_struct(**cache)
+    check(lowram_decode_step(ctx.handle, ctypes.byref(cs), ctypes.byref(params), _ptr(q),
+                             _ptr(out), _ptr(sel_out), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_decode_step")
+
+
+def select_chunks(ctx: Context, landmark, q, sel_out, workspace, stream=None) -> None:
+    check(lowram_select_chunks(ctx.handle, _ptr(landmark), _ptr(q), _ptr(sel_out),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)), "lowram_select_chunks")
+
+
+def attend_selected(ctx: Context, cache: dict, params: lowram_layer_params, q, sel, out,
+                    workspace, stream=None) -> None:
+    cs = cache_struct(**cache)
+    check(lowram_attend_selected(ctx.handle, ctypes.byref(cs), ctypes.byref(params), _ptr(q),
+                                 _ptr(sel), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_attend_selected")
+
+
+def debug_tc_tile(a, b, d, k: int, mode: int, stream=None) -> None:
+    check(lowram_debug_tc_tile(_ptr(a), _ptr(b), _ptr(d), k, mode, _stream(stream)),
+          "lowram_debug_tc_tile")

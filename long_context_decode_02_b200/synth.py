@@ -112,7 +112,7 @@ def group_basis(shape: Shape, group: int, device="cpu") -> torch.Tensor:
     a = torch.randn(shape.kv_dim, shape.rank, generator=g, device=device,
                     dtype=torch.float64)
     q, _ = torch.linalg.qr(a, mode="reduced")
-    return q
+    return q.contiguous()
 
 
 def layer_weights(shape: Shape, layer: int, device="cpu"):

@@ -1,0 +1,102 @@
+"""Shared test plumbing: build one layer's seeded inputs, store them in the workload's
+precision, run the oracle on exactly the stored values, and compare selections with the
+tie rule (an index may differ only if its fp64 score lies within 1e-5 of the k-th)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle.lowram_oracle as O
+from long_context_decode_02_b200 import synth
+
+STORE = {"f32": O.STORE_F32, "bf16": O.STORE_BF16}
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def stored_layer(shape: synth.Shape, layer: int = 0, batch=None):
+    """Stored (storage-dtype) CPU tensors of one layer: k_cache, v [B,T,H,d], basis and
+    weights, plus their exact fp64 values for the oracle."""
+    group = layer // 2
+    basis = synth.group_basis(shape, group)
+    w = synth.layer_weights(shape, layer)
+    bs = range(shape.batch) if batch is None else batch
+    ks, vs = [], []
+    for b in bs:
+        k, v = synth.layer_kv(shape, basis, w, layer, b)
+        ks.append(k)
+        vs.append(v)
+    st = shape.torch_dtype
+    t = {"k": torch.stack(ks), "v": torch.stack(vs), "basis": basis.to(st),
+         "w1": w[0].to(st), "b1": w[1].to(st), "w2": w[2].to(st), "b2": w[3].to(st)}
+    return {n: x.contiguous() for n, x in t.items()}
+
+
+def oracle_params(t):
+    return dict(basis=f64(t["basis"]), w1=f64(t["w1"]), b1=f64(t["b1"]), w2=f64(t["w2"]),
+                b2=f64(t["b2"]))
+
+
+def oracle_encode(shape, t):
+    p = oracle_params(t)
+    return O.encode(f64(t["k"]), f64(t["v"]), p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
+                    chunk=shape.chunk, n_res=shape.n_res, theta=shape.theta, act=shape.act,
+                    store=STORE[shape.dtype])
+
+
+def cache_to_device(shape, cache, device):
+    st = shape.torch_dtype
+
+    def dense(x, dt):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dt).contiguous().to(device)
+    return {
+        "coef": dense(cache["coef"], st),
+        "landmark": dense(cache["landmark"], st),
+        "res_idx": dense(cache["res_idx"], torch.int32),
+        "res_val": dense(cache["res_val"], st),
+        "chunk_ptr": dense(cache["chunk_ptr"], torch.int32),
+    }
+
+
+def cache_to_oracle(cache_dev):
+    return {"coef": f64(cache_dev["coef"]), "landmark": f64(cache_dev["landmark"]),
+            "res_idx": cache_dev["res_idx"].cpu().numpy().astype(np.int64),
+            "res_val": f64(cache_dev["res_val"]),
+            "chunk_ptr": cache_dev["chunk_ptr"].cpu().numpy().astype(np.int64)}
+
+
+def kth_largest(x: np.ndarray, k: int) -> float:
+    return float(np.sort(x)[::-1][min(k, len(x)) - 1])
+
+
+def compare_selection(got: np.ndarray, want: np.ndarray, scores: np.ndarray, k: int,
+                      rel: float = 1e-5, abs_floor: float = 0.0):
+    """Per row: sets must match except indices whose score is within rel*|s_k| (+floor)
+    of the k-th largest score. Returns the number of tie differences; asserts the rest."""
+    got = np.asarray(got).reshape(-1, got.shape[-1])
+    want = np.asarray(want).reshape(-1, want.shape[-1])
+    sc = np.asarray(scores).reshape(-1, scores.shape[-1])
+    ties = 0
+    for r in range(got.shape[0]):
+        assert np.all(np.diff(got[r]) > 0), "selection not strictly ascending"
+        g, w = set(got[r].tolist()), set(want[r].tolist())
+        if g == w:
+            continue
+        sk = kth_largest(sc[r], k)
+        win = rel * abs(sk) + abs_floor
+        for i in g ^ w:
+            assert abs(sc[r][i] - sk) <= win, (
+                f"row {r}: index {i} differs with score {sc[r][i]!r}, k-th {sk!r}")
+            ties += 1
+    return ties
+
+
+def rel_err(got: np.ndarray, want: np.ndarray) -> float:
+    """max |got - want| / RMS(want)."""
+    rms = math.sqrt(float(np.mean(np.asarray(want, np.float64) ** 2)))
+    return float(np.max(np.abs(np.asarray(got, np.float64) - want))) / max(rms, 1e-300)

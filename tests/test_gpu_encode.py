@@ -1,0 +1,101 @@
+"""Encode parity through the C ABI: GPU lowram_encode against the oracle's encode on the
+same stored keys, values, basis and weights.
+
+Bar: residual token indices bit-exact except ties within 1e-5 of the k-th error
+(reported); chunk CSR identical where the indices are; coefficients and landmarks
+within one storage rounding; residual rows within the decode tolerance. End-to-end
+(GPU encode -> GPU decode vs oracle encode -> oracle decode) checks outputs only."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.lowram_oracle as O
+from long_context_decode_02_b200 import synth
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L(cuda_device):
+    from long_context_decode_02_b200 import lowram
+    return lowram
+
+
+def gpu_encode(L, shape, t, device):
+    cfg = L.make_config(shape)
+    ctx = L.Context(cfg, device.index or 0)
+    cache = L.alloc_cache(cfg, device)
+    td = {k: v.to(device) for k, v in t.items()}
+    params = L.layer_params(*(td[n] for n in ("basis", "w1", "b1", "w2", "b2")))
+    ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=device)
+    L.encode(ctx, td["k"], td["v"], params, cache, ws)
+    st = ctx.last_error()
+    assert st == L.OK, L.lowram_status_string(st)
+    return ctx, cfg, cache, td, params
+
+
+def ulp_bound(x, dtype):
+    """One unit in the last place of the storage format at |x|."""
+    mant = 7 if dtype == "bf16" else 23
+    e = np.floor(np.log2(np.maximum(np.abs(x), 1e-30)))
+    return 2.0 ** (e - mant)
+
+
+def check_encode(L, shape, device):
+    t = H.stored_layer(shape, 0)
+    enc = H.oracle_encode(shape, t)
+    ctx, cfg, cache, td, params = gpu_encode(L, shape, t, device)
+    got_idx = cache["res_idx"].cpu().numpy()
+    ties = H.compare_selection(got_idx, enc["res_idx"], enc["err"], shape.n_res)
+    same = np.all(got_idx == enc["res_idx"], axis=-1)
+    ptr = cache["chunk_ptr"].cpu().numpy()
+    assert np.array_equal(ptr[same], enc["chunk_ptr"][same])
+    for b in range(shape.batch):
+        for h in range(shape.n_kv_heads):
+            cnt = np.bincount(got_idx[b, h] // shape.chunk, minlength=shape.n_chunks)
+            assert np.array_equal(np.diff(ptr[b, h]), cnt)
+    # coefficients / landmarks: the GPU's fp32 value rounds to the same storage value, or
+    # to a neighbour when the exact value lies within fp32 error of a rounding midpoint
+    for name in ("coef", "landmark"):
+        g = H.f64(cache[name])
+        w = enc[name]
+        assert np.all(np.abs(g - w) <= ulp_bound(w, shape.dtype) * 1.01 + 1e-6 * np.abs(w).max()), name
+    # residual rows of the tokens both sides picked
+    gv, wv = H.f64(cache["res_val"]), enc["res_val"]
+    assert H.rel_err(gv[same], wv[same]) <= H.TOL[shape.dtype]
+    return ties, ctx, cfg, cache, td, params, t, enc
+
+
+def test_config0_encode(L, cuda_device):
+    ties, *_ = check_encode(L, synth.CONFIGS[0], cuda_device)
+    print("config0 residual tie differences:", ties)
+
+
+def test_config1_encode(L, cuda_device):
+    ties, *_ = check_encode(L, synth.CONFIGS[1], cuda_device)
+    print("config1 residual tie differences:", ties)
+
+
+@pytest.mark.parametrize("cfg_id", [0, 1])
+def test_end_to_end(L, cuda_device, cfg_id):
+    sh = synth.CONFIGS[cfg_id]
+    ties, ctx, cfg, cache, td, params, t, enc = check_encode(L, sh, cuda_device)
+    p = H.oracle_params(t)
+    for step in range(2):
+        q = synth.queries(sh, 0, step)
+        out = torch.empty_like(q, device=cuda_device)
+        ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8,
+                         device=cuda_device)
+        L.decode_step(ctx, cache, params, q.to(cuda_device), out, ws)
+        assert ctx.last_error() == L.OK
+        want, _ = O.decode_step(H.f64(q), enc, p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
+                                chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta, act=sh.act)
+        err = H.rel_err(H.f64(out), want)
+        assert err <= H.TOL[sh.dtype], err
+
+
+def test_encode_edge_budgets(L, cuda_device):
+    for over in (dict(res_frac=0.0), dict(res_frac=1.0), dict(res_frac=1.0 / 1024)):
+        sh = synth.CONFIGS[0].replace(n_tokens=1024, **over)
+        check_encode(L, sh, cuda_device)
