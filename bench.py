@@ -373,13 +373,8 @@ def run_ours(args):
     tokens_per_s = B * world / (ms_step_max / 1e3)
     hbm_gbs = step_bytes / (ms_step_max / 1e3) / 1e9
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get("score_select_kernel")
-        except Exception:
-            traffic = None
+    traffic = measured_traffic("score_select_kernel")
+    traffic_b = measured_traffic("attend_tc_kernel")
 
     ach_a = bytes_a / (ms_a_max / 1e3) / 1e9
     ach_b = bytes_b / (ms_b_max / 1e3) / 1e9
@@ -393,7 +388,7 @@ def run_ours(args):
               "bound": "tensor", "achieved_tflops": round(tflops_b, 1), "peak_tflops": tc_peak,
               "tensor_frac": round(tflops_b / tc_peak, 4), "achieved_gbs": round(ach_b, 1),
               "hbm_frac": round(ach_b / hbm_peak, 4), "hbm_frac_of_8tbs": round(ach_b / NOMINAL_HBM_GBS, 4),
-              "algorithmic_bytes_per_launch": bytes_b,
+              "algorithmic_bytes_per_launch": bytes_b, "traffic": traffic_b,
               "tensor_flops_per_launch": attend_tensor_flops(sh),
               "us_per_launch": round(ms_b_max * 1e3, 2)}
 
@@ -432,6 +427,20 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu capture of `kernel`, or None when the
+    kernel's sources changed since that capture."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+        m = hashlib.sha256()
+        for f in rec["sources"]:
+            m.update(open(os.path.join(ROOT, f), "rb").read())
+        return rec["bytes_per_launch"] if m.hexdigest()[:16] == rec["sources_sha256_16"] else None
+    except Exception:
+        return None
 
 
 def _threads():

@@ -234,8 +234,10 @@ __global__ void __launch_bounds__(256) combine_plain_kernel(const AttendArgs a) 
   for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
     const int g = i / D, j = i - g * D;
     float M = -INFINITY;
+#pragma unroll 8
     for (int t = 0; t < a.n_tiles; ++t) M = fmaxf(M, part[t * tstride + g * (2 + D)]);
     float L = 0.f, O = 0.f;
+#pragma unroll 8
     for (int t = 0; t < a.n_tiles; ++t) {
       const float* pt = part + t * tstride + g * (2 + D);
       const float w = pt[0] == -INFINITY ? 0.f : expf(pt[0] - M);
@@ -248,67 +250,66 @@ __global__ void __launch_bounds__(256) combine_plain_kernel(const AttendArgs a) 
 
 // Combine, W2-after-attention form used by the tensor-core kernel. Partial of a tile:
 // [G][2] (m in log2 units, l), [G][F] sum_t e_t act(h_t), [2][G][D] sum_t e_t R_t.
-//   out_g = (W2 Hs_g + Rs_g) / L_g + b2,   Hs/Rs/L the e^{m_t-M}-weighted tile sums.
+//   out_g = (W2 Hs_g + Rs_g) / L_g + b2,   Hs/Rs/L the 2^(m_t-M)-weighted tile sums.
+// One CTA per (b, h, g); n_tiles <= 64 (checked on the host).
 template <typename T, int D, int FH>
 __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a) {
   const Dims& dm = a.dm;
-  const int p = blockIdx.x, b = p / dm.H, h = p % dm.H, G = dm.G;
+  const int G = dm.G;
+  const int p = blockIdx.x / G, g = blockIdx.x % G;
+  const int b = p / dm.H, h = p % dm.H;
+  const int n = a.n_tiles;
   const size_t tstride = (size_t)G * 2 + (size_t)G * FH + 2 * (size_t)G * D;
-  const float* part = a.part + (size_t)p * a.n_tiles * tstride;
-  __shared__ float s_w[kMaxG][64];
-  __shared__ float s_L[kMaxG];
-  __shared__ float hs[kMaxG * FH];
-  __shared__ float rs[kMaxG * D];
-  const int tid = threadIdx.x;
-  // tile weights (n_tiles <= 64 is checked on the host)
-  if (tid < G) {
-    const int g = tid;
-    float M = -INFINITY;
-    for (int t = 0; t < a.n_tiles; ++t) M = fmaxf(M, part[t * tstride + 2 * g]);
-    float L = 0.f;
-    for (int t = 0; t < a.n_tiles; ++t) {
-      const float m = part[t * tstride + 2 * g];
-      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
-      s_w[g][t] = w;
-      L = fmaf(w, part[t * tstride + 2 * g + 1], L);
-    }
-    s_L[g] = L;
+  const float* part = a.part + (size_t)p * n * tstride;
+  __shared__ float s_w[64];
+  __shared__ float s_L;
+  __shared__ float hs[FH];
+  __shared__ float rs[D];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (warp == 0) {
+    const float m0 = lane < n ? part[lane * tstride + 2 * g] : -INFINITY;
+    const float m1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g] : -INFINITY;
+    const float l0 = lane < n ? part[lane * tstride + 2 * g + 1] : 0.f;
+    const float l1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g + 1] : 0.f;
+    const float M = warp_max(fmaxf(m0, m1));
+    const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+    const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    const float L = warp_sum(w0 * l0 + w1 * l1);
+    s_w[lane] = w0;
+    s_w[lane + 32] = w1;
+    if (lane == 0) s_L = L;
   }
   __syncthreads();
-  for (int i = tid; i < G * FH; i += blockDim.x) {
-    const int g = i / FH;
+  for (int f = tid; f < FH; f += blockDim.x) {
+    const float* src = part + 2 * G + (size_t)g * FH + f;
     float acc = 0.f;
-    for (int t = 0; t < a.n_tiles; ++t) acc = fmaf(s_w[g][t], part[t * tstride + 2 * G + i], acc);
-    hs[i] = acc;
+#pragma unroll 8
+    for (int t = 0; t < n; ++t) acc = fmaf(s_w[t], src[t * tstride], acc);
+    hs[f] = acc;
   }
-  for (int i = tid; i < G * D; i += blockDim.x) {
-    const int g = i / D;
+  for (int j = tid; j < D; j += blockDim.x) {
+    const float* src = part + 2 * G + (size_t)G * FH + (size_t)g * D + j;
     float acc = 0.f;
-    for (int t = 0; t < a.n_tiles; ++t) {
-      const float* pr = part + t * tstride + 2 * G + (size_t)G * FH;
-      acc = fmaf(s_w[g][t], pr[i] + pr[G * D + i], acc);
-    }
-    rs[i] = acc;
+#pragma unroll 8
+    for (int t = 0; t < n; ++t) acc = fmaf(s_w[t], src[t * tstride] + src[t * tstride + G * D], acc);
+    rs[j] = acc;
   }
   __syncthreads();
-  // warp per output row j of W2: lanes split F
-  const int warp = tid >> 5, lane = tid & 31;
+  // warp per output row j of W2; lanes split F with one vector load each
   constexpr int FPL = FH / 32;
+  const float invL = 1.f / s_L;
   for (int j = warp; j < D; j += blockDim.x / 32) {
     const T* wrow = (const T*)a.w2 + ((size_t)h * D + j) * FH + lane * FPL;
     float w[FPL];
 #pragma unroll
-    for (int i = 0; i < FPL; ++i) w[i] = ldf(wrow, i);
-    const float bias = ldf((const T*)a.b2, (size_t)h * D + j);
-    for (int g = 0; g < G; ++g) {
-      float acc = 0.f;
+    for (int i = 0; i < FPL; i += 4) VecLoad<T, 4>::load(wrow + i, w + i);
+    float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < FPL; ++i) acc = fmaf(w[i], hs[g * FH + lane * FPL + i], acc);
-      acc = warp_sum(acc);
-      if (lane == 0)
-        ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] =
-            from_f<T>((acc + rs[g * D + j]) / s_L[g] + bias);
-    }
+    for (int i = 0; i < FPL; ++i) acc = fmaf(w[i], hs[lane * FPL + i], acc);
+    acc = warp_sum(acc);
+    if (lane == 0)
+      ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] =
+          from_f<T>((acc + rs[j]) * invL + ldf((const T*)a.b2, (size_t)h * D + j));
   }
 }
 
@@ -361,7 +362,7 @@ cudaError_t launch_combine(const AttendArgs& a, bool reorder_form, cudaStream_t 
     return cudaGetLastError();
   }
   if (D == 128 && FH == 256 && bf) {
-    combine_reorder_kernel<__nv_bfloat16, 128, 256><<<grid, 256, 0, s>>>(a);
+    combine_reorder_kernel<__nv_bfloat16, 128, 256><<<grid * a.dm.G, 256, 0, s>>>(a);
     return cudaGetLastError();
   }
   return cudaErrorInvalidValue;

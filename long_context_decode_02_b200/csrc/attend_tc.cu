@@ -55,8 +55,20 @@ struct TcMaps {
   CUtensorMap w1;     // [H*F][d] bf16, box 64 x 128, 128B swizzle
 };
 
+// One slot of the producer -> epilogue metadata ring (three slots: the producer fills
+// tile i+1 while the epilogue may still read tiles i-1 and i).
+struct TileMeta {
+  int cid[kChunksPerTile];  // chunk id of each slot of the tile; -1 past the selection
+  int nres;                 // residual rows of the tile
+  int pad[3];
+  int2 res[kTile];          // (row of res_val, token row in the tile); row -1 = skip
+  uint4 q[64];              // the tile's G = 4 query rows, bf16 [4][128]
+};
+static_assert(sizeof(TileMeta) == 2128, "TileMeta layout");
+constexpr int kMetaSlots = 3;
+
 struct Layout {
-  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, bar, total;
+  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, meta, bar, total;
 };
 __host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
@@ -73,7 +85,8 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.b1 = L.q + 2048;            // [256] fp32
   L.zx = L.b1 + 1024;           // [128][4] fp32
   L.red = L.zx + 2048;          // 512 B of reduction scratch
-  L.bar = L.red + 512;          // barriers + TMEM address holder
+  L.meta = L.red + 512;         // kMetaSlots x TileMeta
+  L.bar = L.meta + kMetaSlots * (uint32_t)sizeof(TileMeta);  // barriers + TMEM holder
   L.total = L.bar + 256 + 1024; // + alignment slack of the dynamic base
   return L;
 }
@@ -82,8 +95,10 @@ __host__ __device__ inline Layout make_layout(int r) {
 enum {
   BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
   BAR_KT_EMPTY1, BAR_KBF_FULL0, BAR_KBF_FULL1, BAR_KBF_EMPTY0, BAR_KBF_EMPTY1, BAR_H_FULL,
-  BAR_H_EMPTY, BAR_DRAIN, BAR_COUNT
+  BAR_H_EMPTY, BAR_DRAIN, BAR_META_FULL0, BAR_META_FULL1, BAR_META_FULL2, BAR_META_EMPTY0,
+  BAR_META_EMPTY1, BAR_META_EMPTY2, BAR_COUNT
 };
+static_assert(BAR_COUNT * 8 + 8 <= 256, "barrier area");
 
 template <int ACT>
 __device__ __forceinline__ float act_fast(float x) {
@@ -109,6 +124,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   const int n_items = dm.B * a.n_tiles;
   const int kb_r = dm.r / 32;
   const int ksteps_r = dm.r / 16;
+  int n_mine = 0;
+  for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
 
   auto bar = [&](int i) { return base + L.bar + 8u * (uint32_t)i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + L.bar + 8 * BAR_COUNT);
@@ -118,6 +135,13 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   float* sB1 = reinterpret_cast<float*>(gbase + L.b1);
   float* sZx = reinterpret_cast<float*>(gbase + L.zx);
   float* sRed = reinterpret_cast<float*>(gbase + L.red);  // [4 quadrants][4 g] x 2, ml[2][4][2]
+  TileMeta* meta = reinterpret_cast<TileMeta*>(gbase + L.meta);
+
+  auto item_of = [&](int i, int& b, int& tile) {
+    const int it = cta_in_head + i * cta_per_head;
+    b = it / a.n_tiles;
+    tile = it % a.n_tiles;
+  };
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -135,6 +159,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     mbar_init(bar(BAR_H_FULL), 1);
     mbar_init(bar(BAR_H_EMPTY), 8);
     mbar_init(bar(BAR_DRAIN), 1);
+    for (int i = 0; i < kMetaSlots; ++i) {
+      mbar_init(bar(BAR_META_FULL0 + i), 1);
+      mbar_init(bar(BAR_META_EMPTY0 + i), 8);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -149,6 +177,78 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   const int32_t* sel_all = a.sel;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Tile metadata (chunk ids, the residual rows of its chunks, its queries) goes to the
+    // ring; the coefficient rows of its 16 chunks are TMA-gathered into the tile buffer.
+    const int32_t* ptr_all = a.chunk_ptr;
+    const int32_t* ridx_all = a.res_idx;
+    // returns this lane's chunk id (lanes 0..15) or -1
+    auto build_meta = [&](int i, bool& ok) -> int {
+      int b, tile;
+      item_of(i, b, tile);
+      const int slot = i % kMetaSlots;
+      int got = 0;
+      if (lane == 0)
+        got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
+      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
+      if (!ok) return -1;
+      TileMeta* M = meta + slot;
+      const int p = b * dm.H + h;
+      int cid = -1, e0 = 0, n = 0;
+      if (lane < kChunksPerTile) {
+        const int gs = tile * kChunksPerTile + lane;
+        if (gs < dm.k) {
+          cid = sel_all[(size_t)p * dm.k + gs];
+          if (cid < 0 || cid >= dm.Nc) {
+            raise_status(a.status, kStatusDeviceCheck);
+            cid = -1;
+          }
+        }
+        if (cid >= 0) {
+          const int32_t* ptr = ptr_all + (size_t)p * (dm.Nc + 1);
+          e0 = ptr[cid];
+          const int e1 = ptr[cid + 1];
+          if (e0 < 0 || e1 < e0 || e1 > dm.n_res || e1 - e0 > kChunk) {
+            raise_status(a.status, kStatusDeviceCheck);
+            n = 0;
+          } else {
+            n = e1 - e0;
+          }
+        }
+        M->cid[lane] = cid;
+      }
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int off = incl - n;
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (n > 0) {
+        const int32_t* ridx = ridx_all + (size_t)p * dm.n_res + e0;
+        int t[kChunk];
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+          if (j < n) {
+            const int tt = t[j] - cid * kChunk;
+            const bool good = tt >= 0 && tt < kChunk;
+            if (!good) raise_status(a.status, kStatusDeviceCheck);
+            M->res[off + j] = make_int2(e0 + j, good ? lane * kChunk + tt : -1);
+          }
+        }
+      }
+      if (lane == 0) M->nres = total;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
+      M->q[lane] = qsrc[lane];
+      M->q[lane + 32] = qsrc[lane + 32];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_META_FULL0 + slot));
+      return cid;
+    };
+
     int issued_phase = -1;  // parity of the last coef load issued (for the drain)
     if (lane == 0) {
       mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192 + 65536));
@@ -159,28 +259,25 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
           tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
                       h * kF + hf * 128, bar(BAR_W));
     }
-    int i = 0;
-    for (int it = cta_in_head; it < n_items; it += cta_per_head, ++i) {
-      const int b = it / a.n_tiles, tile = it % a.n_tiles;
+    bool ok = true;
+    int cid = n_mine > 0 ? build_meta(0, ok) : -1;
+    for (int i = 0; ok && i < n_mine; ++i) {
+      int b, tile;
+      item_of(i, b, tile);
       int got = 0;
       if (lane == 0) got = mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      int cid = 0;
-      if (lane < kChunksPerTile) {
-        const int slot = tile * kChunksPerTile + lane;
-        if (slot < dm.k) cid = sel_all[((size_t)b * dm.H + h) * dm.k + slot];
-        if (cid < 0 || cid >= dm.Nc) cid = 0;
-      }
       if (lane == 0)
         mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
       __syncwarp();
       if (lane < kChunksPerTile) {
-        const int row = b * dm.T + cid * kChunk;
+        const int row = b * dm.T + (cid < 0 ? 0 : cid) * kChunk;
         for (int kb = 0; kb < kb_r; ++kb)
           tma_load_2d(base + L.coef + kb * 8192 + lane * 512, &maps.coef, kb * 32, row,
                       bar(BAR_COEF_FULL));
       }
       issued_phase = i & 1;
+      if (i + 1 < n_mine) cid = build_meta(i + 1, ok);
     }
     // drain: a load still in flight (only possible after an abort) must land before exit
     if (lane == 0 && *abort_flag && issued_phase >= 0) {
@@ -225,8 +322,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
         mma_commit(bar(BAR_KBF_EMPTY0 + u));
         return true;
       };
-      int n_mine = 0;
-      for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
       if (ok && n_mine > 0) ok = issue_k(0);
       for (int i = 0; ok && i < n_mine; ++i) {
         if (i + 1 < n_mine) ok = issue_k(i + 1);
@@ -246,43 +341,33 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     const int trow = 32 * qd + lane;     // token row (A) / hidden-unit row within a half (B)
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
-    const int32_t* ptr_all = a.chunk_ptr;
-    const int32_t* ridx_all = a.res_idx;
     const __nv_bfloat16* rval_all = (const __nv_bfloat16*)a.res_val;
-    const __nv_bfloat16* q_all = (const __nv_bfloat16*)a.q;
     float* s_ml = sRed + 64;  // [2][4][2]
 
     for (int i = et; i < kF; i += kEpiThreads)
       sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
-
-    int n_mine = 0;
-    for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
     bool ok = true;
 
-    auto item_of = [&](int i, int& b, int& tile) {
-      const int it = cta_in_head + i * cta_per_head;
-      b = it / a.n_tiles;
-      tile = it % a.n_tiles;
-    };
-
-    // ---- part A of tile i
     // A failed (timed-out) wait never changes the sequence of named barriers: the
     // thread carries on with `good` false so every barrier is still reached.
+    // ---- part A of tile i
     auto part_a = [&](int i) -> bool {
-      bool good = true;
-      int b, tile;
-      item_of(i, b, tile);
       const int u = i & 1;
+      const int slot = i % kMetaSlots;
+      const TileMeta* M = meta + slot;
+      bool good = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
       named_bar_sync(1, kEpiThreads);  // previous readers of sQ / sZx are done
-      for (int e = et; e < kG * kD; e += kEpiThreads)
-        sQ[e] = __bfloat162float(q_all[((size_t)b * dm.Hq + (size_t)h * kG) * kD + e]);
-      const int slot = tile * kChunksPerTile + (trow >> 3);
-      int cid = slot < dm.k ? sel_all[((size_t)b * dm.H + h) * dm.k + slot] : -1;
-      if (cid >= dm.Nc) cid = -1;
+      {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
+        const float2 f = bf2_to_f2(w);
+        sQ[2 * et] = f.x;
+        sQ[2 * et + 1] = f.y;
+      }
+      const int cid = M->cid[trow >> 3];
       const bool valid = cid >= 0;
       const int pos = valid ? cid * kChunk + (trow & 7) : 0;
 
-      good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag);
+      good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
       tc_fence_after();
       float x[32], y[32];
       const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + 32 * hf);
@@ -310,17 +395,32 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL0 + u));
 
       named_bar_sync(1, kEpiThreads);  // sQ ready
-      // RoPE on pairs (32hf + i, 64 + 32hf + i) and partial logits
+      // RoPE on pairs (32hf + e, 64 + 32hf + e) and partial logits; this thread's 32
+      // (cos, sin) pairs are contiguous in both position-major tables
       float z[kG] = {0.f, 0.f, 0.f, 0.f};
+      const float4* lo4 = reinterpret_cast<const float4*>(a.rope.lo32 + (pos & (kRopeLo - 1)) * (kD / 2) + 32 * hf);
+      const float4* hi4 = reinterpret_cast<const float4*>(a.rope.hi32 + (size_t)(pos >> kRopeLoBits) * (kD / 2) + 32 * hf);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int pi = 32 * hf + e;
-        const float2 cs = rope_cs32(a.rope, pi, pos);
-        const float xr = x[e] * cs.x - y[e] * cs.y;
-        const float yr = x[e] * cs.y + y[e] * cs.x;
+      for (int e4 = 0; e4 < 32; e4 += 8) {
+        float4 lo[4], hi[4];
 #pragma unroll
-        for (int g = 0; g < kG; ++g)
-          z[g] = fmaf(sQ[g * kD + pi], xr, fmaf(sQ[g * kD + 64 + pi], yr, z[g]));
+        for (int v = 0; v < 4; ++v) { lo[v] = lo4[e4 / 2 + v]; hi[v] = hi4[e4 / 2 + v]; }
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+#pragma unroll
+          for (int w2 = 0; w2 < 2; ++w2) {
+            const int e = e4 + 2 * v + w2;
+            const float2 lo2 = w2 ? make_float2(lo[v].z, lo[v].w) : make_float2(lo[v].x, lo[v].y);
+            const float2 hi2 = w2 ? make_float2(hi[v].z, hi[v].w) : make_float2(hi[v].x, hi[v].y);
+            const float2 cs = rope_combine(hi2, lo2);
+            const int pi = 32 * hf + e;
+            const float xr = x[e] * cs.x - y[e] * cs.y;
+            const float yr = x[e] * cs.y + y[e] * cs.x;
+#pragma unroll
+            for (int g = 0; g < kG; ++g)
+              z[g] = fmaf(sQ[g * kD + pi], xr, fmaf(sQ[g * kD + 64 + pi], yr, z[g]));
+          }
+        }
       }
       if (hf == 1) *reinterpret_cast<float4*>(sZx + 4 * trow) = make_float4(z[0], z[1], z[2], z[3]);
       named_bar_sync(1, kEpiThreads);
@@ -364,6 +464,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       int b, tile;
       item_of(i, b, tile);
       const int u = i & 1;
+      const int slot = i % kMetaSlots;
+      const TileMeta* M = meta + slot;
       const int p = b * dm.H + h;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
       const bool good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag);
@@ -393,40 +495,36 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 #pragma unroll
       for (int g = 0; g < kG; ++g) part[2 * kG + g * kF + f] = hacc[g];
 
-      // residual rows of the tile's chunks; thread = column j, rows split by half
+      // residual rows of the tile (list built by the producer); thread = column j,
+      // rows split between the two halves, loads issued four at a time
       const int j = trow;
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
-      const int32_t* ptr = ptr_all + (size_t)p * (dm.Nc + 1);
-      const int32_t* ridx = ridx_all + (size_t)p * dm.n_res;
-      const __nv_bfloat16* rval = rval_all + (size_t)p * dm.n_res * kD;
-      for (int slot = 0; slot < kChunksPerTile; ++slot) {
-        const int gs = tile * kChunksPerTile + slot;
-        if (gs >= dm.k) break;
-        const int cid = sel_all[(size_t)p * dm.k + gs];
-        if (cid < 0 || cid >= dm.Nc) continue;
-        const int e0 = ptr[cid], e1 = ptr[cid + 1];
-        if (e0 < 0 || e1 < e0 || e1 > dm.n_res || e1 - e0 > kChunk) {
-          if (j == 0) raise_status(a.status, kStatusDeviceCheck);
-          continue;
+      const int nres = M->nres;
+      for (int e0 = 2 * 0 + hf; e0 < nres; e0 += 8) {
+        int2 ent[4];
+        float rv[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int ei = e0 + 2 * v;
+          ent[v] = ei < nres ? M->res[ei] : make_int2(0, -1);
+          rv[v] = ent[v].y >= 0 ? __bfloat162float(rval_all[((size_t)p * dm.n_res + ent[v].x) * kD + j]) : 0.f;
         }
-        for (int e = e0 + hf; e < e1; e += 2) {
-          const int tt = ridx[e] - cid * kChunk;
-          if (tt < 0 || tt >= kChunk) {
-            if (j == 0) raise_status(a.status, kStatusDeviceCheck);
-            continue;
-          }
-          const float4 pv = P4[slot * kChunk + tt];
-          const float rv = __bfloat162float(rval[(size_t)e * kD + j]);
-          racc[0] = fmaf(pv.x, rv, racc[0]);
-          racc[1] = fmaf(pv.y, rv, racc[1]);
-          racc[2] = fmaf(pv.z, rv, racc[2]);
-          racc[3] = fmaf(pv.w, rv, racc[3]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          if (ent[v].y < 0) continue;
+          const float4 pv = P4[ent[v].y];
+          racc[0] = fmaf(pv.x, rv[v], racc[0]);
+          racc[1] = fmaf(pv.y, rv[v], racc[1]);
+          racc[2] = fmaf(pv.z, rv[v], racc[2]);
+          racc[3] = fmaf(pv.w, rv[v], racc[3]);
         }
       }
       float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
 #pragma unroll
       for (int g = 0; g < kG; ++g) pr[g * kD + j] = racc[g];
       if (ew == 0 && lane < 2 * kG) part[lane] = s_ml[u * 8 + lane];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_META_EMPTY0 + slot));
       return good;
     };
 
@@ -465,7 +563,7 @@ debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_consta
   const uint32_t barf = base + 131072, bard = barf + 8;
   uint32_t* holder = reinterpret_cast<uint32_t*>(gbase + 131072 + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + 131072 + 20);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(barf, 1);
@@ -544,37 +642,6 @@ debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_consta
 }
 
 // --------------------------------------------------------------------- host helpers
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2D bf16 tensor map over a row-major [rows][cols] array.
-bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_cols,
-                 uint32_t box_rows, CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {box_cols, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool attend_tc_supported(const Dims& dm) {
@@ -591,12 +658,9 @@ size_t attend_tc_part_floats(const Dims& dm, int n_tiles) {
 cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   const Dims& dm = a.dm;
   TcMaps maps;
-  if (!make_map_2d(&maps.coef, a.coef, dm.r, (uint64_t)dm.B * dm.T, 32, 8,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_2d(&maps.basis, a.basis, dm.r, (uint64_t)dm.H * kD, 32, 128,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_2d(&maps.w1, a.w1, kD, (uint64_t)dm.H * kF, 64, 128,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tensor_map_2d(&maps.coef, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 32, 8, 64) ||
+      !make_tensor_map_2d(&maps.basis, a.basis, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.H * kD, 32, 128, 64) ||
+      !make_tensor_map_2d(&maps.w1, a.w1, LOWRAM_DTYPE_BF16, kD, (uint64_t)dm.H * kF, 64, 128, 128))
     return cudaErrorInvalidValue;
   const Layout L = make_layout(dm.r);
   const int n_items = dm.B * a.n_tiles;
@@ -622,11 +686,11 @@ cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, 
                                  int* status, cudaStream_t s) {
   CUtensorMap ma, mb;
   if (mode == 0) {
-    if (!make_map_2d(&ma, a, (uint64_t)k, 128, 32, 8, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map_2d(&mb, b, (uint64_t)k, 128, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_tensor_map_2d(&ma, a, LOWRAM_DTYPE_BF16, (uint64_t)k, 128, 32, 8, 64) ||
+        !make_tensor_map_2d(&mb, b, LOWRAM_DTYPE_BF16, (uint64_t)k, 128, 32, 128, 64))
       return cudaErrorInvalidValue;
   } else {
-    if (!make_map_2d(&ma, a, 128, 128, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_tensor_map_2d(&ma, a, LOWRAM_DTYPE_BF16, 128, 128, 64, 128, 128))
       return cudaErrorInvalidValue;
     mb = ma;
   }

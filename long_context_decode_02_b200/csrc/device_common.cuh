@@ -67,13 +67,17 @@ __device__ __forceinline__ void raise_status(int* status, int bit) {
 // ------------------------------------------------------------------ RoPE
 // (cos, sin) of t * theta_i from the two-level tables by angle addition.
 __device__ __forceinline__ float2 rope_cs32(const RopeTables& rt, int i, int t) {
-  const float2 lo = rt.lo32[i * kRopeLo + (t & (kRopeLo - 1))];
-  const float2 hi = rt.hi32[(size_t)i * rt.n_hi + (t >> kRopeLoBits)];
+  const float2 lo = rt.lo32[(t & (kRopeLo - 1)) * rt.half + i];
+  const float2 hi = rt.hi32[(size_t)(t >> kRopeLoBits) * rt.half + i];
+  return make_float2(fmaf(hi.x, lo.x, -hi.y * lo.y), fmaf(hi.y, lo.x, hi.x * lo.y));
+}
+// (cos, sin) combination of a hi and a lo table entry by angle addition.
+__device__ __forceinline__ float2 rope_combine(float2 hi, float2 lo) {
   return make_float2(fmaf(hi.x, lo.x, -hi.y * lo.y), fmaf(hi.y, lo.x, hi.x * lo.y));
 }
 __device__ __forceinline__ double2 rope_cs64(const RopeTables& rt, int i, int t) {
-  const double2 lo = rt.lo64[i * kRopeLo + (t & (kRopeLo - 1))];
-  const double2 hi = rt.hi64[(size_t)i * rt.n_hi + (t >> kRopeLoBits)];
+  const double2 lo = rt.lo64[(t & (kRopeLo - 1)) * rt.half + i];
+  const double2 hi = rt.hi64[(size_t)(t >> kRopeLoBits) * rt.half + i];
   return make_double2(hi.x * lo.x - hi.y * lo.y, hi.y * lo.x + hi.x * lo.y);
 }
 
@@ -99,9 +103,19 @@ __device__ __forceinline__ float key2f(uint32_t k) {
   return __uint_as_float(u);
 }
 
-// ------------------------------------------------------------------ block reductions
-// All helpers below must be called by every thread of the block; blockDim.x is a
-// multiple of 32 and at most 1024. `scratch` is shared memory of at least 33 words.
+// ------------------------------------------------------------------ thread groups
+// A group of whole warps, numbered from 0, synchronised either by __syncthreads (the
+// whole block, id 0) or by named barrier `id` over `nt` threads. The helpers below must
+// be called by every thread of the group.
+struct Grp {
+  int tid, nt, id;
+  __device__ __forceinline__ void sync() const {
+    if (id == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nt) : "memory");
+  }
+};
+__device__ __forceinline__ Grp whole_block() { return Grp{(int)threadIdx.x, (int)blockDim.x, 0}; }
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -113,29 +127,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ inline float block_max(float v, float* scratch) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Max over the group. `scratch`: 33 words of shared memory.
+__device__ inline float group_max(const Grp& g, float v, float* scratch) {
+  const int lane = g.tid & 31, wid = g.tid >> 5, nw = g.nt >> 5;
   v = warp_max(v);
-  __syncthreads();
+  g.sync();
   if (lane == 0) scratch[wid] = v;
-  __syncthreads();
+  g.sync();
   float r = lane < nw ? scratch[lane] : -INFINITY;
-  r = warp_max(r);
-  return r;
+  return warp_max(r);
 }
 
-// Exclusive prefix sum of v over the block in thread order; *total gets the sum.
-__device__ inline int block_exclusive_scan(int v, int* scratch, int* total) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Exclusive prefix sum of v over the group in thread order; *total gets the sum.
+__device__ inline int group_exclusive_scan(const Grp& g, int v, int* scratch, int* total) {
+  const int lane = g.tid & 31, wid = g.tid >> 5, nw = g.nt >> 5;
   int incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     int n = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += n;
   }
-  __syncthreads();
+  g.sync();
   if (lane == 31) scratch[wid] = incl;
-  __syncthreads();
+  g.sync();
   if (wid == 0) {
     int w = lane < nw ? scratch[lane] : 0;
     int wi = w;
@@ -147,10 +161,10 @@ __device__ inline int block_exclusive_scan(int v, int* scratch, int* total) {
     if (lane < nw) scratch[lane] = wi - w;  // exclusive warp offsets
     if (lane == 31) scratch[32] = wi;
   }
-  __syncthreads();
+  g.sync();
   const int res = scratch[wid] + incl - v;
   *total = scratch[32];
-  __syncthreads();
+  g.sync();
   return res;
 }
 
@@ -158,21 +172,21 @@ __device__ inline int block_exclusive_scan(int v, int* scratch, int* total) {
 // key_of(i), by a most-significant-digit-first radix pass over 8-bit digits.
 // `hist` holds 256 words and `bc` 4 words of shared memory.
 template <typename KeyFn>
-__device__ uint32_t block_kth_largest(int n, int k, KeyFn key_of, unsigned* hist,
-                                      unsigned* bc) {
+__device__ uint32_t group_kth_largest(const Grp& g, int n, int k, KeyFn key_of,
+                                      unsigned* hist, unsigned* bc) {
   uint32_t prefix = 0, mask = 0;
   unsigned remaining = (unsigned)k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = g.tid; i < 256; i += g.nt) hist[i] = 0;
+    g.sync();
+    for (int i = g.tid; i < n; i += g.nt) {
       const uint32_t key = key_of(i);
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
-    __syncthreads();
-    if (threadIdx.x < 32) {
+    g.sync();
+    if (g.tid < 32) {
       // lane l owns digits 255-8l .. 248-8l (high digits first)
-      const int lane = threadIdx.x;
+      const int lane = g.tid;
       unsigned own = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) own += hist[255 - 8 * lane - j];
@@ -194,13 +208,52 @@ __device__ uint32_t block_kth_largest(int n, int k, KeyFn key_of, unsigned* hist
         }
       }
     }
-    __syncthreads();
+    g.sync();
     prefix |= bc[0] << shift;
     mask |= 255u << shift;
     remaining = bc[1];
-    __syncthreads();
+    g.sync();
   }
   return prefix;
+}
+
+// Sort n (a power of two) (key, idx) pairs in shared memory so that (key desc, idx asc)
+// comes first.
+__device__ inline void group_sort_desc(const Grp& g, float* key, int* idx, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = g.tid; t < n / 2; t += g.nt) {
+        const int i = 2 * t - (t & (stride - 1));
+        const int j = i + stride;
+        const float ki = key[i], kj = key[j];
+        const int ii = idx[i], ij = idx[j];
+        const bool j_first = (kj > ki) || (kj == ki && ij < ii);
+        const bool i_first = (ki > kj) || (ki == kj && ii < ij);
+        const bool up = (i & size) == 0;
+        if (up ? j_first : i_first) {
+          key[i] = kj; key[j] = ki;
+          idx[i] = ij; idx[j] = ii;
+        }
+      }
+      g.sync();
+    }
+  }
+}
+
+// Ascending sort of n (power of two) ints in shared memory.
+__device__ inline void group_sort_int_asc(const Grp& g, int* v, int n) {
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = g.tid; t < n / 2; t += g.nt) {
+        const int i = 2 * t - (t & (stride - 1));
+        const int j = i + stride;
+        const int a = v[i], b = v[j];
+        const bool up = (i & size) == 0;
+        if (up ? (b < a) : (a < b)) { v[i] = b; v[j] = a; }
+      }
+      g.sync();
+    }
+  }
 }
 
 }  // namespace lowram

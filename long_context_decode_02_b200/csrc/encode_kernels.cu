@@ -189,9 +189,9 @@ __global__ void __launch_bounds__(kSelEncThreads) residual_threshold_kernel(cons
   }
   float mx = 0.f;
   for (int i = tid; i < T; i += blockDim.x) mx = fmaxf(mx, fabsf(e[i]));
-  mx = block_max(mx, fscr);
-  const uint32_t tk = block_kth_largest(T, dm.n_res, [&](int i) { return f2key(e[i]); },
-                                        hist, bc);
+  mx = group_max(whole_block(), mx, fscr);
+  const uint32_t tk = group_kth_largest(whole_block(), T, dm.n_res,
+                                        [&](int i) { return f2key(e[i]); }, hist, bc);
   const double tau = (double)key2f(tk);
   const double delta = 2e-3 * fabs(tau) + 1e-6 * (double)mx + 1e-30;
   const double hi = tau + delta, lo = tau - delta;
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kSelEncThreads) residual_threshold_kernel(cons
     flags[i] = f;
   }
   int total;
-  (void)block_exclusive_scan(n_in, iscr, &total);
+  (void)group_exclusive_scan(whole_block(), n_in, iscr, &total);
   if (tid == 0) { a.in_count[p] = total; a.cand_count[p] = cnt; }
 }
 
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kSelEncThreads) residual_finalize_kernel(const
     const int i = c0 + tid;
     const int f = (i < T && flags[i] == 1) ? 1 : 0;
     int total;
-    const int ex = block_exclusive_scan(f, iscr, &total);
+    const int ex = group_exclusive_scan(whole_block(), f, iscr, &total);
     if (f && base + ex < dm.n_res) ridx[base + ex] = i;
     base += total;
   }

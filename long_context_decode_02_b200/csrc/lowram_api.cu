@@ -130,6 +130,7 @@ RopeTables rope_of(const lowram_ctx* ctx) {
   r.lo64 = ctx->lo64;
   r.hi64 = ctx->hi64;
   r.n_hi = ctx->n_hi;
+  r.half = ctx->cfg.head_dim / 2;
   return r;
 }
 
@@ -231,13 +232,13 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
     const double th = std::pow(c->rope_theta, -2.0 * i / c->head_dim);
     for (int t = 0; t < kRopeLo; ++t) {
       const double ang = (double)t * th;
-      lo64[(size_t)i * kRopeLo + t] = make_double2(std::cos(ang), std::sin(ang));
-      lo32[(size_t)i * kRopeLo + t] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      lo64[(size_t)t * half + i] = make_double2(std::cos(ang), std::sin(ang));
+      lo32[(size_t)t * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
     }
     for (int j = 0; j < ctx->n_hi; ++j) {
       const double ang = (double)j * kRopeLo * th;
-      hi64[(size_t)i * ctx->n_hi + j] = make_double2(std::cos(ang), std::sin(ang));
-      hi32[(size_t)i * ctx->n_hi + j] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      hi64[(size_t)j * half + i] = make_double2(std::cos(ang), std::sin(ang));
+      hi32[(size_t)j * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
     }
   }
   const size_t pairs = (size_t)c->batch * c->n_kv_heads;
@@ -327,9 +328,7 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, 
   sa.counters = ctx->counters;
   sa.sel = sel;
   sa.status = ctx->status;
-  sa.slice_len = 8 * (32 / dm.G) * 4;
-  sa.n_slices = (dm.Nc + sa.slice_len - 1) / sa.slice_len;
-  if (launch_select(sa, s) != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
+  if (launch_select(sa, ctx->num_sms, s) != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;
 }
 

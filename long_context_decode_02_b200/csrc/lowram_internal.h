@@ -2,6 +2,7 @@
 // Not part of the public ABI (include/lowram.h is).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -14,9 +15,10 @@ namespace lowram {
 constexpr int kStatusDeviceCheck = 1;
 constexpr int kStatusTimeout = 2;
 
-// Two-level RoPE tables. For pair i and position t:
-//   lo[i * kRopeLo + (t & (kRopeLo-1))] = (cos, sin)((t mod kRopeLo) * theta_i)
-//   hi[i * n_hi   + (t >> kRopeLoBits)] = (cos, sin)((t - t mod kRopeLo) * theta_i)
+// Two-level RoPE tables, position-major (the d/2 pairs of one position are contiguous,
+// so a thread rotating one token reads them with vector loads). For pair i, position t:
+//   lo[(t & (kRopeLo-1)) * half + i] = (cos, sin)((t mod kRopeLo) * theta_i)
+//   hi[(t >> kRopeLoBits) * half + i] = (cos, sin)((t - t mod kRopeLo) * theta_i)
 // and the angle of t is recovered by the angle-addition formulas. Entries are computed
 // in fp64 on the host, so the fp32 copy carries only its own rounding.
 constexpr int kRopeLoBits = 9;
@@ -28,6 +30,7 @@ struct RopeTables {
   const double2* lo64;
   const double2* hi64;
   int n_hi;
+  int half;   // d / 2
 };
 
 struct Dims {
@@ -46,10 +49,8 @@ struct SelectArgs {
   int* counters;          // ctx [B*H], zero between launches
   int32_t* sel;           // [B*H][k]
   int* status;
-  int slice_len;          // chunks scored per CTA
-  int n_slices;
 };
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
 
 // ---------------- decode: reconstruct + attend ----------------
 struct AttendArgs {
@@ -97,6 +98,11 @@ struct EncodeArgs {
   int* status;
 };
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
+
+// 2D tiled TMA map over a row-major [rows][cols] array of dtype (LOWRAM_DTYPE_*), box
+// box_rows x box_cols, swizzle 0/32/64/128 bytes. False if the driver refuses it.
+bool make_tensor_map_2d(CUtensorMap* m, const void* ptr, int dtype, uint64_t cols,
+                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
 // ---------------- test-only ----------------
 cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, int mode,

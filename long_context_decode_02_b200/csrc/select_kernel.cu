@@ -6,39 +6,73 @@
 // works", Selective reconstruction). With GQA a chunk's score is the max over the
 // group's query heads of q . L_c; ties go to the lower chunk index.
 //
-// Structure (HBM-bound: every landmark byte is read once; ~4 FLOP per byte):
-//  * grid (n_slices, B*H_kv); a CTA scores one slice of one (batch, KV head).
-//    Each warp streams groups of U = 32/G landmarks; lane l holds dims
-//    [l*E, l*E+E) of the G queries in registers (E = d/32) and of each landmark, so the
-//    loads are coalesced rows. The U*G partial dot products of a group are summed across
-//    lanes by a reduce-scatter (31 shuffles per 32 values) that leaves lane l with value
-//    l; a max over G lanes gives the chunk score, written as fp32.
-//  * The last CTA of a (batch, KV head) to finish (atomic counter, no spinning) selects:
-//    radix select of the k-th largest fp32 score tau; chunks with score > tau + delta are
-//    in, chunks within delta of tau are re-scored in fp64 (exact products, fp64 sums)
-//    and ranked by (fp64 score desc, index asc). delta = 1e-3|tau| + 1e-6 max|s| is far
-//    above the fp32 accumulation error, so the result equals the fp64 selection.
-//    The selection is written in ascending chunk order.
+// Structure (HBM-bound: every landmark byte is read once, ~4 FLOP per byte):
+//  * Persistent CTAs (one per SM) split the stream of all (batch, KV head) landmark rows
+//    into contiguous ranges of stages. A producer warp TMA-loads 64 KB stages (the rows
+//    of one (b, h)) into a 3-stage shared-memory ring with the 128-byte swizzle; 256
+//    consumer threads each score one landmark row of a stage (packed fp32x2 FMAs against
+//    the queries held in shared memory) and write the fp32 score. The swizzle makes the
+//    row-per-thread 16-byte reads conflict-free.
+//  * The CTA that completes the last stage of a (b, h) (atomic stage counter, no
+//    spinning) selects on its consumer warps while its producer keeps streaming:
+//    a sorted sample places a threshold, candidates above it are sorted, tau = k-th
+//    score, candidates within delta = 1e-3|tau| + 1e-6 max|s| of tau are re-scored in
+//    fp64 (exact products, fp64 sums) and ranked by (score desc, index asc). delta is far
+//    above the fp32 accumulation error, so the result equals the fp64 selection. When the
+//    candidate set cannot be proven to contain the answer, a radix-select path over all
+//    scores decides instead. The selection is written in ascending chunk order.
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace lowram {
 namespace {
 
-constexpr int kSelThreads = 256;
+using namespace sm100;
 
-// One reduce-scatter step: 2N values per lane -> N, exchanging the half this lane
-// does not keep with the partner lane^off.
-template <int N>
-__device__ __forceinline__ void rs_step(float* v, bool upper, int off) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const float send = upper ? v[i] : v[i + N];
-    const float keep = upper ? v[i + N] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-  }
+constexpr int kConsumers = 256;               // consumer threads (warps 0..7)
+constexpr int kSelThreads = kConsumers + 32;  // + producer warp 8
+constexpr int kStages = 3;
+constexpr int kStageBytes = 65536;
+constexpr int kCap = 2048;                    // candidate capacity of the fast selection
+constexpr int kSample = 1024;                 // sampled scores placing its threshold
+
+template <typename T, int D>
+struct Geom {
+  static constexpr int kRowBytes = D * (int)sizeof(T);
+  static constexpr int kBoxes = kRowBytes / 128;             // 128-byte column boxes per row
+  static constexpr int kBoxCols = 128 / (int)sizeof(T);
+  static constexpr int kLps0 = kStageBytes / kRowBytes;
+  static constexpr int kLps = kLps0 < kConsumers ? kLps0 : kConsumers;  // rows per stage
+  static constexpr int kChunks = kRowBytes / 16;
+};
+
+struct SelSmem {  // offsets from the 1024-aligned dynamic base
+  uint32_t stages, q, ckey, cid, outs, misc, bar, total;
+};
+__host__ __device__ inline SelSmem sel_smem(int G, int D) {
+  SelSmem L{};
+  L.stages = 0;
+  L.q = kStages * kStageBytes;
+  L.ckey = L.q + (uint32_t)(G * D * 4);
+  L.cid = L.ckey + kCap * 4;
+  L.outs = L.cid + kCap * 4;
+  L.misc = L.outs + (kCap / 2) * 4;     // 2 KB of scalars and reduction scratch
+  L.bar = L.misc + 2048;
+  L.total = L.bar + 128 + 1024;
+  return L;
 }
+
+struct Misc {
+  unsigned hist[256];
+  unsigned bc[4];
+  float fscr[33];
+  int iscr[33];
+  int cnt, lo, hi, last;
+  float t0;
+};
+static_assert(sizeof(Misc) <= 2048, "Misc scratch");
 
 template <typename T, int D, int G>
 __device__ double score64(const T* lrow, const T* qb) {
@@ -51,43 +85,41 @@ __device__ double score64(const T* lrow, const T* qb) {
   return best;
 }
 
+__device__ __forceinline__ int next_pow2(int x) {
+  int n = 1;
+  while (n < x) n <<= 1;
+  return n;
+}
+
+// ---------------------------------------------------------------- selection
+// Fallback over all N_c scores: radix select of the k-th largest fp32 score,
+// classification against its window, exact fp64 ranking of the window, ascending
+// compaction through a flag array.
 template <typename T, int D, int G>
-__device__ void select_pair(const SelectArgs& a, int p) {
+__device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc* ms) {
   const Dims& dm = a.dm;
   const int Nc = dm.Nc, k = dm.k;
   int32_t* sel = a.sel + (size_t)p * k;
-  const int tid = threadIdx.x;
-  if (k >= Nc) {
-    for (int i = tid; i < Nc; i += blockDim.x) sel[i] = i;
-    return;
-  }
-  __shared__ unsigned hist[256];
-  __shared__ unsigned bc[4];
-  __shared__ float fscr[33];
-  __shared__ int iscr[33];
-  __shared__ int cnt[2];
   const float* s = a.scores + (size_t)p * Nc;
   uint8_t* flags = a.flags + (size_t)p * Nc;
   int* cidx = a.cand_idx + (size_t)p * Nc;
   double* cs64 = a.cand_s64 + (size_t)p * Nc;
 
   float mx = 0.f;
-  for (int i = tid; i < Nc; i += blockDim.x) mx = fmaxf(mx, fabsf(__ldcg(s + i)));
-  mx = block_max(mx, fscr);
-
-  const uint32_t tk = block_kth_largest(
-      Nc, k, [&](int i) { return f2key(__ldcg(s + i)); }, hist, bc);
+  for (int i = g.tid; i < Nc; i += g.nt) mx = fmaxf(mx, fabsf(__ldcg(s + i)));
+  mx = group_max(g, mx, ms->fscr);
+  const uint32_t tk = group_kth_largest(
+      g, Nc, k, [&](int i) { return f2key(__ldcg(s + i)); }, ms->hist, ms->bc);
   const double tau = (double)key2f(tk);
   const double delta = 1e-3 * fabs(tau) + 1e-6 * (double)mx + 1e-30;
   const double hi = tau + delta, lo = tau - delta;
-
-  if (tid == 0) { cnt[0] = 0; cnt[1] = 0; }
-  __syncthreads();
+  if (g.tid == 0) ms->cnt = 0;
+  g.sync();
   const int b = p / dm.H, h = p % dm.H;
   const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
   const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
   int n_in = 0;
-  for (int i = tid; i < Nc; i += blockDim.x) {
+  for (int i = g.tid; i < Nc; i += g.nt) {
     const double x = (double)__ldcg(s + i);
     uint8_t f = 0;
     if (x > hi) {
@@ -95,18 +127,17 @@ __device__ void select_pair(const SelectArgs& a, int p) {
       ++n_in;
     } else if (x >= lo) {
       f = 2;
-      const int slot = atomicAdd(&cnt[1], 1);
+      const int slot = atomicAdd(&ms->cnt, 1);
       cidx[slot] = i;
       cs64[slot] = score64<T, D, G>(L + (size_t)i * D, qb);
     }
     flags[i] = f;
   }
   int n_in_total;
-  (void)block_exclusive_scan(n_in, iscr, &n_in_total);
-  const int n_w = cnt[1];
+  (void)group_exclusive_scan(g, n_in, ms->iscr, &n_in_total);
+  const int n_w = ms->cnt;
   const int need = k - n_in_total;
-  // rank the window candidates by (fp64 score desc, index asc); keep the first `need`
-  for (int j = tid; j < n_w; j += blockDim.x) {
+  for (int j = g.tid; j < n_w; j += g.nt) {
     const double sj = cs64[j];
     const int ij = cidx[j];
     int rank = 0;
@@ -116,100 +147,304 @@ __device__ void select_pair(const SelectArgs& a, int p) {
     }
     flags[ij] = rank < need ? 1 : 0;
   }
-  __syncthreads();
+  g.sync();
   int base = 0;
-  for (int c0 = 0; c0 < Nc; c0 += blockDim.x) {
-    const int i = c0 + tid;
+  for (int c0 = 0; c0 < Nc; c0 += g.nt) {
+    const int i = c0 + g.tid;
     const int f = (i < Nc && flags[i] == 1) ? 1 : 0;
     int total;
-    const int ex = block_exclusive_scan(f, iscr, &total);
+    const int ex = group_exclusive_scan(g, f, ms->iscr, &total);
     if (f && base + ex < k) sel[base + ex] = i;
     base += total;
   }
 }
 
+// Fast path: the candidate set is all scores (N_c <= kCap) or those at or above a
+// threshold placed from a sorted sample; candidates are sorted, the window around the
+// k-th is re-scored in fp64 and ranked exactly. Returns false (writing nothing) when the
+// candidate set cannot be proven to contain the answer.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kSelThreads, 3) score_select_kernel(const SelectArgs a) {
-  constexpr int E = D / 32;
-  constexpr int U = 32 / G;
+__device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, float* ckey,
+                                 int* cid, int* outs, Misc* ms) {
   const Dims& dm = a.dm;
-  const int p = blockIdx.y;
-  const int b = p / dm.H, h = p % dm.H;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Nc = dm.Nc;
-  const T* L = (const T*)a.landmark + (size_t)p * Nc * D + lane * E;
-
-  float qr[G][E];
-  {
-    const T* qp = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D + lane * E;
-#pragma unroll
-    for (int g = 0; g < G; ++g) VecLoad<T, E>::load(qp + g * D, qr[g]);
-  }
-  const int c_begin = blockIdx.x * a.slice_len;
-  const int c_end = min(Nc, c_begin + a.slice_len);
-  float* out = a.scores + (size_t)p * Nc;
-  constexpr int kWarps = kSelThreads / 32;
-
-  for (int c0 = c_begin + warp * U; c0 < c_end; c0 += kWarps * U) {
-    float lv[U][E];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (c0 + u < c_end) {
-        VecLoad<T, E>::load(L + (size_t)(c0 + u) * D, lv[u]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) lv[u][e] = 0.f;
+  const int Nc = dm.Nc, k = dm.k;
+  const int lane = g.tid & 31;
+  if (k > kCap / 2) return false;
+  const float* s = a.scores + (size_t)p * Nc;
+  int m;
+  float t0 = -INFINITY;
+  const bool sampled = Nc > kCap;
+  if (!sampled) {
+    for (int i = g.tid; i < Nc; i += g.nt) { ckey[i] = __ldcg(s + i); cid[i] = i; }
+    m = Nc;
+  } else {
+    for (int i = g.tid; i < kSample; i += g.nt) {
+      const int j = (int)(((long long)i * Nc) / kSample);
+      ckey[i] = __ldcg(s + j);
+      cid[i] = j;
+    }
+    g.sync();
+    group_sort_desc(g, ckey, cid, kSample);
+    if (g.tid == 0) {
+      int j = (int)((3LL * k * kSample) / (2LL * Nc)) + 16;
+      if (j > kSample - 1) j = kSample - 1;
+      ms->t0 = ckey[j];
+      ms->cnt = 0;
+    }
+    g.sync();
+    t0 = ms->t0;
+    for (int base = 0; base < Nc; base += g.nt) {
+      const int i = base + g.tid;
+      const float x = i < Nc ? __ldcg(s + i) : -INFINITY;
+      const bool keep = i < Nc && x >= t0;
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      int wb = 0;
+      if (lane == 0 && bal) wb = atomicAdd(&ms->cnt, __popc(bal));
+      wb = __shfl_sync(0xffffffffu, wb, 0);
+      if (keep) {
+        const int pos = wb + __popc(bal & ((1u << lane) - 1u));
+        if (pos < kCap) { ckey[pos] = x; cid[pos] = i; }
       }
     }
-    float v[32];
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc = fmaf(qr[g][e], lv[u][e], acc);
-        v[u * G + g] = acc;
-      }
-    rs_step<16>(v, lane & 16, 16);
-    rs_step<8>(v, lane & 8, 8);
-    rs_step<4>(v, lane & 4, 4);
-    rs_step<2>(v, lane & 2, 2);
-    rs_step<1>(v, lane & 1, 1);
-    float x = v[0];  // = score of chunk c0 + lane / G for head lane % G
-#pragma unroll
-    for (int o = 1; o < G; o <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-    const int c = c0 + lane / G;
-    if ((lane % G) == 0 && c < c_end) out[c] = x;
+    g.sync();
+    m = ms->cnt;
+    if (m > kCap || m < k) return false;
   }
-
-  // last CTA of this (batch, KV head) selects
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int t = atomicAdd(a.counters + p, 1);
-    s_last = (t == a.n_slices - 1);
+  const int n = next_pow2(m);
+  for (int i = m + g.tid; i < n; i += g.nt) { ckey[i] = -INFINITY; cid[i] = 0x7fffffff; }
+  g.sync();
+  group_sort_desc(g, ckey, cid, n);
+  const double tau = (double)ckey[k - 1];
+  const double delta = 1e-3 * fabs(tau) + 1e-6 * fmax(fabs((double)ckey[0]), fabs(tau)) + 1e-30;
+  const double hi = tau + delta, lo = tau - delta;
+  if (sampled && (double)t0 > lo) return false;   // the window may reach below the filter
+  if (g.tid == 0) { ms->lo = m; ms->hi = -1; }
+  g.sync();
+  for (int i = g.tid; i < m; i += g.nt) {
+    const double x = (double)ckey[i];
+    if (x <= hi) atomicMin(&ms->lo, i);
+    if (x >= lo) atomicMax(&ms->hi, i);
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  select_pair<T, D, G>(a, p);
-  if (threadIdx.x == 0) a.counters[p] = 0;
+  g.sync();
+  const int p_lo = ms->lo, p_hi = ms->hi, need = k - p_lo, w = p_hi - p_lo + 1;
+  const int b = p / dm.H, h = p % dm.H;
+  const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
+  const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
+  double* s64 = a.cand_s64 + (size_t)p * Nc;
+  for (int i = g.tid; i < w; i += g.nt) s64[i] = score64<T, D, G>(L + (size_t)cid[p_lo + i] * D, qb);
+  for (int i = g.tid; i < p_lo; i += g.nt) outs[i] = cid[i];
+  g.sync();
+  for (int i = g.tid; i < w; i += g.nt) {
+    const double si = s64[i];
+    const int ii = cid[p_lo + i];
+    int rank = 0;
+    for (int j = 0; j < w; ++j) {
+      const double sj = s64[j];
+      rank += (sj > si) || (sj == si && cid[p_lo + j] < ii);
+    }
+    if (rank < need) outs[p_lo + rank] = ii;
+  }
+  g.sync();
+  const int nk = next_pow2(k);
+  for (int i = k + g.tid; i < nk; i += g.nt) outs[i] = 0x7fffffff;
+  g.sync();
+  group_sort_int_asc(g, outs, nk);
+  int32_t* sel = a.sel + (size_t)p * k;
+  for (int i = g.tid; i < k; i += g.nt) sel[i] = outs[i];
+  return true;
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_typed(const SelectArgs& a, cudaStream_t s) {
-  dim3 grid(a.n_slices, a.dm.B * a.dm.H);
-  score_select_kernel<T, D, G><<<grid, kSelThreads, 0, s>>>(a);
+__device__ void select_pair(const Grp& g, const SelectArgs& a, int p, float* ckey, int* cid,
+                            int* outs, Misc* ms) {
+  const int Nc = a.dm.Nc, k = a.dm.k;
+  if (k >= Nc) {
+    int32_t* sel = a.sel + (size_t)p * k;
+    for (int i = g.tid; i < Nc; i += g.nt) sel[i] = i;
+    return;
+  }
+  const bool done = select_pair_fast<T, D, G>(g, a, p, ckey, cid, outs, ms);
+  g.sync();
+  if (!done) select_pair_radix<T, D, G>(g, a, p, ms);
+}
+
+// ---------------------------------------------------------------- scoring
+// Score of landmark row r of a swizzled stage.
+template <typename T, int D, int G>
+__device__ __forceinline__ float score_row(const uint8_t* stage, int r, const float* sQ) {
+  using Gm = Geom<T, D>;
+  float2 acc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < Gm::kChunks; ++c) {
+    const int box = c >> 3, cc = c & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(
+        stage + box * Gm::kLps * 128 + r * 128 + ((cc ^ (r & 7)) << 4));
+    if constexpr (sizeof(T) == 2) {
+      // 8 bf16: chunk c holds dims 8c .. 8c+7
+      const float2 v0 = bf2_to_f2(w.x), v1 = bf2_to_f2(w.y), v2 = bf2_to_f2(w.z), v3 = bf2_to_f2(w.w);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c);
+        const float4 q1 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c + 4);
+        acc[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, acc[g]);
+        acc[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, acc[g]);
+        acc[g] = __ffma2_rn(make_float2(q1.x, q1.y), v2, acc[g]);
+        acc[g] = __ffma2_rn(make_float2(q1.z, q1.w), v3, acc[g]);
+      }
+    } else {
+      // 4 fp32: chunk c holds dims 4c .. 4c+3
+      const float2 v0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+      const float2 v1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 4 * c);
+        acc[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, acc[g]);
+        acc[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, acc[g]);
+      }
+    }
+  }
+  float best = acc[0].x + acc[0].y;
+#pragma unroll
+  for (int g = 1; g < G; ++g) best = fmaxf(best, acc[g].x + acc[g].y);
+  return best;
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kSelThreads, 1)
+score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap) {
+  using Gm = Geom<T, D>;
+  const Dims& dm = a.dm;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const SelSmem L = sel_smem(G, D);
+  float* sQ = reinterpret_cast<float*>(gbase + L.q);
+  float* ckey = reinterpret_cast<float*>(gbase + L.ckey);
+  int* cidv = reinterpret_cast<int*>(gbase + L.cid);
+  int* outs = reinterpret_cast<int*>(gbase + L.outs);
+  Misc* ms = reinterpret_cast<Misc*>(gbase + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.bar + 8 * 2 * kStages);
+  auto full = [&](int s) { return base + L.bar + 8u * (uint32_t)s; };
+  auto empty = [&](int s) { return base + L.bar + 8u * (uint32_t)(kStages + s); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Nc = dm.Nc, P = dm.B * dm.H;
+  const int upp = (Nc + Gm::kLps - 1) / Gm::kLps;    // stages per (b, h)
+  const long long U = (long long)P * upp;
+  const int u_begin = (int)(U * blockIdx.x / gridDim.x);
+  const int u_end = (int)(U * (blockIdx.x + 1) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), kConsumers / 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumers / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int last_i[kStages];
+      for (int s = 0; s < kStages; ++s) last_i[s] = -1;
+      for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait_bounded(empty(s), ((i / kStages) & 1) ^ 1, abort_flag)) break;
+        const int pair = u / upp, st = u % upp;
+        const int row = pair * Nc + st * Gm::kLps;
+        mbar_arrive_expect_tx(full(s), (uint32_t)(Gm::kBoxes * Gm::kLps * 128));
+        for (int bx = 0; bx < Gm::kBoxes; ++bx)
+          tma_load_2d(base + L.stages + s * kStageBytes + bx * Gm::kLps * 128, &lmap,
+                      bx * Gm::kBoxCols, row, full(s));
+        last_i[s] = i;
+      }
+      if (*abort_flag) {   // loads may still be in flight: let them land before exit
+        for (int s = 0; s < kStages; ++s) {
+          if (last_i[s] < 0) continue;
+          int dummy = 0;
+          mbar_wait_bounded(full(s), (last_i[s] / kStages) & 1, (volatile int*)&dummy);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    // Every consumer thread runs the same sequence of group barriers whatever its
+    // waits return, so a timed-out wait never leaves the others at a barrier.
+    const Grp g{(int)threadIdx.x, kConsumers, 1};
+    const int tid = threadIdx.x;
+    int cur = -1, seg = 0;
+    auto finish_segment = [&](int pair, int nst) {
+      __threadfence();
+      g.sync();
+      if (tid == 0) {
+        const int old = atomicAdd(a.counters + pair, nst);
+        ms->last = (old + nst == upp);
+      }
+      g.sync();
+      if (ms->last) {
+        __threadfence();
+        select_pair<T, D, G>(g, a, pair, ckey, cidv, outs, ms);
+        g.sync();
+        if (tid == 0) a.counters[pair] = 0;
+      }
+    };
+    for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
+      const int pair = u / upp, st = u % upp;
+      if (pair != cur) {
+        if (cur >= 0) finish_segment(cur, seg);
+        cur = pair;
+        seg = 0;
+        g.sync();
+        const int b = pair / dm.H, h = pair % dm.H;
+        const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
+        for (int e = tid; e < G * D; e += kConsumers) sQ[e] = ldf(qb, e);
+        g.sync();
+      }
+      const int s = i % kStages;
+      mbar_wait_bounded(full(s), (i / kStages) & 1, abort_flag);
+      const int c = st * Gm::kLps + tid;
+      if (tid < Gm::kLps && c < Nc) {
+        const float sc = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ);
+        a.scores[(size_t)pair * Nc + c] = sc;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(s));
+      ++seg;
+    }
+    if (cur >= 0) finish_segment(cur, seg);
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) raise_status(a.status, kStatusTimeout);
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_typed(const SelectArgs& a, int num_sms, cudaStream_t s) {
+  using Gm = Geom<T, D>;
+  CUtensorMap map;
+  if (!make_tensor_map_2d(&map, a.landmark, a.dm.dtype, (uint64_t)D,
+                          (uint64_t)a.dm.B * a.dm.H * a.dm.Nc, Gm::kBoxCols, Gm::kLps, 128))
+    return cudaErrorInvalidValue;
+  const SelSmem L = sel_smem(G, D);
+  auto kern = score_select_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)L.total);
+  if (e != cudaSuccess) return e;
+  const long long U = (long long)a.dm.B * a.dm.H * ((a.dm.Nc + Gm::kLps - 1) / Gm::kLps);
+  const int grid = (int)(U < num_sms ? U : num_sms);
+  kern<<<grid, kSelThreads, L.total, s>>>(a, map);
   return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_by_shape(const SelectArgs& a, cudaStream_t s) {
+cudaError_t launch_by_shape(const SelectArgs& a, int num_sms, cudaStream_t s) {
   const int D = a.dm.d, G = a.dm.G;
 #define LR_CASE(DD, GG) \
-  if (D == DD && G == GG) return launch_typed<T, DD, GG>(a, s);
+  if (D == DD && G == GG) return launch_typed<T, DD, GG>(a, num_sms, s);
   LR_CASE(64, 1) LR_CASE(64, 2) LR_CASE(64, 4) LR_CASE(64, 8)
   LR_CASE(128, 1) LR_CASE(128, 2) LR_CASE(128, 4) LR_CASE(128, 8)
 #undef LR_CASE
@@ -218,9 +453,9 @@ cudaError_t launch_by_shape(const SelectArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
-  if (a.dm.dtype == LOWRAM_DTYPE_BF16) return launch_by_shape<__nv_bfloat16>(a, s);
-  return launch_by_shape<float>(a, s);
+cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s) {
+  if (a.dm.dtype == LOWRAM_DTYPE_BF16) return launch_by_shape<__nv_bfloat16>(a, num_sms, s);
+  return launch_by_shape<float>(a, num_sms, s);
 }
 
 }  // namespace lowram

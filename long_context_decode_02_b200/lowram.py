@@ -177,7 +177,11 @@ class Context:
 
 
 def layer_params(basis, w1, b1, w2, b2) -> lowram_layer_params:
-    return lowram_layer_params(_ptr(basis), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
+    """Parameter block of one layer. It keeps references to the tensors, so their device
+    memory stays allocated while the block is in use."""
+    p = lowram_layer_params(_ptr(basis), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
+    p._refs = (basis, w1, b1, w2, b2)
+    return p
 
 
 def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr) -> lowram_cache:

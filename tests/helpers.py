@@ -78,8 +78,12 @@ def compare_selection(got: np.ndarray, want: np.ndarray, scores: np.ndarray, k: 
                       rel: float = 1e-5, abs_floor: float = 0.0):
     """Per row: sets must match except indices whose score is within rel*|s_k| (+floor)
     of the k-th largest score. Returns the number of tie differences; asserts the rest."""
-    got = np.asarray(got).reshape(-1, got.shape[-1])
-    want = np.asarray(want).reshape(-1, want.shape[-1])
+    got, want = np.asarray(got), np.asarray(want)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    if got.size == 0:
+        return 0
+    got = got.reshape(-1, got.shape[-1])
+    want = want.reshape(-1, want.shape[-1])
     sc = np.asarray(scores).reshape(-1, scores.shape[-1])
     ties = 0
     for r in range(got.shape[0]):
