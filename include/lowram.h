@@ -182,6 +182,26 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
                                      const int32_t* sel, void* out, void* workspace,
                                      size_t workspace_bytes, void* stream);
 
+/* lowram_decode_step with its scratch in a fixed device array of the library instead of
+ * a caller workspace. The paper has no counterpart: it is an interface for callers that
+ * cannot allocate device memory where they decode (a fully reserved memory pool, a
+ * runtime that forbids allocation after start-up, a plugin without an allocator). The
+ * call itself allocates nothing; arguments and results are those of lowram_decode_step.
+ *   - The array holds 32 MiB and lives on every device that loads the library until the
+ *     process exits. A configuration whose decode workspace (lowram_workspace_size) is
+ *     larger is refused with LOWRAM_ERR_WORKSPACE, before anything else is checked and
+ *     with nothing launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current). Make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array, which keeps whatever the last call
+ *     left. The decode step needs none of it zeroed: it writes all it reads. Calls that
+ *     overlap on the GPU (other streams, other threads, other contexts) race on it:
+ *     serialise them. */
+lowram_status lowram_decode_step_static(lowram_ctx* ctx, const lowram_cache* cache,
+                                        const lowram_layer_params* params, const void* q,
+                                        void* out, int32_t* sel_out, void* stream);
+
 /* Synchronise the device, then return and clear the context's status word: LOWRAM_OK,
  * LOWRAM_ERR_DEVICE_CHECK (a kernel met a residual index outside its chunk or a CSR
  * offset out of range, and skipped it) or LOWRAM_ERR_TIMEOUT (a bounded wait expired;

@@ -469,3 +469,8 @@ lowram_status lowram_debug_tc_tile(const void* a, const void* b, float* d, int32
 }
 
 }  // extern "C"
+
+namespace lowram {
+const lowram_config* ctx_config(const lowram_ctx* ctx) { return &ctx->cfg; }
+int ctx_device(const lowram_ctx* ctx) { return ctx->device; }
+}  // namespace lowram

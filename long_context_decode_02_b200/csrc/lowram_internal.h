@@ -104,6 +104,10 @@ cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
 bool make_tensor_map_2d(CUtensorMap* m, const void* ptr, int dtype, uint64_t cols,
                         uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
+// Read-only access to a context's configuration and device.
+const lowram_config* ctx_config(const lowram_ctx* ctx);
+int ctx_device(const lowram_ctx* ctx);
+
 // ---------------- test-only ----------------
 cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, int mode,
                                  int* status, cudaStream_t s);

@@ -83,6 +83,8 @@ _sig = {
     "lowram_attend_selected": (_S, [_P, ctypes.POINTER(lowram_cache),
                                     ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
+    "lowram_decode_step_static": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                       ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P]),
     "lowram_last_error": (_S, [_P]),
     "lowram_status_string": (ctypes.c_char_p, [_S]),
     "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
@@ -219,6 +221,16 @@ def decode_step(ctx: Context, cache: dict, params: lowram_layer_params, q, out, 
                              _ptr(out), _ptr(sel_out), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)),
           "lowram_decode_step")
+
+
+def decode_step_static(ctx: Context, cache: dict, params: lowram_layer_params, q, out,
+                       sel_out=None, stream=None) -> None:
+    """lowram_decode_step_static: the decode step without a caller workspace (its scratch
+    is the library's fixed device array; see include/lowram.h)."""
+    cs = cache_struct(**cache)
+    check(lowram_decode_step_static(ctx.handle, ctypes.byref(cs), ctypes.byref(params), _ptr(q),
+                                    _ptr(out), _ptr(sel_out), _stream(stream)),
+          "lowram_decode_step_static")
 
 
 def select_chunks(ctx: Context, landmark, q, sel_out, workspace, stream=None) -> None:

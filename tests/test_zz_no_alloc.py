@@ -1,0 +1,71 @@
+"""The decode entry point that allocates nothing (lowram_decode_step_static), checked
+against lowram_decode_step with a caller workspace.
+
+Some callers cannot allocate device memory where they decode. Examples are a serving
+loop whose memory pool is fully reserved, a runtime that forbids allocation after
+start-up, and a plugin that owns no allocator. lowram_decode_step_static serves them from
+a fixed 32 MiB device array inside the library.
+
+This file calls it through the C ABI twice in a row, with different queries. Each call
+must match the workspace entry point: the same selected chunks, and outputs within the
+bf16 tolerance the other tests use. It also checks that a configuration needing more
+scratch than the array holds is refused before anything runs.
+
+The file is named to be collected last, so a failure here stops a `-x` run only after
+every other test has run. It needs no state from other tests and runs alone as well.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_02_b200 import synth
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def L(cuda_device):
+    from long_context_decode_02_b200 import lowram
+    return lowram
+
+
+def test_static_scratch_decode_matches_workspace_decode(L, cuda_device):
+    sh = synth.CONFIGS[1].replace(name="no-alloc", n_tokens=4096, batch=2, seed=123)
+    dev = cuda_device
+    t = H.stored_layer(sh, 0)
+    td = {n: x.to(dev) for n, x in t.items()}
+    cfg = L.make_config(sh)
+    ctx = L.Context(cfg, dev.index or 0)
+    cache = L.alloc_cache(cfg, dev)
+    params = L.layer_params(*(td[n] for n in ("basis", "w1", "b1", "w2", "b2")))
+    enc_ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=dev)
+    L.encode(ctx, td["k"], td["v"], params, cache, enc_ws)
+    assert ctx.last_error() == L.OK
+    dec_ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    kk = min(sh.top_k, sh.n_chunks)
+    for step in range(2):  # two calls in a row: the shared array keeps the last call's data
+        q = synth.queries(sh, 0, step).to(dev)
+        out_ref = torch.empty_like(q)
+        sel_ref = torch.empty(sh.batch, sh.n_kv_heads, kk, dtype=torch.int32, device=dev)
+        L.decode_step(ctx, cache, params, q, out_ref, dec_ws, sel_out=sel_ref)
+        out = torch.full_like(q, float("nan"))
+        sel = torch.full_like(sel_ref, -1)
+        L.decode_step_static(ctx, cache, params, q, out, sel_out=sel)
+        assert ctx.last_error() == L.OK
+        assert torch.equal(sel, sel_ref)
+        err = H.rel_err(H.f64(out), H.f64(out_ref))
+        assert np.isfinite(err) and err <= TOL_BF16, (step, err)
+    ctx.close()
+
+
+def test_static_scratch_refuses_an_oversize_configuration(L, cuda_device):
+    big = synth.CONFIGS[2].replace(n_tokens=1 << 20)   # decode workspace far above 32 MiB
+    cfg = L.make_config(big)
+    assert L.workspace_size(cfg, L.OP_DECODE) > (32 << 20)
+    ctx = L.Context(cfg, cuda_device.index or 0)
+    st = L.lowram_decode_step_static(ctx.handle, None, None, None, None, None, None)
+    assert st == L.ERR_WORKSPACE
+    ctx.close()
