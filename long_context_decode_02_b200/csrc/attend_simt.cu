@@ -251,9 +251,11 @@ __global__ void __launch_bounds__(256) combine_plain_kernel(const AttendArgs a) 
 // Combine, W2-after-attention form used by the tensor-core kernel. Partial of a tile:
 // [G][2] (m in log2 units, l), [G][F] sum_t e_t act(h_t), [2][G][D] sum_t e_t R_t.
 //   out_g = (W2 Hs_g + Rs_g) / L_g + b2,   Hs/Rs/L the 2^(m_t-M)-weighted tile sums.
-// One CTA per (b, h, g); n_tiles <= 64 (checked on the host).
+// One CTA per (b, h, g); n_tiles <= 64 (checked on the host). Every global load of a
+// thread is issued before the arithmetic that needs it: the kernel is a few round trips.
 template <typename T, int D, int FH>
 __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a) {
+  static_assert(FH == 256 && D == 128, "combine shape");
   const Dims& dm = a.dm;
   const int G = dm.G;
   const int p = blockIdx.x / G, g = blockIdx.x % G;
@@ -261,56 +263,69 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
   const int n = a.n_tiles;
   const size_t tstride = (size_t)G * 2 + (size_t)G * FH + 2 * (size_t)G * D;
   const float* part = a.part + (size_t)p * n * tstride;
-  __shared__ float s_w[64];
-  __shared__ float s_L;
   __shared__ float hs[FH];
-  __shared__ float rs[D];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (warp == 0) {
-    const float m0 = lane < n ? part[lane * tstride + 2 * g] : -INFINITY;
-    const float m1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g] : -INFINITY;
-    const float l0 = lane < n ? part[lane * tstride + 2 * g + 1] : 0.f;
-    const float l1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g + 1] : 0.f;
-    const float M = warp_max(fmaxf(m0, m1));
-    const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
-    const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
-    const float L = warp_sum(w0 * l0 + w1 * l1);
-    s_w[lane] = w0;
-    s_w[lane + 32] = w1;
-    if (lane == 0) s_L = L;
-  }
-  __syncthreads();
-  for (int f = tid; f < FH; f += blockDim.x) {
-    const float* src = part + 2 * G + (size_t)g * FH + f;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < n; ++t) acc = fmaf(s_w[t], src[t * tstride], acc);
-    hs[f] = acc;
-  }
-  for (int j = tid; j < D; j += blockDim.x) {
-    const float* src = part + 2 * G + (size_t)G * FH + (size_t)g * D + j;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < n; ++t) acc = fmaf(s_w[t], src[t * tstride] + src[t * tstride + G * D], acc);
-    rs[j] = acc;
-  }
-  __syncthreads();
-  // warp per output row j of W2; lanes split F with one vector load each
-  constexpr int FPL = FH / 32;
-  const float invL = 1.f / s_L;
-  for (int j = warp; j < D; j += blockDim.x / 32) {
-    const T* wrow = (const T*)a.w2 + ((size_t)h * D + j) * FH + lane * FPL;
-    float w[FPL];
+  __shared__ float rs[2][D];
+  __shared__ float s_L;
+  const int tid = threadIdx.x, lane = tid & 31;
+  // this thread's output row j = tid / 2, half of F: 128 bf16 of W2, loaded now
+  const int j = tid >> 1, half = tid & 1;
+  uint4 w2v[FH / 2 / 8];
+  {
+    const uint4* wrow = reinterpret_cast<const uint4*>(
+        (const T*)a.w2 + ((size_t)h * D + j) * FH + half * (FH / 2));
 #pragma unroll
-    for (int i = 0; i < FPL; i += 4) VecLoad<T, 4>::load(wrow + i, w + i);
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < FPL; ++i) acc = fmaf(w[i], hs[lane * FPL + i], acc);
-    acc = warp_sum(acc);
-    if (lane == 0)
-      ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] =
-          from_f<T>((acc + rs[j]) * invL + ldf((const T*)a.b2, (size_t)h * D + j));
+    for (int i = 0; i < FH / 2 / 8; ++i) w2v[i] = wrow[i];
   }
+  const float b2 = ldf((const T*)a.b2, (size_t)h * D + j);
+  // tile weights, computed by every warp: lane t holds tile t (and t + 32)
+  const float m0 = lane < n ? part[lane * tstride + 2 * g] : -INFINITY;
+  const float m1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g] : -INFINITY;
+  const float l0 = lane < n ? part[lane * tstride + 2 * g + 1] : 0.f;
+  const float l1 = lane + 32 < n ? part[(lane + 32) * tstride + 2 * g + 1] : 0.f;
+  const float* hsrc = part + 2 * G + (size_t)g * FH + tid;                       // f = tid
+  const float* rsrc = part + 2 * G + (size_t)G * FH + (size_t)(tid >> 7) * G * D + (size_t)g * D + (tid & 127);
+  float hacc = 0.f, racc = 0.f;
+  const float M = warp_max(fmaxf(m0, m1));
+  const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+  const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+  for (int t0 = 0; t0 < n; t0 += 16) {
+    float hv[16], rv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int t = t0 + u;
+      hv[u] = t < n ? hsrc[t * tstride] : 0.f;
+      rv[u] = t < n ? rsrc[t * tstride] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int t = t0 + u;
+      const float wt = __shfl_sync(0xffffffffu, t < 32 ? w0 : w1, t & 31);
+      hacc = fmaf(wt, hv[u], hacc);
+      racc = fmaf(wt, rv[u], racc);
+    }
+  }
+  const float L = warp_sum(w0 * l0 + w1 * l1);
+  hs[tid] = hacc;
+  rs[tid >> 7][tid & 127] = racc;
+  if (tid == 0) s_L = L;
+  __syncthreads();
+  float acc = 0.f;
+  const float* hh = hs + half * (FH / 2);
+#pragma unroll
+  for (int i = 0; i < FH / 2 / 8; ++i) {
+    float w[8];
+    const uint4 v = w2v[i];
+    if constexpr (sizeof(T) == 2) {
+      const float2 a0 = bf2_to_f2(v.x), a1 = bf2_to_f2(v.y), a2 = bf2_to_f2(v.z), a3 = bf2_to_f2(v.w);
+      w[0] = a0.x; w[1] = a0.y; w[2] = a1.x; w[3] = a1.y; w[4] = a2.x; w[5] = a2.y; w[6] = a3.x; w[7] = a3.y;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc = fmaf(w[e], hh[8 * i + e], acc);
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  if (half == 0)
+    ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] =
+        from_f<T>((acc + rs[0][j] + rs[1][j]) / s_L + b2);
 }
 
 template <typename T, int D, int FH>

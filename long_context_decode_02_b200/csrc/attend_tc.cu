@@ -44,7 +44,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128, kF = 256, kG = 4, kTile = 128, kChunk = 8, kChunksPerTile = 16;
-constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2..9 epilogue
+constexpr int kThreads = 352;  // warp 0 TMA, warp 1 MMA, warp 2 metadata, warps 3..10 epilogue
 constexpr int kEpiThreads = 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 constexpr int kPartFloats = 2 * kG + kG * kF + 2 * kG * kD;
@@ -55,20 +55,23 @@ struct TcMaps {
   CUtensorMap w1;     // [H*F][d] bf16, box 64 x 128, 128B swizzle
 };
 
-// One slot of the producer -> epilogue metadata ring (three slots: the producer fills
-// tile i+1 while the epilogue may still read tiles i-1 and i).
+// One slot of the metadata ring (filled by the metadata warp up to kMetaSlots tiles
+// ahead; read by the TMA warp and the epilogue; released after the epilogue's part B).
 struct TileMeta {
   int cid[kChunksPerTile];  // chunk id of each slot of the tile; -1 past the selection
   int nres;                 // residual rows of the tile
   int pad[3];
-  int2 res[kTile];          // (row of res_val, token row in the tile); row -1 = skip
+  uint32_t res[kTile];      // (row of res_val) << 8 | token row in the tile (255 = skip)
   uint4 q[64];              // the tile's G = 4 query rows, bf16 [4][128]
 };
-static_assert(sizeof(TileMeta) == 2128, "TileMeta layout");
-constexpr int kMetaSlots = 3;
+static_assert(sizeof(TileMeta) == 1616, "TileMeta layout");
+constexpr int kMetaSlots = 4;
+constexpr int kResPrefetch = 16;   // residual rows per thread loaded before the hidden layer
+
+constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in flight
 
 struct Layout {
-  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, meta, bar, total;
+  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, rot, roff, meta, bar, total;
 };
 __host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
@@ -79,13 +82,15 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.basis = 0;
   L.w1 = align_up(L.basis + kb * 8192, 1024);
   L.coef = L.w1 + 65536;
-  L.kbf = align_up(L.coef + kb * 8192, 1024);
-  L.p = L.kbf + 65536;          // [2][128][4] fp32
+  L.kbf = align_up(L.coef + kb * 8192, 1024);   // K~ bf16 [128 tok][128 d], one buffer
+  L.p = L.kbf + 32768;          // [2][128][4] fp32
   L.q = L.p + 4096;             // [4][128] fp32
   L.b1 = L.q + 2048;            // [256] fp32
   L.zx = L.b1 + 1024;           // [128][4] fp32
   L.red = L.zx + 2048;          // 512 B of reduction scratch
-  L.meta = L.red + 512;         // kMetaSlots x TileMeta
+  L.rot = L.red + 512;          // [kRotSlots][16 chunks][64 pairs] float2 (cos, sin)
+  L.roff = L.rot + kRotSlots * kChunksPerTile * (kD / 2) * 8;  // [64 pairs][8] float2
+  L.meta = L.roff + (kD / 2) * kChunk * 8;  // kMetaSlots x TileMeta
   L.bar = L.meta + kMetaSlots * (uint32_t)sizeof(TileMeta);  // barriers + TMEM holder
   L.total = L.bar + 256 + 1024; // + alignment slack of the dynamic base
   return L;
@@ -94,9 +99,10 @@ __host__ __device__ inline Layout make_layout(int r) {
 // barrier slots (8 bytes each) inside L.bar
 enum {
   BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
-  BAR_KT_EMPTY1, BAR_KBF_FULL0, BAR_KBF_FULL1, BAR_KBF_EMPTY0, BAR_KBF_EMPTY1, BAR_H_FULL,
-  BAR_H_EMPTY, BAR_DRAIN, BAR_META_FULL0, BAR_META_FULL1, BAR_META_FULL2, BAR_META_EMPTY0,
-  BAR_META_EMPTY1, BAR_META_EMPTY2, BAR_COUNT
+  BAR_KT_EMPTY1, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN,
+  BAR_ROT_FULL0, BAR_ROT_EMPTY0 = BAR_ROT_FULL0 + kRotSlots,
+  BAR_META_FULL0 = BAR_ROT_EMPTY0 + kRotSlots, BAR_META_EMPTY0 = BAR_META_FULL0 + kMetaSlots,
+  BAR_COUNT = BAR_META_EMPTY0 + kMetaSlots
 };
 static_assert(BAR_COUNT * 8 + 8 <= 256, "barrier area");
 
@@ -136,6 +142,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   float* sZx = reinterpret_cast<float*>(gbase + L.zx);
   float* sRed = reinterpret_cast<float*>(gbase + L.red);  // [4 quadrants][4 g] x 2, ml[2][4][2]
   TileMeta* meta = reinterpret_cast<TileMeta*>(gbase + L.meta);
+  float2* sRot = reinterpret_cast<float2*>(gbase + L.rot);
+  float2* sRoff = reinterpret_cast<float2*>(gbase + L.roff);
 
   auto item_of = [&](int i, int& b, int& tile) {
     const int it = cta_in_head + i * cta_per_head;
@@ -152,10 +160,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     mbar_init(bar(BAR_KT_FULL1), 1);
     mbar_init(bar(BAR_KT_EMPTY0), 8);
     mbar_init(bar(BAR_KT_EMPTY1), 8);
-    mbar_init(bar(BAR_KBF_FULL0), 8);
-    mbar_init(bar(BAR_KBF_FULL1), 8);
-    mbar_init(bar(BAR_KBF_EMPTY0), 1);
-    mbar_init(bar(BAR_KBF_EMPTY1), 1);
+    mbar_init(bar(BAR_KBF_FULL), 8);
+    mbar_init(bar(BAR_KBF_EMPTY), 1);
+    for (int i = 0; i < kRotSlots; ++i) {
+      mbar_init(bar(BAR_ROT_FULL0 + i), 1);
+      mbar_init(bar(BAR_ROT_EMPTY0 + i), 8);
+    }
     mbar_init(bar(BAR_H_FULL), 1);
     mbar_init(bar(BAR_H_EMPTY), 8);
     mbar_init(bar(BAR_DRAIN), 1);
@@ -176,33 +186,91 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 
   const int32_t* sel_all = a.sel;
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Tile metadata (chunk ids, the residual rows of its chunks, its queries) goes to the
-    // ring; the coefficient rows of its 16 chunks are TMA-gathered into the tile buffer.
-    const int32_t* ptr_all = a.chunk_ptr;
-    const int32_t* ridx_all = a.res_idx;
-    // returns this lane's chunk id (lanes 0..15) or -1
-    auto build_meta = [&](int i, bool& ok) -> int {
+    // ------------------------------------------------------------ TMA warp
+    // Weights once; then per tile the coefficient rows of its 16 chunks (chunk ids from
+    // the tile's metadata slot), TMA-gathered into the 64B-swizzled tile buffer.
+    int issued_phase = -1;  // parity of the last coef load issued (for the drain)
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192 + 65536));
+      for (int kb = 0; kb < kb_r; ++kb)
+        tma_load_2d(base + L.basis + kb * 8192, &maps.basis, kb * 32, h * kD, bar(BAR_W));
+      for (int hf = 0; hf < 2; ++hf)
+        for (int kb = 0; kb < 2; ++kb)
+          tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
+                      h * kF + hf * 128, bar(BAR_W));
+    }
+    for (int i = 0; i < n_mine; ++i) {
       int b, tile;
       item_of(i, b, tile);
       const int slot = i % kMetaSlots;
       int got = 0;
       if (lane == 0)
-        got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
-      ok = __shfl_sync(0xffffffffu, got, 0) != 0;
-      if (!ok) return -1;
-      TileMeta* M = meta + slot;
-      const int p = b * dm.H + h;
-      int cid = -1, e0 = 0, n = 0;
+        got = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag) &&
+              mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      const int cid = lane < kChunksPerTile ? meta[slot].cid[lane] : -1;
+      if (lane == 0)
+        mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
+      __syncwarp();
+      if (lane < kChunksPerTile) {
+        const int row = b * dm.T + (cid < 0 ? 0 : cid) * kChunk;
+        for (int kb = 0; kb < kb_r; ++kb)
+          tma_load_2d(base + L.coef + kb * 8192 + lane * 512, &maps.coef, kb * 32, row,
+                      bar(BAR_COEF_FULL));
+      }
+      issued_phase = i & 1;
+    }
+    // drain: a load still in flight (only possible after an abort) must land before exit
+    if (lane == 0 && *abort_flag && issued_phase >= 0) {
+      int dummy = 0;
+      mbar_wait_bounded(bar(BAR_COEF_FULL), (uint32_t)issued_phase, (volatile int*)&dummy);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ metadata warp
+    // Per tile: chunk ids, the residual rows of its chunks (CSR spans, every index
+    // bounds-checked), its queries, and the rotation of each chunk's base position,
+    // up to kMetaSlots (kRotSlots for rotations) tiles ahead of the epilogue. The next
+    // tile's chunk ids are fetched while the current tile is built.
+    const int32_t* ptr_all = a.chunk_ptr;
+    const int32_t* ridx_all = a.res_idx;
+    // theta_i for this lane's pairs (lane, lane + 32)
+    const double th0 = a.rope.theta64[lane], th1 = a.rope.theta64[lane + 32];
+    auto load_cid = [&](int i) -> int {
+      int b, tile;
+      item_of(i, b, tile);
+      int cid = -1;
       if (lane < kChunksPerTile) {
         const int gs = tile * kChunksPerTile + lane;
-        if (gs < dm.k) {
-          cid = sel_all[(size_t)p * dm.k + gs];
-          if (cid < 0 || cid >= dm.Nc) {
-            raise_status(a.status, kStatusDeviceCheck);
-            cid = -1;
-          }
-        }
+        if (gs < dm.k) cid = sel_all[((size_t)b * dm.H + h) * dm.k + gs];
+      }
+      return cid;
+    };
+    int cid_next = n_mine > 0 ? load_cid(0) : -1;
+    for (int i = 0; i < n_mine; ++i) {
+      int b, tile;
+      item_of(i, b, tile);
+      const int slot = i % kMetaSlots;
+      const int p = b * dm.H + h;
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
+      const uint4 q0 = qsrc[lane], q1 = qsrc[lane + 32];
+      int cid = cid_next;
+      if (i + 1 < n_mine) cid_next = load_cid(i + 1);
+      if (lane < kChunksPerTile && cid >= dm.Nc) {
+        raise_status(a.status, kStatusDeviceCheck);
+        cid = -1;
+      }
+      if (cid < -1) {
+        raise_status(a.status, kStatusDeviceCheck);
+        cid = -1;
+      }
+      int got = 0;
+      if (lane == 0)
+        got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      TileMeta* M = meta + slot;
+      int e0 = 0, n = 0;
+      if (lane < kChunksPerTile) {
         if (cid >= 0) {
           const int32_t* ptr = ptr_all + (size_t)p * (dm.Nc + 1);
           e0 = ptr[cid];
@@ -235,54 +303,43 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
             const int tt = t[j] - cid * kChunk;
             const bool good = tt >= 0 && tt < kChunk;
             if (!good) raise_status(a.status, kStatusDeviceCheck);
-            M->res[off + j] = make_int2(e0 + j, good ? lane * kChunk + tt : -1);
+            M->res[off + j] = ((uint32_t)(e0 + j) << 8) | (good ? (uint32_t)(lane * kChunk + tt) : 255u);
           }
         }
       }
       if (lane == 0) M->nres = total;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(
-          (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
-      M->q[lane] = qsrc[lane];
-      M->q[lane + 32] = qsrc[lane + 32];
+      M->q[lane] = q0;
+      M->q[lane + 32] = q1;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_META_FULL0 + slot));
-      return cid;
-    };
-
-    int issued_phase = -1;  // parity of the last coef load issued (for the drain)
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192 + 65536));
-      for (int kb = 0; kb < kb_r; ++kb)
-        tma_load_2d(base + L.basis + kb * 8192, &maps.basis, kb * 32, h * kD, bar(BAR_W));
-      for (int hf = 0; hf < 2; ++hf)
-        for (int kb = 0; kb < 2; ++kb)
-          tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
-                      h * kF + hf * 128, bar(BAR_W));
-    }
-    bool ok = true;
-    int cid = n_mine > 0 ? build_meta(0, ok) : -1;
-    for (int i = 0; ok && i < n_mine; ++i) {
-      int b, tile;
-      item_of(i, b, tile);
-      int got = 0;
-      if (lane == 0) got = mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
-      if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      if (lane == 0)
-        mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
-      __syncwarp();
-      if (lane < kChunksPerTile) {
-        const int row = b * dm.T + (cid < 0 ? 0 : cid) * kChunk;
-        for (int kb = 0; kb < kb_r; ++kb)
-          tma_load_2d(base + L.coef + kb * 8192 + lane * 512, &maps.coef, kb * 32, row,
-                      bar(BAR_COEF_FULL));
+      // chunk-base rotations (cos, sin)(8 cid theta_i): the angle is reduced modulo 2 pi
+      // in fp64 (error ~1e-11 rad) and its sine and cosine taken in fp32 (|err| < 4e-7)
+      {
+        const int rs = i % kRotSlots;
+        int rgot = 0;
+        if (lane == 0)
+          rgot = mbar_wait_bounded(bar(BAR_ROT_EMPTY0 + rs), ((i / kRotSlots) & 1) ^ 1, abort_flag);
+        if (!__shfl_sync(0xffffffffu, rgot, 0)) break;
+        float2* R = sRot + rs * kChunksPerTile * (kD / 2);
+        const double two_pi_hi = 6.283185307179586232, two_pi_lo = 2.4492935982947064e-16;
+        const double inv_two_pi = 0.15915494309189533577;
+#pragma unroll 4
+        for (int c = 0; c < kChunksPerTile; ++c) {
+          const int cc = __shfl_sync(0xffffffffu, cid, c);
+          const double pb = (double)((cc < 0 ? 0 : cc) * kChunk);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const double ang = pb * (w ? th1 : th0);
+            const double kq = rint(ang * inv_two_pi);
+            const float red = (float)fma(-kq, two_pi_lo, fma(-kq, two_pi_hi, ang));
+            float sn, cs;
+            __sincosf(red, &sn, &cs);
+            R[c * (kD / 2) + w * 32 + lane] = make_float2(cs, sn);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_ROT_FULL0 + rs));
       }
-      issued_phase = i & 1;
-      if (i + 1 < n_mine) cid = build_meta(i + 1, ok);
-    }
-    // drain: a load still in flight (only possible after an abort) must land before exit
-    if (lane == 0 && *abort_flag && issued_phase >= 0) {
-      int dummy = 0;
-      mbar_wait_bounded(bar(BAR_COEF_FULL), (uint32_t)issued_phase, (volatile int*)&dummy);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -305,11 +362,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
         return true;
       };
       auto issue_h = [&](int i) -> bool {
-        const int u = i & 1;
-        if (!mbar_wait_bounded(bar(BAR_KBF_FULL0 + u), (i >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_bounded(bar(BAR_KBF_FULL), i & 1, abort_flag)) return false;
         if (!mbar_wait_bounded(bar(BAR_H_EMPTY), (i & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t skb = base + L.kbf + (uint32_t)u * 32768;
+        const uint32_t skb = base + L.kbf;
         for (int hf = 0; hf < 2; ++hf) {
           const uint32_t d_t = tmem + 256u + (uint32_t)hf * 128u;
           for (int s = 0; s < 8; ++s) {
@@ -319,7 +375,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
           }
         }
         mma_commit(bar(BAR_H_FULL));
-        mma_commit(bar(BAR_KBF_EMPTY0 + u));
+        mma_commit(bar(BAR_KBF_EMPTY));
         return true;
       };
       if (ok && n_mine > 0) ok = issue_k(0);
@@ -334,10 +390,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;             // 0..7
+    const int ew = warp - 3;             // 0..7
     const int qd = warp & 3;             // TMEM lane quadrant this warp may access
     const int hf = ew >> 2;              // column half
-    const int et = threadIdx.x - 64;     // 0..255
+    const int et = threadIdx.x - 96;     // 0..255
     const int trow = 32 * qd + lane;     // token row (A) / hidden-unit row within a half (B)
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
@@ -346,6 +402,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 
     for (int i = et; i < kF; i += kEpiThreads)
       sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
+    // in-chunk offsets: sRoff[pair * 8 + j] = (cos, sin)(j theta_pair), j < 8
+    for (int i = et; i < (kD / 2) * kChunk; i += kEpiThreads)
+      sRoff[i] = a.rope.lo32[(i & (kChunk - 1)) * (kD / 2) + (i >> 3)];
     bool ok = true;
 
     // A failed (timed-out) wait never changes the sequence of named barriers: the
@@ -356,6 +415,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       const int slot = i % kMetaSlots;
       const TileMeta* M = meta + slot;
       bool good = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
+      const bool valid = M->cid[trow >> 3] >= 0;
       named_bar_sync(1, kEpiThreads);  // previous readers of sQ / sZx are done
       {
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
@@ -363,9 +423,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
         sQ[2 * et] = f.x;
         sQ[2 * et + 1] = f.y;
       }
-      const int cid = M->cid[trow >> 3];
-      const bool valid = cid >= 0;
-      const int pos = valid ? cid * kChunk + (trow & 7) : 0;
 
       good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
       tc_fence_after();
@@ -378,9 +435,51 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY0 + u));
 
-      // K~_pre in bf16 -> shared memory, 128B-swizzled K-major [tok][d]
-      good = mbar_wait_bounded(bar(BAR_KBF_EMPTY0 + u), ((i >> 1) & 1) ^ 1, abort_flag) && good;
-      const uint32_t skb = base + L.kbf + (uint32_t)u * 32768;
+      const int rs = i % kRotSlots;
+      good = mbar_wait_bounded(bar(BAR_ROT_FULL0 + rs), (i / kRotSlots) & 1, abort_flag) && good;
+      named_bar_sync(1, kEpiThreads);  // sQ ready
+      // RoPE on pairs (32hf + e, 64 + 32hf + e): the chunk-base rotation (from the ring)
+      // times the in-chunk offset (table) by angle addition; partial logits accumulate as
+      // (x, y) pairs with packed fp32x2 FMAs, the queries of 4 pairs in one 16-byte load
+      const float4* rb4 = reinterpret_cast<const float4*>(
+          sRot + (rs * kChunksPerTile + (trow >> 3)) * (kD / 2) + 32 * hf);
+      const float2* ro = sRoff + (32 * hf) * kChunk + (trow & 7);
+      float2 z2[kG];
+#pragma unroll
+      for (int g = 0; g < kG; ++g) z2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int e4 = 0; e4 < 32; e4 += 4) {
+        const float4 b01 = rb4[e4 / 2], b23 = rb4[e4 / 2 + 1];
+        const float2 bs[4] = {make_float2(b01.x, b01.y), make_float2(b01.z, b01.w),
+                              make_float2(b23.x, b23.y), make_float2(b23.z, b23.w)};
+        float2 rot[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int e = e4 + w;
+          const float2 cs = rope_combine(bs[w], ro[e * kChunk]);
+          rot[w] = make_float2(x[e] * cs.x - y[e] * cs.y, x[e] * cs.y + y[e] * cs.x);
+        }
+        const int pi = 32 * hf + e4;
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+          const float4 qx = *reinterpret_cast<const float4*>(sQ + g * kD + pi);
+          const float4 qy = *reinterpret_cast<const float4*>(sQ + g * kD + 64 + pi);
+          z2[g] = __ffma2_rn(make_float2(qx.x, qy.x), rot[0], z2[g]);
+          z2[g] = __ffma2_rn(make_float2(qx.y, qy.y), rot[1], z2[g]);
+          z2[g] = __ffma2_rn(make_float2(qx.z, qy.z), rot[2], z2[g]);
+          z2[g] = __ffma2_rn(make_float2(qx.w, qy.w), rot[3], z2[g]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_ROT_EMPTY0 + rs));
+      float z[kG];
+#pragma unroll
+      for (int g = 0; g < kG; ++g) z[g] = z2[g].x + z2[g].y;
+
+      // K~_pre in bf16 -> shared memory (single buffer, 128B-swizzled K-major [tok][d]);
+      // the hidden-layer MMA of the previous tile has released it by now
+      good = mbar_wait_bounded(bar(BAR_KBF_EMPTY), (i & 1) ^ 1, abort_flag) && good;
+      const uint32_t skb = base + L.kbf;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         st_shared_v4(skb + sw128_offset(trow, 4 * hf + cc),
@@ -392,36 +491,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL0 + u));
+      if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL));
 
-      named_bar_sync(1, kEpiThreads);  // sQ ready
-      // RoPE on pairs (32hf + e, 64 + 32hf + e) and partial logits; this thread's 32
-      // (cos, sin) pairs are contiguous in both position-major tables
-      float z[kG] = {0.f, 0.f, 0.f, 0.f};
-      const float4* lo4 = reinterpret_cast<const float4*>(a.rope.lo32 + (pos & (kRopeLo - 1)) * (kD / 2) + 32 * hf);
-      const float4* hi4 = reinterpret_cast<const float4*>(a.rope.hi32 + (size_t)(pos >> kRopeLoBits) * (kD / 2) + 32 * hf);
-#pragma unroll
-      for (int e4 = 0; e4 < 32; e4 += 8) {
-        float4 lo[4], hi[4];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) { lo[v] = lo4[e4 / 2 + v]; hi[v] = hi4[e4 / 2 + v]; }
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-#pragma unroll
-          for (int w2 = 0; w2 < 2; ++w2) {
-            const int e = e4 + 2 * v + w2;
-            const float2 lo2 = w2 ? make_float2(lo[v].z, lo[v].w) : make_float2(lo[v].x, lo[v].y);
-            const float2 hi2 = w2 ? make_float2(hi[v].z, hi[v].w) : make_float2(hi[v].x, hi[v].y);
-            const float2 cs = rope_combine(hi2, lo2);
-            const int pi = 32 * hf + e;
-            const float xr = x[e] * cs.x - y[e] * cs.y;
-            const float yr = x[e] * cs.y + y[e] * cs.x;
-#pragma unroll
-            for (int g = 0; g < kG; ++g)
-              z[g] = fmaf(sQ[g * kD + pi], xr, fmaf(sQ[g * kD + 64 + pi], yr, z[g]));
-          }
-        }
-      }
       if (hf == 1) *reinterpret_cast<float4*>(sZx + 4 * trow) = make_float4(z[0], z[1], z[2], z[3]);
       named_bar_sync(1, kEpiThreads);
       if (hf == 0) {
@@ -468,56 +539,82 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       const TileMeta* M = meta + slot;
       const int p = b * dm.H + h;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
+      // residual rows of the tile: thread = column j; rows split between the two halves.
+      // The first kResPrefetch of this thread's rows are loaded before the hidden layer.
+      const int j = trow;
+      const int nres = M->nres;
+      const __nv_bfloat16* rbase = rval_all + (size_t)p * dm.n_res * kD + j;
+      float rv[kResPrefetch];
+      int rrow[kResPrefetch];
+#pragma unroll
+      for (int v = 0; v < kResPrefetch; ++v) {
+        const int ei = hf + 2 * v;
+        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
+        rrow[v] = (int)(ent & 255u);
+        rv[v] = rrow[v] != 255 ? __bfloat162float(rbase[(size_t)(ent >> 8) * kD]) : 0.f;
+      }
       const bool good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag);
       tc_fence_after();
       const int f = 128 * hf + trow;
       const float bias = sB1[f];
-      float hacc[kG] = {0.f, 0.f, 0.f, 0.f};
+      float2 hacc01 = make_float2(0.f, 0.f), hacc23 = make_float2(0.f, 0.f);
       const float4* P4 = reinterpret_cast<const float4*>(sP + u * 512);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float hv[32];
         tmem_ld_x32(tmem + lane_addr + 256u + (uint32_t)(hf * 128 + 32 * c), hv);
         tmem_wait_ld();
+        if (ACT == LOWRAM_ACT_SILU) {
+          // two tokens per step: hx = (h + b1)/2, silu = hx + hx tanh(hx)
+          const float2 half2 = make_float2(0.5f, 0.5f);
+          const float2 hb2 = make_float2(0.5f * bias, 0.5f * bias);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float av = act_fast<ACT>(hv[e] + bias);
-          const float4 pv = P4[32 * c + e];
-          hacc[0] = fmaf(pv.x, av, hacc[0]);
-          hacc[1] = fmaf(pv.y, av, hacc[1]);
-          hacc[2] = fmaf(pv.z, av, hacc[2]);
-          hacc[3] = fmaf(pv.w, av, hacc[3]);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 hx = __ffma2_rn(half2, make_float2(hv[e], hv[e + 1]), hb2);
+            const float2 av = __ffma2_rn(hx, make_float2(tanh_approx(hx.x), tanh_approx(hx.y)), hx);
+            const float4 p0 = P4[32 * c + e], p1 = P4[32 * c + e + 1];
+            hacc01 = __ffma2_rn(make_float2(p0.x, p0.y), make_float2(av.x, av.x), hacc01);
+            hacc23 = __ffma2_rn(make_float2(p0.z, p0.w), make_float2(av.x, av.x), hacc23);
+            hacc01 = __ffma2_rn(make_float2(p1.x, p1.y), make_float2(av.y, av.y), hacc01);
+            hacc23 = __ffma2_rn(make_float2(p1.z, p1.w), make_float2(av.y, av.y), hacc23);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float av = act_fast<ACT>(hv[e] + bias);
+            const float4 pv = P4[32 * c + e];
+            hacc01 = __ffma2_rn(make_float2(pv.x, pv.y), make_float2(av, av), hacc01);
+            hacc23 = __ffma2_rn(make_float2(pv.z, pv.w), make_float2(av, av), hacc23);
+          }
         }
       }
+      const float hacc[kG] = {hacc01.x, hacc01.y, hacc23.x, hacc23.y};
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
 #pragma unroll
       for (int g = 0; g < kG; ++g) part[2 * kG + g * kF + f] = hacc[g];
 
-      // residual rows of the tile (list built by the producer); thread = column j,
-      // rows split between the two halves, loads issued four at a time
-      const int j = trow;
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
-      const int nres = M->nres;
-      for (int e0 = 2 * 0 + hf; e0 < nres; e0 += 8) {
-        int2 ent[4];
-        float rv[4];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int ei = e0 + 2 * v;
-          ent[v] = ei < nres ? M->res[ei] : make_int2(0, -1);
-          rv[v] = ent[v].y >= 0 ? __bfloat162float(rval_all[((size_t)p * dm.n_res + ent[v].x) * kD + j]) : 0.f;
-        }
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          if (ent[v].y < 0) continue;
-          const float4 pv = P4[ent[v].y];
-          racc[0] = fmaf(pv.x, rv[v], racc[0]);
-          racc[1] = fmaf(pv.y, rv[v], racc[1]);
-          racc[2] = fmaf(pv.z, rv[v], racc[2]);
-          racc[3] = fmaf(pv.w, rv[v], racc[3]);
-        }
+      for (int v = 0; v < kResPrefetch; ++v) {
+        if (rrow[v] == 255) continue;
+        const float4 pv = P4[rrow[v]];
+        racc[0] = fmaf(pv.x, rv[v], racc[0]);
+        racc[1] = fmaf(pv.y, rv[v], racc[1]);
+        racc[2] = fmaf(pv.z, rv[v], racc[2]);
+        racc[3] = fmaf(pv.w, rv[v], racc[3]);
+      }
+      for (int ei = hf + 2 * kResPrefetch; ei < nres; ei += 2) {   // rows beyond the prefetch
+        const uint32_t ent = M->res[ei];
+        const int row = (int)(ent & 255u);
+        if (row == 255) continue;
+        const float r = __bfloat162float(rbase[(size_t)(ent >> 8) * kD]);
+        const float4 pv = P4[row];
+        racc[0] = fmaf(pv.x, r, racc[0]);
+        racc[1] = fmaf(pv.y, r, racc[1]);
+        racc[2] = fmaf(pv.z, r, racc[2]);
+        racc[3] = fmaf(pv.w, r, racc[3]);
       }
       float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
 #pragma unroll

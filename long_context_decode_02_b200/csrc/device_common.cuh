@@ -217,6 +217,59 @@ __device__ uint32_t group_kth_largest(const Grp& g, int n, int k, KeyFn key_of,
   return prefix;
 }
 
+// Same as group_kth_largest, with warp-aggregated histogram updates: lanes of a warp
+// holding the same digit add their count with one atomic. For key sets concentrated in
+// few digits (scores sharing an exponent).
+template <typename KeyFn>
+__device__ uint32_t group_kth_largest_aggr(const Grp& g, int n, int k, KeyFn key_of,
+                                           unsigned* hist, unsigned* bc) {
+  uint32_t prefix = 0, mask = 0;
+  unsigned remaining = (unsigned)k;
+  const int lane = g.tid & 31;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = g.tid; i < 256; i += g.nt) hist[i] = 0;
+    g.sync();
+    for (int base = 0; base < n; base += g.nt) {
+      const int i = base + g.tid;
+      unsigned digit = 256u;
+      if (i < n) {
+        const uint32_t key = key_of(i);
+        if ((key & mask) == prefix) digit = (key >> shift) & 255u;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+    }
+    g.sync();
+    if (g.tid < 32) {
+      unsigned own = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) own += hist[255 - 8 * lane - j];
+      unsigned incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const unsigned before = incl - own;
+      if (before < remaining && incl >= remaining) {
+        unsigned acc = before;
+        for (int j = 0; j < 8; ++j) {
+          const int dg = 255 - 8 * lane - j;
+          const unsigned c = hist[dg];
+          if (acc + c >= remaining) { bc[0] = (unsigned)dg; bc[1] = remaining - acc; break; }
+          acc += c;
+        }
+      }
+    }
+    g.sync();
+    prefix |= bc[0] << shift;
+    mask |= 255u << shift;
+    remaining = bc[1];
+    g.sync();
+  }
+  return prefix;
+}
+
 // Sort n (a power of two) (key, idx) pairs in shared memory so that (key desc, idx asc)
 // comes first.
 __device__ inline void group_sort_desc(const Grp& g, float* key, int* idx, int n) {

@@ -24,6 +24,7 @@ struct lowram_ctx {
   int n_hi;
   int* status;    // device word
   int* counters;  // device [B*H]
+  double* theta64;  // device [d/2]
 };
 
 namespace {
@@ -131,6 +132,7 @@ RopeTables rope_of(const lowram_ctx* ctx) {
   r.hi64 = ctx->hi64;
   r.n_hi = ctx->n_hi;
   r.half = ctx->cfg.head_dim / 2;
+  r.theta64 = ctx->theta64;
   return r;
 }
 
@@ -228,8 +230,10 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
   // two-level tables, fp64 on the host: theta_i = theta^(-2i/d)
   std::vector<float2> lo32((size_t)half * kRopeLo), hi32((size_t)half * ctx->n_hi);
   std::vector<double2> lo64((size_t)half * kRopeLo), hi64((size_t)half * ctx->n_hi);
+  std::vector<double> th64((size_t)half);
   for (int i = 0; i < half; ++i) {
     const double th = std::pow(c->rope_theta, -2.0 * i / c->head_dim);
+    th64[i] = th;
     for (int t = 0; t < kRopeLo; ++t) {
       const double ang = (double)t * th;
       lo64[(size_t)t * half + i] = make_double2(std::cos(ang), std::sin(ang));
@@ -247,14 +251,16 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->lo64, lo64.size() * sizeof(double2)) == cudaSuccess &&
             cudaMalloc(&ctx->hi64, hi64.size() * sizeof(double2)) == cudaSuccess &&
             cudaMalloc(&ctx->status, sizeof(int)) == cudaSuccess &&
-            cudaMalloc(&ctx->counters, pairs * sizeof(int)) == cudaSuccess;
+            cudaMalloc(&ctx->counters, pairs * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
   ok = ok &&
        cudaMemcpy(ctx->lo32, lo32.data(), lo32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->hi32, hi32.data(), hi32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->lo64, lo64.data(), lo64.size() * sizeof(double2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->hi64, hi64.data(), hi64.size() * sizeof(double2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemset(ctx->status, 0, sizeof(int)) == cudaSuccess &&
-       cudaMemset(ctx->counters, 0, pairs * sizeof(int)) == cudaSuccess;
+       cudaMemset(ctx->counters, 0, pairs * sizeof(int)) == cudaSuccess &&
+       cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     lowram_destroy(ctx);
@@ -273,6 +279,7 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->hi64);
   cudaFree(ctx->status);
   cudaFree(ctx->counters);
+  cudaFree(ctx->theta64);
   delete ctx;
 }
 

@@ -7,7 +7,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include "../../include/lowram.h"
+#include "lowram.h"
 
 namespace lowram {
 
@@ -31,6 +31,7 @@ struct RopeTables {
   const double2* hi64;
   int n_hi;
   int half;   // d / 2
+  const double* theta64;  // theta_i = theta^(-2i/d), i < d/2 (fp64)
 };
 
 struct Dims {

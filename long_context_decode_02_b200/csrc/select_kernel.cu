@@ -37,6 +37,8 @@ constexpr int kStages = 3;
 constexpr int kStageBytes = 65536;
 constexpr int kCap = 2048;                    // candidate capacity of the fast selection
 constexpr int kSample = 1024;                 // sampled scores placing its threshold
+constexpr int kBitmapChunks = 65536;          // chunks the fast path's output bitmap covers
+constexpr int kWindowCap = 256;               // fp64 re-scored candidates of the fast path
 
 template <typename T, int D>
 struct Geom {
@@ -57,9 +59,9 @@ __host__ __device__ inline SelSmem sel_smem(int G, int D) {
   L.q = kStages * kStageBytes;
   L.ckey = L.q + (uint32_t)(G * D * 4);
   L.cid = L.ckey + kCap * 4;
-  L.outs = L.cid + kCap * 4;
-  L.misc = L.outs + (kCap / 2) * 4;     // 2 KB of scalars and reduction scratch
-  L.bar = L.misc + 2048;
+  L.outs = L.cid + kCap * 4;            // chunk bitmap of the fast path
+  L.misc = L.outs + kBitmapChunks / 8;   // scalars, reduction scratch, window list
+  L.bar = L.misc + 3072;
   L.total = L.bar + 128 + 1024;
   return L;
 }
@@ -70,9 +72,10 @@ struct Misc {
   float fscr[33];
   int iscr[33];
   int cnt, lo, hi, last;
-  float t0;
+  float t0, fmax;
+  int wl[kWindowCap];
 };
-static_assert(sizeof(Misc) <= 2048, "Misc scratch");
+static_assert(sizeof(Misc) <= 3072, "Misc scratch");
 
 template <typename T, int D, int G>
 __device__ double score64(const T* lrow, const T* qb) {
@@ -83,12 +86,6 @@ __device__ double score64(const T* lrow, const T* qb) {
     best = fmax(best, acc);
   }
   return best;
-}
-
-__device__ __forceinline__ int next_pow2(int x) {
-  int n = 1;
-  while (n < x) n <<= 1;
-  return n;
 }
 
 // ---------------------------------------------------------------- selection
@@ -159,17 +156,50 @@ __device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc
   }
 }
 
-// Fast path: the candidate set is all scores (N_c <= kCap) or those at or above a
-// threshold placed from a sorted sample; candidates are sorted, the window around the
-// k-th is re-scored in fp64 and ranked exactly. Returns false (writing nothing) when the
-// candidate set cannot be proven to contain the answer.
+// fp64 score of one landmark row against the group's queries held (exactly, as fp32) in
+// shared memory: exact products, one fp64 accumulator per query head.
 template <typename T, int D, int G>
-__device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, float* ckey,
-                                 int* cid, int* outs, Misc* ms) {
+__device__ double score64_row(const T* lrow, const float* sQ) {
+  constexpr int kV = 16 / (int)sizeof(T);
+  double acc[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) acc[g] = 0.0;
+  const uint4* w4 = reinterpret_cast<const uint4*>(lrow);
+#pragma unroll 4
+  for (int c = 0; c < D / kV; ++c) {
+    const uint4 w = w4[c];
+    float v[kV];
+    if constexpr (sizeof(T) == 2) {
+      const float2 a0 = bf2_to_f2(w.x), a1 = bf2_to_f2(w.y), a2 = bf2_to_f2(w.z), a3 = bf2_to_f2(w.w);
+      v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y; v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
+    } else {
+      v[0] = __uint_as_float(w.x); v[1] = __uint_as_float(w.y);
+      v[2] = __uint_as_float(w.z); v[3] = __uint_as_float(w.w);
+    }
+#pragma unroll
+    for (int e = 0; e < kV; ++e)
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = fma((double)sQ[g * D + c * kV + e], (double)v[e], acc[g]);
+  }
+  double best = acc[0];
+#pragma unroll
+  for (int g = 1; g < G; ++g) best = fmax(best, acc[g]);
+  return best;
+}
+
+// Fast path. Candidates: all scores (N_c <= kCap), or every score at or above a
+// threshold t0 = the j-th largest of an evenly spaced sample (radix select). tau = the
+// k-th largest candidate (radix select); candidates above tau + delta are in; the window
+// |s - tau| <= delta is re-scored in fp64 and ranked by (score desc, index asc); the k
+// chosen chunk ids are written ascending through a bitmap scan. Returns false (writing
+// nothing) when the candidate set cannot be proven to contain the answer.
+template <typename T, int D, int G>
+__device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, const float* sQ,
+                                 float* ckey, int* cid, uint32_t* bits, Misc* ms) {
   const Dims& dm = a.dm;
   const int Nc = dm.Nc, k = dm.k;
   const int lane = g.tid & 31;
-  if (k > kCap / 2) return false;
+  if (k > kCap / 2 || Nc > kBitmapChunks) return false;
   const float* s = a.scores + (size_t)p * Nc;
   int m;
   float t0 = -INFINITY;
@@ -177,93 +207,143 @@ __device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, float
   if (!sampled) {
     for (int i = g.tid; i < Nc; i += g.nt) { ckey[i] = __ldcg(s + i); cid[i] = i; }
     m = Nc;
+    g.sync();
   } else {
-    for (int i = g.tid; i < kSample; i += g.nt) {
-      const int j = (int)(((long long)i * Nc) / kSample);
-      ckey[i] = __ldcg(s + j);
-      cid[i] = j;
-    }
+    uint32_t* skey = reinterpret_cast<uint32_t*>(cid);
+    for (int i = g.tid; i < kSample; i += g.nt)
+      skey[i] = f2key(__ldcg(s + (int)(((long long)i * Nc) / kSample)));
     g.sync();
-    group_sort_desc(g, ckey, cid, kSample);
-    if (g.tid == 0) {
-      int j = (int)((3LL * k * kSample) / (2LL * Nc)) + 16;
-      if (j > kSample - 1) j = kSample - 1;
-      ms->t0 = ckey[j];
-      ms->cnt = 0;
-    }
+    int j = (int)((3LL * k * kSample) / (2LL * Nc)) + 16;
+    if (j > kSample) j = kSample;
+    t0 = key2f(group_kth_largest_aggr(g, kSample, j, [&](int i) { return skey[i]; },
+                                      ms->hist, ms->bc));
+    if (g.tid == 0) ms->cnt = 0;
     g.sync();
-    t0 = ms->t0;
-    for (int base = 0; base < Nc; base += g.nt) {
-      const int i = base + g.tid;
-      const float x = i < Nc ? __ldcg(s + i) : -INFINITY;
-      const bool keep = i < Nc && x >= t0;
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      int wb = 0;
-      if (lane == 0 && bal) wb = atomicAdd(&ms->cnt, __popc(bal));
-      wb = __shfl_sync(0xffffffffu, wb, 0);
-      if (keep) {
-        const int pos = wb + __popc(bal & ((1u << lane) - 1u));
-        if (pos < kCap) { ckey[pos] = x; cid[pos] = i; }
+    // every score >= t0 becomes a candidate (warp-aggregated append); each thread issues
+    // 8 independent 16-byte loads before filtering them (rows are 16-byte aligned when
+    // 4 | N_c; otherwise scalar loads)
+    const int n4 = (Nc & 3) == 0 ? Nc / 4 : 0;
+    if (n4 == 0) {
+      for (int i = g.tid; i < Nc; i += g.nt) {
+        const float x = __ldcg(s + i);
+        if (x >= t0) {
+          const int pos = atomicAdd(&ms->cnt, 1);
+          if (pos < kCap) { ckey[pos] = x; cid[pos] = i; }
+        }
+      }
+    }
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    for (int base = 0; base < n4; base += 8 * g.nt) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i4 = base + u * g.nt + g.tid;
+        v[u] = i4 < n4 ? __ldcg(s4 + i4) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i4 = base + u * g.nt + g.tid;
+        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * i4 + e;
+          const bool keep = i < Nc && xs[e] >= t0;
+          const unsigned bal = __ballot_sync(0xffffffffu, keep);
+          if (bal == 0) continue;
+          int wb = 0;
+          if (lane == 0) wb = atomicAdd(&ms->cnt, __popc(bal));
+          wb = __shfl_sync(0xffffffffu, wb, 0);
+          if (keep) {
+            const int pos = wb + __popc(bal & ((1u << lane) - 1u));
+            if (pos < kCap) { ckey[pos] = xs[e]; cid[pos] = i; }
+          }
+        }
       }
     }
     g.sync();
     m = ms->cnt;
     if (m > kCap || m < k) return false;
   }
-  const int n = next_pow2(m);
-  for (int i = m + g.tid; i < n; i += g.nt) { ckey[i] = -INFINITY; cid[i] = 0x7fffffff; }
+  const double tau = (double)key2f(group_kth_largest_aggr(
+      g, m, k, [&](int i) { return f2key(ckey[i]); }, ms->hist, ms->bc));
+  if (g.tid == 0) { ms->cnt = 0; ms->lo = 0; ms->fmax = 0.f; }
   g.sync();
-  group_sort_desc(g, ckey, cid, n);
-  const double tau = (double)ckey[k - 1];
-  const double delta = 1e-3 * fabs(tau) + 1e-6 * fmax(fabs((double)ckey[0]), fabs(tau)) + 1e-30;
+  // |largest candidate| for the window floor
+  {
+    float mx = 0.f;
+    for (int i = g.tid; i < m; i += g.nt) mx = fmaxf(mx, fabsf(ckey[i]));
+    mx = warp_max(mx);
+    if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(mx));
+  }
+  for (int i = g.tid; i < kBitmapChunks / 32; i += g.nt) bits[i] = 0u;
+  g.sync();
+  const double delta = 1e-3 * fabs(tau) + 1e-6 * fmax((double)ms->fmax, fabs(tau)) + 1e-30;
   const double hi = tau + delta, lo = tau - delta;
   if (sampled && (double)t0 > lo) return false;   // the window may reach below the filter
-  if (g.tid == 0) { ms->lo = m; ms->hi = -1; }
-  g.sync();
+  // classify: clearly in -> bitmap; window -> list (chunk ids in wl, positions in ckey)
+  int* wl = reinterpret_cast<int*>(ms->wl);
   for (int i = g.tid; i < m; i += g.nt) {
     const double x = (double)ckey[i];
-    if (x <= hi) atomicMin(&ms->lo, i);
-    if (x >= lo) atomicMax(&ms->hi, i);
+    if (x > hi) {
+      atomicOr(&bits[cid[i] >> 5], 1u << (cid[i] & 31));
+      atomicAdd(&ms->lo, 1);
+    } else if (x >= lo) {
+      const int pos = atomicAdd(&ms->cnt, 1);
+      if (pos < kWindowCap) wl[pos] = cid[i];
+    }
   }
   g.sync();
-  const int p_lo = ms->lo, p_hi = ms->hi, need = k - p_lo, w = p_hi - p_lo + 1;
+  const int n_in = ms->lo, w = ms->cnt, need = k - n_in;
+  if (w > kWindowCap) return false;
   const int b = p / dm.H, h = p % dm.H;
-  const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
   const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
   double* s64 = a.cand_s64 + (size_t)p * Nc;
-  for (int i = g.tid; i < w; i += g.nt) s64[i] = score64<T, D, G>(L + (size_t)cid[p_lo + i] * D, qb);
-  for (int i = g.tid; i < p_lo; i += g.nt) outs[i] = cid[i];
+  for (int i = g.tid; i < w; i += g.nt) s64[i] = score64_row<T, D, G>(L + (size_t)wl[i] * D, sQ);
+  (void)b;
+  (void)h;
   g.sync();
   for (int i = g.tid; i < w; i += g.nt) {
     const double si = s64[i];
-    const int ii = cid[p_lo + i];
+    const int ii = wl[i];
     int rank = 0;
-    for (int j = 0; j < w; ++j) {
-      const double sj = s64[j];
-      rank += (sj > si) || (sj == si && cid[p_lo + j] < ii);
+    for (int j2 = 0; j2 < w; ++j2) {
+      const double sj = s64[j2];
+      rank += (sj > si) || (sj == si && wl[j2] < ii);
     }
-    if (rank < need) outs[p_lo + rank] = ii;
+    if (rank < need) atomicOr(&bits[ii >> 5], 1u << (ii & 31));
   }
   g.sync();
-  const int nk = next_pow2(k);
-  for (int i = k + g.tid; i < nk; i += g.nt) outs[i] = 0x7fffffff;
-  g.sync();
-  group_sort_int_asc(g, outs, nk);
+  // ascending output: exclusive scan of the per-word bit counts
   int32_t* sel = a.sel + (size_t)p * k;
-  for (int i = g.tid; i < k; i += g.nt) sel[i] = outs[i];
+  const int nw = (Nc + 31) / 32;
+  int base = 0;
+  for (int w0 = 0; w0 < nw; w0 += g.nt) {
+    const int wi = w0 + g.tid;
+    const uint32_t word = wi < nw ? bits[wi] : 0u;
+    int total;
+    int pos = base + group_exclusive_scan(g, __popc(word), ms->iscr, &total);
+    uint32_t rem = word;
+    while (rem) {
+      const int bit = __ffs(rem) - 1;
+      rem &= rem - 1;
+      if (pos < k) sel[pos] = wi * 32 + bit;
+      ++pos;
+    }
+    base += total;
+  }
   return true;
 }
 
 template <typename T, int D, int G>
-__device__ void select_pair(const Grp& g, const SelectArgs& a, int p, float* ckey, int* cid,
-                            int* outs, Misc* ms) {
+__device__ void select_pair(const Grp& g, const SelectArgs& a, int p, const float* sQ,
+                            float* ckey, int* cid, uint32_t* bits, Misc* ms) {
   const int Nc = a.dm.Nc, k = a.dm.k;
   if (k >= Nc) {
     int32_t* sel = a.sel + (size_t)p * k;
     for (int i = g.tid; i < Nc; i += g.nt) sel[i] = i;
     return;
   }
-  const bool done = select_pair_fast<T, D, G>(g, a, p, ckey, cid, outs, ms);
+  const bool done = select_pair_fast<T, D, G>(g, a, p, sQ, ckey, cid, bits, ms);
   g.sync();
   if (!done) select_pair_radix<T, D, G>(g, a, p, ms);
 }
@@ -324,7 +404,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
   float* sQ = reinterpret_cast<float*>(gbase + L.q);
   float* ckey = reinterpret_cast<float*>(gbase + L.ckey);
   int* cidv = reinterpret_cast<int*>(gbase + L.cid);
-  int* outs = reinterpret_cast<int*>(gbase + L.outs);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(gbase + L.outs);
   Misc* ms = reinterpret_cast<Misc*>(gbase + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.bar + 8 * 2 * kStages);
   auto full = [&](int s) { return base + L.bar + 8u * (uint32_t)s; };
@@ -388,7 +468,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       g.sync();
       if (ms->last) {
         __threadfence();
-        select_pair<T, D, G>(g, a, pair, ckey, cidv, outs, ms);
+        select_pair<T, D, G>(g, a, pair, sQ, ckey, cidv, bits, ms);
         g.sync();
         if (tid == 0) a.counters[pair] = 0;
       }
