@@ -21,8 +21,9 @@
  *     cfg->dtype (fp32 or bf16); index arrays are int32. Arithmetic is fp32 with fp64
  *     used to settle selections near their threshold.
  *   - The caller owns every buffer (inputs, cache, outputs, workspace). The context owns
- *     only small tables (RoPE cos/sin, a status word, completion counters). Calls
- *     allocate nothing.
+ *     small tables (RoPE cos/sin, a status word, work counters) and the landmark scores
+ *     of one decode step (B*H_kv*N_c floats: 4 MiB at batch 8, 8 KV heads, 128K tokens,
+ *     chunk 8), which it keeps in a reset state between calls. Calls allocate nothing.
  *   - Calls are asynchronous on the given stream (a cudaStream_t passed as void*; NULL =
  *     the legacy default stream). Arguments are validated on the host first; on any
  *     error nothing is launched and the status says why.

@@ -115,6 +115,22 @@ __device__ __forceinline__ float act_fast(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
 
+// Polls *flag until it is non-zero, with acquire semantics (bounded: 2 s, or *abort set;
+// on giving up sets *abort and returns 0).
+__device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0) return 1;
+    if (*abort) return 0;
+    if (global_timer_ns() - t0 > 2000000000ull) break;
+    __nanosleep(256);
+  }
+  *abort = 1;
+  return 0;
+}
+
 template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int cta_per_head) {
@@ -238,10 +254,15 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     auto load_cid = [&](int i) -> int {
       int b, tile;
       item_of(i, b, tile);
+      if (a.wait_ready) {   // the selection kernel may still be running: wait for this pair
+        int ok = 1;
+        if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) return -1;
+      }
       int cid = -1;
       if (lane < kChunksPerTile) {
         const int gs = tile * kChunksPerTile + lane;
-        if (gs < dm.k) cid = sel_all[((size_t)b * dm.H + h) * dm.k + gs];
+        if (gs < dm.k) cid = __ldcg(sel_all + ((size_t)b * dm.H + h) * dm.k + gs);
       }
       return cid;
     };
@@ -765,17 +786,24 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   if (cph < 1) cph = 1;
   if (cph > n_items) cph = n_items;
   cudaError_t e;
-  if (dm.act == LOWRAM_ACT_SILU) {
-    auto kern = attend_tc_kernel<LOWRAM_ACT_SILU>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)L.total)) != cudaSuccess) return e;
-    kern<<<dm.H * cph, kThreads, L.total, s>>>(a, maps, cph);
-  } else {
-    auto kern = attend_tc_kernel<LOWRAM_ACT_GELU_ERF>;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)L.total)) != cudaSuccess) return e;
-    kern<<<dm.H * cph, kThreads, L.total, s>>>(a, maps, cph);
-  }
+  auto kern = dm.act == LOWRAM_ACT_SILU ? attend_tc_kernel<LOWRAM_ACT_SILU>
+                                        : attend_tc_kernel<LOWRAM_ACT_GELU_ERF>;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)L.total)) != cudaSuccess) return e;
+  // after the selection kernel: a programmatic dependent launch, so CTAs start on SMs
+  // the selection kernel has left and overlap its last selections
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(dm.H * cph);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.wait_ready ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, a, maps, cph);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

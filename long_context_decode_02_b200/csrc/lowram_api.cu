@@ -23,7 +23,9 @@ struct lowram_ctx {
   double2* hi64;
   int n_hi;
   int* status;    // device word
-  int* counters;  // device [B*H]
+  int* counters;  // device [4]: the selection kernel's work, exit and pair counters
+  float* scores;  // device [B*H][Nc], the sentinel 0xFFFFFFFF between launches
+  int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   double* theta64;  // device [d/2]
 };
 
@@ -86,7 +88,7 @@ struct DeviceGuard {
 };
 
 struct DecodeWs {
-  size_t scores, cand_s64, cand_idx, flags, sel, part, total;
+  size_t cand_s64, cand_idx, flags, sel, part, total;
 };
 DecodeWs decode_ws(const lowram_config& c) {
   const Dims d = dims_of(c);
@@ -96,7 +98,6 @@ DecodeWs decode_ws(const lowram_config& c) {
                                        : attend_simt_part_floats(d, nt);
   DecodeWs w{};
   size_t o = 0;
-  w.scores = o;   o = align_up(o + pairs * d.Nc * sizeof(float));
   w.cand_s64 = o; o = align_up(o + pairs * d.Nc * sizeof(double));
   w.cand_idx = o; o = align_up(o + pairs * d.Nc * sizeof(int));
   w.flags = o;    o = align_up(o + pairs * d.Nc);
@@ -181,6 +182,8 @@ lowram_status lowram_check_config(const lowram_config* c) {
   if (!pow2_in(c->n_q_heads / c->n_kv_heads, 1, 8)) return LOWRAM_ERR_UNSUPPORTED;
   if (c->n_tokens % 16 != 0 || c->n_tokens > (1 << 24)) return LOWRAM_ERR_UNSUPPORTED;
   if (c->n_kv_heads * c->head_dim > 2048) return LOWRAM_ERR_UNSUPPORTED;
+  if ((size_t)c->batch * c->n_kv_heads * (size_t)(c->n_tokens / c->chunk) > ((size_t)1 << 30))
+    return LOWRAM_ERR_UNSUPPORTED;   // landmark rows of one call, indexed in 32 bits
   if (c->decode_variant == LOWRAM_DECODE_TCGEN05 && !attend_tc_supported(dims_of(*c)))
     return LOWRAM_ERR_UNSUPPORTED;
   return LOWRAM_OK;
@@ -251,7 +254,9 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->lo64, lo64.size() * sizeof(double2)) == cudaSuccess &&
             cudaMalloc(&ctx->hi64, hi64.size() * sizeof(double2)) == cudaSuccess &&
             cudaMalloc(&ctx->status, sizeof(int)) == cudaSuccess &&
-            cudaMalloc(&ctx->counters, pairs * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
   ok = ok &&
        cudaMemcpy(ctx->lo32, lo32.data(), lo32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -259,7 +264,9 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemcpy(ctx->lo64, lo64.data(), lo64.size() * sizeof(double2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->hi64, hi64.data(), hi64.size() * sizeof(double2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemset(ctx->status, 0, sizeof(int)) == cudaSuccess &&
-       cudaMemset(ctx->counters, 0, pairs * sizeof(int)) == cudaSuccess &&
+       cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
+       cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
+       cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -279,6 +286,8 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->hi64);
   cudaFree(ctx->status);
   cudaFree(ctx->counters);
+  cudaFree(ctx->scores);
+  cudaFree(ctx->ready);
   cudaFree(ctx->theta64);
   delete ctx;
 }
@@ -322,18 +331,19 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
 namespace {
 
 lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, int32_t* sel,
-                          uint8_t* ws, const DecodeWs& w, cudaStream_t s) {
+                          uint8_t* ws, const DecodeWs& w, cudaStream_t s, bool set_ready) {
   const Dims dm = dims_of(ctx->cfg);
   SelectArgs sa{};
   sa.dm = dm;
   sa.landmark = landmark;
   sa.q = q;
-  sa.scores = reinterpret_cast<float*>(ws + w.scores);
+  sa.scores = ctx->scores;
   sa.cand_s64 = reinterpret_cast<double*>(ws + w.cand_s64);
   sa.cand_idx = reinterpret_cast<int*>(ws + w.cand_idx);
   sa.flags = ws + w.flags;
   sa.counters = ctx->counters;
   sa.sel = sel;
+  sa.ready = set_ready ? ctx->ready : nullptr;
   sa.status = ctx->status;
   if (launch_select(sa, ctx->num_sms, s) != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;
@@ -341,7 +351,8 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, 
 
 lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
                           const lowram_layer_params* params, const void* q, const int32_t* sel,
-                          void* out, uint8_t* ws, const DecodeWs& w, cudaStream_t s) {
+                          void* out, uint8_t* ws, const DecodeWs& w, cudaStream_t s,
+                          bool after_select) {
   const lowram_config& c = ctx->cfg;
   const Dims dm = dims_of(c);
   AttendArgs aa{};
@@ -360,6 +371,9 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   aa.n_tiles = n_tiles_of(c);
   const bool tc = use_tc(c);
   aa.tile_tokens = tc ? kTcTileTokens : attend_simt_tile_tokens(dm);
+  // right after the selection kernel the tcgen05 kernel overlaps its tail, pair by pair
+  aa.ready = tc && after_select ? ctx->ready : nullptr;
+  aa.wait_ready = aa.ready ? 1 : 0;
   cudaError_t e = tc ? launch_attend_tc(aa, ctx->num_sms, s) : launch_attend_simt(aa, s);
   if (e == cudaSuccess) e = launch_combine(aa, tc, s);
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
@@ -381,7 +395,7 @@ lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark, const 
   DeviceGuard g(ctx->device);
   if (!g.ok) return LOWRAM_ERR_CUDA;
   return select_impl(ctx, landmark, q, sel_out, static_cast<uint8_t*>(workspace), w,
-                     static_cast<cudaStream_t>(stream));
+                     static_cast<cudaStream_t>(stream), false);
 }
 
 lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
@@ -399,7 +413,7 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
   DeviceGuard g(ctx->device);
   if (!g.ok) return LOWRAM_ERR_CUDA;
   return attend_impl(ctx, cache, params, q, sel, out, static_cast<uint8_t*>(workspace), w,
-                     static_cast<cudaStream_t>(stream));
+                     static_cast<cudaStream_t>(stream), false);
 }
 
 lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
@@ -420,8 +434,9 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + w.sel);
-  if ((st = select_impl(ctx, cache->landmark, q, sel, ws, w, s)) != LOWRAM_OK) return st;
-  return attend_impl(ctx, cache, params, q, sel, out, ws, w, s);
+  const bool tc = use_tc(ctx->cfg);
+  if ((st = select_impl(ctx, cache->landmark, q, sel, ws, w, s, tc)) != LOWRAM_OK) return st;
+  return attend_impl(ctx, cache, params, q, sel, out, ws, w, s, tc);
 }
 
 lowram_status lowram_last_error(lowram_ctx* ctx) {

@@ -43,12 +43,13 @@ struct SelectArgs {
   Dims dm;
   const void* landmark;   // [B][H][Nc][d]
   const void* q;          // [B][Hq][d]
-  float* scores;          // ws [B*H][Nc]
+  float* scores;          // ctx [B*H][Nc], the sentinel 0xFFFFFFFF between launches
   double* cand_s64;       // ws [B*H][Nc]
   int* cand_idx;          // ws [B*H][Nc]
   uint8_t* flags;         // ws [B*H][Nc]
-  int* counters;          // ctx [B*H], zero between launches
+  int* counters;          // ctx [4]: work, exit and pair counters, zero between launches
   int32_t* sel;           // [B*H][k]
+  int* ready;             // ctx [B*H] or null: set to 1 once a pair's selection is written
   int* status;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
@@ -70,6 +71,9 @@ struct AttendArgs {
   int* status;
   int n_tiles;            // tiles per (b, h)
   int tile_tokens;
+  int* ready;             // ctx [B*H] or null: per-pair selection flags; combine clears them
+  int wait_ready;         // 1: launched as a programmatic dependent of the selection
+                          // kernel; wait for ready[pair] before reading its selection
 };
 size_t attend_simt_part_floats(const Dims& dm, int n_tiles);
 int attend_simt_tile_tokens(const Dims& dm);

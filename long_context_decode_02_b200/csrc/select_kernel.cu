@@ -7,20 +7,29 @@
 // group's query heads of q . L_c; ties go to the lower chunk index.
 //
 // Structure (HBM-bound: every landmark byte is read once, ~4 FLOP per byte):
-//  * Persistent CTAs (one per SM) split the stream of all (batch, KV head) landmark rows
-//    into contiguous ranges of stages. A producer warp TMA-loads 64 KB stages (the rows
-//    of one (b, h)) into a 3-stage shared-memory ring with the 128-byte swizzle; 256
-//    consumer threads each score one landmark row of a stage (packed fp32x2 FMAs against
-//    the queries held in shared memory) and write the fp32 score. The swizzle makes the
-//    row-per-thread 16-byte reads conflict-free.
-//  * The CTA that completes the last stage of a (b, h) (atomic stage counter, no
-//    spinning) selects on its consumer warps while its producer keeps streaming:
-//    a sorted sample places a threshold, candidates above it are sorted, tau = k-th
-//    score, candidates within delta = 1e-3|tau| + 1e-6 max|s| of tau are re-scored in
-//    fp64 (exact products, fp64 sums) and ranked by (score desc, index asc). delta is far
-//    above the fp32 accumulation error, so the result equals the fp64 selection. When the
-//    candidate set cannot be proven to contain the answer, a radix-select path over all
-//    scores decides instead. The selection is written in ascending chunk order.
+//  * Persistent CTAs (one per SM) take 64 KB stages (up to 256 landmark rows of one
+//    (b, h)) from a global work counter in (b, h)-major order, so the load balances
+//    itself and the (b, h) pairs are completed one after another while the stream runs.
+//    A producer warp TMA-loads each stage into a 3-stage shared-memory ring (128-byte
+//    swizzle) and stages the pair's queries in fp32 beside it; 256 consumer threads
+//    score one row each (packed fp32x2 FMAs) and write the fp32 score.
+//  * Scores live in a context-owned buffer that holds a sentinel bit pattern between
+//    launches (0xFFFFFFFF, a NaN that fp32 arithmetic never produces), so a written score
+//    is its own completion flag: no counters or memory fences on the streaming path.
+//    Three selection warps per CTA take (b, h) pairs in order from a global counter,
+//    wait until the work counter has handed out all of the pair's stages and every score
+//    has landed, select, and put the sentinel back. Selections are spread over the CTAs
+//    and overlap the stream; a selection group only waits for stages held by running
+//    CTAs, and every wait is bounded.
+//  * Selection: the 16-bit key prefix of the j-th largest of 1024 evenly spaced scores
+//    gives a threshold t0; every score >= t0 is a candidate; three radix passes find the
+//    24-bit prefix bucket [tau_lo, tau_hi] holding the k-th largest candidate.
+//    Candidates above tau_hi + delta are in; those in [tau_lo - delta, tau_hi + delta]
+//    are re-scored in fp64 (exact products, fp64 sums) and ranked by (score desc, index
+//    asc). delta = 1e-3|tau| + 1e-6 max|s| is far above the fp32 accumulation error, so
+//    the result equals the selection made in fp64. When the candidate set cannot be
+//    proven to hold the answer, a radix select over all scores decides instead. The
+//    chunk ids are written in ascending order.
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
@@ -32,13 +41,17 @@ namespace {
 using namespace sm100;
 
 constexpr int kConsumers = 256;               // consumer threads (warps 0..7)
-constexpr int kSelThreads = kConsumers + 32;  // + producer warp 8
+constexpr int kSelectors = 96;                // selection threads (warps 9..11)
+constexpr int kSelThreads = kConsumers + 32 + kSelectors;  // + producer warp 8
 constexpr int kStages = 3;
 constexpr int kStageBytes = 65536;
-constexpr int kCap = 2048;                    // candidate capacity of the fast selection
-constexpr int kSample = 1024;                 // sampled scores placing its threshold
+constexpr int kSample = 1024;                 // sampled scores placing the threshold t0
 constexpr int kBitmapChunks = 65536;          // chunks the fast path's output bitmap covers
 constexpr int kWindowCap = 256;               // fp64 re-scored candidates of the fast path
+constexpr int kSmemLimit = 232448;            // opt-in shared memory per block
+
+// Candidate capacity of the fast selection: smaller when the per-stage queries are large.
+__host__ __device__ constexpr int cand_cap(int G, int D) { return G * D <= 512 ? 2048 : 1280; }
 
 template <typename T, int D>
 struct Geom {
@@ -50,32 +63,143 @@ struct Geom {
   static constexpr int kChunks = kRowBytes / 16;
 };
 
-struct SelSmem {  // offsets from the 1024-aligned dynamic base
-  uint32_t stages, q, ckey, cid, outs, misc, bar, total;
-};
-__host__ __device__ inline SelSmem sel_smem(int G, int D) {
-  SelSmem L{};
-  L.stages = 0;
-  L.q = kStages * kStageBytes;
-  L.ckey = L.q + (uint32_t)(G * D * 4);
-  L.cid = L.ckey + kCap * 4;
-  L.outs = L.cid + kCap * 4;            // chunk bitmap of the fast path
-  L.misc = L.outs + kBitmapChunks / 8;   // scalars, reduction scratch, window list
-  L.bar = L.misc + 3072;
-  L.total = L.bar + 128 + 1024;
-  return L;
-}
 
 struct Misc {
-  unsigned hist[256];
+  unsigned hist[512];   // two radix histograms
   unsigned bc[4];
   float fscr[33];
   int iscr[33];
-  int cnt, lo, hi, last;
-  float t0, fmax;
+  int cnt, n_in, nwin;
+  float fmax;
+  int req;              // the selection warps' current request
   int wl[kWindowCap];
 };
-static_assert(sizeof(Misc) <= 3072, "Misc scratch");
+
+struct SelSmem {  // offsets from the 1024-aligned dynamic base
+  uint32_t stages, q, ckey, cid, outs, misc, hdr, bar, total;
+};
+__host__ __device__ inline SelSmem sel_smem(int G, int D) {
+  SelSmem L{};
+  const int cap = cand_cap(G, D);
+  L.stages = 0;
+  L.q = kStages * kStageBytes;                          // fp32 queries per stage
+  L.ckey = L.q + (uint32_t)(kStages * G * D * 4);
+  L.cid = L.ckey + cap * 4;
+  L.outs = L.cid + cap * 4;                              // chunk bitmap of the fast path
+  L.misc = L.outs + kBitmapChunks / 8;
+  L.hdr = L.misc + (uint32_t)((sizeof(Misc) + 15) & ~(size_t)15);   // stage units
+  L.bar = L.hdr + 64;       // full[], empty[], abort word
+  L.total = L.bar + 64 + 1024;
+  return L;
+}
+static_assert(kStages * 4 <= 64 && 2 * kStages * 8 + 4 <= 64, "stage units and barriers");
+
+constexpr uint32_t kScoreEmpty = 0xFFFFFFFFu;   // sentinel of an unwritten score
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 ld_relaxed4(const uint32_t* p) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
+  return v;
+}
+
+// Polls *p until it reaches target (bounded: 2 s, or *abort set; on giving up sets *abort).
+__device__ bool wait_counter_ge(const int* p, int target, volatile int* abort) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if ((int)ld_relaxed(reinterpret_cast<const uint32_t*>(p)) >= target) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 2000000000ull) break;
+    __nanosleep(500);
+  }
+  *abort = 1;
+  return false;
+}
+
+// Waits until none of the n scores at sp holds the sentinel (this thread's share of the
+// group; bounded like wait_counter_ge). Returns false on giving up.
+__device__ bool wait_scores(const Grp& g, const uint32_t* sp, int n, volatile int* abort) {
+  const uint64_t t0 = global_timer_ns();
+  const bool vec = (reinterpret_cast<uintptr_t>(sp) & 15) == 0;
+  for (int i = 4 * g.tid; i < n; i += 4 * g.nt) {
+    for (;;) {
+      bool done;
+      if (vec && i + 4 <= n) {
+        const uint4 v = ld_relaxed4(sp + i);
+        done = v.x != kScoreEmpty && v.y != kScoreEmpty && v.z != kScoreEmpty && v.w != kScoreEmpty;
+      } else {
+        done = true;
+        for (int e = i; e < n && e < i + 4; ++e) done = done && ld_relaxed(sp + e) != kScoreEmpty;
+      }
+      if (done) break;
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > 2000000000ull) { *abort = 1; return false; }
+      __nanosleep(200);
+    }
+  }
+  return true;
+}
+
+// Puts the sentinel back into n scores (this thread's share).
+__device__ void clear_scores(const Grp& g, uint32_t* sp, int n) {
+  const bool vec = (reinterpret_cast<uintptr_t>(sp) & 15) == 0;
+  for (int i = 4 * g.tid; i < n; i += 4 * g.nt) {
+    if (vec && i + 4 <= n)
+      *reinterpret_cast<uint4*>(sp + i) = make_uint4(kScoreEmpty, kScoreEmpty, kScoreEmpty, kScoreEmpty);
+    else
+      for (int e = i; e < n && e < i + 4; ++e) sp[e] = kScoreEmpty;
+  }
+}
+
+// Loads the kN words su[idx[j]] for the bits j of want, polling until none holds the
+// sentinel; returns false if the wait gave up (2 s since t0, or *abort set).
+template <int kN>
+__device__ bool poll_words(const uint32_t* su, const int (&idx)[kN], uint32_t want,
+                           uint32_t (&v)[kN], volatile int* abort, uint64_t t0) {
+  while (want) {
+#pragma unroll
+    for (int j = 0; j < kN; ++j)
+      if ((want >> j) & 1u) v[j] = ld_relaxed(su + idx[j]);
+#pragma unroll
+    for (int j = 0; j < kN; ++j)
+      if (((want >> j) & 1u) && v[j] != kScoreEmpty) want &= ~(1u << j);
+    if (!want) break;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 2000000000ull) { *abort = 1; return false; }
+    __nanosleep(200);
+  }
+  return true;
+}
+
+// The same for kN 16-byte groups su[4 idx[j] .. 4 idx[j] + 3].
+template <int kN>
+__device__ bool poll_vec4(const uint32_t* su, const int (&idx)[kN], uint32_t want,
+                          uint4 (&v)[kN], volatile int* abort, uint64_t t0) {
+  while (want) {
+#pragma unroll
+    for (int j = 0; j < kN; ++j)
+      if ((want >> j) & 1u) v[j] = ld_relaxed4(su + 4 * idx[j]);
+#pragma unroll
+    for (int j = 0; j < kN; ++j)
+      if (((want >> j) & 1u) && v[j].x != kScoreEmpty && v[j].y != kScoreEmpty &&
+          v[j].z != kScoreEmpty && v[j].w != kScoreEmpty)
+        want &= ~(1u << j);
+    if (!want) break;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > 2000000000ull) { *abort = 1; return false; }
+    __nanosleep(200);
+  }
+  return true;
+}
 
 template <typename T, int D, int G>
 __device__ double score64(const T* lrow, const T* qb) {
@@ -156,151 +280,285 @@ __device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc
   }
 }
 
-// fp64 score of one landmark row against the group's queries held (exactly, as fp32) in
-// shared memory: exact products, one fp64 accumulator per query head.
+// fp64 scores of window rows by one warp: lane l holds D/32 consecutive elements of
+// each row and of each query head; exact products, fp64 sums (lane-serial, then a
+// butterfly); lane 0's value is stored. The loads of up to 8 rows are issued together.
 template <typename T, int D, int G>
-__device__ double score64_row(const T* lrow, const float* sQ) {
-  constexpr int kV = 16 / (int)sizeof(T);
-  double acc[G];
+__device__ void score64_rows_warp(const T* Lp, const T* qb, const int* wl, int w, int first,
+                                  int stride, double* s64, int lane) {
+  constexpr int E = D / 32;
+  constexpr int kBatch = 8;
+  float qr[G][E];
 #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = 0.0;
-  const uint4* w4 = reinterpret_cast<const uint4*>(lrow);
-#pragma unroll 4
-  for (int c = 0; c < D / kV; ++c) {
-    const uint4 w = w4[c];
-    float v[kV];
-    if constexpr (sizeof(T) == 2) {
-      const float2 a0 = bf2_to_f2(w.x), a1 = bf2_to_f2(w.y), a2 = bf2_to_f2(w.z), a3 = bf2_to_f2(w.w);
-      v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y; v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
-    } else {
-      v[0] = __uint_as_float(w.x); v[1] = __uint_as_float(w.y);
-      v[2] = __uint_as_float(w.z); v[3] = __uint_as_float(w.w);
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qr[g][e] = ldf(qb, g * D + lane * E + e);
+  for (int r0 = first; r0 < w; r0 += stride * kBatch) {
+    float lv[kBatch][E];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = r0 + j * stride;
+      if (i < w) {
+        const T* row = Lp + (size_t)wl[i] * D;
+#pragma unroll
+        for (int e = 0; e < E; ++e) lv[j][e] = ldf(row, lane * E + e);
+      }
     }
 #pragma unroll
-    for (int e = 0; e < kV; ++e)
+    for (int j = 0; j < kBatch; ++j) {
+      const int i = r0 + j * stride;
+      if (i >= w) break;
+      double best = -INFINITY;
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = fma((double)sQ[g * D + c * kV + e], (double)v[e], acc[g]);
+      for (int g = 0; g < G; ++g) {
+        double acc = 0.0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc = fma((double)qr[g][e], (double)lv[j][e], acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        best = fmax(best, acc);
+      }
+      if (lane == 0) s64[i] = best;
+    }
   }
-  double best = acc[0];
-#pragma unroll
-  for (int g = 1; g < G; ++g) best = fmax(best, acc[g]);
-  return best;
 }
 
-// Fast path. Candidates: all scores (N_c <= kCap), or every score at or above a
-// threshold t0 = the j-th largest of an evenly spaced sample (radix select). tau = the
-// k-th largest candidate (radix select); candidates above tau + delta are in; the window
-// |s - tau| <= delta is re-scored in fp64 and ranked by (score desc, index asc); the k
-// chosen chunk ids are written ascending through a bitmap scan. Returns false (writing
-// nothing) when the candidate set cannot be proven to contain the answer.
+// The top 8 * kPasses bits of the k-th largest (1 <= k <= n) of n uint32 keys, by kPasses
+// 8-bit radix passes (most significant digit first); the lower bits are returned as
+// zero. Two histograms alternate: the one for pass p + 1 is cleared during pass p.
+template <int kPasses, typename KeyFn>
+__device__ uint32_t kth_largest_prefix(const Grp& g, int n, int k, KeyFn key_of, Misc* ms) {
+  const int lane = g.tid & 31;
+  for (int i = g.tid; i < 512; i += g.nt) ms->hist[i] = 0u;
+  g.sync();
+  uint32_t prefix = 0, mask = 0;
+  unsigned remaining = (unsigned)k;
+#pragma unroll
+  for (int pass = 0; pass < kPasses; ++pass) {
+    const int shift = 24 - 8 * pass;
+    unsigned* hist = ms->hist + 256 * (pass & 1);
+    if (pass >= 1 && pass + 1 < kPasses)
+      for (int i = g.tid; i < 256; i += g.nt) ms->hist[256 * ((pass + 1) & 1) + i] = 0u;
+    for (int base = 0; base < n; base += g.nt) {
+      const int i = base + g.tid;
+      unsigned digit = 256u;
+      if (i < n) {
+        const uint32_t key = key_of(i);
+        if ((key & mask) == prefix) digit = (key >> shift) & 255u;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+    }
+    g.sync();
+    if (g.tid < 32) {
+      unsigned own = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) own += hist[255 - 8 * lane - j];
+      unsigned incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const unsigned before = incl - own;
+      if (before < remaining && incl >= remaining) {
+        unsigned acc = before;
+        for (int j = 0; j < 8; ++j) {
+          const int dg = 255 - 8 * lane - j;
+          const unsigned c = hist[dg];
+          if (acc + c >= remaining) { ms->bc[2 * (pass & 1)] = (unsigned)dg; ms->bc[2 * (pass & 1) + 1] = remaining - acc; break; }
+          acc += c;
+        }
+      }
+    }
+    g.sync();
+    prefix |= ms->bc[2 * (pass & 1)] << shift;
+    mask |= 255u << shift;
+    remaining = ms->bc[2 * (pass & 1) + 1];
+  }
+  return prefix;
+}
+
+// Fast path (see the file comment); needs k <= cap/2 and N_c <= kBitmapChunks. Reads each
+// score through a poll that waits out the sentinel, so it needs no separate wait for the
+// pair. Expects ms->cnt, n_in, nwin and fmax at zero. Returns 1 when done; 0, having
+// written no output, when the candidate set cannot be proven to hold the answer (every
+// score has been seen by then); -1 when a wait gave up.
 template <typename T, int D, int G>
-__device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, const float* sQ,
-                                 float* ckey, int* cid, uint32_t* bits, Misc* ms) {
+__device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float* ckey,
+                                int* cid, uint32_t* bits, Misc* ms, volatile int* abort) {
+  constexpr int kCap = cand_cap(G, D);
+  constexpr int kB = 8;   // independent loads in flight per thread
   const Dims& dm = a.dm;
   const int Nc = dm.Nc, k = dm.k;
   const int lane = g.tid & 31;
-  if (k > kCap / 2 || Nc > kBitmapChunks) return false;
-  const float* s = a.scores + (size_t)p * Nc;
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + (size_t)p * Nc);
+  const uint64_t t_start = global_timer_ns();
+  const int nw = (Nc + 31) >> 5;
+  for (int i = g.tid; i < nw; i += g.nt) bits[i] = 0u;
+  bool good = true;
   int m;
   float t0 = -INFINITY;
   const bool sampled = Nc > kCap;
   if (!sampled) {
-    for (int i = g.tid; i < Nc; i += g.nt) { ckey[i] = __ldcg(s + i); cid[i] = i; }
-    m = Nc;
+    float mx = 0.f;
+    for (int base = 0; base < Nc; base += kB * g.nt) {
+      int idx[kB];
+      uint32_t want = 0, v[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        idx[j] = base + j * g.nt + g.tid;
+        if (idx[j] < Nc) want |= 1u << j;
+      }
+      good = good && poll_words<kB>(su, idx, want, v, abort, t_start);
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+        if ((want >> j) & 1u) {
+          const float x = __uint_as_float(v[j]);
+          ckey[idx[j]] = x;
+          cid[idx[j]] = idx[j];
+          mx = fmaxf(mx, fabsf(x));
+        }
+    }
+    mx = warp_max(mx);
+    if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(mx));
+    if (!good) ms->cnt = -1;
     g.sync();
+    if (ms->cnt < 0) return -1;
+    m = Nc;
   } else {
     uint32_t* skey = reinterpret_cast<uint32_t*>(cid);
-    for (int i = g.tid; i < kSample; i += g.nt)
-      skey[i] = f2key(__ldcg(s + (int)(((long long)i * Nc) / kSample)));
+    for (int base = 0; base < kSample; base += kB * g.nt) {
+      int idx[kB];
+      uint32_t want = 0, v[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const int i = base + j * g.nt + g.tid;
+        idx[j] = (int)(((long long)i * Nc) / kSample);
+        if (i < kSample) want |= 1u << j;
+      }
+      good = good && poll_words<kB>(su, idx, want, v, abort, t_start);
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+        if ((want >> j) & 1u) skey[base + j * g.nt + g.tid] = f2key(__uint_as_float(v[j]));
+    }
+    if (!good) ms->cnt = -1;
     g.sync();
+    if (ms->cnt < 0) return -1;
     int j = (int)((3LL * k * kSample) / (2LL * Nc)) + 16;
     if (j > kSample) j = kSample;
-    t0 = key2f(group_kth_largest_aggr(g, kSample, j, [&](int i) { return skey[i]; },
-                                      ms->hist, ms->bc));
-    if (g.tid == 0) ms->cnt = 0;
-    g.sync();
-    // every score >= t0 becomes a candidate (warp-aggregated append); each thread issues
-    // 8 independent 16-byte loads before filtering them (rows are 16-byte aligned when
-    // 4 | N_c; otherwise scalar loads)
-    const int n4 = (Nc & 3) == 0 ? Nc / 4 : 0;
-    if (n4 == 0) {
-      for (int i = g.tid; i < Nc; i += g.nt) {
-        const float x = __ldcg(s + i);
-        if (x >= t0) {
-          const int pos = atomicAdd(&ms->cnt, 1);
-          if (pos < kCap) { ckey[pos] = x; cid[pos] = i; }
-        }
-      }
-    }
-    const float4* s4 = reinterpret_cast<const float4*>(s);
-    for (int base = 0; base < n4; base += 8 * g.nt) {
-      float4 v[8];
+    t0 = key2f(kth_largest_prefix<2>(g, kSample, j, [&](int i) { return skey[i]; }, ms));
+    // every score >= t0 becomes a candidate: each thread filters 32 scores from 8
+    // independent 16-byte loads, then one warp scan and one shared atomic per warp place
+    // them (16-byte groups when 4 | N_c and the row is 16-byte aligned; else single words)
+    float mx = 0.f;
+    const bool vec = (Nc & 3) == 0 && (reinterpret_cast<uintptr_t>(su) & 15) == 0;
+    const int n4 = vec ? Nc / 4 : (Nc + 3) / 4;
+    for (int base = 0; base < n4; base += kB * g.nt) {
+      int idx[kB];
+      uint32_t want = 0;
+      uint4 v[kB];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i4 = base + u * g.nt + g.tid;
-        v[u] = i4 < n4 ? __ldcg(s4 + i4) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      for (int j = 0; j < kB; ++j) {
+        idx[j] = base + j * g.nt + g.tid;
+        if (idx[j] < n4) want |= 1u << j;
       }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i4 = base + u * g.nt + g.tid;
-        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      if (vec) {
+        good = good && poll_vec4<kB>(su, idx, want, v, abort, t_start);
+      } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 4 * i4 + e;
-          const bool keep = i < Nc && xs[e] >= t0;
-          const unsigned bal = __ballot_sync(0xffffffffu, keep);
-          if (bal == 0) continue;
-          int wb = 0;
-          if (lane == 0) wb = atomicAdd(&ms->cnt, __popc(bal));
-          wb = __shfl_sync(0xffffffffu, wb, 0);
-          if (keep) {
-            const int pos = wb + __popc(bal & ((1u << lane) - 1u));
-            if (pos < kCap) { ckey[pos] = xs[e]; cid[pos] = i; }
+          int ie[kB];
+          uint32_t we = 0, ve[kB];
+#pragma unroll
+          for (int j = 0; j < kB; ++j) {
+            ie[j] = 4 * idx[j] + e;
+            if (((want >> j) & 1u) && ie[j] < Nc) we |= 1u << j;
+          }
+          good = good && poll_words<kB>(su, ie, we, ve, abort, t_start);
+#pragma unroll
+          for (int j = 0; j < kB; ++j) {
+            const uint32_t x = ((we >> j) & 1u) ? ve[j] : __float_as_uint(-INFINITY);
+            if (e == 0) v[j].x = x; else if (e == 1) v[j].y = x; else if (e == 2) v[j].z = x; else v[j].w = x;
+          }
+        }
+      }
+      uint32_t keep = 0;
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        if (!((want >> j) & 1u)) continue;
+        keep |= (__uint_as_float(v[j].x) >= t0 ? 1u : 0u) << (4 * j);
+        keep |= (__uint_as_float(v[j].y) >= t0 ? 1u : 0u) << (4 * j + 1);
+        keep |= (__uint_as_float(v[j].z) >= t0 ? 1u : 0u) << (4 * j + 2);
+        keep |= (__uint_as_float(v[j].w) >= t0 ? 1u : 0u) << (4 * j + 3);
+      }
+      const int c = __popc(keep);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int wb = 0;
+      if (lane == 31 && incl > 0) wb = atomicAdd(&ms->cnt, incl);
+      wb = __shfl_sync(0xffffffffu, wb, 31);
+      if (keep == 0) continue;
+      int pos = wb + incl - c;
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        const float xs[4] = {__uint_as_float(v[j].x), __uint_as_float(v[j].y),
+                             __uint_as_float(v[j].z), __uint_as_float(v[j].w)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((keep >> (4 * j + e)) & 1u) {
+            if (pos < kCap) { ckey[pos] = xs[e]; cid[pos] = 4 * idx[j] + e; }
+            ++pos;
+            mx = fmaxf(mx, fabsf(xs[e]));
           }
         }
       }
     }
-    g.sync();
-    m = ms->cnt;
-    if (m > kCap || m < k) return false;
-  }
-  const double tau = (double)key2f(group_kth_largest_aggr(
-      g, m, k, [&](int i) { return f2key(ckey[i]); }, ms->hist, ms->bc));
-  if (g.tid == 0) { ms->cnt = 0; ms->lo = 0; ms->fmax = 0.f; }
-  g.sync();
-  // |largest candidate| for the window floor
-  {
-    float mx = 0.f;
-    for (int i = g.tid; i < m; i += g.nt) mx = fmaxf(mx, fabsf(ckey[i]));
     mx = warp_max(mx);
     if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(mx));
+    if (!good) ms->n_in = -1;
+    g.sync();
+    if (ms->n_in < 0) return -1;
+    m = ms->cnt;
+    if (m > kCap || m < k) return 0;
   }
-  for (int i = g.tid; i < kBitmapChunks / 32; i += g.nt) bits[i] = 0u;
-  g.sync();
-  const double delta = 1e-3 * fabs(tau) + 1e-6 * fmax((double)ms->fmax, fabs(tau)) + 1e-30;
-  const double hi = tau + delta, lo = tau - delta;
-  if (sampled && (double)t0 > lo) return false;   // the window may reach below the filter
-  // classify: clearly in -> bitmap; window -> list (chunk ids in wl, positions in ckey)
-  int* wl = reinterpret_cast<int*>(ms->wl);
-  for (int i = g.tid; i < m; i += g.nt) {
-    const double x = (double)ckey[i];
-    if (x > hi) {
-      atomicOr(&bits[cid[i] >> 5], 1u << (cid[i] & 31));
-      atomicAdd(&ms->lo, 1);
-    } else if (x >= lo) {
-      const int pos = atomicAdd(&ms->cnt, 1);
-      if (pos < kWindowCap) wl[pos] = cid[i];
+  const uint32_t tp = kth_largest_prefix<3>(g, m, k, [&](int i) { return f2key(ckey[i]); }, ms);
+  const double tau_lo = (double)key2f(tp), tau_hi = (double)key2f(tp | 0xFFu);
+  if (!(tau_lo <= tau_hi)) return 0;   // a non-finite bucket
+  const double tmag = fmax(fabs(tau_lo), fabs(tau_hi));
+  const double delta = 1e-3 * tmag + 1e-6 * fmax((double)ms->fmax, tmag) + 1e-30;
+  const double hi = tau_hi + delta, lo = tau_lo - delta;
+  if (sampled && (double)t0 > lo) return 0;   // the window may reach below the filter
+  // classify: clearly in -> bitmap; window -> list (warp-aggregated counts)
+  int* wl = ms->wl;
+  for (int base = 0; base < m; base += g.nt) {
+    const int i = base + g.tid;
+    const double x = i < m ? (double)ckey[i] : -INFINITY;
+    const bool in = i < m && x > hi;
+    const bool win = i < m && !in && x >= lo;
+    const unsigned bin = __ballot_sync(0xffffffffu, in), bwin = __ballot_sync(0xffffffffu, win);
+    if (in) atomicOr(&bits[cid[i] >> 5], 1u << (cid[i] & 31));
+    if (lane == 0 && bin) atomicAdd(&ms->n_in, __popc(bin));
+    if (bwin) {
+      int wb = 0;
+      if (lane == 0) wb = atomicAdd(&ms->nwin, __popc(bwin));
+      wb = __shfl_sync(0xffffffffu, wb, 0);
+      const int pos = wb + __popc(bwin & ((1u << lane) - 1u));
+      if (win && pos < kWindowCap) wl[pos] = cid[i];
     }
   }
   g.sync();
-  const int n_in = ms->lo, w = ms->cnt, need = k - n_in;
-  if (w > kWindowCap) return false;
-  const int b = p / dm.H, h = p % dm.H;
-  const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
-  double* s64 = a.cand_s64 + (size_t)p * Nc;
-  for (int i = g.tid; i < w; i += g.nt) s64[i] = score64_row<T, D, G>(L + (size_t)wl[i] * D, sQ);
-  (void)b;
-  (void)h;
+  const int n_in = ms->n_in, w = ms->nwin, need = k - n_in;
+  if (w > kWindowCap) return 0;
+  // window: one warp per row re-scores in fp64 (queries read as stored)
+  const T* qb = (const T*)a.q + ((size_t)(p / dm.H) * dm.Hq + (size_t)(p % dm.H) * G) * D;
+  const T* Lp = (const T*)a.landmark + (size_t)p * Nc * D;
+  double* s64 = reinterpret_cast<double*>(ckey);   // candidates are no longer needed
+  score64_rows_warp<T, D, G>(Lp, qb, wl, w, g.tid >> 5, g.nt >> 5, s64, lane);
   g.sync();
   for (int i = g.tid; i < w; i += g.nt) {
     const double si = s64[i];
@@ -313,39 +571,56 @@ __device__ bool select_pair_fast(const Grp& g, const SelectArgs& a, int p, const
     if (rank < need) atomicOr(&bits[ii >> 5], 1u << (ii & 31));
   }
   g.sync();
-  // ascending output: exclusive scan of the per-word bit counts
+  // ascending output: each thread owns a run of bitmap words; one scan of their counts
   int32_t* sel = a.sel + (size_t)p * k;
-  const int nw = (Nc + 31) / 32;
-  int base = 0;
-  for (int w0 = 0; w0 < nw; w0 += g.nt) {
-    const int wi = w0 + g.tid;
-    const uint32_t word = wi < nw ? bits[wi] : 0u;
-    int total;
-    int pos = base + group_exclusive_scan(g, __popc(word), ms->iscr, &total);
-    uint32_t rem = word;
+  const int wpt = (nw + g.nt - 1) / g.nt;
+  int cnt = 0;
+  for (int j = 0; j < wpt; ++j) {
+    const int wi = g.tid * wpt + j;
+    if (wi < nw) cnt += __popc(bits[wi]);
+  }
+  int total;
+  int pos = group_exclusive_scan(g, cnt, ms->iscr, &total);
+  for (int j = 0; j < wpt; ++j) {
+    const int wi = g.tid * wpt + j;
+    uint32_t rem = wi < nw ? bits[wi] : 0u;
     while (rem) {
       const int bit = __ffs(rem) - 1;
       rem &= rem - 1;
       if (pos < k) sel[pos] = wi * 32 + bit;
       ++pos;
     }
-    base += total;
   }
-  return true;
+  return 1;
 }
 
+// Selects (b, h) pair p from its scores, waiting for them as it reads; leaves the scratch
+// counters at zero. Returns false if a wait gave up.
 template <typename T, int D, int G>
-__device__ void select_pair(const Grp& g, const SelectArgs& a, int p, const float* sQ,
-                            float* ckey, int* cid, uint32_t* bits, Misc* ms) {
+__device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* ckey, int* cid,
+                            uint32_t* bits, Misc* ms, volatile int* abort) {
+  constexpr int kCap = cand_cap(G, D);
   const int Nc = a.dm.Nc, k = a.dm.k;
-  if (k >= Nc) {
-    int32_t* sel = a.sel + (size_t)p * k;
-    for (int i = g.tid; i < Nc; i += g.nt) sel[i] = i;
-    return;
+  const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + (size_t)p * Nc);
+  int r = 0;   // 1 done, 0 radix path, -1 gave up
+  if (k < Nc && k <= kCap / 2 && Nc <= kBitmapChunks) {
+    r = select_pair_fast<T, D, G>(g, a, p, ckey, cid, bits, ms, abort);
+  } else {
+    if (!wait_scores(g, su, Nc, abort)) ms->n_in = -1;   // every score, before any is used
+    g.sync();
+    r = ms->n_in < 0 ? -1 : 0;
+    if (r == 0 && k >= Nc) {
+      int32_t* sel = a.sel + (size_t)p * k;
+      for (int i = g.tid; i < Nc; i += g.nt) sel[i] = i;
+      r = 1;
+    }
   }
-  const bool done = select_pair_fast<T, D, G>(g, a, p, sQ, ckey, cid, bits, ms);
   g.sync();
-  if (!done) select_pair_radix<T, D, G>(g, a, p, ms);
+  if (r == 0) select_pair_radix<T, D, G>(g, a, p, ms);
+  g.sync();
+  if (g.tid == 0) { ms->cnt = 0; ms->n_in = 0; ms->nwin = 0; ms->fmax = 0.f; }
+  g.sync();
+  return r >= 0;
 }
 
 // ---------------------------------------------------------------- scoring
@@ -395,6 +670,8 @@ template <typename T, int D, int G>
 __global__ void __launch_bounds__(kSelThreads, 1)
 score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap) {
   using Gm = Geom<T, D>;
+  constexpr int kQ = G * D;        // query values per (b, h); a multiple of 32
+  constexpr int kQL = kQ / 32;     // per producer lane
   const Dims& dm = a.dm;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -406,6 +683,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
   int* cidv = reinterpret_cast<int*>(gbase + L.cid);
   uint32_t* bits = reinterpret_cast<uint32_t*>(gbase + L.outs);
   Misc* ms = reinterpret_cast<Misc*>(gbase + L.misc);
+  int* stage_unit = reinterpret_cast<int*>(gbase + L.hdr);   // [kStages]; -2: no more
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.bar + 8 * 2 * kStages);
   auto full = [&](int s) { return base + L.bar + 8u * (uint32_t)s; };
   auto empty = [&](int s) { return base + L.bar + 8u * (uint32_t)(kStages + s); };
@@ -413,28 +691,67 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Nc = dm.Nc, P = dm.B * dm.H;
   const int upp = (Nc + Gm::kLps - 1) / Gm::kLps;    // stages per (b, h)
-  const long long U = (long long)P * upp;
-  const int u_begin = (int)(U * blockIdx.x / gridDim.x);
-  const int u_end = (int)(U * (blockIdx.x + 1) / gridDim.x);
+  const int U = P * upp;
+  int* grab = a.counters;        // next stage to hand out
+  int* exits = a.counters + 1;   // CTAs finished
+  int* q_head = a.counters + 2;  // next (b, h) to select
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full(s), 1);
-      mbar_init(empty(s), kConsumers / 32);
+      mbar_init(full(s), 32);                 // the producer warp's lanes
+      mbar_init(empty(s), kConsumers / 32);   // one arrival per consumer warp
     }
     fence_mbar_init();
+    ms->cnt = 0;
+    ms->n_in = 0;
+    ms->nwin = 0;
+    ms->fmax = 0.f;
   }
   __syncthreads();
+  // a programmatic dependent (the reconstruct-and-attend kernel) may start as SMs free
+  // up; it reads a pair's selection only after that pair's ready flag is set
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == kConsumers / 32) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer warp
+    // Lane 0 takes stages two fills ahead and issues their loads; every lane loads the
+    // queries of the next fill's (b, h) one fill ahead and stages them.
+    int last_i[kStages];
+    for (int s = 0; s < kStages; ++s) last_i[s] = -1;
+    bool ok = true;
+    auto load_q = [&](int unit, float* qv) {
+      const int pair = unit / upp;
+      const T* qb = (const T*)a.q + ((size_t)(pair / dm.H) * dm.Hq + (size_t)(pair % dm.H) * G) * D;
+#pragma unroll
+      for (int j = 0; j < kQL; ++j) qv[j] = ldf(qb, lane + 32 * j);
+    };
+    // u: this fill's stage, un: the next one; lane 0's grab_pend is the take for the fill
+    // after that, issued one fill earlier and read one fill later.
+    int u = U, un = U, grab_pend = U;
     if (lane == 0) {
-      int last_i[kStages];
-      for (int s = 0; s < kStages; ++s) last_i[s] = -1;
-      for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait_bounded(empty(s), ((i / kStages) & 1) ^ 1, abort_flag)) break;
+      u = atomicAdd(grab, 1);
+      if (u < U) un = atomicAdd(grab, 1);
+      if (un < U) grab_pend = atomicAdd(grab, 1);
+    }
+    u = __shfl_sync(0xffffffffu, u, 0);
+    un = __shfl_sync(0xffffffffu, un, 0);
+    float qa[kQL], qb[kQL];
+    if (u < U) load_q(u, qa);
+    int i = 0;
+    // One fill; qc holds this fill's queries, qn receives the next fill's. Returns 0 to go
+    // on, 1 when no stages are left (fill i's slot is free), 2 on a failed wait.
+    auto step = [&](float (&qc)[kQL], float (&qn)[kQL]) -> int {
+      const int s = i % kStages;
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait_bounded(empty(s), ((i / kStages) & 1) ^ 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, okw, 0)) return 2;
+      if (u >= U) return 1;   // slot s is free for the closing fill
+      float* q_s = sQ + s * kQ;
+#pragma unroll
+      for (int j = 0; j < kQL; ++j) q_s[lane + 32 * j] = qc[j];
+      if (lane == 0) {
+        stage_unit[s] = u;
         const int pair = u / upp, st = u % upp;
         const int row = pair * Nc + st * Gm::kLps;
         mbar_arrive_expect_tx(full(s), (uint32_t)(Gm::kBoxes * Gm::kLps * 128));
@@ -442,64 +759,105 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
           tma_load_2d(base + L.stages + s * kStageBytes + bx * Gm::kLps * 128, &lmap,
                       bx * Gm::kBoxCols, row, full(s));
         last_i[s] = i;
+      } else {
+        mbar_arrive(full(s));
       }
-      if (*abort_flag) {   // loads may still be in flight: let them land before exit
-        for (int s = 0; s < kStages; ++s) {
-          if (last_i[s] < 0) continue;
-          int dummy = 0;
-          mbar_wait_bounded(full(s), (last_i[s] / kStages) & 1, (volatile int*)&dummy);
-        }
+      // the next fill's queries and the take after the next
+      if (un < U) load_q(un, qn);
+      int unn = U;
+      if (lane == 0 && un < U) {
+        unn = grab_pend;
+        grab_pend = unn < U ? atomicAdd(grab, 1) : U;
+      }
+      u = un;
+      un = __shfl_sync(0xffffffffu, unn, 0);
+      ++i;
+      return 0;
+    };
+    for (;;) {
+      int r = step(qa, qb);
+      if (r == 0) r = step(qb, qa);
+      if (r == 0) continue;
+      ok = r == 1;
+      break;
+    }
+    if (ok) {   // closing fill: no stages left
+      const int s = i % kStages;
+      if (lane == 0) stage_unit[s] = -2;
+      mbar_arrive(full(s));
+    }
+    if (lane == 0 && *abort_flag) {   // loads may still be in flight: let them land
+      for (int s = 0; s < kStages; ++s) {
+        if (last_i[s] < 0) continue;
+        int dummy = 0;
+        mbar_wait_bounded(full(s), (last_i[s] / kStages) & 1, (volatile int*)&dummy);
       }
     }
-  } else {
+  } else if (warp < kConsumers / 32) {
     // ------------------------------------------------------------ consumers
-    // Every consumer thread runs the same sequence of group barriers whatever its
-    // waits return, so a timed-out wait never leaves the others at a barrier.
-    const Grp g{(int)threadIdx.x, kConsumers, 1};
     const int tid = threadIdx.x;
-    int cur = -1, seg = 0;
-    auto finish_segment = [&](int pair, int nst) {
-      __threadfence();
-      g.sync();
-      if (tid == 0) {
-        const int old = atomicAdd(a.counters + pair, nst);
-        ms->last = (old + nst == upp);
-      }
-      g.sync();
-      if (ms->last) {
-        __threadfence();
-        select_pair<T, D, G>(g, a, pair, sQ, ckey, cidv, bits, ms);
-        g.sync();
-        if (tid == 0) a.counters[pair] = 0;
-      }
-    };
-    for (int u = u_begin, i = 0; u < u_end; ++u, ++i) {
-      const int pair = u / upp, st = u % upp;
-      if (pair != cur) {
-        if (cur >= 0) finish_segment(cur, seg);
-        cur = pair;
-        seg = 0;
-        g.sync();
-        const int b = pair / dm.H, h = pair % dm.H;
-        const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
-        for (int e = tid; e < G * D; e += kConsumers) sQ[e] = ldf(qb, e);
-        g.sync();
-      }
+    for (int i = 0;; ++i) {
       const int s = i % kStages;
-      mbar_wait_bounded(full(s), (i / kStages) & 1, abort_flag);
+      const bool okw = mbar_wait_bounded(full(s), (i / kStages) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      const int u = stage_unit[s];
+      if (u < 0) break;
+      const int pair = u / upp, st = u % upp;
       const int c = st * Gm::kLps + tid;
       if (tid < Gm::kLps && c < Nc) {
-        const float sc = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ);
+        const float sc = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
         a.scores[(size_t)pair * Nc + c] = sc;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
-      ++seg;
     }
-    if (cur >= 0) finish_segment(cur, seg);
+  } else {
+    // ------------------------------------------------------------ selection warps
+    // Take the next (b, h), wait until all of its stages are handed out and all of its
+    // scores have landed, select, restore the sentinel. One verdict per step for the
+    // whole group keeps its barrier sequence uniform.
+    const Grp g{(int)threadIdx.x - (kConsumers + 32), kSelectors, 2};
+    for (;;) {
+      if (g.tid == 0) {
+        int pair = -1;
+        const int at = atomicAdd(q_head, 1);
+        if (at < P && wait_counter_ge(grab, (at + 1) * upp, abort_flag)) pair = at;
+        ms->req = pair;
+      }
+      g.sync();
+      const int pair = ms->req;
+      g.sync();
+      if (pair < 0) break;
+      uint32_t* sp = reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc);
+      if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) break;
+      clear_scores(g, sp, Nc);
+      if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
+        __threadfence();
+        st_release(a.ready + pair, 1);
+      }
+    }
   }
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) raise_status(a.status, kStatusTimeout);
+  if (threadIdx.x == 0) {
+    if (*abort_flag) raise_status(a.status, kStatusTimeout);
+    // the last CTA out resets the counters and, after a failure, every score
+    __threadfence();
+    const bool last = atomicAdd(exits, 1) == (int)gridDim.x - 1;
+    bool failed = false;
+    if (last) {
+      __threadfence();
+      failed = *(volatile int*)a.status != 0;
+      atomicExch(grab, 0);
+      atomicExch(q_head, 0);
+      atomicExch(exits, 0);
+    }
+    ms->req = failed ? 1 : 0;
+  }
+  __syncthreads();
+  if (ms->req) {
+    const Grp all{(int)threadIdx.x, (int)blockDim.x, 0};
+    clear_scores(all, reinterpret_cast<uint32_t*>(a.scores), P * Nc);
+  }
 }
 
 template <typename T, int D, int G>
@@ -510,6 +868,7 @@ cudaError_t launch_typed(const SelectArgs& a, int num_sms, cudaStream_t s) {
                           (uint64_t)a.dm.B * a.dm.H * a.dm.Nc, Gm::kBoxCols, Gm::kLps, 128))
     return cudaErrorInvalidValue;
   const SelSmem L = sel_smem(G, D);
+  if (L.total > (uint32_t)kSmemLimit) return cudaErrorInvalidValue;
   auto kern = score_select_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L.total);
