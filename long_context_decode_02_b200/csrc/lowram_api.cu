@@ -24,7 +24,8 @@ struct lowram_ctx {
   int n_hi;
   int* status;    // device word
   int* counters;  // device [4]: the selection kernel's work, exit and pair counters
-  float* scores;  // device [B*H][Nc], the sentinel 0xFFFFFFFF between launches
+  float* scores;   // device [B*H][Nc], all bits set between launches
+  float* norms;    // device [B*H][stages][8], all bits set between launches
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   double* theta64;  // device [d/2]
 };
@@ -257,6 +258,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
+            cudaMalloc(&ctx->norms, pairs * 8 * (size_t)select_stages_per_pair(dims_of(*c)) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
   ok = ok &&
        cudaMemcpy(ctx->lo32, lo32.data(), lo32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -267,6 +269,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
+       cudaMemset(ctx->norms, 0xff, pairs * 8 * (size_t)select_stages_per_pair(dims_of(*c)) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -287,6 +290,7 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->status);
   cudaFree(ctx->counters);
   cudaFree(ctx->scores);
+  cudaFree(ctx->norms);
   cudaFree(ctx->ready);
   cudaFree(ctx->theta64);
   delete ctx;
@@ -338,6 +342,7 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, 
   sa.landmark = landmark;
   sa.q = q;
   sa.scores = ctx->scores;
+  sa.norms = ctx->norms;
   sa.cand_s64 = reinterpret_cast<double*>(ws + w.cand_s64);
   sa.cand_idx = reinterpret_cast<int*>(ws + w.cand_idx);
   sa.flags = ws + w.flags;

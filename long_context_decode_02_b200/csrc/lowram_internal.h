@@ -43,7 +43,9 @@ struct SelectArgs {
   Dims dm;
   const void* landmark;   // [B][H][Nc][d]
   const void* q;          // [B][Hq][d]
-  float* scores;          // ctx [B*H][Nc], the sentinel 0xFFFFFFFF between launches
+  float* scores;          // ctx [B*H][Nc], all bits set between launches
+  float* norms;           // ctx [B*H][stages][8]: largest |L|_2 per stage and consumer warp,
+                          // all bits set between launches
   double* cand_s64;       // ws [B*H][Nc]
   int* cand_idx;          // ws [B*H][Nc]
   uint8_t* flags;         // ws [B*H][Nc]
@@ -53,6 +55,14 @@ struct SelectArgs {
   int* status;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
+// Stages of landmark rows per (b, h) in the selection kernel: a stage is
+// min(65536 / row bytes, 256) rows.
+__host__ __device__ inline int select_stages_per_pair(const Dims& dm) {
+  const int row_bytes = dm.d * (dm.dtype == LOWRAM_DTYPE_BF16 ? 2 : 4);
+  int rows = 65536 / row_bytes;
+  if (rows > 256) rows = 256;
+  return (dm.Nc + rows - 1) / rows;
+}
 
 // ---------------- decode: reconstruct + attend ----------------
 struct AttendArgs {

@@ -15,7 +15,9 @@
 //    score one row each (packed fp32x2 FMAs) and write the fp32 score.
 //  * Scores live in a context-owned buffer that holds a sentinel bit pattern between
 //    launches (0xFFFFFFFF, a NaN that fp32 arithmetic never produces), so a written score
-//    is its own completion flag: no counters or memory fences on the streaming path.
+//    is its own completion flag: no counters or memory fences on the streaming path. Each
+//    consumer warp also writes the largest |L|_2 of its rows in each stage to a second
+//    sentinel-initialised buffer (the norms bound the fp32 error below).
 //    Three selection warps per CTA take (b, h) pairs in order from a global counter,
 //    wait until the work counter has handed out all of the pair's stages and every score
 //    has landed, select, and put the sentinel back. Selections are spread over the CTAs
@@ -26,10 +28,13 @@
 //    24-bit prefix bucket [tau_lo, tau_hi] holding the k-th largest candidate.
 //    Candidates above tau_hi + delta are in; those in [tau_lo - delta, tau_hi + delta]
 //    are re-scored in fp64 (exact products, fp64 sums) and ranked by (score desc, index
-//    asc). delta = 1e-3|tau| + 1e-6 max|s| is far above the fp32 accumulation error, so
-//    the result equals the selection made in fp64. When the candidate set cannot be
-//    proven to hold the answer, a radix select over all scores decides instead. The
-//    chunk ids are written in ascending order.
+//    asc). delta is twice a rigorous bound on the fp32 score error: an fp32 dot product of
+//    D terms accumulated with fused multiply-adds is within gamma_D * sum|q_i L_i| <=
+//    gamma_D * |q|_2 |L|_2 of the exact value (gamma_n = n u / (1 - n u), u = 2^-24). So the
+//    result equals the selection made in fp64, and the window usually holds exactly the
+//    rows still needed, which then need no re-scoring. When the candidate set cannot be proven to
+//    hold the answer, a radix select over all scores decides instead. The chunk ids are
+//    written in ascending order.
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
@@ -70,7 +75,7 @@ struct Misc {
   float fscr[33];
   int iscr[33];
   int cnt, n_in, nwin;
-  float fmax;
+  float fmax;           // largest landmark norm among the candidates
   int req;              // the selection warps' current request
   int wl[kWindowCap];
 };
@@ -201,6 +206,41 @@ __device__ bool poll_vec4(const uint32_t* su, const int (&idx)[kN], uint32_t wan
   return true;
 }
 
+// This lane's slice of the group's queries: qr[g][e] = q[g][lane * D/32 + e].
+template <typename T, int D, int G>
+__device__ __forceinline__ void load_q_slice(const T* qb, int lane, float (&qr)[G][D / 32]) {
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) qr[g][e] = ldf(qb, g * D + lane * (D / 32) + e);
+}
+
+// max_g |q_g|_2 from every lane's slice (fp64 sums, a butterfly; the same in every lane).
+template <int D, int G>
+__device__ __forceinline__ double q_norm_max(const float (&qr)[G][D / 32]) {
+  double best = 0.0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    double ss = 0.0;
+#pragma unroll
+    for (int e = 0; e < D / 32; ++e) ss = fma((double)qr[g][e], (double)qr[g][e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    best = fmax(best, sqrt(ss));
+  }
+  return best;
+}
+
+// Twice a bound on |fl32(q . L) - q . L| for every row with |L|_2 <= lmax: gamma_D *
+// sum|q_i L_i| <= gamma_D |q|_2 |L|_2 (FMA accumulation of D exact-input products), with
+// margins for the fp32 norm itself and for the fp64 re-score.
+template <int D>
+__device__ __forceinline__ double score_error_window(double qmax, double lmax) {
+  const double u = 5.9604644775390625e-8;   // 2^-24
+  const double gam = D * u / (1.0 - D * u);
+  return 2.0 * (gam * 1.001 + 1e-12) * qmax * lmax + 1e-300;
+}
+
 template <typename T, int D, int G>
 __device__ double score64(const T* lrow, const T* qb) {
   double best = -INFINITY;
@@ -225,20 +265,23 @@ __device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc
   uint8_t* flags = a.flags + (size_t)p * Nc;
   int* cidx = a.cand_idx + (size_t)p * Nc;
   double* cs64 = a.cand_s64 + (size_t)p * Nc;
-
-  float mx = 0.f;
-  for (int i = g.tid; i < Nc; i += g.nt) mx = fmaxf(mx, fabsf(__ldcg(s + i)));
-  mx = group_max(g, mx, ms->fscr);
-  const uint32_t tk = group_kth_largest(
-      g, Nc, k, [&](int i) { return f2key(__ldcg(s + i)); }, ms->hist, ms->bc);
-  const double tau = (double)key2f(tk);
-  const double delta = 1e-3 * fabs(tau) + 1e-6 * (double)mx + 1e-30;
-  const double hi = tau + delta, lo = tau - delta;
-  if (g.tid == 0) ms->cnt = 0;
-  g.sync();
   const int b = p / dm.H, h = p % dm.H;
   const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
   const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
+
+  const int n_norm = 8 * select_stages_per_pair(dm);
+  float lmax = 0.f;
+  for (int i = g.tid; i < n_norm; i += g.nt) lmax = fmaxf(lmax, __ldcg(a.norms + (size_t)p * n_norm + i));
+  lmax = group_max(g, lmax, ms->fscr);
+  float qr[G][D / 32];
+  load_q_slice<T, D, G>(qb, g.tid & 31, qr);
+  const uint32_t tk = group_kth_largest(
+      g, Nc, k, [&](int i) { return f2key(__ldcg(s + i)); }, ms->hist, ms->bc);
+  const double tau = (double)key2f(tk);
+  const double delta = score_error_window<D>(q_norm_max<D, G>(qr), (double)lmax);
+  const double hi = tau + delta, lo = tau - delta;
+  if (g.tid == 0) ms->cnt = 0;
+  g.sync();
   int n_in = 0;
   for (int i = g.tid; i < Nc; i += g.nt) {
     const double x = (double)__ldcg(s + i);
@@ -281,18 +324,14 @@ __device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc
 }
 
 // fp64 scores of window rows by one warp: lane l holds D/32 consecutive elements of
-// each row and of each query head; exact products, fp64 sums (lane-serial, then a
-// butterfly); lane 0's value is stored. The loads of up to 8 rows are issued together.
+// each row and the same slice of each query head (qr); exact products, fp64 sums
+// (lane-serial, then a butterfly); lane 0's value is stored. The loads of up to 8 rows
+// are issued together.
 template <typename T, int D, int G>
-__device__ void score64_rows_warp(const T* Lp, const T* qb, const int* wl, int w, int first,
-                                  int stride, double* s64, int lane) {
+__device__ void score64_rows_warp(const T* Lp, const float (&qr)[G][D / 32], const int* wl,
+                                  int w, int first, int stride, double* s64, int lane) {
   constexpr int E = D / 32;
   constexpr int kBatch = 8;
-  float qr[G][E];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < E; ++e) qr[g][e] = ldf(qb, g * D + lane * E + e);
   for (int r0 = first; r0 < w; r0 += stride * kBatch) {
     float lv[kBatch][E];
 #pragma unroll
@@ -380,10 +419,10 @@ __device__ uint32_t kth_largest_prefix(const Grp& g, int n, int k, KeyFn key_of,
 }
 
 // Fast path (see the file comment); needs k <= cap/2 and N_c <= kBitmapChunks. Reads each
-// score through a poll that waits out the sentinel, so it needs no separate wait for the
+// entry through a poll that waits out the sentinel, so it needs no separate wait for the
 // pair. Expects ms->cnt, n_in, nwin and fmax at zero. Returns 1 when done; 0, having
 // written no output, when the candidate set cannot be proven to hold the answer (every
-// score has been seen by then); -1 when a wait gave up.
+// entry has been seen by then); -1 when a wait gave up.
 template <typename T, int D, int G>
 __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float* ckey,
                                 int* cid, uint32_t* bits, Misc* ms, volatile int* abort) {
@@ -393,15 +432,40 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
   const int Nc = dm.Nc, k = dm.k;
   const int lane = g.tid & 31;
   const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + (size_t)p * Nc);
+  const T* qb = (const T*)a.q + ((size_t)(p / dm.H) * dm.Hq + (size_t)(p % dm.H) * G) * D;
   const uint64_t t_start = global_timer_ns();
+  double qmax;   // max_g |q_g|_2, for the error window
+  {
+    float qr[G][D / 32];
+    load_q_slice<T, D, G>(qb, lane, qr);
+    qmax = q_norm_max<D, G>(qr);
+  }
   const int nw = (Nc + 31) >> 5;
   for (int i = g.tid; i < nw; i += g.nt) bits[i] = 0u;
   bool good = true;
+  // largest |L|_2 of the pair, from the consumer warps' per-stage maxima
+  float lmax = 0.f;
+  {
+    const int n_norm = 8 * select_stages_per_pair(dm);
+    const uint32_t* nu = reinterpret_cast<const uint32_t*>(a.norms + (size_t)p * n_norm);
+    for (int base = 0; base < n_norm; base += kB * g.nt) {
+      int idx[kB];
+      uint32_t want = 0, v[kB];
+#pragma unroll
+      for (int j = 0; j < kB; ++j) {
+        idx[j] = base + j * g.nt + g.tid;
+        if (idx[j] < n_norm) want |= 1u << j;
+      }
+      good = good && poll_words<kB>(nu, idx, want, v, abort, t_start);
+#pragma unroll
+      for (int j = 0; j < kB; ++j)
+        if ((want >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(v[j]));
+    }
+  }
   int m;
   float t0 = -INFINITY;
   const bool sampled = Nc > kCap;
   if (!sampled) {
-    float mx = 0.f;
     for (int base = 0; base < Nc; base += kB * g.nt) {
       int idx[kB];
       uint32_t want = 0, v[kB];
@@ -414,14 +478,10 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
 #pragma unroll
       for (int j = 0; j < kB; ++j)
         if ((want >> j) & 1u) {
-          const float x = __uint_as_float(v[j]);
-          ckey[idx[j]] = x;
+          ckey[idx[j]] = __uint_as_float(v[j]);
           cid[idx[j]] = idx[j];
-          mx = fmaxf(mx, fabsf(x));
         }
     }
-    mx = warp_max(mx);
-    if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(mx));
     if (!good) ms->cnt = -1;
     g.sync();
     if (ms->cnt < 0) return -1;
@@ -448,42 +508,31 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
     int j = (int)((3LL * k * kSample) / (2LL * Nc)) + 16;
     if (j > kSample) j = kSample;
     t0 = key2f(kth_largest_prefix<2>(g, kSample, j, [&](int i) { return skey[i]; }, ms));
-    // every score >= t0 becomes a candidate: each thread filters 32 scores from 8
-    // independent 16-byte loads, then one warp scan and one shared atomic per warp place
-    // them (16-byte groups when 4 | N_c and the row is 16-byte aligned; else single words)
-    float mx = 0.f;
+    // every score >= t0 becomes a candidate. Each thread polls 8 independent 16-byte
+    // groups (4 scores; single scores when 4 does not divide N_c), keeps a mask of its
+    // candidates, and one warp scan and one shared atomic per warp place them.
     const bool vec = (Nc & 3) == 0 && (reinterpret_cast<uintptr_t>(su) & 15) == 0;
-    const int n4 = vec ? Nc / 4 : (Nc + 3) / 4;
-    for (int base = 0; base < n4; base += kB * g.nt) {
+    const int per = vec ? 4 : 1;   // scores per polled group
+    const int n_groups = Nc / per;
+    for (int base = 0; base < n_groups; base += kB * g.nt) {
       int idx[kB];
       uint32_t want = 0;
       uint4 v[kB];
 #pragma unroll
       for (int j = 0; j < kB; ++j) {
         idx[j] = base + j * g.nt + g.tid;
-        if (idx[j] < n4) want |= 1u << j;
+        if (idx[j] < n_groups) want |= 1u << j;
       }
       if (vec) {
         good = good && poll_vec4<kB>(su, idx, want, v, abort, t_start);
       } else {
+        uint32_t v1[kB];
+        good = good && poll_words<kB>(su, idx, want, v1, abort, t_start);
+        const uint32_t ninf = __float_as_uint(-INFINITY);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int ie[kB];
-          uint32_t we = 0, ve[kB];
-#pragma unroll
-          for (int j = 0; j < kB; ++j) {
-            ie[j] = 4 * idx[j] + e;
-            if (((want >> j) & 1u) && ie[j] < Nc) we |= 1u << j;
-          }
-          good = good && poll_words<kB>(su, ie, we, ve, abort, t_start);
-#pragma unroll
-          for (int j = 0; j < kB; ++j) {
-            const uint32_t x = ((we >> j) & 1u) ? ve[j] : __float_as_uint(-INFINITY);
-            if (e == 0) v[j].x = x; else if (e == 1) v[j].y = x; else if (e == 2) v[j].z = x; else v[j].w = x;
-          }
-        }
+        for (int j = 0; j < kB; ++j) v[j] = make_uint4(v1[j], ninf, ninf, ninf);
       }
-      uint32_t keep = 0;
+      uint32_t keep = 0;   // bit 4j + e: score per * idx[j] + e
 #pragma unroll
       for (int j = 0; j < kB; ++j) {
         if (!((want >> j) & 1u)) continue;
@@ -506,31 +555,30 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
       int pos = wb + incl - c;
 #pragma unroll
       for (int j = 0; j < kB; ++j) {
-        const float xs[4] = {__uint_as_float(v[j].x), __uint_as_float(v[j].y),
-                             __uint_as_float(v[j].z), __uint_as_float(v[j].w)};
+        const uint32_t xs[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           if ((keep >> (4 * j + e)) & 1u) {
-            if (pos < kCap) { ckey[pos] = xs[e]; cid[pos] = 4 * idx[j] + e; }
+            if (pos < kCap) { ckey[pos] = __uint_as_float(xs[e]); cid[pos] = per * idx[j] + e; }
             ++pos;
-            mx = fmaxf(mx, fabsf(xs[e]));
           }
         }
       }
     }
-    mx = warp_max(mx);
-    if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(mx));
     if (!good) ms->n_in = -1;
-    g.sync();
-    if (ms->n_in < 0) return -1;
+  }
+  lmax = warp_max(lmax);
+  if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(lmax));
+  g.sync();
+  if (ms->n_in < 0) return -1;
+  if (sampled) {
     m = ms->cnt;
     if (m > kCap || m < k) return 0;
   }
   const uint32_t tp = kth_largest_prefix<3>(g, m, k, [&](int i) { return f2key(ckey[i]); }, ms);
   const double tau_lo = (double)key2f(tp), tau_hi = (double)key2f(tp | 0xFFu);
   if (!(tau_lo <= tau_hi)) return 0;   // a non-finite bucket
-  const double tmag = fmax(fabs(tau_lo), fabs(tau_hi));
-  const double delta = 1e-3 * tmag + 1e-6 * fmax((double)ms->fmax, tmag) + 1e-30;
+  const double delta = score_error_window<D>(qmax, (double)ms->fmax);
   const double hi = tau_hi + delta, lo = tau_lo - delta;
   if (sampled && (double)t0 > lo) return 0;   // the window may reach below the filter
   // classify: clearly in -> bitmap; window -> list (warp-aggregated counts)
@@ -554,23 +602,31 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
   g.sync();
   const int n_in = ms->n_in, w = ms->nwin, need = k - n_in;
   if (w > kWindowCap) return 0;
-  // window: one warp per row re-scores in fp64 (queries read as stored)
-  const T* qb = (const T*)a.q + ((size_t)(p / dm.H) * dm.Hq + (size_t)(p % dm.H) * G) * D;
-  const T* Lp = (const T*)a.landmark + (size_t)p * Nc * D;
-  double* s64 = reinterpret_cast<double*>(ckey);   // candidates are no longer needed
-  score64_rows_warp<T, D, G>(Lp, qb, wl, w, g.tid >> 5, g.nt >> 5, s64, lane);
-  g.sync();
-  for (int i = g.tid; i < w; i += g.nt) {
-    const double si = s64[i];
-    const int ii = wl[i];
-    int rank = 0;
-    for (int j2 = 0; j2 < w; ++j2) {
-      const double sj = s64[j2];
-      rank += (sj > si) || (sj == si && wl[j2] < ii);
+  // window: when it holds exactly the rows still needed (the usual case: the k-th row
+  // alone) all are in. Otherwise one warp per row re-scores in fp64 (queries as stored)
+  // and the rows are ranked by (score desc, index asc).
+  if (w == need) {
+    for (int i = g.tid; i < w; i += g.nt) atomicOr(&bits[wl[i] >> 5], 1u << (wl[i] & 31));
+    g.sync();
+  } else if (w > 0) {
+    const T* Lp = (const T*)a.landmark + (size_t)p * Nc * D;
+    double* s64 = reinterpret_cast<double*>(ckey);   // candidates are no longer needed
+    float qr[G][D / 32];
+    load_q_slice<T, D, G>(qb, lane, qr);
+    score64_rows_warp<T, D, G>(Lp, qr, wl, w, g.tid >> 5, g.nt >> 5, s64, lane);
+    g.sync();
+    for (int i = g.tid; i < w; i += g.nt) {
+      const double si = s64[i];
+      const int ii = wl[i];
+      int rank = 0;
+      for (int j2 = 0; j2 < w; ++j2) {
+        const double sj = s64[j2];
+        rank += (sj > si) || (sj == si && wl[j2] < ii);
+      }
+      if (rank < need) atomicOr(&bits[ii >> 5], 1u << (ii & 31));
     }
-    if (rank < need) atomicOr(&bits[ii >> 5], 1u << (ii & 31));
+    g.sync();
   }
-  g.sync();
   // ascending output: each thread owns a run of bitmap words; one scan of their counts
   int32_t* sel = a.sel + (size_t)p * k;
   const int wpt = (nw + g.nt - 1) / g.nt;
@@ -606,7 +662,10 @@ __device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* cke
   if (k < Nc && k <= kCap / 2 && Nc <= kBitmapChunks) {
     r = select_pair_fast<T, D, G>(g, a, p, ckey, cid, bits, ms, abort);
   } else {
-    if (!wait_scores(g, su, Nc, abort)) ms->n_in = -1;   // every score, before any is used
+    const int n_norm = 8 * select_stages_per_pair(a.dm);   // every score and norm, before use
+    if (!wait_scores(g, su, Nc, abort) ||
+        !wait_scores(g, reinterpret_cast<const uint32_t*>(a.norms + (size_t)p * n_norm), n_norm, abort))
+      ms->n_in = -1;
     g.sync();
     r = ms->n_in < 0 ? -1 : 0;
     if (r == 0 && k >= Nc) {
@@ -624,11 +683,12 @@ __device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* cke
 }
 
 // ---------------------------------------------------------------- scoring
-// Score of landmark row r of a swizzled stage.
+// {score, |L|_2} of landmark row r of a swizzled stage.
 template <typename T, int D, int G>
-__device__ __forceinline__ float score_row(const uint8_t* stage, int r, const float* sQ) {
+__device__ __forceinline__ float2 score_row(const uint8_t* stage, int r, const float* sQ) {
   using Gm = Geom<T, D>;
   float2 acc[G];
+  float2 nn = make_float2(0.f, 0.f);
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
 #pragma unroll
@@ -639,6 +699,10 @@ __device__ __forceinline__ float score_row(const uint8_t* stage, int r, const fl
     if constexpr (sizeof(T) == 2) {
       // 8 bf16: chunk c holds dims 8c .. 8c+7
       const float2 v0 = bf2_to_f2(w.x), v1 = bf2_to_f2(w.y), v2 = bf2_to_f2(w.z), v3 = bf2_to_f2(w.w);
+      nn = __ffma2_rn(v0, v0, nn);
+      nn = __ffma2_rn(v1, v1, nn);
+      nn = __ffma2_rn(v2, v2, nn);
+      nn = __ffma2_rn(v3, v3, nn);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c);
@@ -652,6 +716,8 @@ __device__ __forceinline__ float score_row(const uint8_t* stage, int r, const fl
       // 4 fp32: chunk c holds dims 4c .. 4c+3
       const float2 v0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
       const float2 v1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+      nn = __ffma2_rn(v0, v0, nn);
+      nn = __ffma2_rn(v1, v1, nn);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 4 * c);
@@ -663,7 +729,7 @@ __device__ __forceinline__ float score_row(const uint8_t* stage, int r, const fl
   float best = acc[0].x + acc[0].y;
 #pragma unroll
   for (int g = 1; g < G; ++g) best = fmaxf(best, acc[g].x + acc[g].y);
-  return best;
+  return make_float2(best, sqrtf(nn.x + nn.y));
 }
 
 template <typename T, int D, int G>
@@ -690,7 +756,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Nc = dm.Nc, P = dm.B * dm.H;
-  const int upp = (Nc + Gm::kLps - 1) / Gm::kLps;    // stages per (b, h)
+  const int upp = select_stages_per_pair(dm);   // stages of Gm::kLps rows per (b, h)
   const int U = P * upp;
   int* grab = a.counters;        // next stage to hand out
   int* exits = a.counters + 1;   // CTAs finished
@@ -804,10 +870,14 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (u < 0) break;
       const int pair = u / upp, st = u % upp;
       const int c = st * Gm::kLps + tid;
+      float nrm = 0.f;
       if (tid < Gm::kLps && c < Nc) {
-        const float sc = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
-        a.scores[(size_t)pair * Nc + c] = sc;
+        const float2 r = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
+        a.scores[(size_t)pair * Nc + c] = r.x;
+        nrm = r.y;
       }
+      nrm = warp_max(nrm);   // this warp's largest |L|_2 in the stage
+      if (lane == 0) a.norms[((size_t)pair * upp + st) * 8 + warp] = nrm;
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
     }
@@ -828,9 +898,9 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       const int pair = ms->req;
       g.sync();
       if (pair < 0) break;
-      uint32_t* sp = reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc);
       if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) break;
-      clear_scores(g, sp, Nc);
+      clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
+      clear_scores(g, reinterpret_cast<uint32_t*>(a.norms + (size_t)pair * upp * 8), upp * 8);
       if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
         __threadfence();
         st_release(a.ready + pair, 1);
@@ -857,6 +927,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
   if (ms->req) {
     const Grp all{(int)threadIdx.x, (int)blockDim.x, 0};
     clear_scores(all, reinterpret_cast<uint32_t*>(a.scores), P * Nc);
+    clear_scores(all, reinterpret_cast<uint32_t*>(a.norms), P * upp * 8);
   }
 }
 
