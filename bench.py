@@ -246,7 +246,8 @@ def run_ours(args):
 
     def select_calls():
         for layer in range(n_layers):
-            L.select_chunks(ctx, layers[layer]["cache"]["landmark"], q_buf[layer],
+            L.select_chunks(ctx, layers[layer]["cache"]["landmark"],
+                            layers[layer]["cache"]["landmark_norm"], q_buf[layer],
                             sel_buf[layer], dec_ws)
 
     def attend_calls():

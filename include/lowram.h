@@ -103,8 +103,14 @@ typedef struct lowram_layer_params {
  *   res_idx   [B][H_kv][n_res]   int32 token indices of the residual rows, ascending
  *   res_val   [B][H_kv][n_res][d] residual corrections V_t - V_hat_t
  *   chunk_ptr [B][H_kv][T/C + 1] int32 CSR: rows of chunk c are ptr[c] .. ptr[c+1]-1
+ *   landmark_norm [B][H_kv]      fp32 upper bound of max_c |landmark_c|_2 of each (b, h).
+ *                                Not part of the method: decode uses it to bound the fp32
+ *                                score error near the top-k threshold. lowram_encode
+ *                                writes it; lowram_landmark_norms recomputes it for a
+ *                                cache built elsewhere. A value below the true maximum
+ *                                can change the selection.
  * The layout is fixed by these shapes, so a cache can be saved and restored byte for
- * byte (lowram_cache_layout gives the five sizes). res_idx and res_val may be NULL when
+ * byte (lowram_cache_layout gives the six sizes). res_idx and res_val may be NULL when
  * n_res == 0. */
 typedef struct lowram_cache {
   void* coef;
@@ -112,6 +118,7 @@ typedef struct lowram_cache {
   int32_t* res_idx;
   void* res_val;
   int32_t* chunk_ptr;
+  float* landmark_norm;
 } lowram_cache;
 
 typedef struct lowram_ctx lowram_ctx;
@@ -129,8 +136,9 @@ lowram_status lowram_create(const lowram_config* cfg, int device, lowram_ctx** o
  * stream still using the context. NULL is accepted. */
 void lowram_destroy(lowram_ctx* ctx);
 
-/* Host only. bytes_out[0..4] = sizes of coef, landmark, res_idx, res_val, chunk_ptr. */
-lowram_status lowram_cache_layout(const lowram_config* cfg, size_t bytes_out[5]);
+/* Host only. bytes_out[0..5] = sizes of coef, landmark, res_idx, res_val, chunk_ptr,
+ * landmark_norm. */
+lowram_status lowram_cache_layout(const lowram_config* cfg, size_t bytes_out[6]);
 
 /* Host only. Workspace bytes needed by op (LOWRAM_OP_ENCODE or LOWRAM_OP_DECODE). The
  * workspace needs no initialisation and holds nothing between calls. */
@@ -168,11 +176,18 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
 /* Decode sub-step 1 (kernel (a) alone): score every chunk by max over the GQA group of
  * q . landmark and write the top-k chunks per (batch, KV head), ascending, ties to the
  * lower chunk (agihunt summary, key paragraph; cctest "Selective reconstruction").
- *   landmark [B][H_kv][T/C][d]; q [B][H_q][d]; sel_out [B][H_kv][k] int32 (written).
+ *   landmark [B][H_kv][T/C][d]; landmark_norm [B][H_kv] fp32 (the cache field);
+ *   q [B][H_q][d]; sel_out [B][H_kv][k] int32 (written).
  * Uses the decode workspace. lowram_decode_step = this + lowram_attend_selected. */
-lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark, const void* q,
-                                   int32_t* sel_out, void* workspace, size_t workspace_bytes,
-                                   void* stream);
+lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark,
+                                   const float* landmark_norm, const void* q, int32_t* sel_out,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Write landmark_norm [B][H_kv] (fp32, rounded up) = max over chunks c of |landmark_c|_2,
+ * summed in fp64, for a cache whose landmarks were produced outside lowram_encode (which
+ * writes the field itself). landmark [B][H_kv][T/C][d] is read only. */
+lowram_status lowram_landmark_norms(lowram_ctx* ctx, const void* landmark, float* landmark_norm,
+                                    void* stream);
 
 /* Decode sub-step 2 (kernel (b) + split-K combine): rebuild the chunks listed in sel
  * ([B][H_kv][k] int32, k = min(top_k, T/C), each entry in 0 .. T/C-1; out-of-range

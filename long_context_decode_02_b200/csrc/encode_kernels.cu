@@ -399,6 +399,44 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// landmark_norm[p] = max over chunks of |L_pc|_2, one warp per row (exact squares, fp64
+// sums), rounded up to fp32 with a margin for the fp64 rounding.
+template <typename T>
+__global__ void __launch_bounds__(256) landmark_norm_kernel(const Dims dm, const T* landmark,
+                                                            float* norm) {
+  const int p = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const T* Lp = landmark + (size_t)p * dm.Nc * dm.d;
+  double best = 0.0;
+  for (int c = warp; c < dm.Nc; c += blockDim.x >> 5) {
+    const T* row = Lp + (size_t)c * dm.d;
+    double ss = 0.0;
+    for (int j = lane; j < dm.d; j += 32) {
+      const double x = ldd(row, j);
+      ss = fma(x, x, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    best = fmax(best, ss);
+  }
+  __shared__ double wmax[8];
+  if (lane == 0) wmax[warp] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = fmax(best, wmax[w]);
+    norm[p] = __double2float_ru(sqrt(best) * (1.0 + 1e-12));
+  }
+}
+
+cudaError_t launch_landmark_norms(const Dims& dm, const void* landmark, float* norm,
+                                  cudaStream_t s) {
+  const int pairs = dm.B * dm.H;
+  if (dm.dtype == LOWRAM_DTYPE_BF16)
+    landmark_norm_kernel<__nv_bfloat16><<<pairs, 256, 0, s>>>(dm, (const __nv_bfloat16*)landmark, norm);
+  else
+    landmark_norm_kernel<float><<<pairs, 256, 0, s>>>(dm, (const float*)landmark, norm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s) {
   const bool bf = a.dm.dtype == LOWRAM_DTYPE_BF16;
   const int D = a.dm.d, FH = a.dm.F;

@@ -25,7 +25,6 @@ struct lowram_ctx {
   int* status;    // device word
   int* counters;  // device [4]: the selection kernel's work, exit and pair counters
   float* scores;   // device [B*H][Nc], all bits set between launches
-  float* norms;    // device [B*H][stages][8], all bits set between launches
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   double* theta64;  // device [d/2]
 };
@@ -148,10 +147,11 @@ lowram_status check_layer_params(const lowram_layer_params* p) {
 
 // res_idx / res_val may be NULL when the configuration keeps no residual rows.
 lowram_status check_cache(const lowram_cache* c, int n_res) {
-  if (!c || !c->coef || !c->landmark || !c->chunk_ptr) return LOWRAM_ERR_INVALID_ARG;
+  if (!c || !c->coef || !c->landmark || !c->chunk_ptr || !c->landmark_norm)
+    return LOWRAM_ERR_INVALID_ARG;
   if (n_res > 0 && (!c->res_idx || !c->res_val)) return LOWRAM_ERR_INVALID_ARG;
   if (!aligned16(c->coef) || !aligned16(c->landmark) || !aligned16(c->res_idx) ||
-      !aligned16(c->res_val) || !aligned16(c->chunk_ptr))
+      !aligned16(c->res_val) || !aligned16(c->chunk_ptr) || !aligned16(c->landmark_norm))
     return LOWRAM_ERR_ALIGN;
   return LOWRAM_OK;
 }
@@ -190,7 +190,7 @@ lowram_status lowram_check_config(const lowram_config* c) {
   return LOWRAM_OK;
 }
 
-lowram_status lowram_cache_layout(const lowram_config* c, size_t bytes_out[5]) {
+lowram_status lowram_cache_layout(const lowram_config* c, size_t bytes_out[6]) {
   if (!bytes_out) return LOWRAM_ERR_INVALID_ARG;
   const lowram_status st = lowram_check_config(c);
   if (st != LOWRAM_OK) return st;
@@ -201,6 +201,7 @@ lowram_status lowram_cache_layout(const lowram_config* c, size_t bytes_out[5]) {
   bytes_out[2] = B * H * (size_t)c->n_res * sizeof(int32_t);
   bytes_out[3] = B * H * (size_t)c->n_res * d * es;
   bytes_out[4] = B * H * (T / c->chunk + 1) * sizeof(int32_t);
+  bytes_out[5] = B * H * sizeof(float);
   return LOWRAM_OK;
 }
 
@@ -258,7 +259,6 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
-            cudaMalloc(&ctx->norms, pairs * 8 * (size_t)select_stages_per_pair(dims_of(*c)) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
   ok = ok &&
        cudaMemcpy(ctx->lo32, lo32.data(), lo32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -269,7 +269,6 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
-       cudaMemset(ctx->norms, 0xff, pairs * 8 * (size_t)select_stages_per_pair(dims_of(*c)) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -290,7 +289,6 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->status);
   cudaFree(ctx->counters);
   cudaFree(ctx->scores);
-  cudaFree(ctx->norms);
   cudaFree(ctx->ready);
   cudaFree(ctx->theta64);
   delete ctx;
@@ -325,7 +323,10 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
   a.in_count = reinterpret_cast<int*>(ws + w.in_count);
   a.rope = rope_of(ctx);
   a.status = ctx->status;
-  const cudaError_t e = launch_encode(a, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_encode(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess)
+    e = launch_landmark_norms(dims_of(c), out->landmark, out->landmark_norm,
+                              static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;
 }
@@ -334,7 +335,8 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
 
 namespace {
 
-lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, int32_t* sel,
+lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const float* landmark_norm,
+                          const void* q, int32_t* sel,
                           uint8_t* ws, const DecodeWs& w, cudaStream_t s, bool set_ready) {
   const Dims dm = dims_of(ctx->cfg);
   SelectArgs sa{};
@@ -342,7 +344,7 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const void* q, 
   sa.landmark = landmark;
   sa.q = q;
   sa.scores = ctx->scores;
-  sa.norms = ctx->norms;
+  sa.landmark_norm = landmark_norm;
   sa.cand_s64 = reinterpret_cast<double*>(ws + w.cand_s64);
   sa.cand_idx = reinterpret_cast<int*>(ws + w.cand_idx);
   sa.flags = ws + w.flags;
@@ -389,18 +391,35 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
 
 extern "C" {
 
-lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark, const void* q,
-                                   int32_t* sel_out, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
-  if (!ctx || !landmark || !q || !sel_out || !workspace) return LOWRAM_ERR_INVALID_ARG;
-  if (!aligned16(landmark) || !aligned16(q) || !aligned16(sel_out) || !aligned16(workspace))
+lowram_status lowram_select_chunks(lowram_ctx* ctx, const void* landmark,
+                                   const float* landmark_norm, const void* q, int32_t* sel_out,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx || !landmark || !landmark_norm || !q || !sel_out || !workspace)
+    return LOWRAM_ERR_INVALID_ARG;
+  if (!aligned16(landmark) || !aligned16(landmark_norm) || !aligned16(q) ||
+      !aligned16(sel_out) || !aligned16(workspace))
     return LOWRAM_ERR_ALIGN;
   const DecodeWs w = decode_ws(ctx->cfg);
   if (workspace_bytes < w.total) return LOWRAM_ERR_WORKSPACE;
   DeviceGuard g(ctx->device);
   if (!g.ok) return LOWRAM_ERR_CUDA;
-  return select_impl(ctx, landmark, q, sel_out, static_cast<uint8_t*>(workspace), w,
-                     static_cast<cudaStream_t>(stream), false);
+  return select_impl(ctx, landmark, landmark_norm, q, sel_out,
+                     static_cast<uint8_t*>(workspace), w, static_cast<cudaStream_t>(stream),
+                     false);
+}
+
+lowram_status lowram_landmark_norms(lowram_ctx* ctx, const void* landmark, float* landmark_norm,
+                                    void* stream) {
+  if (!ctx || !landmark || !landmark_norm) return LOWRAM_ERR_INVALID_ARG;
+  if (!aligned16(landmark) || !aligned16(landmark_norm)) return LOWRAM_ERR_ALIGN;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  if (launch_landmark_norms(dims_of(ctx->cfg), landmark, landmark_norm,
+                            static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
 }
 
 lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
@@ -440,7 +459,9 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + w.sel);
   const bool tc = use_tc(ctx->cfg);
-  if ((st = select_impl(ctx, cache->landmark, q, sel, ws, w, s, tc)) != LOWRAM_OK) return st;
+  if ((st = select_impl(ctx, cache->landmark, cache->landmark_norm, q, sel, ws, w, s, tc)) !=
+      LOWRAM_OK)
+    return st;
   return attend_impl(ctx, cache, params, q, sel, out, ws, w, s, tc);
 }
 

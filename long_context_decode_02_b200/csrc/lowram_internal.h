@@ -44,8 +44,7 @@ struct SelectArgs {
   const void* landmark;   // [B][H][Nc][d]
   const void* q;          // [B][Hq][d]
   float* scores;          // ctx [B*H][Nc], all bits set between launches
-  float* norms;           // ctx [B*H][stages][8]: largest |L|_2 per stage and consumer warp,
-                          // all bits set between launches
+  const float* landmark_norm;  // cache [B*H]: bound of the largest |L|_2 of each pair
   double* cand_s64;       // ws [B*H][Nc]
   int* cand_idx;          // ws [B*H][Nc]
   uint8_t* flags;         // ws [B*H][Nc]
@@ -55,6 +54,9 @@ struct SelectArgs {
   int* status;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
+// landmark_norm[p] = max_c |landmark[p][c]|_2 rounded up to fp32 (fp64 sums).
+cudaError_t launch_landmark_norms(const Dims& dm, const void* landmark, float* norm,
+                                  cudaStream_t s);
 // Stages of landmark rows per (b, h) in the selection kernel: a stage is
 // min(65536 / row bytes, 256) rows.
 __host__ __device__ inline int select_stages_per_pair(const Dims& dm) {

@@ -15,9 +15,7 @@
 //    score one row each (packed fp32x2 FMAs) and write the fp32 score.
 //  * Scores live in a context-owned buffer that holds a sentinel bit pattern between
 //    launches (0xFFFFFFFF, a NaN that fp32 arithmetic never produces), so a written score
-//    is its own completion flag: no counters or memory fences on the streaming path. Each
-//    consumer warp also writes the largest |L|_2 of its rows in each stage to a second
-//    sentinel-initialised buffer (the norms bound the fp32 error below).
+//    is its own completion flag: no counters or memory fences on the streaming path.
 //    Three selection warps per CTA take (b, h) pairs in order from a global counter,
 //    wait until the work counter has handed out all of the pair's stages and every score
 //    has landed, select, and put the sentinel back. Selections are spread over the CTAs
@@ -30,8 +28,9 @@
 //    are re-scored in fp64 (exact products, fp64 sums) and ranked by (score desc, index
 //    asc). delta is twice a rigorous bound on the fp32 score error: an fp32 dot product of
 //    D terms accumulated with fused multiply-adds is within gamma_D * sum|q_i L_i| <=
-//    gamma_D * |q|_2 |L|_2 of the exact value (gamma_n = n u / (1 - n u), u = 2^-24). So the
-//    result equals the selection made in fp64, and the window usually holds exactly the
+//    gamma_D * |q|_2 |L|_2 of the exact value (gamma_n = n u / (1 - n u), u = 2^-24), with
+//    |L|_2 bounded by the cache's per-pair landmark norm. So the result equals the
+//    selection made in fp64, and the window usually holds exactly the
 //    rows still needed, which then need no re-scoring. When the candidate set cannot be proven to
 //    hold the answer, a radix select over all scores decides instead. The chunk ids are
 //    written in ascending order.
@@ -238,7 +237,8 @@ template <int D>
 __device__ __forceinline__ double score_error_window(double qmax, double lmax) {
   const double u = 5.9604644775390625e-8;   // 2^-24
   const double gam = D * u / (1.0 - D * u);
-  return 2.0 * (gam * 1.001 + 1e-12) * qmax * lmax + 1e-300;
+  const double w = 2.0 * (gam * 1.001 + 1e-12) * qmax * lmax + 1e-300;
+  return w < INFINITY ? w : INFINITY;   // non-finite inputs: everything is in the window
 }
 
 template <typename T, int D, int G>
@@ -269,10 +269,7 @@ __device__ void select_pair_radix(const Grp& g, const SelectArgs& a, int p, Misc
   const T* qb = (const T*)a.q + ((size_t)b * dm.Hq + (size_t)h * G) * D;
   const T* L = (const T*)a.landmark + (size_t)p * Nc * D;
 
-  const int n_norm = 8 * select_stages_per_pair(dm);
-  float lmax = 0.f;
-  for (int i = g.tid; i < n_norm; i += g.nt) lmax = fmaxf(lmax, __ldcg(a.norms + (size_t)p * n_norm + i));
-  lmax = group_max(g, lmax, ms->fscr);
+  const float lmax = __ldg(a.landmark_norm + p);
   float qr[G][D / 32];
   load_q_slice<T, D, G>(qb, g.tid & 31, qr);
   const uint32_t tk = group_kth_largest(
@@ -443,25 +440,6 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
   const int nw = (Nc + 31) >> 5;
   for (int i = g.tid; i < nw; i += g.nt) bits[i] = 0u;
   bool good = true;
-  // largest |L|_2 of the pair, from the consumer warps' per-stage maxima
-  float lmax = 0.f;
-  {
-    const int n_norm = 8 * select_stages_per_pair(dm);
-    const uint32_t* nu = reinterpret_cast<const uint32_t*>(a.norms + (size_t)p * n_norm);
-    for (int base = 0; base < n_norm; base += kB * g.nt) {
-      int idx[kB];
-      uint32_t want = 0, v[kB];
-#pragma unroll
-      for (int j = 0; j < kB; ++j) {
-        idx[j] = base + j * g.nt + g.tid;
-        if (idx[j] < n_norm) want |= 1u << j;
-      }
-      good = good && poll_words<kB>(nu, idx, want, v, abort, t_start);
-#pragma unroll
-      for (int j = 0; j < kB; ++j)
-        if ((want >> j) & 1u) lmax = fmaxf(lmax, __uint_as_float(v[j]));
-    }
-  }
   int m;
   float t0 = -INFINITY;
   const bool sampled = Nc > kCap;
@@ -567,8 +545,6 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
     }
     if (!good) ms->n_in = -1;
   }
-  lmax = warp_max(lmax);
-  if (lane == 0) atomicMax(reinterpret_cast<int*>(&ms->fmax), __float_as_int(lmax));
   g.sync();
   if (ms->n_in < 0) return -1;
   if (sampled) {
@@ -578,7 +554,7 @@ __device__ int select_pair_fast(const Grp& g, const SelectArgs& a, int p, float*
   const uint32_t tp = kth_largest_prefix<3>(g, m, k, [&](int i) { return f2key(ckey[i]); }, ms);
   const double tau_lo = (double)key2f(tp), tau_hi = (double)key2f(tp | 0xFFu);
   if (!(tau_lo <= tau_hi)) return 0;   // a non-finite bucket
-  const double delta = score_error_window<D>(qmax, (double)ms->fmax);
+  const double delta = score_error_window<D>(qmax, (double)__ldg(a.landmark_norm + p));
   const double hi = tau_hi + delta, lo = tau_lo - delta;
   if (sampled && (double)t0 > lo) return 0;   // the window may reach below the filter
   // classify: clearly in -> bitmap; window -> list (warp-aggregated counts)
@@ -662,10 +638,7 @@ __device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* cke
   if (k < Nc && k <= kCap / 2 && Nc <= kBitmapChunks) {
     r = select_pair_fast<T, D, G>(g, a, p, ckey, cid, bits, ms, abort);
   } else {
-    const int n_norm = 8 * select_stages_per_pair(a.dm);   // every score and norm, before use
-    if (!wait_scores(g, su, Nc, abort) ||
-        !wait_scores(g, reinterpret_cast<const uint32_t*>(a.norms + (size_t)p * n_norm), n_norm, abort))
-      ms->n_in = -1;
+    if (!wait_scores(g, su, Nc, abort)) ms->n_in = -1;   // every score, before any is used
     g.sync();
     r = ms->n_in < 0 ? -1 : 0;
     if (r == 0 && k >= Nc) {
@@ -683,12 +656,11 @@ __device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* cke
 }
 
 // ---------------------------------------------------------------- scoring
-// {score, |L|_2} of landmark row r of a swizzled stage.
+// Score of landmark row r of a swizzled stage.
 template <typename T, int D, int G>
-__device__ __forceinline__ float2 score_row(const uint8_t* stage, int r, const float* sQ) {
+__device__ __forceinline__ float score_row(const uint8_t* stage, int r, const float* sQ) {
   using Gm = Geom<T, D>;
   float2 acc[G];
-  float2 nn = make_float2(0.f, 0.f);
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
 #pragma unroll
@@ -699,10 +671,6 @@ __device__ __forceinline__ float2 score_row(const uint8_t* stage, int r, const f
     if constexpr (sizeof(T) == 2) {
       // 8 bf16: chunk c holds dims 8c .. 8c+7
       const float2 v0 = bf2_to_f2(w.x), v1 = bf2_to_f2(w.y), v2 = bf2_to_f2(w.z), v3 = bf2_to_f2(w.w);
-      nn = __ffma2_rn(v0, v0, nn);
-      nn = __ffma2_rn(v1, v1, nn);
-      nn = __ffma2_rn(v2, v2, nn);
-      nn = __ffma2_rn(v3, v3, nn);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c);
@@ -716,8 +684,6 @@ __device__ __forceinline__ float2 score_row(const uint8_t* stage, int r, const f
       // 4 fp32: chunk c holds dims 4c .. 4c+3
       const float2 v0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
       const float2 v1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
-      nn = __ffma2_rn(v0, v0, nn);
-      nn = __ffma2_rn(v1, v1, nn);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 4 * c);
@@ -729,7 +695,7 @@ __device__ __forceinline__ float2 score_row(const uint8_t* stage, int r, const f
   float best = acc[0].x + acc[0].y;
 #pragma unroll
   for (int g = 1; g < G; ++g) best = fmaxf(best, acc[g].x + acc[g].y);
-  return make_float2(best, sqrtf(nn.x + nn.y));
+  return best;
 }
 
 template <typename T, int D, int G>
@@ -870,14 +836,9 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (u < 0) break;
       const int pair = u / upp, st = u % upp;
       const int c = st * Gm::kLps + tid;
-      float nrm = 0.f;
-      if (tid < Gm::kLps && c < Nc) {
-        const float2 r = score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
-        a.scores[(size_t)pair * Nc + c] = r.x;
-        nrm = r.y;
-      }
-      nrm = warp_max(nrm);   // this warp's largest |L|_2 in the stage
-      if (lane == 0) a.norms[((size_t)pair * upp + st) * 8 + warp] = nrm;
+      if (tid < Gm::kLps && c < Nc)
+        a.scores[(size_t)pair * Nc + c] =
+            score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
     }
@@ -900,7 +861,6 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (pair < 0) break;
       if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) break;
       clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
-      clear_scores(g, reinterpret_cast<uint32_t*>(a.norms + (size_t)pair * upp * 8), upp * 8);
       if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
         __threadfence();
         st_release(a.ready + pair, 1);
@@ -927,7 +887,6 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
   if (ms->req) {
     const Grp all{(int)threadIdx.x, (int)blockDim.x, 0};
     clear_scores(all, reinterpret_cast<uint32_t*>(a.scores), P * Nc);
-    clear_scores(all, reinterpret_cast<uint32_t*>(a.norms), P * upp * 8);
   }
 }
 

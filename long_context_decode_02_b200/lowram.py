@@ -62,7 +62,7 @@ class lowram_layer_params(ctypes.Structure):
 class lowram_cache(ctypes.Structure):
     _fields_ = [("coef", ctypes.c_void_p), ("landmark", ctypes.c_void_p),
                 ("res_idx", ctypes.c_void_p), ("res_val", ctypes.c_void_p),
-                ("chunk_ptr", ctypes.c_void_p)]
+                ("chunk_ptr", ctypes.c_void_p), ("landmark_norm", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -79,7 +79,8 @@ _sig = {
     "lowram_decode_step": (_S, [_P, ctypes.POINTER(lowram_cache),
                                 ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P,
                                 ctypes.c_size_t, _P]),
-    "lowram_select_chunks": (_S, [_P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_select_chunks": (_S, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_landmark_norms": (_S, [_P, _P, _P, _P]),
     "lowram_attend_selected": (_S, [_P, ctypes.POINTER(lowram_cache),
                                     ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P,
                                     ctypes.c_size_t, _P]),
@@ -140,7 +141,7 @@ def _stream(stream):
 
 
 def cache_layout(cfg: lowram_config):
-    out = (ctypes.c_size_t * 5)()
+    out = (ctypes.c_size_t * 6)()
     check(lowram_cache_layout(ctypes.byref(cfg), out), "lowram_cache_layout")
     return list(out)
 
@@ -186,9 +187,9 @@ def layer_params(basis, w1, b1, w2, b2) -> lowram_layer_params:
     return p
 
 
-def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr) -> lowram_cache:
+def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr, landmark_norm) -> lowram_cache:
     return lowram_cache(_ptr(coef), _ptr(landmark), _ptr(res_idx), _ptr(res_val),
-                        _ptr(chunk_ptr))
+                        _ptr(chunk_ptr), _ptr(landmark_norm))
 
 
 def alloc_cache(cfg: lowram_config, device):
@@ -203,6 +204,7 @@ def alloc_cache(cfg: lowram_config, device):
         "res_idx": torch.empty(B, H, cfg.n_res, dtype=torch.int32, device=device),
         "res_val": torch.empty(B, H, cfg.n_res, d, dtype=dt, device=device),
         "chunk_ptr": torch.empty(B, H, nc + 1, dtype=torch.int32, device=device),
+        "landmark_norm": torch.empty(B, H, dtype=torch.float32, device=device),
     }
 
 
@@ -233,10 +235,18 @@ def decode_step_static(ctx: Context, cache: dict, params: lowram_layer_params, q
           "lowram_decode_step_static")
 
 
-def select_chunks(ctx: Context, landmark, q, sel_out, workspace, stream=None) -> None:
-    check(lowram_select_chunks(ctx.handle, _ptr(landmark), _ptr(q), _ptr(sel_out),
-                               _ptr(workspace), workspace.numel() * workspace.element_size(),
-                               _stream(stream)), "lowram_select_chunks")
+def select_chunks(ctx: Context, landmark, landmark_norm, q, sel_out, workspace,
+                  stream=None) -> None:
+    check(lowram_select_chunks(ctx.handle, _ptr(landmark), _ptr(landmark_norm), _ptr(q),
+                               _ptr(sel_out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_select_chunks")
+
+
+def landmark_norms(ctx: Context, landmark, out, stream=None) -> None:
+    """lowram_landmark_norms: out [B][H_kv] fp32 = max_c |landmark_c|_2, rounded up."""
+    check(lowram_landmark_norms(ctx.handle, _ptr(landmark), _ptr(out), _stream(stream)),
+          "lowram_landmark_norms")
 
 
 def attend_selected(ctx: Context, cache: dict, params: lowram_layer_params, q, sel, out,

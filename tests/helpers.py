@@ -49,6 +49,18 @@ def oracle_encode(shape, t):
                     store=STORE[shape.dtype])
 
 
+def landmark_norm_bound(landmark):
+    """The cache's landmark_norm field for host-built caches: max over chunks of |L_c|_2
+    per (b, h), fp64 sums, times (1 + 1e-12), rounded up to fp32 (the definition in
+    include/lowram.h, written out)."""
+    lm = np.asarray(landmark, dtype=np.float64)
+    n = np.sqrt(np.max(np.sum(lm * lm, axis=-1), axis=-1)) * (1.0 + 1e-12)
+    n32 = n.astype(np.float32)
+    up = n32.astype(np.float64) < n
+    n32[up] = np.nextafter(n32[up], np.float32(np.inf))
+    return n32
+
+
 def cache_to_device(shape, cache, device):
     st = shape.torch_dtype
 
@@ -60,6 +72,7 @@ def cache_to_device(shape, cache, device):
         "res_idx": dense(cache["res_idx"], torch.int32),
         "res_val": dense(cache["res_val"], st),
         "chunk_ptr": dense(cache["chunk_ptr"], torch.int32),
+        "landmark_norm": dense(landmark_norm_bound(cache["landmark"]), torch.float32),
     }
 
 

@@ -69,7 +69,7 @@ def test_cache_layout_and_workspace(L):
     B, T, H, d, r = 1, 32768, 8, 128, 160
     n_res = int(0.2 * T)
     assert sizes == [B * T * r * 2, B * H * (T // 8) * d * 2, B * H * n_res * 4,
-                     B * H * n_res * d * 2, B * H * (T // 8 + 1) * 4]
+                     B * H * n_res * d * 2, B * H * (T // 8 + 1) * 4, B * H * 4]
     for op in (L.OP_ENCODE, L.OP_DECODE):
         assert L.workspace_size(c, op) > 0
     n = ctypes.c_size_t()

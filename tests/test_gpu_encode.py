@@ -61,6 +61,13 @@ def check_encode(L, shape, device):
         g, w = H.f64(cache[name]), enc[name]
         bound = ulp_bound(w, shape.dtype) * 1.01 + 1e-6 * np.abs(w).max()
         assert np.all(np.abs(g - w) <= bound), (name, float(np.max(np.abs(g - w) - bound)))
+    # landmark_norm: an upper bound of max_c |L_c|_2 of the stored landmarks, within two
+    # fp32 steps of the definition written out on the host
+    got_n = cache["landmark_norm"].cpu().numpy().astype(np.float64)
+    lm = H.f64(cache["landmark"])
+    exact = np.sqrt(np.max(np.sum(lm * lm, axis=-1), axis=-1))
+    assert np.all(got_n >= exact)
+    assert np.all(got_n <= H.landmark_norm_bound(lm).astype(np.float64) * (1 + 2.0 ** -22))
     # residual rows: R = V - MLP_h(B_h coef_stored) against the coefficients this side
     # stored (which may differ from the oracle's by one rounding), exact in fp64, then
     # compared with the stored row within one rounding step
