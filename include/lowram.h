@@ -234,7 +234,10 @@ const char* lowram_status_string(lowram_status status);
  *   mode 0: K % 32 == 0, 32 <= K <= 256; a and b TMA-loaded with the 64-byte swizzle
  *           (a in 8-row boxes like the gathered coefficients, b like the basis);
  *   mode 1: K == 128; a TMA-loaded with the 128-byte swizzle (like W1), b stored by
- *           threads in the 128-byte-swizzled layout (like the rebuilt keys).
+ *           threads in the 128-byte-swizzled layout (like the rebuilt keys);
+ *   mode 2: K == 128; a stored by threads into Tensor Memory (row m in lane m, two bf16
+ *           per column) and used as the MMA's A operand, b rows 0..15 stored by threads
+ *           with the 128-byte swizzle; only d[m][0..15] is written.
  * Synchronous: returns after the kernel finished. */
 lowram_status lowram_debug_tc_tile(const void* a, const void* b, float* d, int32_t k,
                                    int32_t mode, void* stream);

@@ -669,10 +669,13 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 // d[m][n] = sum_k a[m][k] b[n][k]. mode 0: both operands TMA-loaded with the 64B swizzle
 // exactly as coef (8-row boxes) and basis (128-row boxes) in the decode kernel; mode 1:
 // a TMA-loaded with the 128B swizzle like W1, b written by threads with the 128B swizzle
-// like K~bf16 (K = 128).
+// like K~bf16 (K = 128); mode 2: a (128 x 128) written by threads into TMEM as bf16
+// pairs and read by the MMA from there, b (16 x 128) written by threads with the 128B
+// swizzle, D = 128 x 16.
 __global__ void __launch_bounds__(128, 1)
 debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_constant__ CUtensorMap mb,
-                     const __nv_bfloat16* bsrc, float* d, int K, int mode, int* status) {
+                     const __nv_bfloat16* asrc, const __nv_bfloat16* bsrc, float* d, int K,
+                     int mode, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = align_up(raw, 1024);
@@ -706,10 +709,37 @@ debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_consta
     }
     fence_proxy_async_smem();
   }
+  if (mode == 2) {
+    // a row m = threadIdx.x -> TMEM lane m, columns 0..63 (two bf16 per column)
+    const uint32_t* arow = reinterpret_cast<const uint32_t*>(asrc + (size_t)threadIdx.x * 128);
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[16];
+      for (int j = 0; j < 16; ++j) v[j] = arow[16 * c + j];
+      tmem_st_x16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)(16 * c), v);
+    }
+    tmem_wait_st();
+    // b rows 0..15, 128B-swizzled K-major, two 64-wide K blocks of 16 rows
+    if (threadIdx.x < 16) {
+      const int n = threadIdx.x;
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(bsrc + (size_t)n * 128 + 8 * c);
+        st_shared_v4(sb + (c >> 3) * 2048 + sw128_offset(n, c & 7), v.x, v.y, v.z, v.w);
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
-    bool ok;
-    if (mode == 0) {
+    bool ok = true;
+    if (mode == 2) {
+      tc_fence_after();
+      for (int s = 0; s < 8; ++s)
+        mma_bf16_ta(tmem + 64u, tmem + (uint32_t)(8 * s),
+                    smem_desc_kmajor(sb + (uint32_t)((s >> 2) * 2048 + (s & 3) * 32), 1024,
+                                     kSwizzle128B),
+                    idesc_bf16_f32(128, 16), s > 0);
+    } else if (mode == 0) {
       mbar_arrive_expect_tx(barf, (uint32_t)(2 * kb32 * 8192));
       for (int kb = 0; kb < kb32; ++kb) {
         for (int c = 0; c < 16; ++c) tma_load_2d(sa + kb * 8192 + c * 512, &ma, kb * 32, c * 8, barf);
@@ -719,8 +749,8 @@ debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_consta
       mbar_arrive_expect_tx(barf, 2u * 16384u);
       for (int kb = 0; kb < 2; ++kb) tma_load_2d(sa + kb * 16384, &ma, kb * 64, 0, barf);
     }
-    ok = mbar_wait_bounded(barf, 0, abort_flag);
-    if (ok) {
+    if (mode != 2) ok = mbar_wait_bounded(barf, 0, abort_flag);
+    if (ok && mode != 2) {
       tc_fence_after();
       if (mode == 0) {
         for (int s = 0; s < K / 16; ++s) {
@@ -742,7 +772,12 @@ debug_tc_tile_kernel(const __grid_constant__ CUtensorMap ma, const __grid_consta
   }
   __syncthreads();
   tc_fence_after();
-  if (!*abort_flag) {
+  if (!*abort_flag && mode == 2) {
+    float v[32];
+    tmem_ld_x32(tmem + ((uint32_t)(32 * warp) << 16) + 64u, v);
+    tmem_wait_ld();
+    for (int e = 0; e < 16; ++e) d[(size_t)threadIdx.x * 128 + e] = v[e];
+  } else if (!*abort_flag) {
     const int m = threadIdx.x;  // warp w reads lanes 32w..32w+31
     for (int c = 0; c < 4; ++c) {
       float v[32];
@@ -810,7 +845,10 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
 cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, int mode,
                                  int* status, cudaStream_t s) {
   CUtensorMap ma, mb;
-  if (mode == 0) {
+  if (mode == 2) {
+    memset(&ma, 0, sizeof(ma));
+    mb = ma;
+  } else if (mode == 0) {
     if (!make_tensor_map_2d(&ma, a, LOWRAM_DTYPE_BF16, (uint64_t)k, 128, 32, 8, 64) ||
         !make_tensor_map_2d(&mb, b, LOWRAM_DTYPE_BF16, (uint64_t)k, 128, 32, 128, 64))
       return cudaErrorInvalidValue;
@@ -823,7 +861,8 @@ cudaError_t launch_debug_tc_tile(const void* a, const void* b, float* d, int k, 
   cudaError_t e = cudaFuncSetAttribute(debug_tc_tile_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  debug_tc_tile_kernel<<<1, 128, smem, s>>>(ma, mb, (const __nv_bfloat16*)b, d, k, mode, status);
+  debug_tc_tile_kernel<<<1, 128, smem, s>>>(ma, mb, (const __nv_bfloat16*)a,
+                                            (const __nv_bfloat16*)b, d, k, mode, status);
   return cudaGetLastError();
 }
 

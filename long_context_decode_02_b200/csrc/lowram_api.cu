@@ -501,8 +501,8 @@ lowram_status lowram_debug_tc_tile(const void* a, const void* b, float* d, int32
   if (!a || !b || !d) return LOWRAM_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return LOWRAM_ERR_ALIGN;
   if (mode == 0 && (k % 32 != 0 || k < 32 || k > 256)) return LOWRAM_ERR_UNSUPPORTED;
-  if (mode == 1 && k != 128) return LOWRAM_ERR_UNSUPPORTED;
-  if (mode != 0 && mode != 1) return LOWRAM_ERR_INVALID_ARG;
+  if ((mode == 1 || mode == 2) && k != 128) return LOWRAM_ERR_UNSUPPORTED;
+  if (mode < 0 || mode > 2) return LOWRAM_ERR_INVALID_ARG;
   int* st = nullptr;
   if (cudaMalloc(&st, sizeof(int)) != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
