@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
   const int n = a.n_tiles;
   const size_t tstride = (size_t)G * 2 + (size_t)G * FH + 2 * (size_t)G * D;
   if (a.ready && g == 0 && threadIdx.x == 0) a.ready[p] = 0;   // the next step's flags
+  if (a.item_ctr && p < dm.H && g == 0 && threadIdx.x == 0) a.item_ctr[p] = 0;   // tile counters
   const float* part = a.part + (size_t)p * n * tstride;
   __shared__ float hs[FH];
   __shared__ float rs[2][D];

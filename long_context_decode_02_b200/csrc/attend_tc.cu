@@ -60,7 +60,8 @@ struct TcMaps {
 struct TileMeta {
   int cid[kChunksPerTile];  // chunk id of each slot of the tile; -1 past the selection
   int nres;                 // residual rows of the tile
-  int pad[3];
+  int item;                 // b * n_tiles + tile; -1: this CTA has no more tiles
+  int pad[2];
   uint32_t res[kTile];      // (row of res_val) << 8 | token row in the tile (255 = skip)
   uint4 q[64];              // the tile's G = 4 query rows, bf16 [4][128]
 };
@@ -133,7 +134,7 @@ __device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
 
 template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
-attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int cta_per_head) {
+attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   const Dims& dm = a.dm;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -141,13 +142,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   uint8_t* gbase = smem_raw + (base - raw);
   const Layout L = make_layout(dm.r);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x / cta_per_head;
-  const int cta_in_head = blockIdx.x % cta_per_head;
+  // KV heads interleaved over the grid, so CTAs that start early (beside a still running
+  // selection kernel) serve every head; each head's tiles are taken from its counter
+  const int h = blockIdx.x % dm.H;
   const int n_items = dm.B * a.n_tiles;
   const int kb_r = dm.r / 32;
   const int ksteps_r = dm.r / 16;
-  int n_mine = 0;
-  for (int it = cta_in_head; it < n_items; it += cta_per_head) ++n_mine;
 
   auto bar = [&](int i) { return base + L.bar + 8u * (uint32_t)i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + L.bar + 8 * BAR_COUNT);
@@ -161,8 +161,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
   float2* sRot = reinterpret_cast<float2*>(gbase + L.rot);
   float2* sRoff = reinterpret_cast<float2*>(gbase + L.roff);
 
-  auto item_of = [&](int i, int& b, int& tile) {
-    const int it = cta_in_head + i * cta_per_head;
+  auto item_of = [&](int it, int& b, int& tile) {
     b = it / a.n_tiles;
     tile = it % a.n_tiles;
   };
@@ -215,15 +214,18 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
           tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
                       h * kF + hf * 128, bar(BAR_W));
     }
-    for (int i = 0; i < n_mine; ++i) {
-      int b, tile;
-      item_of(i, b, tile);
+    for (int i = 0;; ++i) {
       const int slot = i % kMetaSlots;
-      int got = 0;
-      if (lane == 0)
-        got = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag) &&
-              mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
-      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      int got = 0, it = -1;
+      if (lane == 0) {
+        got = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
+        it = got ? meta[slot].item : -1;
+        if (it >= 0) got = mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
+      }
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (!__shfl_sync(0xffffffffu, got, 0) || it < 0) break;
+      int b, tile;
+      item_of(it, b, tile);
       const int cid = lane < kChunksPerTile ? meta[slot].cid[lane] : -1;
       if (lane == 0)
         mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
@@ -251,9 +253,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
     const int32_t* ridx_all = a.res_idx;
     // theta_i for this lane's pairs (lane, lane + 32)
     const double th0 = a.rope.theta64[lane], th1 = a.rope.theta64[lane + 32];
-    auto load_cid = [&](int i) -> int {
+    auto load_cid = [&](int it) -> int {
       int b, tile;
-      item_of(i, b, tile);
+      item_of(it, b, tile);
       if (a.wait_ready) {   // the selection kernel may still be running: wait for this pair
         int ok = 1;
         if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
@@ -266,17 +268,36 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       }
       return cid;
     };
-    int cid_next = n_mine > 0 ? load_cid(0) : -1;
-    for (int i = 0; i < n_mine; ++i) {
-      int b, tile;
-      item_of(i, b, tile);
+    // tiles come from this head's counter, one taken ahead
+    auto take = [&]() -> int {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(a.item_ctr + h, 1);
+      return __shfl_sync(0xffffffffu, it, 0);
+    };
+    int it_next = take();
+    int cid_next = it_next < n_items ? load_cid(it_next) : -1;
+    for (int i = 0;; ++i) {
+      const int it = it_next;
       const int slot = i % kMetaSlots;
+      if (it >= n_items) {   // no more tiles: post the end marker
+        int got = 0;
+        if (lane == 0)
+          got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
+        if (__shfl_sync(0xffffffffu, got, 0) && lane == 0) {
+          meta[slot].item = -1;
+          mbar_arrive(bar(BAR_META_FULL0 + slot));
+        }
+        break;
+      }
+      int b, tile;
+      item_of(it, b, tile);
       const int p = b * dm.H + h;
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
       const uint4 q0 = qsrc[lane], q1 = qsrc[lane + 32];
       int cid = cid_next;
-      if (i + 1 < n_mine) cid_next = load_cid(i + 1);
+      it_next = take();
+      if (it_next < n_items) cid_next = load_cid(it_next);
       if (lane < kChunksPerTile && cid >= dm.Nc) {
         raise_status(a.status, kStatusDeviceCheck);
         cid = -1;
@@ -328,7 +349,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
           }
         }
       }
-      if (lane == 0) M->nres = total;
+      if (lane == 0) {
+        M->nres = total;
+        M->item = it;
+      }
       M->q[lane] = q0;
       M->q[lane + 32] = q1;
       __syncwarp();
@@ -399,9 +423,18 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
         mma_commit(bar(BAR_KBF_EMPTY));
         return true;
       };
-      if (ok && n_mine > 0) ok = issue_k(0);
-      for (int i = 0; ok && i < n_mine; ++i) {
-        if (i + 1 < n_mine) ok = issue_k(i + 1);
+      // whether tile i exists, from its metadata slot (read before the slot can recycle)
+      auto exists = [&](int i) -> bool {
+        const int slot = i % kMetaSlots;
+        if (!mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag))
+          return false;
+        return meta[slot].item >= 0;
+      };
+      bool more = ok && exists(0);
+      if (more) ok = issue_k(0);
+      for (int i = 0; ok && more; ++i) {
+        more = exists(i + 1);
+        if (more) ok = issue_k(i + 1);
         if (ok) ok = issue_h(i);
       }
       // drain every MMA this thread issued before TMEM is released
@@ -428,16 +461,51 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       sRoff[i] = a.rope.lo32[(i & (kChunk - 1)) * (kD / 2) + (i >> 3)];
     bool ok = true;
 
+    // Residual rows of a tile, first kResPrefetch of this thread's: row entries (token row
+    // byte, 255 = none) and raw bf16 values, packed. Loaded while the previous part runs
+    // (at the start of part A of the next tile, or of part B for the last tile) so the
+    // random HBM reads overlap work.
+    uint32_t pre_row[kResPrefetch / 4], pre_val[kResPrefetch / 2];
+    auto prefetch_res = [&](int i) {
+      const TileMeta* M = meta + i % kMetaSlots;
+      int b, tile;
+      item_of(M->item, b, tile);
+      const int nres = M->nres;
+      const __nv_bfloat16* rbase = rval_all + (size_t)(b * dm.H + h) * dm.n_res * kD + trow;
+#pragma unroll
+      for (int w = 0; w < kResPrefetch / 4; ++w) pre_row[w] = 0xFFFFFFFFu;
+#pragma unroll
+      for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
+#pragma unroll
+      for (int v = 0; v < kResPrefetch; ++v) {
+        const int ei = hf + 2 * v;
+        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
+        const uint32_t row = ent & 255u;
+        pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
+        if (row != 255u) {
+          const uint32_t raw =
+              __ldg(reinterpret_cast<const unsigned short*>(rbase + (size_t)(ent >> 8) * kD));
+          pre_val[v >> 1] |= raw << (16 * (v & 1));
+        }
+      }
+    };
+
     // A failed (timed-out) wait never changes the sequence of named barriers: the
     // thread carries on with `good` false so every barrier is still reached.
-    // ---- part A of tile i
+    // ---- part A of tile i; false when the tile does not exist (the end marker) or a wait
+    // gave up, decided by one vote of all epilogue threads
     auto part_a = [&](int i) -> bool {
+      if (i > 0) prefetch_res(i - 1);   // for part B of the previous tile
       const int u = i & 1;
       const int slot = i % kMetaSlots;
       const TileMeta* M = meta + slot;
       bool good = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
+      // the vote is also the barrier after which the previous readers of sQ / sZx are done
+      if (named_bar_red_or(1, kEpiThreads, !good || M->item < 0)) {
+        if (!good) *abort_flag = 1;
+        return false;
+      }
       const bool valid = M->cid[trow >> 3] >= 0;
-      named_bar_sync(1, kEpiThreads);  // previous readers of sQ / sZx are done
       {
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
         const float2 f = bf2_to_f2(w);
@@ -553,27 +621,18 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 
     // ---- part B of tile i
     auto part_b = [&](int i) -> bool {
-      int b, tile;
-      item_of(i, b, tile);
       const int u = i & 1;
       const int slot = i % kMetaSlots;
       const TileMeta* M = meta + slot;
+      int b, tile;
+      item_of(M->item, b, tile);
       const int p = b * dm.H + h;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
       // residual rows of the tile: thread = column j; rows split between the two halves.
-      // The first kResPrefetch of this thread's rows are loaded before the hidden layer.
+      // The first kResPrefetch of this thread's rows were loaded earlier (prefetch_res).
       const int j = trow;
       const int nres = M->nres;
       const __nv_bfloat16* rbase = rval_all + (size_t)p * dm.n_res * kD + j;
-      float rv[kResPrefetch];
-      int rrow[kResPrefetch];
-#pragma unroll
-      for (int v = 0; v < kResPrefetch; ++v) {
-        const int ei = hf + 2 * v;
-        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
-        rrow[v] = (int)(ent & 255u);
-        rv[v] = rrow[v] != 255 ? __bfloat162float(rbase[(size_t)(ent >> 8) * kD]) : 0.f;
-      }
       const bool good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag);
       tc_fence_after();
       const int f = 128 * hf + trow;
@@ -619,12 +678,14 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int v = 0; v < kResPrefetch; ++v) {
-        if (rrow[v] == 255) continue;
-        const float4 pv = P4[rrow[v]];
-        racc[0] = fmaf(pv.x, rv[v], racc[0]);
-        racc[1] = fmaf(pv.y, rv[v], racc[1]);
-        racc[2] = fmaf(pv.z, rv[v], racc[2]);
-        racc[3] = fmaf(pv.w, rv[v], racc[3]);
+        const uint32_t row = (pre_row[v >> 2] >> (8 * (v & 3))) & 255u;
+        if (row == 255u) continue;
+        const float4 pv = P4[row];
+        const float r = __uint_as_float(((pre_val[v >> 1] >> (16 * (v & 1))) & 0xFFFFu) << 16);
+        racc[0] = fmaf(pv.x, r, racc[0]);
+        racc[1] = fmaf(pv.y, r, racc[1]);
+        racc[2] = fmaf(pv.z, r, racc[2]);
+        racc[3] = fmaf(pv.w, r, racc[3]);
       }
       for (int ei = hf + 2 * kResPrefetch; ei < nres; ei += 2) {   // rows beyond the prefetch
         const uint32_t ent = M->res[ei];
@@ -648,10 +709,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps, int ct
 
     // Every epilogue thread runs the full sequence; once the abort flag is set, the
     // remaining waits return at once and the results are discarded by the caller.
-    if (n_mine > 0) ok = part_a(0) && ok;
-    for (int i = 0; i < n_mine; ++i) {
-      if (i + 1 < n_mine) ok = part_a(i + 1) && ok;
+    bool more = part_a(0);
+    for (int i = 0; more; ++i) {
+      const bool next = part_a(i + 1);   // or the end marker (it also prefetches for B(i))
       ok = part_b(i) && ok;
+      more = next;
     }
     if (!ok) *abort_flag = 1;
   }
@@ -837,7 +899,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.wait_ready ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, a, maps, cph);
+  e = cudaLaunchKernelEx(&cfg, kern, a, maps);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

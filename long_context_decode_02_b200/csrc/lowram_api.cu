@@ -26,6 +26,7 @@ struct lowram_ctx {
   int* counters;  // device [4]: the selection kernel's work, exit and pair counters
   float* scores;   // device [B*H][Nc], all bits set between launches
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
+  int* item_ctr;  // device [H]: tile counters of the tcgen05 attend kernel, 0 between calls
   double* theta64;  // device [d/2]
 };
 
@@ -258,6 +259,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->status, sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->item_ctr, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
   ok = ok &&
@@ -268,6 +270,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->status, 0, sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
+       cudaMemset(ctx->item_ctr, 0, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
@@ -290,6 +293,7 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->counters);
   cudaFree(ctx->scores);
   cudaFree(ctx->ready);
+  cudaFree(ctx->item_ctr);
   cudaFree(ctx->theta64);
   delete ctx;
 }
@@ -381,6 +385,7 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   // right after the selection kernel the tcgen05 kernel overlaps its tail, pair by pair
   aa.ready = tc && after_select ? ctx->ready : nullptr;
   aa.wait_ready = aa.ready ? 1 : 0;
+  aa.item_ctr = tc ? ctx->item_ctr : nullptr;
   cudaError_t e = tc ? launch_attend_tc(aa, ctx->num_sms, s) : launch_attend_simt(aa, s);
   if (e == cudaSuccess) e = launch_combine(aa, tc, s);
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }

@@ -86,6 +86,8 @@ struct AttendArgs {
   int* ready;             // ctx [B*H] or null: per-pair selection flags; combine clears them
   int wait_ready;         // 1: launched as a programmatic dependent of the selection
                           // kernel; wait for ready[pair] before reading its selection
+  int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); combine
+                          // clears them
 };
 size_t attend_simt_part_floats(const Dims& dm, int n_tiles);
 int attend_simt_tile_tokens(const Dims& dm);
