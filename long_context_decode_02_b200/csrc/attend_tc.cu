@@ -50,7 +50,8 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 constexpr int kPartFloats = 2 * kG + kG * kF + 2 * kG * kD;
 
 struct TcMaps {
-  CUtensorMap coef;   // [B*T][r] bf16, box 32 x 8,   64B swizzle
+  CUtensorMap coef;   // [B*T][r] bf16, box 64 x 8,  128B swizzle (64-column blocks)
+  CUtensorMap coef64; // [B*T][r] bf16, box 32 x 8,   64B swizzle (a last 32-column block)
   CUtensorMap basis;  // [H*d][r] bf16, box 32 x 128, 64B swizzle
   CUtensorMap w1;     // [H*F][d] bf16, box 64 x 128, 128B swizzle
 };
@@ -148,6 +149,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   const int n_items = dm.B * a.n_tiles;
   const int kb_r = dm.r / 32;
   const int ksteps_r = dm.r / 16;
+  const int n128 = dm.r / 64;            // 64-column coefficient blocks (128B swizzle)
+  const bool has64 = (dm.r & 63) != 0;   // and a last 32-column block (64B swizzle)
 
   auto bar = [&](int i) { return base + L.bar + 8u * (uint32_t)i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + L.bar + 8 * BAR_COUNT);
@@ -227,13 +230,18 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       int b, tile;
       item_of(it, b, tile);
       const int cid = lane < kChunksPerTile ? meta[slot].cid[lane] : -1;
+      // each chunk: r/64 boxes of 64 columns (128B swizzle) and, when 64 does not divide
+      // r, one box of the last 32 columns (64B swizzle): 3 boxes per chunk at r = 160
       if (lane == 0)
         mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
       __syncwarp();
       if (lane < kChunksPerTile) {
         const int row = b * dm.T + (cid < 0 ? 0 : cid) * kChunk;
-        for (int kb = 0; kb < kb_r; ++kb)
-          tma_load_2d(base + L.coef + kb * 8192 + lane * 512, &maps.coef, kb * 32, row,
+        for (int c2 = 0; c2 < n128; ++c2)
+          tma_load_2d(base + L.coef + c2 * 16384 + lane * 1024, &maps.coef, c2 * 64, row,
+                      bar(BAR_COEF_FULL));
+        if (has64)
+          tma_load_2d(base + L.coef + n128 * 16384 + lane * 512, &maps.coef64, n128 * 64, row,
                       bar(BAR_COEF_FULL));
       }
       issued_phase = i & 1;
@@ -398,9 +406,14 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         tc_fence_after();
         const uint32_t d_t = tmem + (uint32_t)(u * 128);
         for (int s = 0; s < ksteps_r; ++s) {
-          const uint32_t off = (uint32_t)((s >> 1) * 8192 + (s & 1) * 32);
-          mma_bf16(d_t, smem_desc_kmajor(sc + off, 512, kSwizzle64B),
-                   smem_desc_kmajor(sb + off, 512, kSwizzle64B), kIdesc, s > 0);
+          const uint32_t off = (uint32_t)((s >> 1) * 8192 + (s & 1) * 32);   // basis
+          const uint64_t adesc =
+              s < 4 * n128
+                  ? smem_desc_kmajor(sc + (uint32_t)((s >> 2) * 16384 + (s & 3) * 32), 1024,
+                                     kSwizzle128B)
+                  : smem_desc_kmajor(sc + (uint32_t)(n128 * 16384 + (s & 1) * 32), 512,
+                                     kSwizzle64B);
+          mma_bf16(d_t, adesc, smem_desc_kmajor(sb + off, 512, kSwizzle64B), kIdesc, s > 0);
         }
         mma_commit(bar(BAR_KT_FULL0 + u));
         mma_commit(bar(BAR_COEF_EMPTY));
@@ -873,7 +886,8 @@ size_t attend_tc_part_floats(const Dims& dm, int n_tiles) {
 cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   const Dims& dm = a.dm;
   TcMaps maps;
-  if (!make_tensor_map_2d(&maps.coef, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 32, 8, 64) ||
+  if (!make_tensor_map_2d(&maps.coef, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 64, 8, 128) ||
+      !make_tensor_map_2d(&maps.coef64, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 32, 8, 64) ||
       !make_tensor_map_2d(&maps.basis, a.basis, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.H * kD, 32, 128, 64) ||
       !make_tensor_map_2d(&maps.w1, a.w1, LOWRAM_DTYPE_BF16, kD, (uint64_t)dm.H * kF, 64, 128, 128))
     return cudaErrorInvalidValue;
