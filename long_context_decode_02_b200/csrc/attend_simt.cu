@@ -262,8 +262,6 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
   const int b = p / dm.H, h = p % dm.H;
   const int n = a.n_tiles;
   const size_t tstride = (size_t)G * 2 + (size_t)G * FH + 2 * (size_t)G * D;
-  if (a.ready && g == 0 && threadIdx.x == 0) a.ready[p] = 0;   // the next step's flags
-  if (a.item_ctr && p < dm.H && g == 0 && threadIdx.x == 0) a.item_ctr[p] = 0;   // tile counters
   const float* part = a.part + (size_t)p * n * tstride;
   __shared__ float hs[FH];
   __shared__ float rs[2][D];
@@ -278,6 +276,11 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
 #pragma unroll
     for (int i = 0; i < FH / 2 / 8; ++i) w2v[i] = wrow[i];
   }
+  // launched as a programmatic dependent of the attend kernel: W2 above is independent
+  // of it; the partials, flags and counters below are not
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (a.ready && g == 0 && threadIdx.x == 0) a.ready[p] = 0;   // the next step's flags
+  if (a.item_ctr && p < dm.H && g == 0 && threadIdx.x == 0) a.item_ctr[p] = 0;   // tile counters
   const float b2 = ldf((const T*)a.b2, (size_t)h * D + j);
   // tile weights, computed by every warp: lane t holds tile t (and t + 32)
   const float m0 = lane < n ? part[lane * tstride + 2 * g] : -INFINITY;
@@ -379,7 +382,18 @@ cudaError_t launch_combine(const AttendArgs& a, bool reorder_form, cudaStream_t 
     return cudaGetLastError();
   }
   if (D == 128 && FH == 256 && bf) {
-    combine_reorder_kernel<__nv_bfloat16, 128, 256><<<grid * a.dm.G, 256, 0, s>>>(a);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid * a.dm.G);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_reorder_kernel<__nv_bfloat16, 128, 256>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
   return cudaErrorInvalidValue;

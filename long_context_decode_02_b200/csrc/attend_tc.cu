@@ -71,6 +71,9 @@ constexpr int kMetaSlots = 4;
 constexpr int kResPrefetch = 16;   // residual rows per thread loaded before the hidden layer
 
 constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in flight
+// float2 stride of a chunk's 64 rotations: padded by 2 so the four chunks one warp reads
+// fall in different shared-memory banks
+constexpr int kRotStride = kD / 2 + 2;
 
 struct Layout {
   uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, rot, roff, meta, bar, total;
@@ -90,8 +93,8 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.b1 = L.q + 2048;            // [256] fp32
   L.zx = L.b1 + 1024;           // [128][4] fp32
   L.red = L.zx + 2048;          // 512 B of reduction scratch
-  L.rot = L.red + 512;          // [kRotSlots][16 chunks][64 pairs] float2 (cos, sin)
-  L.roff = L.rot + kRotSlots * kChunksPerTile * (kD / 2) * 8;  // [64 pairs][8] float2
+  L.rot = L.red + 512;          // [kRotSlots][16 chunks][kRotStride] float2 (cos, sin)
+  L.roff = L.rot + kRotSlots * kChunksPerTile * kRotStride * 8;  // [64 pairs][8] float2
   L.meta = L.roff + (kD / 2) * kChunk * 8;  // kMetaSlots x TileMeta
   L.bar = L.meta + kMetaSlots * (uint32_t)sizeof(TileMeta);  // barriers + TMEM holder
   L.total = L.bar + 256 + 1024; // + alignment slack of the dynamic base
@@ -201,6 +204,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // the combine kernel may start on SMs this kernel leaves; it waits for this grid's
+  // completion before it reads the partials
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int32_t* sel_all = a.sel;
   if (warp == 0) {
@@ -373,7 +379,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         if (lane == 0)
           rgot = mbar_wait_bounded(bar(BAR_ROT_EMPTY0 + rs), ((i / kRotSlots) & 1) ^ 1, abort_flag);
         if (!__shfl_sync(0xffffffffu, rgot, 0)) break;
-        float2* R = sRot + rs * kChunksPerTile * (kD / 2);
+        float2* R = sRot + rs * kChunksPerTile * kRotStride;
         const double two_pi_hi = 6.283185307179586232, two_pi_lo = 2.4492935982947064e-16;
         const double inv_two_pi = 0.15915494309189533577;
 #pragma unroll 4
@@ -387,7 +393,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
             const float red = (float)fma(-kq, two_pi_lo, fma(-kq, two_pi_hi, ang));
             float sn, cs;
             __sincosf(red, &sn, &cs);
-            R[c * (kD / 2) + w * 32 + lane] = make_float2(cs, sn);
+            R[c * kRotStride + w * 32 + lane] = make_float2(cs, sn);
           }
         }
         __syncwarp();
@@ -544,7 +550,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       // times the in-chunk offset (table) by angle addition; partial logits accumulate as
       // (x, y) pairs with packed fp32x2 FMAs, the queries of 4 pairs in one 16-byte load
       const float4* rb4 = reinterpret_cast<const float4*>(
-          sRot + (rs * kChunksPerTile + (trow >> 3)) * (kD / 2) + 32 * hf);
+          sRot + (rs * kChunksPerTile + (trow >> 3)) * kRotStride + 32 * hf);
       const float2* ro = sRoff + (32 * hf) * kChunk + (trow & 7);
       float2 z2[kG];
 #pragma unroll
@@ -738,6 +744,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // when launched as a programmatic dependent of the selection kernel, finish only after
+  // it has: the kernels that follow in the stream then find it complete as well
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // --------------------------------------------------------------------- debug tile
