@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
   const int p = blockIdx.x / G, g = blockIdx.x % G;
   const int b = p / dm.H, h = p % dm.H;
   const int n = a.n_tiles;
-  const size_t tstride = (size_t)G * 2 + (size_t)G * FH + 2 * (size_t)G * D;
+  const size_t tstride = (size_t)G * 2 + (size_t)G * FH + (size_t)kTcResSlots * G * D;
   const float* part = a.part + (size_t)p * n * tstride;
   __shared__ float hs[FH];
   __shared__ float rs[2][D];
@@ -299,7 +299,8 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
     for (int u = 0; u < 16; ++u) {
       const int t = t0 + u;
       hv[u] = t < n ? hsrc[t * tstride] : 0.f;
-      rv[u] = t < n ? rsrc[t * tstride] : 0.f;
+      // this thread sums residual slots (tid >> 7) and (tid >> 7) + 2
+      rv[u] = t < n ? rsrc[t * tstride] + rsrc[t * tstride + 2 * (size_t)G * D] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) {

@@ -44,10 +44,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128, kF = 256, kG = 4, kTile = 128, kChunk = 8, kChunksPerTile = 16;
-constexpr int kThreads = 352;  // warp 0 TMA, warp 1 MMA, warp 2 metadata, warps 3..10 epilogue
-constexpr int kEpiThreads = 256;
+constexpr int kThreads = 608;  // warp 0 TMA, warp 1 MMA, warp 2 metadata, warps 3..18 epilogue
+constexpr int kEpiThreads = 512;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
-constexpr int kPartFloats = 2 * kG + kG * kF + 2 * kG * kD;
+constexpr int kPartFloats = 2 * kG + kG * kF + kTcResSlots * kG * kD;
 
 struct TcMaps {
   CUtensorMap coef;   // [B*T][r] bf16, box 64 x 8,  128B swizzle (64-column blocks)
@@ -68,7 +68,7 @@ struct TileMeta {
 };
 static_assert(sizeof(TileMeta) == 1616, "TileMeta layout");
 constexpr int kMetaSlots = 4;
-constexpr int kResPrefetch = 16;   // residual rows per thread loaded before the hidden layer
+constexpr int kResPrefetch = 8;   // residual rows per thread loaded before the hidden layer
 
 constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in flight
 // float2 stride of a chunk's 64 rotations: padded by 2 so the four chunks one warp reads
@@ -91,8 +91,8 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.p = L.kbf + 32768;          // [2][128][4] fp32
   L.q = L.p + 4096;             // [4][128] fp32
   L.b1 = L.q + 2048;            // [256] fp32
-  L.zx = L.b1 + 1024;           // [128][4] fp32
-  L.red = L.zx + 2048;          // 512 B of reduction scratch
+  L.zx = L.b1 + 1024;           // [3][128][4] fp32: partial logits; part B: [2][128][4]
+  L.red = L.zx + 6144;          // 512 B of reduction scratch
   L.rot = L.red + 512;          // [kRotSlots][16 chunks][kRotStride] float2 (cos, sin)
   L.roff = L.rot + kRotSlots * kChunksPerTile * kRotStride * 8;  // [64 pairs][8] float2
   L.meta = L.roff + (kD / 2) * kChunk * 8;  // kMetaSlots x TileMeta
@@ -179,20 +179,20 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     mbar_init(bar(BAR_COEF_EMPTY), 1);
     mbar_init(bar(BAR_KT_FULL0), 1);
     mbar_init(bar(BAR_KT_FULL1), 1);
-    mbar_init(bar(BAR_KT_EMPTY0), 8);
-    mbar_init(bar(BAR_KT_EMPTY1), 8);
-    mbar_init(bar(BAR_KBF_FULL), 8);
+    mbar_init(bar(BAR_KT_EMPTY0), kEpiThreads / 32);
+    mbar_init(bar(BAR_KT_EMPTY1), kEpiThreads / 32);
+    mbar_init(bar(BAR_KBF_FULL), kEpiThreads / 32);
     mbar_init(bar(BAR_KBF_EMPTY), 1);
     for (int i = 0; i < kRotSlots; ++i) {
       mbar_init(bar(BAR_ROT_FULL0 + i), 1);
-      mbar_init(bar(BAR_ROT_EMPTY0 + i), 8);
+      mbar_init(bar(BAR_ROT_EMPTY0 + i), kEpiThreads / 32);
     }
     mbar_init(bar(BAR_H_FULL), 1);
-    mbar_init(bar(BAR_H_EMPTY), 8);
+    mbar_init(bar(BAR_H_EMPTY), kEpiThreads / 32);
     mbar_init(bar(BAR_DRAIN), 1);
     for (int i = 0; i < kMetaSlots; ++i) {
       mbar_init(bar(BAR_META_FULL0 + i), 1);
-      mbar_init(bar(BAR_META_EMPTY0 + i), 8);
+      mbar_init(bar(BAR_META_EMPTY0 + i), kEpiThreads / 32);
     }
     fence_mbar_init();
   }
@@ -463,10 +463,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 3;             // 0..7
+    // 16 warps, four per TMEM lane quadrant; quarter qt of a quadrant's warps takes 16 of
+    // the 64 RoPE pairs in part A and one (hidden half, token half) of H^T in part B
+    const int ew = warp - 3;             // 0..15
     const int qd = warp & 3;             // TMEM lane quadrant this warp may access
-    const int hf = ew >> 2;              // column half
-    const int et = threadIdx.x - 96;     // 0..255
+    const int qt = ew >> 2;              // quarter
+    const int et = threadIdx.x - 96;     // 0..511
     const int trow = 32 * qd + lane;     // token row (A) / hidden-unit row within a half (B)
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
@@ -480,10 +482,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       sRoff[i] = a.rope.lo32[(i & (kChunk - 1)) * (kD / 2) + (i >> 3)];
     bool ok = true;
 
-    // Residual rows of a tile, first kResPrefetch of this thread's: row entries (token row
-    // byte, 255 = none) and raw bf16 values, packed. Loaded while the previous part runs
-    // (at the start of part A of the next tile, or of part B for the last tile) so the
-    // random HBM reads overlap work.
+    // Residual rows of a tile, first kResPrefetch of this thread's (rows qt, qt + 4, ...):
+    // row entries (token row byte, 255 = none) and raw bf16 values, packed. Loaded at the
+    // start of part A of the next tile (or of the end marker), so the random HBM reads
+    // overlap work.
     uint32_t pre_row[kResPrefetch / 4], pre_val[kResPrefetch / 2];
     auto prefetch_res = [&](int i) {
       const TileMeta* M = meta + i % kMetaSlots;
@@ -497,7 +499,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
 #pragma unroll
       for (int v = 0; v < kResPrefetch; ++v) {
-        const int ei = hf + 2 * v;
+        const int ei = qt + 4 * v;
         const uint32_t ent = ei < nres ? M->res[ei] : 255u;
         const uint32_t row = ent & 255u;
         pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
@@ -525,7 +527,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         return false;
       }
       const bool valid = M->cid[trow >> 3] >= 0;
-      {
+      if (et < 256) {
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
         const float2 f = bf2_to_f2(w);
         sQ[2 * et] = f.x;
@@ -534,10 +536,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
 
       good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
       tc_fence_after();
-      float x[32], y[32];
-      const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + 32 * hf);
-      tmem_ld_x32(tcol, x);
-      tmem_ld_x32(tcol + 64, y);
+      float x[16], y[16];
+      const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + 16 * qt);
+      tmem_ld_x16(tcol, x);
+      tmem_ld_x16(tcol + 64, y);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -546,17 +548,17 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       const int rs = i % kRotSlots;
       good = mbar_wait_bounded(bar(BAR_ROT_FULL0 + rs), (i / kRotSlots) & 1, abort_flag) && good;
       named_bar_sync(1, kEpiThreads);  // sQ ready
-      // RoPE on pairs (32hf + e, 64 + 32hf + e): the chunk-base rotation (from the ring)
+      // RoPE on pairs (16qt + e, 64 + 16qt + e): the chunk-base rotation (from the ring)
       // times the in-chunk offset (table) by angle addition; partial logits accumulate as
       // (x, y) pairs with packed fp32x2 FMAs, the queries of 4 pairs in one 16-byte load
       const float4* rb4 = reinterpret_cast<const float4*>(
-          sRot + (rs * kChunksPerTile + (trow >> 3)) * kRotStride + 32 * hf);
-      const float2* ro = sRoff + (32 * hf) * kChunk + (trow & 7);
+          sRot + (rs * kChunksPerTile + (trow >> 3)) * kRotStride + 16 * qt);
+      const float2* ro = sRoff + (16 * qt) * kChunk + (trow & 7);
       float2 z2[kG];
 #pragma unroll
       for (int g = 0; g < kG; ++g) z2[g] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int e4 = 0; e4 < 32; e4 += 4) {
+      for (int e4 = 0; e4 < 16; e4 += 4) {
         const float4 b01 = rb4[e4 / 2], b23 = rb4[e4 / 2 + 1];
         const float2 bs[4] = {make_float2(b01.x, b01.y), make_float2(b01.z, b01.w),
                               make_float2(b23.x, b23.y), make_float2(b23.z, b23.w)};
@@ -567,7 +569,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           const float2 cs = rope_combine(bs[w], ro[e * kChunk]);
           rot[w] = make_float2(x[e] * cs.x - y[e] * cs.y, x[e] * cs.y + y[e] * cs.x);
         }
-        const int pi = 32 * hf + e4;
+        const int pi = 16 * qt + e4;
 #pragma unroll
         for (int g = 0; g < kG; ++g) {
           const float4 qx = *reinterpret_cast<const float4*>(sQ + g * kD + pi);
@@ -589,11 +591,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       good = mbar_wait_bounded(bar(BAR_KBF_EMPTY), (i & 1) ^ 1, abort_flag) && good;
       const uint32_t skb = base + L.kbf;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        st_shared_v4(skb + sw128_offset(trow, 4 * hf + cc),
+      for (int cc = 0; cc < 2; ++cc) {
+        st_shared_v4(skb + sw128_offset(trow, 2 * qt + cc),
                      pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]), pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]),
                      pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]), pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]));
-        st_shared_v4(skb + 16384 + sw128_offset(trow, 4 * hf + cc),
+        st_shared_v4(skb + 16384 + sw128_offset(trow, 2 * qt + cc),
                      pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]), pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]),
                      pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]), pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]));
       }
@@ -601,14 +603,20 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL));
 
-      if (hf == 1) *reinterpret_cast<float4*>(sZx + 4 * trow) = make_float4(z[0], z[1], z[2], z[3]);
+      // partial logits of quarters 1..3 -> sZx[qt - 1][trow]; quarter 0 adds them
+      if (qt > 0) *reinterpret_cast<float4*>(sZx + ((qt - 1) * kTile + trow) * 4) = make_float4(z[0], z[1], z[2], z[3]);
       named_bar_sync(1, kEpiThreads);
-      if (hf == 0) {
-        const float4 o = *reinterpret_cast<const float4*>(sZx + 4 * trow);
-        z[0] = valid ? (z[0] + o.x) * zscale : -INFINITY;
-        z[1] = valid ? (z[1] + o.y) * zscale : -INFINITY;
-        z[2] = valid ? (z[2] + o.z) * zscale : -INFINITY;
-        z[3] = valid ? (z[3] + o.w) * zscale : -INFINITY;
+      if (qt == 0) {
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+          const float4 v = *reinterpret_cast<const float4*>(sZx + (o * kTile + trow) * 4);
+          z[0] += v.x;
+          z[1] += v.y;
+          z[2] += v.z;
+          z[3] += v.w;
+        }
+#pragma unroll
+        for (int g = 0; g < kG; ++g) z[g] = valid ? z[g] * zscale : -INFINITY;
 #pragma unroll
         for (int g = 0; g < kG; ++g) {
           const float m = warp_max(z[g]);
@@ -638,7 +646,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       return good;
     };
 
-    // ---- part B of tile i
+    // ---- part B of tile i: quarter qt takes hidden half hf = qt / 2 and token half
+    // th = qt % 2 of H^T; the token halves' sums meet in shared memory
     auto part_b = [&](int i) -> bool {
       const int u = i & 1;
       const int slot = i % kMetaSlots;
@@ -646,8 +655,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       int b, tile;
       item_of(M->item, b, tile);
       const int p = b * dm.H + h;
+      const int hf = qt >> 1, th = qt & 1;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
-      // residual rows of the tile: thread = column j; rows split between the two halves.
+      // residual rows of the tile: thread = column j; rows split between the quarters.
       // The first kResPrefetch of this thread's rows were loaded earlier (prefetch_res).
       const int j = trow;
       const int nres = M->nres;
@@ -659,7 +669,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       float2 hacc01 = make_float2(0.f, 0.f), hacc23 = make_float2(0.f, 0.f);
       const float4* P4 = reinterpret_cast<const float4*>(sP + u * 512);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * th; c < 2 * th + 2; ++c) {
         float hv[32];
         tmem_ld_x32(tmem + lane_addr + 256u + (uint32_t)(hf * 128 + 32 * c), hv);
         tmem_wait_ld();
@@ -687,12 +697,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           }
         }
       }
-      const float hacc[kG] = {hacc01.x, hacc01.y, hacc23.x, hacc23.y};
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
-#pragma unroll
-      for (int g = 0; g < kG; ++g) part[2 * kG + g * kF + f] = hacc[g];
+      // token half 1 hands its sums to token half 0 (sZx is free until the next part A)
+      float4* hx4 = reinterpret_cast<float4*>(sZx) + hf * kTile + trow;
+      if (th == 1) *hx4 = make_float4(hacc01.x, hacc01.y, hacc23.x, hacc23.y);
 
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -706,7 +716,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         racc[2] = fmaf(pv.z, r, racc[2]);
         racc[3] = fmaf(pv.w, r, racc[3]);
       }
-      for (int ei = hf + 2 * kResPrefetch; ei < nres; ei += 2) {   // rows beyond the prefetch
+      for (int ei = qt + 4 * kResPrefetch; ei < nres; ei += 4) {   // rows beyond the prefetch
         const uint32_t ent = M->res[ei];
         const int row = (int)(ent & 255u);
         if (row == 255) continue;
@@ -717,9 +727,17 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         racc[2] = fmaf(pv.z, r, racc[2]);
         racc[3] = fmaf(pv.w, r, racc[3]);
       }
-      float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
+      float* pr = part + 2 * kG + kG * kF + (size_t)qt * kG * kD;
 #pragma unroll
       for (int g = 0; g < kG; ++g) pr[g * kD + j] = racc[g];
+      named_bar_sync(1, kEpiThreads);   // token half 1's sums are in shared memory
+      if (th == 0) {
+        const float4 o = *hx4;
+        part[2 * kG + 0 * kF + f] = hacc01.x + o.x;
+        part[2 * kG + 1 * kF + f] = hacc01.y + o.y;
+        part[2 * kG + 2 * kF + f] = hacc23.x + o.z;
+        part[2 * kG + 3 * kF + f] = hacc23.y + o.w;
+      }
       if (ew == 0 && lane < 2 * kG) part[lane] = s_ml[u * 8 + lane];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_META_EMPTY0 + slot));
