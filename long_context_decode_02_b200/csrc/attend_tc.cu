@@ -44,7 +44,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128, kF = 256, kG = 4, kTile = 128, kChunk = 8, kChunksPerTile = 16;
-constexpr int kThreads = 608;  // warp 0 TMA, warp 1 MMA, warp 2 metadata, warps 3..18 epilogue
+// warp 0 TMA, warp 1 K-MMA issuer + TMEM owner, warp 2 metadata, warps 3..18 epilogue,
+// warp 19 hidden-layer MMA issuer
+constexpr int kThreads = 640;
+constexpr int kHWarp = 19;
 constexpr int kEpiThreads = 512;
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 constexpr int kPartFloats = 2 * kG + kG * kF + kTcResSlots * kG * kD;
@@ -104,7 +107,7 @@ __host__ __device__ inline Layout make_layout(int r) {
 // barrier slots (8 bytes each) inside L.bar
 enum {
   BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
-  BAR_KT_EMPTY1, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN,
+  BAR_KT_EMPTY1, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN, BAR_DRAIN_H,
   BAR_ROT_FULL0, BAR_ROT_EMPTY0 = BAR_ROT_FULL0 + kRotSlots,
   BAR_META_FULL0 = BAR_ROT_EMPTY0 + kRotSlots, BAR_META_EMPTY0 = BAR_META_FULL0 + kMetaSlots,
   BAR_COUNT = BAR_META_EMPTY0 + kMetaSlots
@@ -188,6 +191,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       mbar_init(bar(BAR_ROT_EMPTY0 + i), kEpiThreads / 32);
     }
     mbar_init(bar(BAR_H_FULL), 1);
+    mbar_init(bar(BAR_DRAIN_H), 1);
     mbar_init(bar(BAR_H_EMPTY), kEpiThreads / 32);
     mbar_init(bar(BAR_DRAIN), 1);
     for (int i = 0; i < kMetaSlots; ++i) {
@@ -404,7 +408,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait_bounded(bar(BAR_W), 0, abort_flag);
-      const uint32_t sb = base + L.basis, sw1 = base + L.w1, sc = base + L.coef;
+      const uint32_t sb = base + L.basis, sc = base + L.coef;
       auto issue_k = [&](int i) -> bool {
         const int u = i & 1;
         if (!mbar_wait_bounded(bar(BAR_COEF_FULL), i & 1, abort_flag)) return false;
@@ -425,11 +429,33 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         mma_commit(bar(BAR_COEF_EMPTY));
         return true;
       };
-      auto issue_h = [&](int i) -> bool {
-        if (!mbar_wait_bounded(bar(BAR_KBF_FULL), i & 1, abort_flag)) return false;
-        if (!mbar_wait_bounded(bar(BAR_H_EMPTY), (i & 1) ^ 1, abort_flag)) return false;
+      // whether tile i exists, from its metadata slot (read before the slot can recycle)
+      auto exists = [&](int i) -> bool {
+        const int slot = i % kMetaSlots;
+        if (!mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag))
+          return false;
+        return meta[slot].item >= 0;
+      };
+      // the K~ GEMMs run ahead on their own: the hidden-layer GEMMs have their own issuer
+      for (int i = 0; ok && exists(i); ++i) ok = issue_k(i);
+      // drain every MMA this thread issued before TMEM is released
+      mma_commit(bar(BAR_DRAIN));
+      int dummy = 0;
+      mbar_wait_bounded(bar(BAR_DRAIN), 0, (volatile int*)&dummy);
+    }
+  } else if (warp == kHWarp) {
+    // ------------------------------------------------------------ hidden-layer MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait_bounded(bar(BAR_W), 0, abort_flag);
+      const uint32_t sw1 = base + L.w1, skb = base + L.kbf;
+      for (int i = 0; ok; ++i) {
+        const int slot = i % kMetaSlots;
+        if (!mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag) ||
+            meta[slot].item < 0)
+          break;
+        if (!mbar_wait_bounded(bar(BAR_KBF_FULL), i & 1, abort_flag)) break;
+        if (!mbar_wait_bounded(bar(BAR_H_EMPTY), (i & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t skb = base + L.kbf;
         for (int hf = 0; hf < 2; ++hf) {
           const uint32_t d_t = tmem + 256u + (uint32_t)hf * 128u;
           for (int s = 0; s < 8; ++s) {
@@ -440,26 +466,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         }
         mma_commit(bar(BAR_H_FULL));
         mma_commit(bar(BAR_KBF_EMPTY));
-        return true;
-      };
-      // whether tile i exists, from its metadata slot (read before the slot can recycle)
-      auto exists = [&](int i) -> bool {
-        const int slot = i % kMetaSlots;
-        if (!mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag))
-          return false;
-        return meta[slot].item >= 0;
-      };
-      bool more = ok && exists(0);
-      if (more) ok = issue_k(0);
-      for (int i = 0; ok && more; ++i) {
-        more = exists(i + 1);
-        if (more) ok = issue_k(i + 1);
-        if (ok) ok = issue_h(i);
       }
-      // drain every MMA this thread issued before TMEM is released
-      mma_commit(bar(BAR_DRAIN));
+      mma_commit(bar(BAR_DRAIN_H));
       int dummy = 0;
-      mbar_wait_bounded(bar(BAR_DRAIN), 0, (volatile int*)&dummy);
+      mbar_wait_bounded(bar(BAR_DRAIN_H), 0, (volatile int*)&dummy);
     }
   } else {
     // ------------------------------------------------------------ epilogue
