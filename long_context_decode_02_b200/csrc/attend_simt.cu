@@ -299,8 +299,11 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
     for (int u = 0; u < 16; ++u) {
       const int t = t0 + u;
       hv[u] = t < n ? hsrc[t * tstride] : 0.f;
-      // this thread sums residual slots (tid >> 7) and (tid >> 7) + 2
-      rv[u] = t < n ? rsrc[t * tstride] + rsrc[t * tstride + 2 * (size_t)G * D] : 0.f;
+      // this thread sums residual slots (tid >> 7), (tid >> 7) + 2, ...
+      float r = 0.f;
+      if (t < n)
+        for (int sl = 0; sl + (tid >> 7) < kTcResSlots; sl += 2) r += rsrc[t * tstride + (size_t)sl * G * D];
+      rv[u] = r;
     }
 #pragma unroll
     for (int u = 0; u < 16; ++u) {

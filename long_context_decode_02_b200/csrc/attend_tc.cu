@@ -44,11 +44,12 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128, kF = 256, kG = 4, kTile = 128, kChunk = 8, kChunksPerTile = 16;
-// warp 0 TMA, warp 1 K-MMA issuer + TMEM owner, warp 2 metadata, warps 3..18 epilogue,
-// warp 19 hidden-layer MMA issuer
-constexpr int kThreads = 640;
-constexpr int kHWarp = 19;
-constexpr int kEpiThreads = 512;
+// warp 0 TMA, warp 1 K-MMA issuer + TMEM owner, warp 2 metadata, warps 3..10 epilogue
+// part A, warps 11..18 epilogue part B, warp 19 hidden-layer MMA issuer
+constexpr int kEpiWarpsA = 8, kEpiWarpsB = 8;
+constexpr int kEpiThreadsA = 32 * kEpiWarpsA, kEpiThreadsB = 32 * kEpiWarpsB;
+constexpr int kHWarp = 3 + kEpiWarpsA + kEpiWarpsB;
+constexpr int kThreads = 32 * (kHWarp + 1);
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128);
 constexpr int kPartFloats = 2 * kG + kG * kF + kTcResSlots * kG * kD;
 
@@ -71,7 +72,7 @@ struct TileMeta {
 };
 static_assert(sizeof(TileMeta) == 1616, "TileMeta layout");
 constexpr int kMetaSlots = 4;
-constexpr int kResPrefetch = 8;   // residual rows per thread loaded before the hidden layer
+constexpr int kResPrefetch = 16;   // residual rows per thread loaded before the hidden layer
 
 constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in flight
 // float2 stride of a chunk's 64 rotations: padded by 2 so the four chunks one warp reads
@@ -94,8 +95,8 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.p = L.kbf + 32768;          // [2][128][4] fp32
   L.q = L.p + 4096;             // [4][128] fp32
   L.b1 = L.q + 2048;            // [256] fp32
-  L.zx = L.b1 + 1024;           // [3][128][4] fp32: partial logits; part B: [2][128][4]
-  L.red = L.zx + 6144;          // 512 B of reduction scratch
+  L.zx = L.b1 + 1024;           // [128][4] fp32: the second pair half's partial logits
+  L.red = L.zx + 2048;          // 512 B of reduction scratch
   L.rot = L.red + 512;          // [kRotSlots][16 chunks][kRotStride] float2 (cos, sin)
   L.roff = L.rot + kRotSlots * kChunksPerTile * kRotStride * 8;  // [64 pairs][8] float2
   L.meta = L.roff + (kD / 2) * kChunk * 8;  // kMetaSlots x TileMeta
@@ -108,6 +109,7 @@ __host__ __device__ inline Layout make_layout(int r) {
 enum {
   BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
   BAR_KT_EMPTY1, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN, BAR_DRAIN_H,
+  BAR_P_FULL0, BAR_P_FULL1, BAR_P_EMPTY0, BAR_P_EMPTY1,
   BAR_ROT_FULL0, BAR_ROT_EMPTY0 = BAR_ROT_FULL0 + kRotSlots,
   BAR_META_FULL0 = BAR_ROT_EMPTY0 + kRotSlots, BAR_META_EMPTY0 = BAR_META_FULL0 + kMetaSlots,
   BAR_COUNT = BAR_META_EMPTY0 + kMetaSlots
@@ -182,21 +184,25 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     mbar_init(bar(BAR_COEF_EMPTY), 1);
     mbar_init(bar(BAR_KT_FULL0), 1);
     mbar_init(bar(BAR_KT_FULL1), 1);
-    mbar_init(bar(BAR_KT_EMPTY0), kEpiThreads / 32);
-    mbar_init(bar(BAR_KT_EMPTY1), kEpiThreads / 32);
-    mbar_init(bar(BAR_KBF_FULL), kEpiThreads / 32);
+    mbar_init(bar(BAR_KT_EMPTY0), kEpiWarpsA);
+    mbar_init(bar(BAR_KT_EMPTY1), kEpiWarpsA);
+    mbar_init(bar(BAR_KBF_FULL), kEpiWarpsA);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(BAR_P_FULL0 + i), 1);
+      mbar_init(bar(BAR_P_EMPTY0 + i), kEpiWarpsB);
+    }
     mbar_init(bar(BAR_KBF_EMPTY), 1);
     for (int i = 0; i < kRotSlots; ++i) {
       mbar_init(bar(BAR_ROT_FULL0 + i), 1);
-      mbar_init(bar(BAR_ROT_EMPTY0 + i), kEpiThreads / 32);
+      mbar_init(bar(BAR_ROT_EMPTY0 + i), kEpiWarpsA);
     }
     mbar_init(bar(BAR_H_FULL), 1);
     mbar_init(bar(BAR_DRAIN_H), 1);
-    mbar_init(bar(BAR_H_EMPTY), kEpiThreads / 32);
+    mbar_init(bar(BAR_H_EMPTY), kEpiWarpsB);
     mbar_init(bar(BAR_DRAIN), 1);
     for (int i = 0; i < kMetaSlots; ++i) {
       mbar_init(bar(BAR_META_FULL0 + i), 1);
-      mbar_init(bar(BAR_META_EMPTY0 + i), kEpiThreads / 32);
+      mbar_init(bar(BAR_META_EMPTY0 + i), kEpiWarpsB);
     }
     fence_mbar_init();
   }
@@ -471,167 +477,135 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       int dummy = 0;
       mbar_wait_bounded(bar(BAR_DRAIN_H), 0, (volatile int*)&dummy);
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    // 16 warps, four per TMEM lane quadrant; quarter qt of a quadrant's warps takes 16 of
-    // the 64 RoPE pairs in part A and one (hidden half, token half) of H^T in part B
-    const int ew = warp - 3;             // 0..15
+  } else if (warp < 3 + kEpiWarpsA) {
+    // ------------------------------------------------------------ epilogue, part A
+    // 8 warps, two per TMEM lane quadrant: pair half ha of the tile's tokens' K~ rows;
+    // RoPE, logits, K~ in bf16 for the hidden-layer GEMM, softmax weights P. Part B runs
+    // concurrently on its own 8 warps; P passes between them through a 2-slot ring.
+    const int ea = warp - 3;             // 0..7
     const int qd = warp & 3;             // TMEM lane quadrant this warp may access
-    const int qt = ew >> 2;              // quarter
-    const int et = threadIdx.x - 96;     // 0..511
-    const int trow = 32 * qd + lane;     // token row (A) / hidden-unit row within a half (B)
+    const int ha = ea >> 2;              // pair half
+    const int et = threadIdx.x - 96;     // 0..255
+    const int trow = 32 * qd + lane;     // token row
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
-    const __nv_bfloat16* rval_all = (const __nv_bfloat16*)a.res_val;
     float* s_ml = sRed + 64;  // [2][4][2]
-
-    for (int i = et; i < kF; i += kEpiThreads)
-      sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
     // in-chunk offsets: sRoff[pair * 8 + j] = (cos, sin)(j theta_pair), j < 8
-    for (int i = et; i < (kD / 2) * kChunk; i += kEpiThreads)
+    for (int i = et; i < (kD / 2) * kChunk; i += kEpiThreadsA)
       sRoff[i] = a.rope.lo32[(i & (kChunk - 1)) * (kD / 2) + (i >> 3)];
-    bool ok = true;
-
-    // Residual rows of a tile, first kResPrefetch of this thread's (rows qt, qt + 4, ...):
-    // row entries (token row byte, 255 = none) and raw bf16 values, packed. Loaded at the
-    // start of part A of the next tile (or of the end marker), so the random HBM reads
-    // overlap work.
-    uint32_t pre_row[kResPrefetch / 4], pre_val[kResPrefetch / 2];
-    auto prefetch_res = [&](int i) {
-      const TileMeta* M = meta + i % kMetaSlots;
-      int b, tile;
-      item_of(M->item, b, tile);
-      const int nres = M->nres;
-      const __nv_bfloat16* rbase = rval_all + (size_t)(b * dm.H + h) * dm.n_res * kD + trow;
-#pragma unroll
-      for (int w = 0; w < kResPrefetch / 4; ++w) pre_row[w] = 0xFFFFFFFFu;
-#pragma unroll
-      for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
-#pragma unroll
-      for (int v = 0; v < kResPrefetch; ++v) {
-        const int ei = qt + 4 * v;
-        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
-        const uint32_t row = ent & 255u;
-        pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
-        if (row != 255u) {
-          const uint32_t raw =
-              __ldg(reinterpret_cast<const unsigned short*>(rbase + (size_t)(ent >> 8) * kD));
-          pre_val[v >> 1] |= raw << (16 * (v & 1));
-        }
-      }
-    };
-
     // A failed (timed-out) wait never changes the sequence of named barriers: the
-    // thread carries on with `good` false so every barrier is still reached.
-    // ---- part A of tile i; false when the tile does not exist (the end marker) or a wait
-    // gave up, decided by one vote of all epilogue threads
+    // thread carries on with `good` false so every barrier is still reached. Returns false
+    // when the tile does not exist (the end marker) or a wait gave up, decided by one vote.
     auto part_a = [&](int i) -> bool {
-      if (i > 0) prefetch_res(i - 1);   // for part B of the previous tile
       const int u = i & 1;
       const int slot = i % kMetaSlots;
       const TileMeta* M = meta + slot;
       bool good = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
       // the vote is also the barrier after which the previous readers of sQ / sZx are done
-      if (named_bar_red_or(1, kEpiThreads, !good || M->item < 0)) {
+      if (named_bar_red_or(1, kEpiThreadsA, !good || M->item < 0)) {
         if (!good) *abort_flag = 1;
         return false;
       }
       const bool valid = M->cid[trow >> 3] >= 0;
-      if (et < 256) {
+      {
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
         const float2 f = bf2_to_f2(w);
         sQ[2 * et] = f.x;
         sQ[2 * et + 1] = f.y;
       }
-
       good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
-      tc_fence_after();
-      float x[16], y[16];
-      const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + 16 * qt);
-      tmem_ld_x16(tcol, x);
-      tmem_ld_x16(tcol + 64, y);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY0 + u));
-
       const int rs = i % kRotSlots;
       good = mbar_wait_bounded(bar(BAR_ROT_FULL0 + rs), (i / kRotSlots) & 1, abort_flag) && good;
-      named_bar_sync(1, kEpiThreads);  // sQ ready
-      // RoPE on pairs (16qt + e, 64 + 16qt + e): the chunk-base rotation (from the ring)
-      // times the in-chunk offset (table) by angle addition; partial logits accumulate as
-      // (x, y) pairs with packed fp32x2 FMAs, the queries of 4 pairs in one 16-byte load
-      const float4* rb4 = reinterpret_cast<const float4*>(
-          sRot + (rs * kChunksPerTile + (trow >> 3)) * kRotStride + 16 * qt);
-      const float2* ro = sRoff + (16 * qt) * kChunk + (trow & 7);
+      named_bar_sync(1, kEpiThreadsA);  // sQ ready
+      // K~_pre in bf16 goes to shared memory (single buffer, 128B-swizzled K-major
+      // [tok][d]) once the previous tile's hidden-layer MMA has released it
+      good = mbar_wait_bounded(bar(BAR_KBF_EMPTY), (i & 1) ^ 1, abort_flag) && good;
+      tc_fence_after();
+      const uint32_t skb = base + L.kbf;
+      const float4* rbase4 = reinterpret_cast<const float4*>(
+          sRot + (rs * kChunksPerTile + (trow >> 3)) * kRotStride);
       float2 z2[kG];
 #pragma unroll
       for (int g = 0; g < kG; ++g) z2[g] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int e4 = 0; e4 < 16; e4 += 4) {
-        const float4 b01 = rb4[e4 / 2], b23 = rb4[e4 / 2 + 1];
-        const float2 bs[4] = {make_float2(b01.x, b01.y), make_float2(b01.z, b01.w),
-                              make_float2(b23.x, b23.y), make_float2(b23.z, b23.w)};
-        float2 rot[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int e = e4 + w;
-          const float2 cs = rope_combine(bs[w], ro[e * kChunk]);
-          rot[w] = make_float2(x[e] * cs.x - y[e] * cs.y, x[e] * cs.y + y[e] * cs.x);
+#pragma unroll 1
+      for (int sb = 0; sb < 2; ++sb) {
+        // pairs p0 .. p0 + 15 of this thread's token: K~ columns p0.. and 64 + p0..
+        const int p0 = 32 * ha + 16 * sb;
+        float x[16], y[16];
+        const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + p0);
+        tmem_ld_x16(tcol, x);
+        tmem_ld_x16(tcol + 64, y);
+        tmem_wait_ld();
+        if (sb == 1) {   // both halves of this thread's K~ columns are in registers
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY0 + u));
         }
-        const int pi = 16 * qt + e4;
+        // RoPE on pairs (p0 + e, 64 + p0 + e): the chunk-base rotation (from the ring)
+        // times the in-chunk offset (table) by angle addition; partial logits accumulate as
+        // (x, y) pairs with packed fp32x2 FMAs, the queries of 4 pairs in one 16-byte load
+        const float4* rb4 = rbase4 + p0 / 2;
+        const float2* ro = sRoff + p0 * kChunk + (trow & 7);
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-          const float4 qx = *reinterpret_cast<const float4*>(sQ + g * kD + pi);
-          const float4 qy = *reinterpret_cast<const float4*>(sQ + g * kD + 64 + pi);
-          z2[g] = __ffma2_rn(make_float2(qx.x, qy.x), rot[0], z2[g]);
-          z2[g] = __ffma2_rn(make_float2(qx.y, qy.y), rot[1], z2[g]);
-          z2[g] = __ffma2_rn(make_float2(qx.z, qy.z), rot[2], z2[g]);
-          z2[g] = __ffma2_rn(make_float2(qx.w, qy.w), rot[3], z2[g]);
+        for (int e4 = 0; e4 < 16; e4 += 4) {
+          const float4 b01 = rb4[e4 / 2], b23 = rb4[e4 / 2 + 1];
+          const float2 bs[4] = {make_float2(b01.x, b01.y), make_float2(b01.z, b01.w),
+                                make_float2(b23.x, b23.y), make_float2(b23.z, b23.w)};
+          float2 rot[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int e = e4 + w;
+            const float2 cs = rope_combine(bs[w], ro[e * kChunk]);
+            rot[w] = make_float2(x[e] * cs.x - y[e] * cs.y, x[e] * cs.y + y[e] * cs.x);
+          }
+          const int pi = p0 + e4;
+#pragma unroll
+          for (int g = 0; g < kG; ++g) {
+            const float4 qx = *reinterpret_cast<const float4*>(sQ + g * kD + pi);
+            const float4 qy = *reinterpret_cast<const float4*>(sQ + g * kD + 64 + pi);
+            z2[g] = __ffma2_rn(make_float2(qx.x, qy.x), rot[0], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qx.y, qy.y), rot[1], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qx.z, qy.z), rot[2], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qx.w, qy.w), rot[3], z2[g]);
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int ch = (p0 >> 3) + cc;   // 16-byte chunk of the 64-dim block
+          st_shared_v4(skb + sw128_offset(trow, ch),
+                       pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]), pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]),
+                       pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]), pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]));
+          st_shared_v4(skb + 16384 + sw128_offset(trow, ch),
+                       pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]), pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]),
+                       pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]), pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]));
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_ROT_EMPTY0 + rs));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL));
       float z[kG];
 #pragma unroll
       for (int g = 0; g < kG; ++g) z[g] = z2[g].x + z2[g].y;
 
-      // K~_pre in bf16 -> shared memory (single buffer, 128B-swizzled K-major [tok][d]);
-      // the hidden-layer MMA of the previous tile has released it by now
-      good = mbar_wait_bounded(bar(BAR_KBF_EMPTY), (i & 1) ^ 1, abort_flag) && good;
-      const uint32_t skb = base + L.kbf;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        st_shared_v4(skb + sw128_offset(trow, 2 * qt + cc),
-                     pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]), pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]),
-                     pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]), pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]));
-        st_shared_v4(skb + 16384 + sw128_offset(trow, 2 * qt + cc),
-                     pack_bf16x2(y[8 * cc + 0], y[8 * cc + 1]), pack_bf16x2(y[8 * cc + 2], y[8 * cc + 3]),
-                     pack_bf16x2(y[8 * cc + 4], y[8 * cc + 5]), pack_bf16x2(y[8 * cc + 6], y[8 * cc + 7]));
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_KBF_FULL));
-
-      // partial logits of quarters 1..3 -> sZx[qt - 1][trow]; quarter 0 adds them
-      if (qt > 0) *reinterpret_cast<float4*>(sZx + ((qt - 1) * kTile + trow) * 4) = make_float4(z[0], z[1], z[2], z[3]);
-      named_bar_sync(1, kEpiThreads);
-      if (qt == 0) {
-#pragma unroll
-        for (int o = 0; o < 3; ++o) {
-          const float4 v = *reinterpret_cast<const float4*>(sZx + (o * kTile + trow) * 4);
-          z[0] += v.x;
-          z[1] += v.y;
-          z[2] += v.z;
-          z[3] += v.w;
-        }
-#pragma unroll
-        for (int g = 0; g < kG; ++g) z[g] = valid ? z[g] * zscale : -INFINITY;
+      if (ha == 1) *reinterpret_cast<float4*>(sZx + 4 * trow) = make_float4(z[0], z[1], z[2], z[3]);
+      named_bar_sync(1, kEpiThreadsA);
+      if (ha == 0) {
+        const float4 o = *reinterpret_cast<const float4*>(sZx + 4 * trow);
+        z[0] = valid ? (z[0] + o.x) * zscale : -INFINITY;
+        z[1] = valid ? (z[1] + o.y) * zscale : -INFINITY;
+        z[2] = valid ? (z[2] + o.z) * zscale : -INFINITY;
+        z[3] = valid ? (z[3] + o.w) * zscale : -INFINITY;
 #pragma unroll
         for (int g = 0; g < kG; ++g) {
           const float m = warp_max(z[g]);
           if (lane == 0) sRed[qd * 4 + g] = m;
         }
+        // P slot u is free once part B has finished with tile i - 2
+        int pe = 1;
+        if (lane == 0) pe = mbar_wait_bounded(bar(BAR_P_EMPTY0 + u), ((i >> 1) & 1) ^ 1, abort_flag);
+        good = __shfl_sync(0xffffffffu, pe, 0) && good;
         named_bar_sync(2, 128);
         float m[kG], pv[kG];
 #pragma unroll
@@ -646,40 +620,81 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           if (lane == 0) sRed[16 + qd * 4 + g] = l;
         }
         named_bar_sync(2, 128);
-        if (ew == 0 && lane < kG) {
+        if (ea == 0 && lane < kG) {
           const int g = lane;
           s_ml[u * 8 + g * 2 + 0] = m[g];
           s_ml[u * 8 + g * 2 + 1] = sRed[16 + g] + sRed[20 + g] + sRed[24 + g] + sRed[28 + g];
         }
       }
-      named_bar_sync(1, kEpiThreads);  // P and (m, l) of tile i visible to all
-      return good;
+      named_bar_sync(1, kEpiThreadsA);  // P and (m, l) of tile i written
+      if (et == 0) mbar_arrive(bar(BAR_P_FULL0 + u));
+      if (!good) *abort_flag = 1;
+      return true;
     };
-
-    // ---- part B of tile i: quarter qt takes hidden half hf = qt / 2 and token half
-    // th = qt % 2 of H^T; the token halves' sums meet in shared memory
+    // after a failed wait every later wait returns at once and the vote ends the loop
+    for (int i = 0; part_a(i); ++i) {
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue, part B
+    // 8 warps, two per TMEM lane quadrant: hidden half hf of H^T (lane = hidden unit f,
+    // columns = the tile's 128 tokens): act(h + b1) and Hacc_g[f] += p_g(t) act, a
+    // reduction along each thread's own TMEM row; and the residual rows of the tile.
+    const int eb = warp - 3 - kEpiWarpsA;   // 0..7
+    const int qd = warp & 3;
+    const int hf = eb >> 2;
+    const int etb = threadIdx.x - 96 - kEpiThreadsA;   // 0..255
+    const int trow = 32 * qd + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
+    const __nv_bfloat16* rval_all = (const __nv_bfloat16*)a.res_val;
+    const float* s_ml = sRed + 64;
+    for (int i = etb; i < kF; i += kEpiThreadsB)
+      sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
+    named_bar_sync(3, kEpiThreadsB);
     auto part_b = [&](int i) -> bool {
       const int u = i & 1;
       const int slot = i % kMetaSlots;
       const TileMeta* M = meta + slot;
+      bool good = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
+      if (named_bar_red_or(3, kEpiThreadsB, !good || M->item < 0)) {
+        if (!good) *abort_flag = 1;
+        return false;
+      }
       int b, tile;
       item_of(M->item, b, tile);
       const int p = b * dm.H + h;
-      const int hf = qt >> 1, th = qt & 1;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
-      // residual rows of the tile: thread = column j; rows split between the quarters.
-      // The first kResPrefetch of this thread's rows were loaded earlier (prefetch_res).
+      // residual rows of the tile: thread = column j; rows split between the two halves.
+      // The first kResPrefetch of this thread's rows are loaded now, as raw bf16 bits:
+      // nothing waits for them until the residual sum after the hidden layer.
       const int j = trow;
       const int nres = M->nres;
       const __nv_bfloat16* rbase = rval_all + (size_t)p * dm.n_res * kD + j;
-      const bool good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag);
+      uint32_t pre_row[kResPrefetch / 4], pre_val[kResPrefetch / 2];
+#pragma unroll
+      for (int w = 0; w < kResPrefetch / 4; ++w) pre_row[w] = 0xFFFFFFFFu;
+#pragma unroll
+      for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
+#pragma unroll
+      for (int v = 0; v < kResPrefetch; ++v) {
+        const int ei = hf + 2 * v;
+        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
+        const uint32_t row = ent & 255u;
+        pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
+        if (row != 255u) {
+          const uint32_t raw =
+              __ldg(reinterpret_cast<const unsigned short*>(rbase + (size_t)(ent >> 8) * kD));
+          pre_val[v >> 1] |= raw << (16 * (v & 1));
+        }
+      }
+      good = mbar_wait_bounded(bar(BAR_P_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
+      good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag) && good;
       tc_fence_after();
       const int f = 128 * hf + trow;
       const float bias = sB1[f];
       float2 hacc01 = make_float2(0.f, 0.f), hacc23 = make_float2(0.f, 0.f);
       const float4* P4 = reinterpret_cast<const float4*>(sP + u * 512);
 #pragma unroll 1
-      for (int c = 2 * th; c < 2 * th + 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
         float hv[32];
         tmem_ld_x32(tmem + lane_addr + 256u + (uint32_t)(hf * 128 + 32 * c), hv);
         tmem_wait_ld();
@@ -710,9 +725,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
-      // token half 1 hands its sums to token half 0 (sZx is free until the next part A)
-      float4* hx4 = reinterpret_cast<float4*>(sZx) + hf * kTile + trow;
-      if (th == 1) *hx4 = make_float4(hacc01.x, hacc01.y, hacc23.x, hacc23.y);
+      part[2 * kG + 0 * kF + f] = hacc01.x;
+      part[2 * kG + 1 * kF + f] = hacc01.y;
+      part[2 * kG + 2 * kF + f] = hacc23.x;
+      part[2 * kG + 3 * kF + f] = hacc23.y;
 
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -726,7 +742,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         racc[2] = fmaf(pv.z, r, racc[2]);
         racc[3] = fmaf(pv.w, r, racc[3]);
       }
-      for (int ei = qt + 4 * kResPrefetch; ei < nres; ei += 4) {   // rows beyond the prefetch
+      for (int ei = hf + 2 * kResPrefetch; ei < nres; ei += 2) {   // rows beyond the prefetch
         const uint32_t ent = M->res[ei];
         const int row = (int)(ent & 255u);
         if (row == 255) continue;
@@ -737,32 +753,20 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         racc[2] = fmaf(pv.z, r, racc[2]);
         racc[3] = fmaf(pv.w, r, racc[3]);
       }
-      float* pr = part + 2 * kG + kG * kF + (size_t)qt * kG * kD;
+      float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
 #pragma unroll
       for (int g = 0; g < kG; ++g) pr[g * kD + j] = racc[g];
-      named_bar_sync(1, kEpiThreads);   // token half 1's sums are in shared memory
-      if (th == 0) {
-        const float4 o = *hx4;
-        part[2 * kG + 0 * kF + f] = hacc01.x + o.x;
-        part[2 * kG + 1 * kF + f] = hacc01.y + o.y;
-        part[2 * kG + 2 * kF + f] = hacc23.x + o.z;
-        part[2 * kG + 3 * kF + f] = hacc23.y + o.w;
-      }
-      if (ew == 0 && lane < 2 * kG) part[lane] = s_ml[u * 8 + lane];
+      if (eb == 0 && lane < 2 * kG) part[lane] = s_ml[u * 8 + lane];
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_META_EMPTY0 + slot));
-      return good;
+      if (lane == 0) {
+        mbar_arrive(bar(BAR_P_EMPTY0 + u));
+        mbar_arrive(bar(BAR_META_EMPTY0 + slot));
+      }
+      if (!good) *abort_flag = 1;
+      return true;
     };
-
-    // Every epilogue thread runs the full sequence; once the abort flag is set, the
-    // remaining waits return at once and the results are discarded by the caller.
-    bool more = part_a(0);
-    for (int i = 0; more; ++i) {
-      const bool next = part_a(i + 1);   // or the end marker (it also prefetches for B(i))
-      ok = part_b(i) && ok;
-      more = next;
+    for (int i = 0; part_b(i); ++i) {
     }
-    if (!ok) *abort_flag = 1;
   }
 
   tc_fence_before();

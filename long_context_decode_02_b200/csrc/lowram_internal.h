@@ -94,8 +94,8 @@ int attend_simt_tile_tokens(const Dims& dm);
 cudaError_t launch_attend_simt(const AttendArgs& a, cudaStream_t s);
 
 bool attend_tc_supported(const Dims& dm);
-// residual-sum slots in a tcgen05 partial (one per epilogue quarter)
-constexpr int kTcResSlots = 4;
+// residual-sum slots in a tcgen05 partial (one per half of the residual rows)
+constexpr int kTcResSlots = 2;
 size_t attend_tc_part_floats(const Dims& dm, int n_tiles);
 constexpr int kTcTileTokens = 128;
 cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s);
