@@ -57,7 +57,6 @@ struct TcMaps {
   CUtensorMap coef;   // [B*T][r] bf16, box 64 x 8,  128B swizzle (64-column blocks)
   CUtensorMap coef64; // [B*T][r] bf16, box 32 x 8,   64B swizzle (a last 32-column block)
   CUtensorMap basis;  // [H*d][r] bf16, box 32 x 128, 64B swizzle
-  CUtensorMap w1;     // [H*F][d] bf16, box 64 x 128, 128B swizzle
 };
 
 // One slot of the metadata ring (filled by the metadata warp up to kMetaSlots tiles
@@ -80,7 +79,7 @@ constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in fli
 constexpr int kRotStride = kD / 2 + 2;
 
 struct Layout {
-  uint32_t basis, w1, coef, kbf, p, q, b1, zx, red, rot, roff, meta, bar, total;
+  uint32_t basis, coef, kbf, p, p2, q, b1, zx, red, rot, roff, meta, bar, total;
 };
 __host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
@@ -89,11 +88,11 @@ __host__ __device__ inline Layout make_layout(int r) {
   Layout L{};
   const uint32_t kb = (uint32_t)r / 32;
   L.basis = 0;
-  L.w1 = align_up(L.basis + kb * 8192, 1024);
-  L.coef = L.w1 + 65536;
-  L.kbf = align_up(L.coef + kb * 8192, 1024);   // K~ bf16 [128 tok][128 d], one buffer
+  L.coef = align_up(L.basis + kb * 8192, 1024);   // two coefficient tile buffers
+  L.kbf = align_up(L.coef + 2 * kb * 8192, 1024);  // K~ bf16 [128 tok][128 d], one buffer
   L.p = L.kbf + 32768;          // [2][128][4] fp32
-  L.q = L.p + 4096;             // [4][128] fp32
+  L.p2 = L.p + 4096;            // [2][64 token pairs][4][2] fp32: P by token pairs
+  L.q = L.p2 + 4096;            // [4][64][2] fp32: (q_x, q_y) of each rotary pair
   L.b1 = L.q + 2048;            // [256] fp32
   L.zx = L.b1 + 1024;           // [128][4] fp32: the second pair half's partial logits
   L.red = L.zx + 2048;          // 512 B of reduction scratch
@@ -107,8 +106,8 @@ __host__ __device__ inline Layout make_layout(int r) {
 
 // barrier slots (8 bytes each) inside L.bar
 enum {
-  BAR_W = 0, BAR_COEF_FULL, BAR_COEF_EMPTY, BAR_KT_FULL0, BAR_KT_FULL1, BAR_KT_EMPTY0,
-  BAR_KT_EMPTY1, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN, BAR_DRAIN_H,
+  BAR_W = 0, BAR_W1T, BAR_COEF_FULL0, BAR_COEF_FULL1, BAR_COEF_EMPTY0, BAR_COEF_EMPTY1,
+  BAR_KT_FULL, BAR_KT_EMPTY, BAR_KBF_FULL, BAR_KBF_EMPTY, BAR_H_FULL, BAR_H_EMPTY, BAR_DRAIN, BAR_DRAIN_H,
   BAR_P_FULL0, BAR_P_FULL1, BAR_P_EMPTY0, BAR_P_EMPTY1,
   BAR_ROT_FULL0, BAR_ROT_EMPTY0 = BAR_ROT_FULL0 + kRotSlots,
   BAR_META_FULL0 = BAR_ROT_EMPTY0 + kRotSlots, BAR_META_EMPTY0 = BAR_META_FULL0 + kMetaSlots,
@@ -165,6 +164,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.bar + 8 * BAR_COUNT + 4);
   float* sP = reinterpret_cast<float*>(gbase + L.p);
   float* sQ = reinterpret_cast<float*>(gbase + L.q);
+  float* sP2 = reinterpret_cast<float*>(gbase + L.p2);
   float* sB1 = reinterpret_cast<float*>(gbase + L.b1);
   float* sZx = reinterpret_cast<float*>(gbase + L.zx);
   float* sRed = reinterpret_cast<float*>(gbase + L.red);  // [4 quadrants][4 g] x 2, ml[2][4][2]
@@ -180,12 +180,13 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(BAR_W), 1);
-    mbar_init(bar(BAR_COEF_FULL), 1);
-    mbar_init(bar(BAR_COEF_EMPTY), 1);
-    mbar_init(bar(BAR_KT_FULL0), 1);
-    mbar_init(bar(BAR_KT_FULL1), 1);
-    mbar_init(bar(BAR_KT_EMPTY0), kEpiWarpsA);
-    mbar_init(bar(BAR_KT_EMPTY1), kEpiWarpsA);
+    mbar_init(bar(BAR_W1T), kEpiWarpsA + kEpiWarpsB);
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(bar(BAR_COEF_FULL0 + c), 1);
+      mbar_init(bar(BAR_COEF_EMPTY0 + c), 1);
+    }
+    mbar_init(bar(BAR_KT_FULL), 1);
+    mbar_init(bar(BAR_KT_EMPTY), kEpiWarpsA);
     mbar_init(bar(BAR_KBF_FULL), kEpiWarpsA);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(BAR_P_FULL0 + i), 1);
@@ -219,19 +220,40 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int32_t* sel_all = a.sel;
+  // W1_h into Tensor Memory as the hidden-layer GEMM's A operand: row f = 128 hf + lane
+  // of half hf in lane `lane`, columns 128 + 64 hf + (0..63) holding bf16 pairs along d.
+  // Each epilogue warp (quadrant of trow, half hf, d-half dh) writes 32 columns from one
+  // batch of eight 16-byte loads per thread.
+  auto w1_to_tmem = [&](int hf, int dh, int trow, uint32_t lane_addr) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(
+        (const __nv_bfloat16*)a.w1 + ((size_t)h * kF + 128 * hf + trow) * kD + 64 * dh);
+    uint32_t v[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 x = __ldg(wrow + j);
+      v[4 * j] = x.x;
+      v[4 * j + 1] = x.y;
+      v[4 * j + 2] = x.z;
+      v[4 * j + 3] = x.w;
+    }
+    const uint32_t col = tmem + lane_addr + 128u + (uint32_t)(64 * hf + 32 * dh);
+    tmem_st_x16(col, v);
+    tmem_st_x16(col + 16, v + 16);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar(BAR_W1T));
+  };
   if (warp == 0) {
     // ------------------------------------------------------------ TMA warp
-    // Weights once; then per tile the coefficient rows of its 16 chunks (chunk ids from
-    // the tile's metadata slot), TMA-gathered into the 64B-swizzled tile buffer.
-    int issued_phase = -1;  // parity of the last coef load issued (for the drain)
+    // The basis once; then per tile the coefficient rows of its 16 chunks (chunk ids from
+    // the tile's metadata slot), TMA-gathered into one of two tile buffers, so the next
+    // tile's gather overlaps this tile's GEMM.
+    int last0 = -1, last1 = -1;   // last tile loaded into each buffer (for the drain)
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192 + 65536));
+      mbar_arrive_expect_tx(bar(BAR_W), (uint32_t)(kb_r * 8192));
       for (int kb = 0; kb < kb_r; ++kb)
         tma_load_2d(base + L.basis + kb * 8192, &maps.basis, kb * 32, h * kD, bar(BAR_W));
-      for (int hf = 0; hf < 2; ++hf)
-        for (int kb = 0; kb < 2; ++kb)
-          tma_load_2d(base + L.w1 + (hf * 2 + kb) * 16384, &maps.w1, kb * 64,
-                      h * kF + hf * 128, bar(BAR_W));
     }
     for (int i = 0;; ++i) {
       const int slot = i % kMetaSlots;
@@ -239,7 +261,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       if (lane == 0) {
         got = mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag);
         it = got ? meta[slot].item : -1;
-        if (it >= 0) got = mbar_wait_bounded(bar(BAR_COEF_EMPTY), (i & 1) ^ 1, abort_flag);
+        if (it >= 0)
+          got = mbar_wait_bounded(bar(BAR_COEF_EMPTY0 + (i & 1)), ((i >> 1) & 1) ^ 1, abort_flag);
       }
       it = __shfl_sync(0xffffffffu, it, 0);
       if (!__shfl_sync(0xffffffffu, got, 0) || it < 0) break;
@@ -248,43 +271,47 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       const int cid = lane < kChunksPerTile ? meta[slot].cid[lane] : -1;
       // each chunk: r/64 boxes of 64 columns (128B swizzle) and, when 64 does not divide
       // r, one box of the last 32 columns (64B swizzle): 3 boxes per chunk at r = 160
-      if (lane == 0)
-        mbar_arrive_expect_tx(bar(BAR_COEF_FULL), (uint32_t)(kChunksPerTile * kb_r * 512));
+      const uint32_t cbuf = base + L.coef + (uint32_t)((i & 1) * kb_r * 8192);
+      const uint32_t cfull = bar(BAR_COEF_FULL0 + (i & 1));
+      if (lane == 0) mbar_arrive_expect_tx(cfull, (uint32_t)(kChunksPerTile * kb_r * 512));
       __syncwarp();
       if (lane < kChunksPerTile) {
         const int row = b * dm.T + (cid < 0 ? 0 : cid) * kChunk;
         for (int c2 = 0; c2 < n128; ++c2)
-          tma_load_2d(base + L.coef + c2 * 16384 + lane * 1024, &maps.coef, c2 * 64, row,
-                      bar(BAR_COEF_FULL));
+          tma_load_2d(cbuf + c2 * 16384 + lane * 1024, &maps.coef, c2 * 64, row, cfull);
         if (has64)
-          tma_load_2d(base + L.coef + n128 * 16384 + lane * 512, &maps.coef64, n128 * 64, row,
-                      bar(BAR_COEF_FULL));
+          tma_load_2d(cbuf + n128 * 16384 + lane * 512, &maps.coef64, n128 * 64, row, cfull);
       }
-      issued_phase = i & 1;
+      if (i & 1) last1 = i; else last0 = i;
     }
-    // drain: a load still in flight (only possible after an abort) must land before exit
-    if (lane == 0 && *abort_flag && issued_phase >= 0) {
-      int dummy = 0;
-      mbar_wait_bounded(bar(BAR_COEF_FULL), (uint32_t)issued_phase, (volatile int*)&dummy);
+    // drain: loads still in flight (only possible after an abort) must land before exit
+    if (lane == 0 && *abort_flag) {
+      for (int c = 0; c < 2; ++c) {
+        const int li = c ? last1 : last0;
+        if (li < 0) continue;
+        int dummy = 0;
+        mbar_wait_bounded(bar(BAR_COEF_FULL0 + c), (uint32_t)((li >> 1) & 1),
+                          (volatile int*)&dummy);
+      }
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ metadata warp
     // Per tile: chunk ids, the residual rows of its chunks (CSR spans, every index
     // bounds-checked), its queries, and the rotation of each chunk's base position,
-    // up to kMetaSlots (kRotSlots for rotations) tiles ahead of the epilogue. The next
-    // tile's chunk ids are fetched while the current tile is built.
+    // up to kMetaSlots (kRotSlots for rotations) tiles ahead of the epilogue.
+    // The four dependent global reads of a tile (its item from the head's counter, its
+    // chunk ids, their CSR spans, the residual rows) are software-pipelined over four
+    // tiles: one pass of the loop issues the counter take of tile j + 3, the chunk ids of
+    // j + 2, the spans of j + 1 and the residual rows of j, so a tile costs about one
+    // memory round trip instead of four.
     const int32_t* ptr_all = a.chunk_ptr;
     const int32_t* ridx_all = a.res_idx;
-    // theta_i for this lane's pairs (lane, lane + 32)
-    const double th0 = a.rope.theta64[lane], th1 = a.rope.theta64[lane + 32];
+    // tiles come from this head's counter (lane 0 takes, the warp learns it later)
+    auto take_raw = [&]() -> int { return lane == 0 ? atomicAdd(a.item_ctr + h, 1) : 0; };
+    // chunk ids of item `it` (issued, not waited for); -1 past the selection
     auto load_cid = [&](int it) -> int {
       int b, tile;
       item_of(it, b, tile);
-      if (a.wait_ready) {   // the selection kernel may still be running: wait for this pair
-        int ok = 1;
-        if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) return -1;
-      }
       int cid = -1;
       if (lane < kChunksPerTile) {
         const int gs = tile * kChunksPerTile + lane;
@@ -292,16 +319,50 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       }
       return cid;
     };
-    // tiles come from this head's counter, one taken ahead
-    auto take = [&]() -> int {
-      int it = 0;
-      if (lane == 0) it = atomicAdd(a.item_ctr + h, 1);
-      return __shfl_sync(0xffffffffu, it, 0);
+    // when the selection kernel may still be running: wait until item it's pair is
+    // published (acquire); false after a timeout (the abort flag is then set)
+    auto pair_ready = [&](int it) -> bool {
+      if (!a.wait_ready) return true;
+      int b, tile;
+      item_of(it, b, tile);
+      int ok = 1;
+      if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
-    int it_next = take();
-    int cid_next = it_next < n_items ? load_cid(it_next) : -1;
+    // an id outside [-1, Nc) is reported and dropped (the chunk is skipped)
+    auto sanitize = [&](int cid) -> int {
+      if (lane < kChunksPerTile && (cid >= dm.Nc || cid < -1)) {
+        raise_status(a.status, kStatusDeviceCheck);
+        return -1;
+      }
+      return cid;
+    };
+    // CSR span reads of item it's chunk cid (issued, validated one stage later)
+    auto load_span = [&](int it, int cid, int& e0, int& e1) {
+      e0 = 0;
+      e1 = 0;
+      if (it < n_items && lane < kChunksPerTile && cid >= 0) {
+        int b, tile;
+        item_of(it, b, tile);
+        const int32_t* ptr = ptr_all + (size_t)(b * dm.H + h) * (dm.Nc + 1);
+        e0 = ptr[cid];
+        e1 = ptr[cid + 1];
+      }
+    };
+    int rot_issued = -1;   // last tile whose rotations were requested (for the drain)
+    // prologue: items of tiles 0..2, chunk ids of 0 and 1, spans of 0
+    int tk0 = take_raw(), tk1 = take_raw(), tk2 = take_raw();
+    int it0 = __shfl_sync(0xffffffffu, tk0, 0);
+    int it1 = __shfl_sync(0xffffffffu, tk1, 0);
+    int it2 = __shfl_sync(0xffffffffu, tk2, 0);
+    int cid0 = -1, cid1 = -1;
+    if (it0 < n_items && pair_ready(it0)) cid0 = load_cid(it0);
+    if (it1 < n_items && pair_ready(it1)) cid1 = load_cid(it1);
+    cid0 = sanitize(cid0);
+    int e0r, e1r;
+    load_span(it0, cid0, e0r, e1r);
     for (int i = 0;; ++i) {
-      const int it = it_next;
+      const int it = it0;
       const int slot = i % kMetaSlots;
       if (it >= n_items) {   // no more tiles: post the end marker
         int got = 0;
@@ -313,64 +374,55 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         }
         break;
       }
+      // issue: the take of tile i + 3, the queries and residual rows of tile i, the spans
+      // of tile i + 1, the chunk ids of tile i + 2
+      const int tk3 = take_raw();
       int b, tile;
       item_of(it, b, tile);
       const int p = b * dm.H + h;
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
       const uint4 q0 = qsrc[lane], q1 = qsrc[lane + 32];
-      int cid = cid_next;
-      it_next = take();
-      if (it_next < n_items) cid_next = load_cid(it_next);
-      if (lane < kChunksPerTile && cid >= dm.Nc) {
-        raise_status(a.status, kStatusDeviceCheck);
-        cid = -1;
+      const int cid = cid0;
+      int e0 = 0, n = 0;
+      if (lane < kChunksPerTile && cid >= 0) {
+        if (e0r < 0 || e1r < e0r || e1r > dm.n_res || e1r - e0r > kChunk) {
+          raise_status(a.status, kStatusDeviceCheck);
+        } else {
+          e0 = e0r;
+          n = e1r - e0r;
+        }
       }
-      if (cid < -1) {
-        raise_status(a.status, kStatusDeviceCheck);
-        cid = -1;
-      }
+      const int32_t* ridx = ridx_all + (size_t)p * dm.n_res + e0;
+      int t[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
+      cid1 = sanitize(cid1);
+      load_span(it1, cid1, e0r, e1r);
+      int cid2 = -1;
+      if (it2 < n_items && pair_ready(it2)) cid2 = load_cid(it2);
+
       int got = 0;
       if (lane == 0)
         got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       TileMeta* M = meta + slot;
-      int e0 = 0, n = 0;
-      if (lane < kChunksPerTile) {
-        if (cid >= 0) {
-          const int32_t* ptr = ptr_all + (size_t)p * (dm.Nc + 1);
-          e0 = ptr[cid];
-          const int e1 = ptr[cid + 1];
-          if (e0 < 0 || e1 < e0 || e1 > dm.n_res || e1 - e0 > kChunk) {
-            raise_status(a.status, kStatusDeviceCheck);
-            n = 0;
-          } else {
-            n = e1 - e0;
-          }
-        }
-        M->cid[lane] = cid;
-      }
+      if (lane < kChunksPerTile) M->cid[lane] = cid;
       int incl = n;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
       const int off = incl - n;
       const int total = __shfl_sync(0xffffffffu, incl, 31);
-      if (n > 0) {
-        const int32_t* ridx = ridx_all + (size_t)p * dm.n_res + e0;
-        int t[kChunk];
 #pragma unroll
-        for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
-#pragma unroll
-        for (int j = 0; j < kChunk; ++j) {
-          if (j < n) {
-            const int tt = t[j] - cid * kChunk;
-            const bool good = tt >= 0 && tt < kChunk;
-            if (!good) raise_status(a.status, kStatusDeviceCheck);
-            M->res[off + j] = ((uint32_t)(e0 + j) << 8) | (good ? (uint32_t)(lane * kChunk + tt) : 255u);
-          }
+      for (int j = 0; j < kChunk; ++j) {
+        if (j < n) {
+          const int tt = t[j] - cid * kChunk;
+          const bool good = tt >= 0 && tt < kChunk;
+          if (!good) raise_status(a.status, kStatusDeviceCheck);
+          M->res[off + j] = ((uint32_t)(e0 + j) << 8) | (good ? (uint32_t)(lane * kChunk + tt) : 255u);
         }
       }
       if (lane == 0) {
@@ -381,46 +433,51 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       M->q[lane + 32] = q1;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_META_FULL0 + slot));
-      // chunk-base rotations (cos, sin)(8 cid theta_i): the angle is reduced modulo 2 pi
-      // in fp64 (error ~1e-11 rad) and its sine and cosine taken in fp32 (|err| < 4e-7)
+      // chunk-base rotations (cos, sin)(C cid theta_i) of the tile's chunks: one 512-byte
+      // row of the context's table per chunk, copied by the TMA engine (row 0 for a slot
+      // past the selection)
       {
         const int rs = i % kRotSlots;
         int rgot = 0;
         if (lane == 0)
           rgot = mbar_wait_bounded(bar(BAR_ROT_EMPTY0 + rs), ((i / kRotSlots) & 1) ^ 1, abort_flag);
         if (!__shfl_sync(0xffffffffu, rgot, 0)) break;
-        float2* R = sRot + rs * kChunksPerTile * kRotStride;
-        const double two_pi_hi = 6.283185307179586232, two_pi_lo = 2.4492935982947064e-16;
-        const double inv_two_pi = 0.15915494309189533577;
-#pragma unroll 4
-        for (int c = 0; c < kChunksPerTile; ++c) {
-          const int cc = __shfl_sync(0xffffffffu, cid, c);
-          const double pb = (double)((cc < 0 ? 0 : cc) * kChunk);
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const double ang = pb * (w ? th1 : th0);
-            const double kq = rint(ang * inv_two_pi);
-            const float red = (float)fma(-kq, two_pi_lo, fma(-kq, two_pi_hi, ang));
-            float sn, cs;
-            __sincosf(red, &sn, &cs);
-            R[c * kRotStride + w * 32 + lane] = make_float2(cs, sn);
-          }
-        }
+        const uint32_t rfull = bar(BAR_ROT_FULL0 + rs);
+        if (lane == 0) mbar_arrive_expect_tx(rfull, (uint32_t)(kChunksPerTile * (kD / 2) * 8));
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_ROT_FULL0 + rs));
+        if (lane < kChunksPerTile)
+          bulk_load(smem_u32(sRot + (rs * kChunksPerTile + lane) * kRotStride),
+                    a.rope.chunk32 + (size_t)(cid < 0 ? 0 : cid) * (kD / 2), (kD / 2) * 8, rfull);
+        rot_issued = i;
+      }
+      // advance the pipeline
+      it0 = it1;
+      it1 = it2;
+      it2 = __shfl_sync(0xffffffffu, tk3, 0);
+      cid0 = cid1;
+      cid1 = cid2;
+    }
+    // drain: rotation copies still in flight (only possible after an abort) land first
+    if (lane == 0 && *abort_flag) {
+      for (int t = rot_issued - kRotSlots + 1; t <= rot_issued; ++t) {
+        if (t < 0) continue;
+        int dummy = 0;
+        mbar_wait_bounded(bar(BAR_ROT_FULL0 + t % kRotSlots), (uint32_t)((t / kRotSlots) & 1),
+                          (volatile int*)&dummy);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait_bounded(bar(BAR_W), 0, abort_flag);
-      const uint32_t sb = base + L.basis, sc = base + L.coef;
+      const uint32_t sb = base + L.basis, sc0 = base + L.coef;
       auto issue_k = [&](int i) -> bool {
-        const int u = i & 1;
-        if (!mbar_wait_bounded(bar(BAR_COEF_FULL), i & 1, abort_flag)) return false;
-        if (!mbar_wait_bounded(bar(BAR_KT_EMPTY0 + u), ((i >> 1) & 1) ^ 1, abort_flag)) return false;
+        const int c = i & 1;   // coefficient buffer
+        if (!mbar_wait_bounded(bar(BAR_COEF_FULL0 + c), (i >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_bounded(bar(BAR_KT_EMPTY), (i & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t d_t = tmem + (uint32_t)(u * 128);
+        const uint32_t d_t = tmem;   // K~ (one buffer, columns 0..127)
+        const uint32_t sc = sc0 + (uint32_t)(c * kb_r * 8192);
         for (int s = 0; s < ksteps_r; ++s) {
           const uint32_t off = (uint32_t)((s >> 1) * 8192 + (s & 1) * 32);   // basis
           const uint64_t adesc =
@@ -431,8 +488,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
                                      kSwizzle64B);
           mma_bf16(d_t, adesc, smem_desc_kmajor(sb + off, 512, kSwizzle64B), kIdesc, s > 0);
         }
-        mma_commit(bar(BAR_KT_FULL0 + u));
-        mma_commit(bar(BAR_COEF_EMPTY));
+        mma_commit(bar(BAR_KT_FULL));
+        mma_commit(bar(BAR_COEF_EMPTY0 + c));
         return true;
       };
       // whether tile i exists, from its metadata slot (read before the slot can recycle)
@@ -452,8 +509,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   } else if (warp == kHWarp) {
     // ------------------------------------------------------------ hidden-layer MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait_bounded(bar(BAR_W), 0, abort_flag);
-      const uint32_t sw1 = base + L.w1, skb = base + L.kbf;
+      // W1_h is the A operand, in Tensor Memory (columns 128 + 64 hf ..), written there by
+      // the part-A warps at the start
+      bool ok = mbar_wait_bounded(bar(BAR_W1T), 0, abort_flag);
+      const uint32_t skb = base + L.kbf;
       for (int i = 0; ok; ++i) {
         const int slot = i % kMetaSlots;
         if (!mbar_wait_bounded(bar(BAR_META_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag) ||
@@ -466,8 +525,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           const uint32_t d_t = tmem + 256u + (uint32_t)hf * 128u;
           for (int s = 0; s < 8; ++s) {
             const uint32_t off = (uint32_t)((s >> 2) * 16384 + (s & 3) * 32);
-            mma_bf16(d_t, smem_desc_kmajor(sw1 + hf * 32768 + off, 1024, kSwizzle128B),
-                     smem_desc_kmajor(skb + off, 1024, kSwizzle128B), kIdesc, s > 0);
+            mma_bf16_ta(d_t, tmem + 128u + (uint32_t)(hf * 64 + 8 * s),
+                        smem_desc_kmajor(skb + off, 1024, kSwizzle128B), kIdesc, s > 0);
           }
         }
         mma_commit(bar(BAR_H_FULL));
@@ -490,6 +549,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const float zscale = 1.4426950408889634f * rsqrtf((float)kD);
     float* s_ml = sRed + 64;  // [2][4][2]
+    w1_to_tmem(ha, 0, trow, lane_addr);
     // in-chunk offsets: sRoff[pair * 8 + j] = (cos, sin)(j theta_pair), j < 8
     for (int i = et; i < (kD / 2) * kChunk; i += kEpiThreadsA)
       sRoff[i] = a.rope.lo32[(i & (kChunk - 1)) * (kD / 2) + (i >> 3)];
@@ -507,13 +567,14 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         return false;
       }
       const bool valid = M->cid[trow >> 3] >= 0;
-      {
+      {   // sQ[g][i][w] = q_g[i + 64 w]: each rotary pair's two query components adjacent
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
         const float2 f = bf2_to_f2(w);
-        sQ[2 * et] = f.x;
-        sQ[2 * et + 1] = f.y;
+        const int g = et >> 6, d0 = 2 * (et & 63), hw = d0 >> 6, i0 = d0 & 63;
+        sQ[g * kD + 2 * i0 + hw] = f.x;
+        sQ[g * kD + 2 * i0 + 2 + hw] = f.y;
       }
-      good = mbar_wait_bounded(bar(BAR_KT_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
+      good = mbar_wait_bounded(bar(BAR_KT_FULL), i & 1, abort_flag) && good;
       const int rs = i % kRotSlots;
       good = mbar_wait_bounded(bar(BAR_ROT_FULL0 + rs), (i / kRotSlots) & 1, abort_flag) && good;
       named_bar_sync(1, kEpiThreadsA);  // sQ ready
@@ -532,14 +593,14 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         // pairs p0 .. p0 + 15 of this thread's token: K~ columns p0.. and 64 + p0..
         const int p0 = 32 * ha + 16 * sb;
         float x[16], y[16];
-        const uint32_t tcol = tmem + lane_addr + (uint32_t)(u * 128 + p0);
+        const uint32_t tcol = tmem + lane_addr + (uint32_t)p0;
         tmem_ld_x16(tcol, x);
         tmem_ld_x16(tcol + 64, y);
         tmem_wait_ld();
         if (sb == 1) {   // both halves of this thread's K~ columns are in registers
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY0 + u));
+          if (lane == 0) mbar_arrive(bar(BAR_KT_EMPTY));
         }
         // RoPE on pairs (p0 + e, 64 + p0 + e): the chunk-base rotation (from the ring)
         // times the in-chunk offset (table) by angle addition; partial logits accumulate as
@@ -561,12 +622,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           const int pi = p0 + e4;
 #pragma unroll
           for (int g = 0; g < kG; ++g) {
-            const float4 qx = *reinterpret_cast<const float4*>(sQ + g * kD + pi);
-            const float4 qy = *reinterpret_cast<const float4*>(sQ + g * kD + 64 + pi);
-            z2[g] = __ffma2_rn(make_float2(qx.x, qy.x), rot[0], z2[g]);
-            z2[g] = __ffma2_rn(make_float2(qx.y, qy.y), rot[1], z2[g]);
-            z2[g] = __ffma2_rn(make_float2(qx.z, qy.z), rot[2], z2[g]);
-            z2[g] = __ffma2_rn(make_float2(qx.w, qy.w), rot[3], z2[g]);
+            const float4 qa = *reinterpret_cast<const float4*>(sQ + g * kD + 2 * pi);
+            const float4 qb = *reinterpret_cast<const float4*>(sQ + g * kD + 2 * pi + 4);
+            z2[g] = __ffma2_rn(make_float2(qa.x, qa.y), rot[0], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qa.z, qa.w), rot[1], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qb.x, qb.y), rot[2], z2[g]);
+            z2[g] = __ffma2_rn(make_float2(qb.z, qb.w), rot[3], z2[g]);
           }
         }
 #pragma unroll
@@ -614,6 +675,16 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           pv[g] = valid ? ex2_approx(z[g] - m[g]) : 0.f;
         }
         *reinterpret_cast<float4*>(sP + u * 512 + 4 * trow) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+        {   // sP2[u][t / 2][g][t % 2]: the weights of tokens 2m and 2m + 1 side by side
+          float po[kG];
+#pragma unroll
+          for (int g = 0; g < kG; ++g) po[g] = __shfl_down_sync(0xffffffffu, pv[g], 1);
+          if ((lane & 1) == 0) {
+            float4* d2 = reinterpret_cast<float4*>(sP2 + u * 512 + 4 * trow);
+            d2[0] = make_float4(pv[0], po[0], pv[1], po[1]);
+            d2[1] = make_float4(pv[2], po[2], pv[3], po[3]);
+          }
+        }
 #pragma unroll
         for (int g = 0; g < kG; ++g) {
           const float l = warp_sum(pv[g]);
@@ -647,6 +718,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     const uint32_t lane_addr = (uint32_t)(32 * qd) << 16;
     const __nv_bfloat16* rval_all = (const __nv_bfloat16*)a.res_val;
     const float* s_ml = sRed + 64;
+    w1_to_tmem(hf, 1, trow, lane_addr);
     for (int i = etb; i < kF; i += kEpiThreadsB)
       sB1[i] = __bfloat162float(((const __nv_bfloat16*)a.b1)[(size_t)h * kF + i]);
     named_bar_sync(3, kEpiThreadsB);
@@ -692,7 +764,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       const int f = 128 * hf + trow;
       const float bias = sB1[f];
       float2 hacc01 = make_float2(0.f, 0.f), hacc23 = make_float2(0.f, 0.f);
+      float2 acc2[kG];   // per head: (even tokens, odd tokens)
+#pragma unroll
+      for (int g = 0; g < kG; ++g) acc2[g] = make_float2(0.f, 0.f);
       const float4* P4 = reinterpret_cast<const float4*>(sP + u * 512);
+      const float4* P2 = reinterpret_cast<const float4*>(sP2 + u * 512);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float hv[32];
@@ -706,11 +782,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           for (int e = 0; e < 32; e += 2) {
             const float2 hx = __ffma2_rn(half2, make_float2(hv[e], hv[e + 1]), hb2);
             const float2 av = __ffma2_rn(hx, make_float2(tanh_approx(hx.x), tanh_approx(hx.y)), hx);
-            const float4 p0 = P4[32 * c + e], p1 = P4[32 * c + e + 1];
-            hacc01 = __ffma2_rn(make_float2(p0.x, p0.y), make_float2(av.x, av.x), hacc01);
-            hacc23 = __ffma2_rn(make_float2(p0.z, p0.w), make_float2(av.x, av.x), hacc23);
-            hacc01 = __ffma2_rn(make_float2(p1.x, p1.y), make_float2(av.y, av.y), hacc01);
-            hacc23 = __ffma2_rn(make_float2(p1.z, p1.w), make_float2(av.y, av.y), hacc23);
+            const float4 pa = P2[32 * c + e], pb = P2[32 * c + e + 1];   // tokens (e, e + 1)
+            acc2[0] = __ffma2_rn(make_float2(pa.x, pa.y), av, acc2[0]);
+            acc2[1] = __ffma2_rn(make_float2(pa.z, pa.w), av, acc2[1]);
+            acc2[2] = __ffma2_rn(make_float2(pb.x, pb.y), av, acc2[2]);
+            acc2[3] = __ffma2_rn(make_float2(pb.z, pb.w), av, acc2[3]);
           }
         } else {
 #pragma unroll
@@ -725,6 +801,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
+      if (ACT == LOWRAM_ACT_SILU) {
+        hacc01 = make_float2(acc2[0].x + acc2[0].y, acc2[1].x + acc2[1].y);
+        hacc23 = make_float2(acc2[2].x + acc2[2].y, acc2[3].x + acc2[3].y);
+      }
       part[2 * kG + 0 * kF + f] = hacc01.x;
       part[2 * kG + 1 * kF + f] = hacc01.y;
       part[2 * kG + 2 * kF + f] = hacc23.x;
@@ -929,8 +1009,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   TcMaps maps;
   if (!make_tensor_map_2d(&maps.coef, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 64, 8, 128) ||
       !make_tensor_map_2d(&maps.coef64, a.coef, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.B * dm.T, 32, 8, 64) ||
-      !make_tensor_map_2d(&maps.basis, a.basis, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.H * kD, 32, 128, 64) ||
-      !make_tensor_map_2d(&maps.w1, a.w1, LOWRAM_DTYPE_BF16, kD, (uint64_t)dm.H * kF, 64, 128, 128))
+      !make_tensor_map_2d(&maps.basis, a.basis, LOWRAM_DTYPE_BF16, dm.r, (uint64_t)dm.H * kD, 32, 128, 64))
     return cudaErrorInvalidValue;
   const Layout L = make_layout(dm.r);
   const int n_items = dm.B * a.n_tiles;

@@ -28,6 +28,7 @@ struct lowram_ctx {
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   int* item_ctr;  // device [H]: tile counters of the tcgen05 attend kernel, 0 between calls
   double* theta64;  // device [d/2]
+  float2* chunk32;  // device [T/C][d/2]: (cos, sin)(c C theta_i)
 };
 
 namespace {
@@ -135,6 +136,7 @@ RopeTables rope_of(const lowram_ctx* ctx) {
   r.n_hi = ctx->n_hi;
   r.half = ctx->cfg.head_dim / 2;
   r.theta64 = ctx->theta64;
+  r.chunk32 = ctx->chunk32;
   return r;
 }
 
@@ -237,6 +239,8 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
   std::vector<float2> lo32((size_t)half * kRopeLo), hi32((size_t)half * ctx->n_hi);
   std::vector<double2> lo64((size_t)half * kRopeLo), hi64((size_t)half * ctx->n_hi);
   std::vector<double> th64((size_t)half);
+  const size_t n_chunks = (size_t)(c->n_tokens / c->chunk);
+  std::vector<float2> chunk32(n_chunks * half);
   for (int i = 0; i < half; ++i) {
     const double th = std::pow(c->rope_theta, -2.0 * i / c->head_dim);
     th64[i] = th;
@@ -250,6 +254,10 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
       hi64[(size_t)j * half + i] = make_double2(std::cos(ang), std::sin(ang));
       hi32[(size_t)j * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
     }
+    for (size_t cc = 0; cc < n_chunks; ++cc) {
+      const double ang = (double)(cc * (size_t)c->chunk) * th;
+      chunk32[cc * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
   }
   const size_t pairs = (size_t)c->batch * c->n_kv_heads;
   bool ok = cudaMalloc(&ctx->lo32, lo32.size() * sizeof(float2)) == cudaSuccess &&
@@ -261,7 +269,8 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->item_ctr, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
-            cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess;
+            cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess &&
+            cudaMalloc(&ctx->chunk32, chunk32.size() * sizeof(float2)) == cudaSuccess;
   ok = ok &&
        cudaMemcpy(ctx->lo32, lo32.data(), lo32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->hi32, hi32.data(), hi32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -272,7 +281,8 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->item_ctr, 0, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
-       cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess;
+       cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess &&
+       cudaMemcpy(ctx->chunk32, chunk32.data(), chunk32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     lowram_destroy(ctx);
@@ -295,6 +305,7 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->ready);
   cudaFree(ctx->item_ctr);
   cudaFree(ctx->theta64);
+  cudaFree(ctx->chunk32);
   delete ctx;
 }
 

@@ -32,6 +32,9 @@ struct RopeTables {
   int n_hi;
   int half;   // d / 2
   const double* theta64;  // theta_i = theta^(-2i/d), i < d/2 (fp64)
+  // chunk-base rotations: chunk32[c * half + i] = (cos, sin)(c C theta_i), c < T / C,
+  // from fp64 on the host
+  const float2* chunk32;
 };
 
 struct Dims {

@@ -46,6 +46,8 @@ using namespace sm100;
 
 constexpr int kConsumers = 256;               // consumer threads (warps 0..7)
 constexpr int kSelectors = 96;                // selection threads (warps 9..11)
+constexpr int kLateWaves = 6;                 // stages per CTA that count as the last wave
+constexpr int kJoinBar = 3;                   // named barrier of the joint selection group
 constexpr int kSelThreads = kConsumers + 32 + kSelectors;  // + producer warp 8
 constexpr int kStages = 3;
 constexpr int kStageBytes = 65536;
@@ -71,11 +73,13 @@ struct Geom {
 struct Misc {
   unsigned hist[512];   // two radix histograms
   unsigned bc[4];
+  unsigned kr[2];       // smallest and largest key of a radix search
   float fscr[33];
   int iscr[33];
   int cnt, n_in, nwin;
   float fmax;           // largest landmark norm among the candidates
-  int req;              // the selection warps' current request
+  int req;              // the selection group's current request
+  int carry;            // a claimed pair handed from the selection warps to the whole group
   int wl[kWindowCap];
 };
 
@@ -359,31 +363,50 @@ __device__ void score64_rows_warp(const T* Lp, const float (&qr)[G][D / 32], con
   }
 }
 
-// The top 8 * kPasses bits of the k-th largest (1 <= k <= n) of n uint32 keys, by kPasses
-// 8-bit radix passes (most significant digit first); the lower bits are returned as
-// zero. Two histograms alternate: the one for pass p + 1 is cleared during pass p.
+// A prefix of the k-th largest (1 <= k <= n) of n uint32 keys, exact in (at least) its
+// top 8 * kPasses bits, the bits below the last resolved digit returned as zero. The bits
+// that all n keys share (above the highest bit where the smallest and the largest key
+// differ) are taken at once; 8-bit radix passes (most significant digit first) resolve
+// the rest, so at most kPasses passes run and usually one fewer. Two histograms
+// alternate: the one for pass p + 1 is cleared during pass p.
 template <int kPasses, typename KeyFn>
 __device__ uint32_t kth_largest_prefix(const Grp& g, int n, int k, KeyFn key_of, Misc* ms) {
   const int lane = g.tid & 31;
   for (int i = g.tid; i < 512; i += g.nt) ms->hist[i] = 0u;
+  if (g.tid == 0) {
+    ms->kr[0] = 0xFFFFFFFFu;
+    ms->kr[1] = 0u;
+  }
   g.sync();
-  uint32_t prefix = 0, mask = 0;
+  {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = g.tid; i < n; i += g.nt) {
+      const uint32_t key = key_of(i);
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      atomicMin(&ms->kr[0], kmin);
+      atomicMax(&ms->kr[1], kmax);
+    }
+  }
+  g.sync();
+  const uint32_t kmin = ms->kr[0], diff = kmin ^ ms->kr[1];
+  const int lb = 32 - 8 * kPasses;                  // lowest bit that must be resolved
+  int hi = diff ? 31 - __clz(diff) : -1;             // highest bit not shared by all keys
+  const uint32_t common = hi < 0 ? 0xFFFFFFFFu : (hi >= 31 ? 0u : ~((2u << hi) - 1u));
+  uint32_t prefix = kmin & common, mask = common;
   unsigned remaining = (unsigned)k;
-#pragma unroll
-  for (int pass = 0; pass < kPasses; ++pass) {
-    const int shift = 24 - 8 * pass;
+  for (int pass = 0; hi >= lb; ++pass) {
+    const int shift = hi - 7;                        // >= 0: hi >= lb >= 8
     unsigned* hist = ms->hist + 256 * (pass & 1);
-    if (pass >= 1 && pass + 1 < kPasses)
+    if (pass >= 1)
       for (int i = g.tid; i < 256; i += g.nt) ms->hist[256 * ((pass + 1) & 1) + i] = 0u;
-    for (int base = 0; base < n; base += g.nt) {
-      const int i = base + g.tid;
-      unsigned digit = 256u;
-      if (i < n) {
-        const uint32_t key = key_of(i);
-        if ((key & mask) == prefix) digit = (key >> shift) & 255u;
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, digit);
-      if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+    for (int i = g.tid; i < n; i += g.nt) {
+      const uint32_t key = key_of(i);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     g.sync();
     if (g.tid < 32) {
@@ -411,6 +434,7 @@ __device__ uint32_t kth_largest_prefix(const Grp& g, int n, int k, KeyFn key_of,
     prefix |= ms->bc[2 * (pass & 1)] << shift;
     mask |= 255u << shift;
     remaining = ms->bc[2 * (pass & 1) + 1];
+    hi = shift - 1;
   }
   return prefix;
 }
@@ -739,6 +763,7 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
     ms->n_in = 0;
     ms->nwin = 0;
     ms->fmax = 0.f;
+    ms->carry = -1;
   }
   __syncthreads();
   // a programmatic dependent (the reconstruct-and-attend kernel) may start as SMs free
@@ -842,24 +867,50 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
     }
-  } else {
-    // ------------------------------------------------------------ selection warps
-    // Take the next (b, h), wait until all of its stages are handed out and all of its
-    // scores have landed, select, restore the sentinel. One verdict per step for the
-    // whole group keeps its barrier sequence uniform.
-    const Grp g{(int)threadIdx.x - (kConsumers + 32), kSelectors, 2};
+  }
+  if (warp != kConsumers / 32) {
+    // ------------------------------------------------------------ selection
+    // The selection warps take the next (b, h), wait until all of its stages are handed
+    // out and all of its scores have landed, select, and restore the sentinel; one
+    // verdict per step for the whole group keeps its barrier sequence uniform. A pair
+    // whose scoring ends in the last wave of stages (about the last kLateWaves stages of
+    // every CTA) is not selected by these three warps: it is handed over, claimed, to the
+    // consumers and the selection warps together (all but the producer), who meet once
+    // the consumers have no stages left and select it several times faster right when
+    // its last scores land, then any pairs still in the queue. The selection warps also
+    // hand over (with no pair) when the queue is empty, so the meeting always happens.
+    const bool sel_warp = warp > kConsumers / 32;
+    const long long late_from = (long long)U - (long long)kLateWaves * gridDim.x;
+    bool joined = !sel_warp;
+    if (!sel_warp) named_bar_sync(kJoinBar, kConsumers + kSelectors);
     for (;;) {
+      const Grp g = joined ? Grp{(int)threadIdx.x < kConsumers ? (int)threadIdx.x
+                                                               : (int)threadIdx.x - 32,
+                                 kConsumers + kSelectors, kJoinBar}
+                           : Grp{(int)threadIdx.x - (kConsumers + 32), kSelectors, 2};
       if (g.tid == 0) {
         int pair = -1;
-        const int at = atomicAdd(q_head, 1);
-        if (at < P && wait_counter_ge(grab, (at + 1) * upp, abort_flag)) pair = at;
+        if (joined && ms->carry >= 0) {
+          pair = ms->carry;
+          ms->carry = -1;
+        } else if (!joined || !*abort_flag) {
+          const int at = atomicAdd(q_head, 1);
+          if (at < P && wait_counter_ge(grab, (at + 1) * upp, abort_flag)) pair = at;
+        }
         ms->req = pair;
       }
       g.sync();
       const int pair = ms->req;
       g.sync();
+      if (!joined && (pair < 0 || (long long)(pair + 1) * upp > late_from)) {
+        if (g.tid == 0) ms->carry = pair;
+        named_bar_sync(kJoinBar, kConsumers + kSelectors);
+        joined = true;
+        continue;
+      }
       if (pair < 0) break;
-      if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) break;
+      // a failed wait has raised the abort flag: the next step ends the loop
+      if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) continue;
       clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
       if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
         __threadfence();
