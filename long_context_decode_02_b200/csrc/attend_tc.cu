@@ -126,6 +126,20 @@ __device__ __forceinline__ float act_fast(float x) {
 
 // Polls *flag until it is non-zero, with acquire semantics (bounded: 2 s, or *abort set;
 // on giving up sets *abort and returns 0).
+// Reduces four values per lane over the warp in one reduce-scatter (6 shuffles instead
+// of 4 x 5): every lane of lane group lane >> 3 gets the reduction of value lane >> 3.
+template <typename Op>
+__device__ __forceinline__ float warp_reduce4_scatter(const float (&v)[4], int lane, Op op) {
+  const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0;
+  const float u0 = op(b4 ? v[2] : v[0], __shfl_xor_sync(0xffffffffu, b4 ? v[0] : v[2], 16));
+  const float u1 = op(b4 ? v[3] : v[1], __shfl_xor_sync(0xffffffffu, b4 ? v[1] : v[3], 16));
+  float w = op(b3 ? u1 : u0, __shfl_xor_sync(0xffffffffu, b3 ? u0 : u1, 8));
+  w = op(w, __shfl_xor_sync(0xffffffffu, w, 4));
+  w = op(w, __shfl_xor_sync(0xffffffffu, w, 2));
+  w = op(w, __shfl_xor_sync(0xffffffffu, w, 1));
+  return w;
+}
+
 __device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -658,10 +672,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         z[1] = valid ? (z[1] + o.y) * zscale : -INFINITY;
         z[2] = valid ? (z[2] + o.z) * zscale : -INFINITY;
         z[3] = valid ? (z[3] + o.w) * zscale : -INFINITY;
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-          const float m = warp_max(z[g]);
-          if (lane == 0) sRed[qd * 4 + g] = m;
+        {   // per-quadrant maxima of the four heads
+          const float m = warp_reduce4_scatter(z, lane, [](float x, float y) { return fmaxf(x, y); });
+          if ((lane & 7) == 0) sRed[qd * 4 + (lane >> 3)] = m;
         }
         // P slot u is free once part B has finished with tile i - 2
         int pe = 1;
@@ -685,10 +698,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
             d2[1] = make_float4(pv[2], po[2], pv[3], po[3]);
           }
         }
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-          const float l = warp_sum(pv[g]);
-          if (lane == 0) sRed[16 + qd * 4 + g] = l;
+        {   // per-quadrant sums of the four heads' weights
+          const float l = warp_reduce4_scatter(pv, lane, [](float x, float y) { return x + y; });
+          if ((lane & 7) == 0) sRed[16 + qd * 4 + (lane >> 3)] = l;
         }
         named_bar_sync(2, 128);
         if (ea == 0 && lane < kG) {
