@@ -46,7 +46,7 @@ using namespace sm100;
 
 constexpr int kConsumers = 256;               // consumer threads (warps 0..7)
 constexpr int kSelectors = 96;                // selection threads (warps 9..11)
-constexpr int kLateWaves = 6;                 // stages per CTA that count as the last wave
+constexpr int kLateWaves = 10;                // stages per CTA that count as the last wave
 constexpr int kJoinBar = 3;                   // named barrier of the joint selection group
 constexpr int kSelThreads = kConsumers + 32 + kSelectors;  // + producer warp 8
 constexpr int kStages = 3;
