@@ -21,7 +21,7 @@
  *     cfg->dtype (fp32 or bf16); index arrays are int32. Arithmetic is fp32 with fp64
  *     used to settle selections near their threshold.
  *   - The caller owns every buffer (inputs, cache, outputs, workspace). The context owns
- *     small tables (RoPE cos/sin, a status word, work counters) and the landmark scores
+ *     tables (RoPE cos/sin, a status word, work counters) and the landmark scores
  *     of one decode step (B*H_kv*N_c floats: 4 MiB at batch 8, 8 KV heads, 128K tokens,
  *     chunk 8), which it keeps in a reset state between calls. Calls allocate nothing.
  *   - Calls are asynchronous on the given stream (a cudaStream_t passed as void*; NULL =
@@ -128,8 +128,10 @@ typedef struct lowram_ctx lowram_ctx;
 lowram_status lowram_check_config(const lowram_config* cfg);
 
 /* Create a context on `device`: checks cfg, builds the RoPE tables (two-level cos/sin of
- * t*theta_i computed in fp64 on the host, stored fp32 and fp64 on the device) and the
- * counters. *out is set only on success. Destroy with lowram_destroy. */
+ * t*theta_i, and the chunk-base cos/sin of c*C*theta_i for every chunk c < N_c:
+ * N_c*d/2 fp32 pairs, 8 MiB at 128K tokens, chunk 8, d 128; all computed in fp64 on the
+ * host, stored fp32 and fp64 on the device) and the counters. *out is set only on
+ * success. Destroy with lowram_destroy. */
 lowram_status lowram_create(const lowram_config* cfg, int device, lowram_ctx** out);
 
 /* Free the context's tables. Waits for nothing: the caller must have synchronised any
