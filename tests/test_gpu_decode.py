@@ -125,7 +125,8 @@ SMALL = synth.CONFIGS[1].replace(name="small", n_tokens=2048, batch=2, seed=77)
     dict(res_frac=0.0),           # no residuals
     dict(res_frac=1.0),           # every token a residual
     dict(rank=128, act=synth.ACT_GELU_ERF),
-], ids=["all", "ragged", "k1", "nores", "allres", "r128gelu"])
+    dict(batch=20, top_k=37),     # 160 (b, h) pairs: more than one per SM
+], ids=["all", "ragged", "k1", "nores", "allres", "r128gelu", "manypairs"])
 def test_edge_cases(L, cuda_device, variant, over):
     sh = SMALL.replace(**over)
     v = L.DECODE_TCGEN05 if variant == "tc" else L.DECODE_SIMT
