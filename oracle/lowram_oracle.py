@@ -144,6 +144,40 @@ def rebuild_keys(coef: np.ndarray, basis: np.ndarray, h: int, d: int) -> np.ndar
     return np.asarray(coef, dtype=np.float64) @ bh.T
 
 
+def cholesky_qr(y: np.ndarray) -> np.ndarray:
+    """Orthonormal basis of the columns of y (full column rank) by Cholesky-QR: with R
+    the upper Cholesky factor of the Gram matrix y^T y (y^T y = R^T R), Q = y R^-1."""
+    y = np.asarray(y, dtype=np.float64)
+    r_up = np.linalg.cholesky(y.T @ y).T
+    return np.linalg.solve(r_up.T, y.T).T
+
+
+def fit_basis(k_pre_rows: np.ndarray, rank: int, omega: np.ndarray,
+              n_power: int = 2) -> np.ndarray:
+    """The xKV basis of one layer group from its keys, by a randomised range finder with
+    Cholesky-QR in place of an exact SVD ([keys]: adjacent layers share one SVD basis,
+    and a randomised Cholesky-QR replaces the exact SVD).
+
+    Reading: the basis is the top-`rank` right singular subspace of A = k_pre_rows (every
+    token of every layer of the group as one row of the flattened D = H_kv*d pre-RoPE
+    key), found by subspace iteration on A^T A:
+      Y = A^T (A omega);  Q = CholQR2(Y);
+      n_power times:  Q = CholQR2(A^T (A Q));
+      Rayleigh-Ritz:  S = (A Q)^T (A Q), U = its eigenvectors by decreasing eigenvalue;
+      basis = Q U[:, :rank]  (orthonormal columns).
+    CholQR2 is Cholesky-QR applied twice. omega [D][l], l >= rank, is the random test
+    matrix, passed in. Returns [D][rank].
+    """
+    a = np.asarray(k_pre_rows, dtype=np.float64)
+    q = cholesky_qr(cholesky_qr(a.T @ (a @ np.asarray(omega, dtype=np.float64))))
+    for _ in range(n_power):
+        q = cholesky_qr(cholesky_qr(a.T @ (a @ q)))
+    aq = a @ q
+    evals, evecs = np.linalg.eigh(aq.T @ aq)
+    order = np.argsort(-evals, kind="stable")
+    return q @ evecs[:, order[:rank]]
+
+
 # ----------------------------------------------------------------------------------
 # chunk landmarks and top-k chunk selection [keys], [how: Selective reconstruction]
 # ----------------------------------------------------------------------------------

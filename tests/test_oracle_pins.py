@@ -251,9 +251,70 @@ def check_selection_and_edges(M):
     assert np.all(np.isfinite(out0))
 
 
+def check_cholesky_qr(M):
+    """Cholesky-QR is the thin QR factorisation with a positive diagonal in R: equal to
+    numpy's QR (a library routine) once the signs of its R diagonal are fixed."""
+    rng = np.random.default_rng(21)
+    y = rng.standard_normal((40, 7)) @ np.diag([5, 4, 3, 2, 1, 0.5, 0.25])
+    q = M.cholesky_qr(y)
+    qn, rn = np.linalg.qr(y)
+    qn = qn * np.sign(np.diag(rn))
+    assert np.allclose(q, qn, atol=1e-10)
+    assert np.allclose(q.T @ q, np.eye(7), atol=1e-12)
+
+
+def check_fit_basis(M):
+    """The randomised range finder returns the top-r right singular subspace of the key
+    rows: exactly for an exactly rank-r matrix, exactly (via Rayleigh-Ritz) when the test
+    matrix spans everything, and to numpy's SVD (a library routine) with oversampling."""
+    rng = np.random.default_rng(22)
+    D, r, N = 32, 5, 400
+    sig = np.array([10.0, 8.0, 6.0, 5.0, 4.0])
+    # planted exact rank r, no oversampling (Cholesky-QR needs full column rank)
+    V, _ = np.linalg.qr(rng.standard_normal((D, r)))
+    A = (rng.standard_normal((N, r)) * sig) @ V.T
+    B = M.fit_basis(A, r, rng.standard_normal((D, r)))
+    assert B.shape == (D, r)
+    assert np.allclose(B.T @ B, np.eye(r), atol=1e-12)
+    assert np.allclose(B @ B.T, V @ V.T, atol=1e-12)
+    # a full-width test matrix and no power step: Rayleigh-Ritz over all of R^D gives the
+    # SVD subspace exactly even though the spectrum has no real gap
+    Vf, _ = np.linalg.qr(rng.standard_normal((D, D)))
+    A = (rng.standard_normal((N, D)) * np.linspace(4.0, 1.0, D)) @ Vf.T
+    vr = np.linalg.svd(A, full_matrices=False)[2][:r].T
+    B = M.fit_basis(A, r, rng.standard_normal((D, D)), n_power=0)
+    assert np.allclose(B @ B.T, vr @ vr.T, atol=1e-10)
+    # oversampled, noisy, with a gap
+    A = (rng.standard_normal((N, r)) * sig) @ V.T + 0.01 * rng.standard_normal((N, D))
+    vr = np.linalg.svd(A, full_matrices=False)[2][:r].T
+    B = M.fit_basis(A, r, rng.standard_normal((D, r + 4)))
+    assert np.allclose(B @ B.T, vr @ vr.T, atol=1e-8)
+
+
+def check_fit_basis_recovers_generator(M):
+    """Fitted on the pre-RoPE keys of a synthetic two-layer group (keys = c B_g^T +
+    0.05 noise), the basis spans the generator's B_g to within the noise."""
+    sh = tiny_shape(n_tokens=256, n_layers=2, rank=5, res_frac=0.1)
+    basis = synth.group_basis(sh, 0)
+    rows = []
+    for layer in range(2):
+        w = synth.layer_weights(sh, layer)
+        for b in range(sh.batch):
+            k, _ = synth.layer_kv(sh, basis, w, layer, b)
+            k = _np(k)
+            pos = np.arange(k.shape[0])[:, None]
+            rows.append(M.rope_rotate(k, pos, sh.theta, inverse=True).reshape(k.shape[0], -1))
+    a = np.concatenate(rows)
+    rng = np.random.default_rng(23)
+    B = M.fit_basis(a, sh.rank, rng.standard_normal((a.shape[1], sh.rank + 4)))
+    bg = _np(basis)
+    assert np.linalg.norm(B @ B.T - bg @ bg.T, 2) < 0.03
+
+
 ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
               check_landmarks_and_scores, check_topk, check_predictor,
-              check_full_rank_exactness, check_residual_pick, check_selection_and_edges]
+              check_full_rank_exactness, check_residual_pick, check_selection_and_edges,
+              check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -367,3 +428,34 @@ def test_mutation_landmark_of_prerope_keys(monkeypatch):
     def bad(k_cache, chunk):
         return orig(k_cache, chunk) * 1.0001
     _fails(check_landmarks_and_scores, monkeypatch, "chunk_landmarks", bad)
+
+
+def _range_finder_q(a, omega, n_power):
+    a = np.asarray(a, np.float64)
+    q = O.cholesky_qr(O.cholesky_qr(a.T @ (a @ omega)))
+    for _ in range(n_power):
+        q = O.cholesky_qr(O.cholesky_qr(a.T @ (a @ q)))
+    return a, q
+
+
+def test_mutation_basis_without_rayleigh_ritz(monkeypatch):
+    def bad(a, rank, omega, n_power=2):
+        _, q = _range_finder_q(a, omega, n_power)
+        return q[:, :rank]
+    _fails(check_fit_basis, monkeypatch, "fit_basis", bad)
+
+
+def test_mutation_basis_smallest_ritz_vectors(monkeypatch):
+    def bad(a, rank, omega, n_power=2):
+        a, q = _range_finder_q(a, omega, n_power)
+        aq = a @ q
+        return q @ np.linalg.eigh(aq.T @ aq)[1][:, :rank]
+    _fails(check_fit_basis, monkeypatch, "fit_basis", bad)
+
+
+def test_mutation_cholesky_qr_wrong_factor(monkeypatch):
+    def bad(y):
+        y = np.asarray(y, np.float64)
+        r_up = np.linalg.cholesky(y.T @ y).T
+        return np.linalg.solve(r_up, y.T).T
+    _fails(check_cholesky_qr, monkeypatch, "cholesky_qr", bad)
