@@ -42,6 +42,10 @@ design notes of the repository):
 - A chunk's score is the max over the GQA group's query heads of q . landmark; the
   k highest-scoring chunks are selected, ties to the lower chunk index.
 - Attention is softmax(q . K_rot / sqrt(d)) over the selected tokens only.
+- The group basis, where it is computed rather than given, is the top-r right singular
+  subspace of the group's stacked pre-RoPE key rows, found by a randomised range finder
+  (subspace iteration, Cholesky-QR applied twice, a Rayleigh-Ritz step) whose random
+  test matrix is an input.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against something other
 than itself (closed forms, brute force, invariants, library routines); none is
