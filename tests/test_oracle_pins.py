@@ -131,6 +131,23 @@ def check_landmarks_and_scores(M):
     assert np.allclose(s, brute, atol=1e-14)
 
 
+def check_encode_landmarks(M):
+    """encode's landmarks are the chunk means of the POST-RoPE keys it is given, per KV
+    head (brute-force fsum over the chunk's rows of k_cache), stored unrounded at f64."""
+    sh = tiny_shape(res_frac=0.25, rank=6)
+    L = make_layer(sh)
+    cache = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                     store=M.STORE_F64, chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    k, C = L["k"], sh.chunk
+    assert cache["landmark"].shape == (sh.batch, sh.n_kv_heads, sh.n_chunks, sh.head_dim)
+    for b in range(sh.batch):
+        for h in range(sh.n_kv_heads):
+            for c in range(sh.n_chunks):
+                brute = [math.fsum(k[b, c * C + i, h, j] for i in range(C)) / C
+                         for j in range(sh.head_dim)]
+                assert np.allclose(cache["landmark"][b, h, c], brute, rtol=0, atol=1e-15)
+
+
 def check_topk(M):
     rng = np.random.default_rng(4)
     for n, k in [(50, 7), (50, 50), (50, 80), (200, 1)]:
@@ -312,7 +329,7 @@ def check_fit_basis_recovers_generator(M):
 
 
 ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
-              check_landmarks_and_scores, check_topk, check_predictor,
+              check_landmarks_and_scores, check_encode_landmarks, check_topk, check_predictor,
               check_full_rank_exactness, check_residual_pick, check_selection_and_edges,
               check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator]
 
@@ -422,12 +439,25 @@ def test_mutation_errors_from_rounded_coef(monkeypatch):
     _fails(check_residual_pick, monkeypatch, "residual_errors", bad)
 
 
-def test_mutation_landmark_of_prerope_keys(monkeypatch):
+def test_mutation_landmark_scaled(monkeypatch):
     orig = O.chunk_landmarks
 
     def bad(k_cache, chunk):
         return orig(k_cache, chunk) * 1.0001
     _fails(check_landmarks_and_scores, monkeypatch, "chunk_landmarks", bad)
+
+
+def test_mutation_landmark_of_prerope_keys(monkeypatch):
+    """encode averaging the inverse-rotated (pre-RoPE) keys instead of the keys it was
+    given: the chunk means differ wherever the rotation angle is non-zero."""
+    orig = O.chunk_landmarks
+    theta = tiny_shape().theta
+
+    def bad(k_cache, chunk):
+        T = k_cache.shape[1]
+        k_pre = O.rope_rotate(k_cache, np.arange(T)[None, :, None], theta, inverse=True)
+        return orig(k_pre, chunk)
+    _fails(check_encode_landmarks, monkeypatch, "chunk_landmarks", bad)
 
 
 def _range_finder_q(a, omega, n_power):
