@@ -206,12 +206,14 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
  * runtime that forbids allocation after start-up, a plugin without an allocator). The
  * call itself allocates nothing; arguments and results are those of lowram_decode_step.
  *   - The array holds 32 MiB and lives on every device that loads the library until the
- *     process exits. A configuration whose decode workspace (lowram_workspace_size) is
- *     larger is refused with LOWRAM_ERR_WORKSPACE, before anything else is checked and
- *     with nothing launched.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current). Make that first call before any
- *     stream capture.
+ *     process exits (or the device's context is destroyed, e.g. by cudaDeviceReset). A
+ *     configuration whose decode workspace (lowram_workspace_size) is larger is refused
+ *     with LOWRAM_ERR_WORKSPACE, before anything else is checked and with nothing
+ *     launched.
+ *   - The first call on a device, and the first call after that device's context was
+ *     destroyed and created again, looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); the address is cached with the
+ *     context's unique id. Make such a first call before any stream capture.
  *   - Every call on a device shares the one array, which keeps whatever the last call
  *     left. The decode step needs none of it zeroed: it writes all it reads. Calls that
  *     overlap on the GPU (other streams, other threads, other contexts) race on it:

@@ -8,8 +8,10 @@
 // input and output buffers.
 //
 // The scratch is a file-scope array of kStaticScratchBytes (32 MiB). Every GPU that loads
-// the library holds it until the process exits. It is as large as the decode workspace of
-// a 128K-token, batch-8 Llama-3-8B-shaped layer.
+// the library holds it until the process exits (or until the device's context is
+// destroyed, e.g. by cudaDeviceReset). It is as large as the decode workspace of a
+// 128K-token, batch-8 Llama-3-8B-shaped layer.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -22,29 +24,75 @@ constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
 
 // Device-side scratch. In host code this name is only a stand-in: its device address
-// comes from cudaGetSymbolAddress, once per device.
+// comes from cudaGetSymbolAddress, with the device current.
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
+// The address is cached per device together with the unique id of the CUDA context it
+// was looked up in. A device reset destroys that context and the module with it; the
+// array can then sit at a new address in the next context, whose id differs, so the next
+// call looks the address up again instead of using a stale one.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void* addr;
+};
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch on `device` (looked up on first use, with that device
-// current), or nullptr when the runtime refuses.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context (0 when it cannot be read).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || !c ||
+      get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch on `device` in its current context, looked up with that
+// device current on the first call in each context; nullptr when the runtime refuses.
 void* scratch_on(int device) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (device < 0 || device >= kMaxDevices) return nullptr;
-  if (g_scratch_addr[device]) return g_scratch_addr[device];
   int prev = -1;
   if (cudaGetDevice(&prev) != cudaSuccess) return nullptr;
-  if (prev != device && cudaSetDevice(device) != cudaSuccess) return nullptr;
+  // since CUDA 12, cudaSetDevice also makes the device's primary context current
+  if (cudaSetDevice(device) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
   void* p = nullptr;
-  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  cudaError_t e = cudaSuccess;
+  const unsigned long long id = current_ctx_id();
+  ScratchEntry& ent = g_scratch[device];
+  if (id != 0 && ent.ctx_id == id && ent.addr) {
+    p = ent.addr;
+  } else {
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e == cudaSuccess) {
+      ent.ctx_id = current_ctx_id();   // 0 (unreadable) never matches: looked up again
+      ent.addr = p;
+    }
+  }
   if (prev != device) cudaSetDevice(prev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return nullptr;
   }
-  g_scratch_addr[device] = p;
   return p;
 }
 
