@@ -15,7 +15,7 @@ Multi-GPU (torchrun): every rank decodes its own batch of 8 (independent seeds):
 scaling, no collective on the data path; time = max over ranks.
 
 --impl reference times the CPU oracle (oracle/) on the host cores on a bounded sample
-of the same workload (one batch element, one layer per step).
+of the same workload (one batch element's token through the layer calls per step).
 """
 from __future__ import annotations
 
@@ -193,6 +193,7 @@ def run_ours(args):
 
     # ---- compressed caches of every layer, encoded on the device
     layers = []
+    kv0 = None
     enc_ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=dev)
     enc_ms = []
     basis64 = basis_dev = None
@@ -209,6 +210,8 @@ def run_ours(args):
                                     compute_dtype=torch.float32)
             k[b], v[b] = kb, vb
             del kb, vb
+        if layer == 0 and rank == 0 and world == 1 and not args.no_cpu_baseline:
+            kv0 = (k[0].cpu(), v[0].cpu())   # the oracle's residual-pick check (cpu leg)
         cache = L.alloc_cache(cfg, dev)
         params = L.layer_params(basis_dev, *wd)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -393,9 +396,18 @@ def run_ours(args):
               "tensor_flops_per_launch": attend_tensor_flops(sh),
               "us_per_launch": round(ms_b_max * 1e3, 2)}
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_from_device(sh, layers, q_all, W, n_layers, args.cpu_baseline_seconds)
+        # the selections and outputs of one eager step on the first timed query, for the
+        # sampled comparison with the oracle
+        with torch.cuda.stream(stream):
+            q_buf.copy_(q_all[W])
+            step_calls()
+        torch.cuda.synchronize()
+        assert ctx.last_error() == L.OK
+        cpu, parity = cpu_baseline_from_device(sh, layers, q_all, W, n_layers,
+                                               args.cpu_baseline_seconds, sel_buf, out_buf)
+        parity["residual_pick"] = residual_pick_vs_oracle(sh, layers[0], kv0)
 
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s",
@@ -414,6 +426,7 @@ def run_ours(args):
         "roofline": roofline,
         "roofline_reconstruct_attend": roof_b,
         "cpu_baseline": cpu,
+        "parity_vs_oracle": parity,
         "e2e": e2e,
         "gpu_launches": 3 * n_layers * K,
         "clocks": clocks,
@@ -459,9 +472,55 @@ def _oracle_unit(O, sh, q, cache_np, p):
                          chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta, act=sh.act)
 
 
-def cpu_baseline_from_device(sh, layers, q_all, W, n_layers, seconds):
+def compare_to_oracle_selection(got, want, scores, k, rel=1e-5):
+    """Per row: index sets must match except indices whose fp64 score lies within
+    rel*|s_k| of the k-th largest score (ties, reported). Returns (ties, other)."""
+    import numpy as np
+    got = np.asarray(got).reshape(-1, np.asarray(got).shape[-1])
+    want = np.asarray(want).reshape(got.shape)
+    sc = np.asarray(scores).reshape(got.shape[0], -1)
+    ties = other = 0
+    for r in range(got.shape[0]):
+        diff = set(got[r].tolist()) ^ set(want[r].tolist())
+        if not diff:
+            continue
+        sk = float(np.sort(sc[r])[::-1][min(k, sc.shape[1]) - 1])
+        for i in diff:
+            if abs(sc[r][i] - sk) <= rel * abs(sk):
+                ties += 1
+            else:
+                other += 1
+    return ties, other
+
+
+def residual_pick_vs_oracle(sh, layer0, kv0):
+    """Residual token indices that lowram_encode picked for batch element 0 of layer 0
+    against the oracle's encode of the same stored keys and values (all KV heads)."""
+    import numpy as np
+    import torch
+
+    import oracle.lowram_oracle as O
+    if kv0 is None:
+        return None
+
+    def f64(t):
+        return t.detach().to("cpu", torch.float64).numpy()
+    basis_dev, wd = layer0["keep"]
+    t0 = time.perf_counter()
+    enc = O.encode(f64(kv0[0])[None], f64(kv0[1])[None], f64(basis_dev), *(f64(w) for w in wd),
+                   chunk=sh.chunk, n_res=sh.n_res, theta=sh.theta, act=sh.act,
+                   store=O.STORE_BF16)
+    got = layer0["cache"]["res_idx"][0:1].cpu().numpy()
+    ties, other = compare_to_oracle_selection(got, enc["res_idx"], enc["err"], sh.n_res)
+    return {"rows": int(got.shape[1]), "tie_differences": ties, "other_differences": other,
+            "sample": "batch element 0 of layer 0, every KV head",
+            "oracle_seconds": round(time.perf_counter() - t0, 1)}
+
+
+def cpu_baseline_from_device(sh, layers, q_all, W, n_layers, seconds, sel_buf, out_buf):
     """The oracle, as it stands, on host cores: decode units of (batch element 0, layer l)
-    with the same stored caches and queries, until ~`seconds` of CPU work."""
+    with the same stored caches and queries, until ~`seconds` of CPU work. Also compares
+    each unit's selection and output with what the GPU step computed for that query."""
     import numpy as np
     import torch
 
@@ -471,6 +530,8 @@ def cpu_baseline_from_device(sh, layers, q_all, W, n_layers, seconds):
         return t.detach().to("cpu", torch.float64).numpy()
 
     units, t_total = 0, 0.0
+    ties = other = 0
+    max_err = 0.0
     layer = 0
     while t_total < seconds and units < 4 * n_layers:
         Ld = layers[layer % n_layers]
@@ -484,15 +545,33 @@ def cpu_baseline_from_device(sh, layers, q_all, W, n_layers, seconds):
              "b2": f64(wd[3])}
         q = f64(q_all[W, layer % n_layers, 0:1])
         t0 = time.perf_counter()
-        _oracle_unit(O, sh, q, cache_np, p)
+        want, _ = _oracle_unit(O, sh, q, cache_np, p)
         t_total += time.perf_counter() - t0
+        if layer < n_layers:   # each layer's GPU result is compared once
+            osel, scores = O.select_chunks(q, cache_np["landmark"], sh.top_k)
+            gsel = sel_buf[layer, 0:1].cpu().numpy()
+            tt, oo = compare_to_oracle_selection(gsel, osel, scores, min(sh.top_k, sh.n_chunks))
+            ties, other = ties + tt, other + oo
+            want_g, _ = O.decode_step(q, cache_np, p["basis"], p["w1"], p["b1"], p["w2"],
+                                      p["b2"], chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta,
+                                      act=sh.act, sel=gsel.astype(np.int64))
+            g = f64(out_buf[layer, 0:1])
+            rms = float(np.sqrt(np.mean(want_g ** 2)))
+            max_err = max(max_err, float(np.max(np.abs(g - want_g))) / rms)
         units += 1
         layer += 1
     per_unit = t_total / units
-    return {"value": round(1.0 / (per_unit * n_layers), 4), "unit": "tokens/s",
-            "cores": _threads(), "host_cpus": os.cpu_count(), "kind": "oracle",
-            "sample": f"{units} (batch element 0, layer) decode units of the same workload "
-                      f"({t_total:.1f} s); tokens/s = units/s / {n_layers} layers"}
+    n_cmp = min(units, n_layers)
+    cpu = {"value": round(1.0 / (per_unit * n_layers), 4), "unit": "tokens/s",
+           "cores": _threads(), "host_cpus": os.cpu_count(), "kind": "oracle",
+           "sample": f"{units} (batch element 0, layer) decode units of the same workload "
+                     f"({t_total:.1f} s); tokens/s = units/s / {n_layers} layers"}
+    parity = {"chunk_selection": {"rows": n_cmp * sh.n_kv_heads, "tie_differences": ties,
+                                  "other_differences": other,
+                                  "sample": f"batch element 0 of layers 0..{n_cmp - 1}, every "
+                                            f"KV head, first timed query"},
+              "output_max_rel_err": round(max_err, 6), "output_tolerance": 2e-2}
+    return cpu, parity
 
 
 # ----------------------------------------------------------------------------------
@@ -523,26 +602,41 @@ def run_reference(args):
                      store=O.STORE_BF16)
     del k, v
     W, K = args.warmup, args.steps
-    qs = [synth.queries(sh, 0, i).to(torch.float64).numpy() for i in range(W + K)]
+    # a step is one batch element's token through the layer calls (the layer-0 cache
+    # stands in for every layer), each call with its own query; when K + W steps of
+    # n_layers calls would run past ~150 s, a step runs fewer calls and tokens/s counts
+    # the fraction of a token it decoded
+    q_of = lambda i: synth.queries(sh, 0, i).to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    _oracle_unit(O, sh, q_of(10 ** 6), cache, p)
+    t_unit = time.perf_counter() - t0
+    per_step = int(max(1, min(n_layers, 150.0 / max(1, W + K) / max(t_unit, 1e-6))))
+    n = 0
     for i in range(W):
-        _oracle_unit(O, sh, qs[i], cache, p)
+        for _ in range(per_step):
+            _oracle_unit(O, sh, q_of(n), cache, p)
+            n += 1
     t0 = time.perf_counter()
     for i in range(K):
-        _oracle_unit(O, sh, qs[W + i], cache, p)
-    per_unit = (time.perf_counter() - t0) / K
-    value = 1.0 / (per_unit * n_layers)
+        for _ in range(per_step):
+            _oracle_unit(O, sh, q_of(n), cache, p)
+            n += 1
+    ms_step = (time.perf_counter() - t0) / K * 1e3
+    tokens_per_step = per_step / n_layers
+    value = tokens_per_step / (ms_step / 1e3)
+    sample = (f"each step = {per_step} oracle decode calls (batch element 0, the layer-0 "
+              f"cache, a fresh query per call) = {tokens_per_step:g} token(s) of one "
+              f"sequence through {n_layers} layers")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K, "warmup": W,
-        "ms_per_step": round(per_unit * n_layers * 1e3, 2), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "ms_per_step": round(ms_step, 2), "tokens_per_step": tokens_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, encoded by the oracle",
         "config": {"workload": base.name, "batch_per_gpu": base.batch, "context": base.n_tokens,
-                   "layers": n_layers, "sampled": "one batch element of layer 0 per step"},
+                   "layers": n_layers, "sampled": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": _threads(),
-                         "host_cpus": os.cpu_count(), "kind": "oracle",
-                         "sample": f"each step = oracle decode of 1 (batch element, layer) "
-                                   f"unit; tokens/s = units/s / {n_layers} layers"},
+                         "host_cpus": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -231,6 +231,38 @@ lowram_status lowram_last_error(lowram_ctx* ctx);
 /* Static string naming a status. */
 const char* lowram_status_string(lowram_status status);
 
+/* Test only: lowram_attend_selected on the tensor-core kernel (LOWRAM_ERR_UNSUPPORTED
+ * where it does not apply) that also stores the rows it rebuilds, at the points where its
+ * epilogue holds them, so they can be compared element by element with the method's
+ * rebuilt keys and values ("rebuild only the top-k chunks", agihunt summary, key
+ * paragraph; cctest "Residuals for difficult tokens"). Rows are in selection order:
+ * row = (b*H_kv + h)*k*C + s*C + j for token j of the chunk sel[b][h][s]; rows = B*H_kv*k*C
+ * with k = min(top_k, T/C). All three outputs are device fp32 arrays, zeroed first:
+ *   k_rot [rows][d]  the rebuilt key with RoPE re-applied (epilogue part A);
+ *   h_act [rows][F]  act(W1 K~_pre + b1), the hidden layer (epilogue part B);
+ *   v_rec [rows][d]  the rebuilt value W2 h_act + b2 + R_t (R_t: the token's stored
+ *                    residual row, read where part B reads it; W2 and b2 applied by a
+ *                    small separate kernel, since the decode kernel applies W2 only after
+ *                    the attention sum).
+ * out is written as by lowram_attend_selected. */
+lowram_status lowram_debug_reconstruct(lowram_ctx* ctx, const lowram_cache* cache,
+                                      const lowram_layer_params* params, const void* q,
+                                      const int32_t* sel, void* out, float* k_rot,
+                                      float* h_act, float* v_rec, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
+/* Test only: the tensor-core attend kernel launched as if it followed a selection launch
+ * in the same decode step, so it waits on every (batch, KV head)'s ready flag; no
+ * selection runs in this call and the flags stay clear, so its first wait gives up after
+ * its bound (about 2 s), the kernel drains its own copies and MMAs, frees its Tensor
+ * Memory and returns. lowram_last_error then reports LOWRAM_ERR_TIMEOUT, out is not
+ * valid, and the context serves the next call normally. LOWRAM_ERR_UNSUPPORTED where the
+ * tensor-core kernel does not apply. */
+lowram_status lowram_debug_attend_unpublished(lowram_ctx* ctx, const lowram_cache* cache,
+                                              const lowram_layer_params* params, const void* q,
+                                              const int32_t* sel, void* out, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
 /* Test only (no counterpart in the method): one 128 x 128 tcgen05 tile product
  * d[m][n] = sum_k a[m][k] * b[n][k] with a [128][K], b [128][K] bf16 row-major (device)
  * and d [128][128] fp32 (device), staged through the same shared-memory layouts and

@@ -154,7 +154,9 @@ __device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
   return 0;
 }
 
-template <int ACT>
+// DBG (test only): also store the rebuilt rows (a.dbg_k, a.dbg_h, a.dbg_v) where the
+// epilogue holds them; the product instantiation has DBG = false and stores nothing.
+template <int ACT, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   const Dims& dm = a.dm;
@@ -581,6 +583,13 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         return false;
       }
       const bool valid = M->cid[trow >> 3] >= 0;
+      float* dbg_krow = nullptr;   // this token's K~_rot row (DBG only)
+      if constexpr (DBG) {
+        int b, tile;
+        item_of(M->item, b, tile);
+        if (valid)
+          dbg_krow = a.dbg_k + (((size_t)b * dm.H + h) * dm.k * kChunk + (size_t)tile * kTile + trow) * kD;
+      }
       {   // sQ[g][i][w] = q_g[i + 64 w]: each rotary pair's two query components adjacent
         const uint32_t w = reinterpret_cast<const uint32_t*>(M->q)[et];
         const float2 f = bf2_to_f2(w);
@@ -632,6 +641,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
             const int e = e4 + w;
             const float2 cs = rope_combine(bs[w], ro[e * kChunk]);
             rot[w] = make_float2(x[e] * cs.x - y[e] * cs.y, x[e] * cs.y + y[e] * cs.x);
+            if constexpr (DBG) {
+              if (dbg_krow) {
+                dbg_krow[p0 + e] = rot[w].x;
+                dbg_krow[kD / 2 + p0 + e] = rot[w].y;
+              }
+            }
           }
           const int pi = p0 + e4;
 #pragma unroll
@@ -747,6 +762,8 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       item_of(M->item, b, tile);
       const int p = b * dm.H + h;
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
+      // first debug row of this tile (DBG only); a row is stored only if its chunk exists
+      const size_t dbg_row0 = ((size_t)p * dm.k * kChunk + (size_t)tile * kTile);
       // residual rows of the tile: thread = column j; rows split between the two halves.
       // The first kResPrefetch of this thread's rows are loaded now, as raw bf16 bits:
       // nothing waits for them until the residual sum after the hidden layer.
@@ -794,6 +811,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           for (int e = 0; e < 32; e += 2) {
             const float2 hx = __ffma2_rn(half2, make_float2(hv[e], hv[e + 1]), hb2);
             const float2 av = __ffma2_rn(hx, make_float2(tanh_approx(hx.x), tanh_approx(hx.y)), hx);
+            if constexpr (DBG) {
+              const int t0 = 32 * c + e;
+              if (M->cid[t0 >> 3] >= 0) a.dbg_h[(dbg_row0 + t0) * kF + f] = av.x;
+              if (M->cid[(t0 + 1) >> 3] >= 0) a.dbg_h[(dbg_row0 + t0 + 1) * kF + f] = av.y;
+            }
             const float4 pa = P2[32 * c + e], pb = P2[32 * c + e + 1];   // tokens (e, e + 1)
             acc2[0] = __ffma2_rn(make_float2(pa.x, pa.y), av, acc2[0]);
             acc2[1] = __ffma2_rn(make_float2(pa.z, pa.w), av, acc2[1]);
@@ -804,6 +826,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float av = act_fast<ACT>(hv[e] + bias);
+            if constexpr (DBG) {
+              if (M->cid[(32 * c + e) >> 3] >= 0) a.dbg_h[(dbg_row0 + 32 * c + e) * kF + f] = av;
+            }
             const float4 pv = P4[32 * c + e];
             hacc01 = __ffma2_rn(make_float2(pv.x, pv.y), make_float2(av, av), hacc01);
             hacc23 = __ffma2_rn(make_float2(pv.z, pv.w), make_float2(av, av), hacc23);
@@ -829,6 +854,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         if (row == 255u) continue;
         const float4 pv = P4[row];
         const float r = __uint_as_float(((pre_val[v >> 1] >> (16 * (v & 1))) & 0xFFFFu) << 16);
+        if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r;
         racc[0] = fmaf(pv.x, r, racc[0]);
         racc[1] = fmaf(pv.y, r, racc[1]);
         racc[2] = fmaf(pv.z, r, racc[2]);
@@ -839,6 +865,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         const int row = (int)(ent & 255u);
         if (row == 255) continue;
         const float r = __bfloat162float(rbase[(size_t)(ent >> 8) * kD]);
+        if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r;
         const float4 pv = P4[row];
         racc[0] = fmaf(pv.x, r, racc[0]);
         racc[1] = fmaf(pv.y, r, racc[1]);
@@ -1029,8 +1056,11 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   if (cph < 1) cph = 1;
   if (cph > n_items) cph = n_items;
   cudaError_t e;
-  auto kern = dm.act == LOWRAM_ACT_SILU ? attend_tc_kernel<LOWRAM_ACT_SILU>
-                                        : attend_tc_kernel<LOWRAM_ACT_GELU_ERF>;
+  const bool dbg = a.dbg_k != nullptr;
+  auto kern = dm.act == LOWRAM_ACT_SILU
+                  ? (dbg ? attend_tc_kernel<LOWRAM_ACT_SILU, true> : attend_tc_kernel<LOWRAM_ACT_SILU, false>)
+                  : (dbg ? attend_tc_kernel<LOWRAM_ACT_GELU_ERF, true>
+                         : attend_tc_kernel<LOWRAM_ACT_GELU_ERF, false>);
   if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)L.total)) != cudaSuccess) return e;
   // after the selection kernel: a programmatic dependent launch, so CTAs start on SMs
@@ -1047,6 +1077,27 @@ cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s) {
   cfg.numAttrs = a.wait_ready ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, kern, a, maps);
   if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Test only: v[row][j] += b2_h[j] + sum_f W2_h[j][f] act[row][f] for every rebuilt row
+// (one CTA per row, thread j), in fp32 from the stored bf16 weights.
+__global__ void __launch_bounds__(kD) debug_values_kernel(const AttendArgs a) {
+  const Dims& dm = a.dm;
+  const size_t row = blockIdx.x;
+  const int h = (int)((row / ((size_t)dm.k * kChunk)) % dm.H);
+  const int j = threadIdx.x;
+  const float* hr = a.dbg_h + row * kF;
+  const __nv_bfloat16* w2 = (const __nv_bfloat16*)a.w2 + ((size_t)h * kD + j) * kF;
+  float acc = __bfloat162float(((const __nv_bfloat16*)a.b2)[(size_t)h * kD + j]);
+  for (int f = 0; f < kF; ++f) acc = fmaf(__bfloat162float(w2[f]), hr[f], acc);
+  a.dbg_v[row * kD + j] += acc;
+}
+
+cudaError_t launch_debug_values(const AttendArgs& a, cudaStream_t s) {
+  const size_t rows = (size_t)a.dm.B * a.dm.H * a.dm.k * kChunk;
+  if (rows == 0) return cudaSuccess;
+  debug_values_kernel<<<(unsigned)rows, kD, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -371,10 +371,11 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const float* la
   return LOWRAM_OK;
 }
 
+// dbg (test only, else null): {k_rot, h_act, v_rec} rows written by the tcgen05 kernel
 lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
                           const lowram_layer_params* params, const void* q, const int32_t* sel,
                           void* out, uint8_t* ws, const DecodeWs& w, cudaStream_t s,
-                          bool after_select) {
+                          bool after_select, float* const* dbg = nullptr) {
   const lowram_config& c = ctx->cfg;
   const Dims dm = dims_of(c);
   AttendArgs aa{};
@@ -397,8 +398,14 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   aa.ready = tc && after_select ? ctx->ready : nullptr;
   aa.wait_ready = aa.ready ? 1 : 0;
   aa.item_ctr = tc ? ctx->item_ctr : nullptr;
+  if (dbg) {
+    aa.dbg_k = dbg[0];
+    aa.dbg_h = dbg[1];
+    aa.dbg_v = dbg[2];
+  }
   cudaError_t e = tc ? launch_attend_tc(aa, ctx->num_sms, s) : launch_attend_simt(aa, s);
   if (e == cudaSuccess) e = launch_combine(aa, tc, s);
+  if (e == cudaSuccess && dbg) e = launch_debug_values(aa, s);
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;
 }
@@ -454,6 +461,58 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
   if (!g.ok) return LOWRAM_ERR_CUDA;
   return attend_impl(ctx, cache, params, q, sel, out, static_cast<uint8_t*>(workspace), w,
                      static_cast<cudaStream_t>(stream), false);
+}
+
+lowram_status lowram_debug_reconstruct(lowram_ctx* ctx, const lowram_cache* cache,
+                                      const lowram_layer_params* params, const void* q,
+                                      const int32_t* sel, void* out, float* k_rot,
+                                      float* h_act, float* v_rec, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!ctx || !q || !sel || !out || !workspace || !k_rot || !h_act || !v_rec)
+    return LOWRAM_ERR_INVALID_ARG;
+  lowram_status st = check_layer_params(params);
+  if (st != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if (!aligned16(q) || !aligned16(sel) || !aligned16(out) || !aligned16(workspace) ||
+      !aligned16(k_rot) || !aligned16(h_act) || !aligned16(v_rec))
+    return LOWRAM_ERR_ALIGN;
+  if (!use_tc(ctx->cfg)) return LOWRAM_ERR_UNSUPPORTED;
+  const DecodeWs w = decode_ws(ctx->cfg);
+  if (workspace_bytes < w.total) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  const Dims dm = dims_of(ctx->cfg);
+  const size_t rows = (size_t)dm.B * dm.H * dm.k * dm.C;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(k_rot, 0, rows * dm.d * sizeof(float), s) != cudaSuccess ||
+      cudaMemsetAsync(h_act, 0, rows * dm.F * sizeof(float), s) != cudaSuccess ||
+      cudaMemsetAsync(v_rec, 0, rows * dm.d * sizeof(float), s) != cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  float* const dbg[3] = {k_rot, h_act, v_rec};
+  return attend_impl(ctx, cache, params, q, sel, out, static_cast<uint8_t*>(workspace), w, s,
+                     false, dbg);
+}
+
+lowram_status lowram_debug_attend_unpublished(lowram_ctx* ctx, const lowram_cache* cache,
+                                              const lowram_layer_params* params, const void* q,
+                                              const int32_t* sel, void* out, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (!ctx || !q || !sel || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
+  lowram_status st = check_layer_params(params);
+  if (st != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if (!aligned16(q) || !aligned16(sel) || !aligned16(out) || !aligned16(workspace))
+    return LOWRAM_ERR_ALIGN;
+  if (!use_tc(ctx->cfg)) return LOWRAM_ERR_UNSUPPORTED;
+  const DecodeWs w = decode_ws(ctx->cfg);
+  if (workspace_bytes < w.total) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  // as right after a selection launch, but none ran: the ready flags stay 0
+  return attend_impl(ctx, cache, params, q, sel, out, static_cast<uint8_t*>(workspace), w,
+                     static_cast<cudaStream_t>(stream), true);
 }
 
 lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,

@@ -91,6 +91,12 @@ struct AttendArgs {
                           // kernel; wait for ready[pair] before reading its selection
   int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); combine
                           // clears them
+  // test only (lowram_debug_reconstruct), null otherwise: rebuilt rows of the selected
+  // chunks in selection order, row = (b*H + h)*k*C + slot*C + j (j = token in chunk):
+  float* dbg_k;           // [rows][d]  K~_rot, as epilogue part A holds it
+  float* dbg_h;           // [rows][F]  act(W1 K~_pre + b1), as epilogue part B holds it
+  float* dbg_v;           // [rows][d]  the residual row of each token (0 if none); the
+                          //            debug value kernel adds W2 h + b2
 };
 size_t attend_simt_part_floats(const Dims& dm, int n_tiles);
 int attend_simt_tile_tokens(const Dims& dm);
@@ -104,6 +110,8 @@ constexpr int kTcTileTokens = 128;
 cudaError_t launch_attend_tc(const AttendArgs& a, int num_sms, cudaStream_t s);
 
 cudaError_t launch_combine(const AttendArgs& a, bool reorder_form, cudaStream_t s);
+// test only: dbg_v[row] += W2_h dbg_h[row] + b2_h for every row of a.dbg_h
+cudaError_t launch_debug_values(const AttendArgs& a, cudaStream_t s);
 
 // ---------------- encode ----------------
 struct EncodeArgs {

@@ -89,6 +89,12 @@ _sig = {
     "lowram_last_error": (_S, [_P]),
     "lowram_status_string": (ctypes.c_char_p, [_S]),
     "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
+    "lowram_debug_reconstruct": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                      ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P, _P,
+                                      _P, _P, ctypes.c_size_t, _P]),
+    "lowram_debug_attend_unpublished": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                             ctypes.POINTER(lowram_layer_params), _P, _P, _P,
+                                             _P, ctypes.c_size_t, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -261,3 +267,25 @@ def attend_selected(ctx: Context, cache: dict, params: lowram_layer_params, q, s
 def debug_tc_tile(a, b, d, k: int, mode: int, stream=None) -> None:
     check(lowram_debug_tc_tile(_ptr(a), _ptr(b), _ptr(d), k, mode, _stream(stream)),
           "lowram_debug_tc_tile")
+
+
+def debug_reconstruct(ctx: Context, cache: dict, params: lowram_layer_params, q, sel, out,
+                      k_rot, h_act, v_rec, workspace, stream=None) -> None:
+    """Test only: lowram_debug_reconstruct (attend + the rebuilt rows; include/lowram.h)."""
+    cs = cache_struct(**cache)
+    check(lowram_debug_reconstruct(ctx.handle, ctypes.byref(cs), ctypes.byref(params), _ptr(q),
+                                   _ptr(sel), _ptr(out), _ptr(k_rot), _ptr(h_act), _ptr(v_rec),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream)),
+          "lowram_debug_reconstruct")
+
+
+def debug_attend_unpublished(ctx: Context, cache: dict, params: lowram_layer_params, q, sel,
+                             out, workspace, stream=None) -> None:
+    """Test only: lowram_debug_attend_unpublished (a wait that runs out; include/lowram.h)."""
+    cs = cache_struct(**cache)
+    check(lowram_debug_attend_unpublished(ctx.handle, ctypes.byref(cs), ctypes.byref(params),
+                                          _ptr(q), _ptr(sel), _ptr(out), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)),
+          "lowram_debug_attend_unpublished")

@@ -113,6 +113,15 @@ def compare_selection(got: np.ndarray, want: np.ndarray, scores: np.ndarray, k: 
     return ties
 
 
+def assert_ties_bounded(n_ties: int, n_rows: int, where: str) -> None:
+    """Report the tie differences of a selection check and bound them: at most one per
+    100 selection rows (at least one allowed). With exact fp64 settling on the GPU side a
+    tie difference needs two fp64 scores within 1e-5 relative of the k-th, which these
+    continuous synthetic scores make rare; many would mean the settling is broken."""
+    print(f"{where}: {n_ties} tie differences over {n_rows} selection rows")
+    assert n_ties <= max(1, n_rows // 100), (where, n_ties, n_rows)
+
+
 def rel_err(got: np.ndarray, want: np.ndarray) -> float:
     """max |got - want| / RMS(want)."""
     rms = math.sqrt(float(np.mean(np.asarray(want, np.float64) ** 2)))

@@ -74,7 +74,8 @@ def test_config0_fp32_two_layers_four_steps(L, cuda_device):
         for step in range(sh.steps):
             q = synth.queries(sh, layer, step)
             check_step(L, sh, cdev, t_dev, t, co, q, L.DECODE_AUTO, ties)
-    print("config0 tie differences:", sum(ties))
+    H.assert_ties_bounded(sum(ties), sh.n_layers * sh.steps * sh.batch * sh.n_kv_heads,
+                          "config0 chunk selection")
 
 
 @pytest.fixture(scope="module")
@@ -93,7 +94,9 @@ def test_config1_bf16(L, config1_layers, variant):
             q = synth.queries(sh, layer, step)
             err, _ = check_step(L, sh, cdev, t_dev, t, co, q, v, ties)
             errs.append(err)
-    print(f"config1 {variant}: max rel err {max(errs):.3e}, tie differences {sum(ties)}")
+    print(f"config1 {variant}: max rel err {max(errs):.3e}")
+    H.assert_ties_bounded(sum(ties), len(layers) * 2 * sh.batch * sh.n_kv_heads,
+                          f"config1 {variant} chunk selection")
 
 
 def test_config1_tc_and_simt_agree(L, config1_layers):

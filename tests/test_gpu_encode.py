@@ -90,13 +90,15 @@ def check_encode(L, shape, device):
 
 
 def test_config0_encode(L, cuda_device):
-    ties, *_ = check_encode(L, synth.CONFIGS[0], cuda_device)
-    print("config0 residual tie differences:", ties)
+    sh = synth.CONFIGS[0]
+    ties, *_ = check_encode(L, sh, cuda_device)
+    H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, "config0 residual pick")
 
 
 def test_config1_encode(L, cuda_device):
-    ties, *_ = check_encode(L, synth.CONFIGS[1], cuda_device)
-    print("config1 residual tie differences:", ties)
+    sh = synth.CONFIGS[1]
+    ties, *_ = check_encode(L, sh, cuda_device)
+    H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, "config1 residual pick")
 
 
 @pytest.mark.parametrize("cfg_id", [0, 1])

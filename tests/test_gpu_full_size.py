@@ -1,7 +1,9 @@
-"""Full-size parity at the headline shape (Llama-3-8B-shaped layer, batch 8, 128K context,
-rank 160, top-256 chunks, 20% residuals, bf16), in the launch configuration the bench
-times. The oracle checks sampled (batch, KV head) pairs one by one, and properties that
-hold at any size check the rest."""
+"""Full-size parity, in the launch configuration the bench times, at two shapes: the
+headline Llama-3-8B-shaped layer (batch 8, 128K context, rank 160, top-256 chunks, 20%
+residuals, bf16) and the Mistral-7B-shaped long-context layer (batch 4, 262144 tokens,
+RoPE theta 1e6, rank 128, 15% residuals), whose RoPE angles reach position 262143. The
+oracle checks sampled (batch, KV head) pairs one by one, and properties that hold at any
+size check the rest."""
 import numpy as np
 import pytest
 import torch
@@ -19,9 +21,9 @@ def L(cuda_device):
     return lowram
 
 
-@pytest.fixture(scope="module")
-def full_layer(L, cuda_device):
-    sh = synth.CONFIGS[2]
+@pytest.fixture(scope="module", params=[2, 3], ids=["llama8b-b8-128k", "mistral7b-b4-262k"])
+def full_layer(L, cuda_device, request):
+    sh = synth.CONFIGS[request.param]
     dev = cuda_device
     basis = synth.group_basis(sh, 0)
     w = synth.layer_weights(sh, 0)
@@ -46,7 +48,10 @@ def full_layer(L, cuda_device):
     return sh, ctx, cfg, cache, td, params, k, v
 
 
-SAMPLED_PAIRS = [(0, 0), (3, 5), (7, 7)]
+def sampled_pairs(sh):
+    """Eight (batch, KV head) pairs spread over the batch and the heads."""
+    B, Hk = sh.batch, sh.n_kv_heads
+    return sorted({(i * B // 8, (3 * i + i // 4) % Hk) for i in range(8)} | {(B - 1, Hk - 1)})
 
 
 def test_encode_properties_and_sampled_errors(full_layer):
@@ -63,7 +68,7 @@ def test_encode_properties_and_sampled_errors(full_layer):
     basis = H.f64(td["basis"])
     w1, b1, w2, b2 = (H.f64(td[n]) for n in ("w1", "b1", "w2", "b2"))
     d = sh.head_dim
-    for b, h in SAMPLED_PAIRS:
+    for b, h in sampled_pairs(sh):
         toks = np.sort(rng.choice(sh.n_tokens, 96, replace=False))
         kt = H.f64(k[b, toks])                                     # [n, H, d]
         vt = H.f64(v[b, toks, h])
@@ -84,34 +89,44 @@ def test_encode_properties_and_sampled_errors(full_layer):
 def test_decode_sampled_pairs_match_oracle(L, full_layer):
     sh, ctx, cfg, cache, td, params, k, v = full_layer
     dev = k.device
-    q = synth.queries(sh, 0, 0).to(dev)
-    out = torch.empty_like(q)
     kk = min(sh.top_k, sh.n_chunks)
-    sel = torch.empty(sh.batch, sh.n_kv_heads, kk, dtype=torch.int32, device=dev)
     ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
-    L.decode_step(ctx, cache, params, q, out, ws, sel_out=sel)
-    assert ctx.last_error() == L.OK
     G, d = sh.group, sh.head_dim
     basis = H.f64(td["basis"])
     w1, b1, w2, b2 = (H.f64(td[n]) for n in ("w1", "b1", "w2", "b2"))
+    pairs = sampled_pairs(sh)
+    subs = {}
+    for b, h in pairs:
+        subs[b, h] = {
+            "coef": H.f64(cache["coef"][b:b + 1]),
+            "landmark": H.f64(cache["landmark"][b:b + 1, h:h + 1]),
+            "res_idx": cache["res_idx"][b:b + 1, h:h + 1].cpu().numpy().astype(np.int64),
+            "res_val": H.f64(cache["res_val"][b:b + 1, h:h + 1]),
+            "chunk_ptr": cache["chunk_ptr"][b:b + 1, h:h + 1].cpu().numpy().astype(np.int64)}
     ties = 0
-    for b, h in SAMPLED_PAIRS:
-        qb = H.f64(q[b:b + 1, h * G:(h + 1) * G])
-        sub = {"coef": H.f64(cache["coef"][b:b + 1]),
-               "landmark": H.f64(cache["landmark"][b:b + 1, h:h + 1]),
-               "res_idx": cache["res_idx"][b:b + 1, h:h + 1].cpu().numpy().astype(np.int64),
-               "res_val": H.f64(cache["res_val"][b:b + 1, h:h + 1]),
-               "chunk_ptr": cache["chunk_ptr"][b:b + 1, h:h + 1].cpu().numpy().astype(np.int64)}
-        osel, scores = O.select_chunks(qb, sub["landmark"], sh.top_k)
-        gsel = sel[b:b + 1, h:h + 1].cpu().numpy()
-        ties += H.compare_selection(gsel, osel, scores, kk)
-        want, _ = O.decode_step(qb, sub, basis[h * d:(h + 1) * d], w1[h:h + 1], b1[h:h + 1],
-                                w2[h:h + 1], b2[h:h + 1], chunk=sh.chunk, top_k=sh.top_k,
-                                theta=sh.theta, act=sh.act, sel=gsel.astype(np.int64))
-        err = H.rel_err(H.f64(out[b:b + 1, h * G:(h + 1) * G]), want)
-        assert err <= 2e-2, (b, h, err)
-    print("full-size sampled tie differences:", ties)
-    # properties over all pairs: selections ascending, in range, distinct
-    s = sel.cpu().numpy()
-    assert np.all(np.diff(s, axis=-1) > 0) and s.min() >= 0 and s.max() < sh.n_chunks
-    assert torch.isfinite(out.float()).all()
+    worst = 0.0
+    for step in range(2):
+        q = synth.queries(sh, 0, step).to(dev)
+        out = torch.empty_like(q)
+        sel = torch.empty(sh.batch, sh.n_kv_heads, kk, dtype=torch.int32, device=dev)
+        L.decode_step(ctx, cache, params, q, out, ws, sel_out=sel)
+        assert ctx.last_error() == L.OK
+        for b, h in pairs:
+            sub = subs[b, h]
+            qb = H.f64(q[b:b + 1, h * G:(h + 1) * G])
+            osel, scores = O.select_chunks(qb, sub["landmark"], sh.top_k)
+            gsel = sel[b:b + 1, h:h + 1].cpu().numpy()
+            ties += H.compare_selection(gsel, osel, scores, kk)
+            want, _ = O.decode_step(qb, sub, basis[h * d:(h + 1) * d], w1[h:h + 1],
+                                    b1[h:h + 1], w2[h:h + 1], b2[h:h + 1], chunk=sh.chunk,
+                                    top_k=sh.top_k, theta=sh.theta, act=sh.act,
+                                    sel=gsel.astype(np.int64))
+            err = H.rel_err(H.f64(out[b:b + 1, h * G:(h + 1) * G]), want)
+            worst = max(worst, err)
+            assert err <= 2e-2, (step, b, h, err)
+        # properties over all pairs: selections ascending, in range, distinct
+        s = sel.cpu().numpy()
+        assert np.all(np.diff(s, axis=-1) > 0) and s.min() >= 0 and s.max() < sh.n_chunks
+        assert torch.isfinite(out.float()).all()
+    print(f"{sh.name}: sampled max rel err {worst:.3e}")
+    H.assert_ties_bounded(ties, 2 * len(pairs), f"{sh.name} sampled chunk selection")

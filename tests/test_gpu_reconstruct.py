@@ -1,0 +1,197 @@
+"""The rows the tensor-core decode kernel rebuilds, compared element by element with the
+oracle, through the C ABI (lowram_debug_reconstruct stores them where the kernel's
+epilogue holds them: K~_rot in part A, act(W1 K~_pre + b1) and the residual row in
+part B); the tensor-core kernel at full rank against exact dense attention; and a
+bounded wait that runs out on purpose.
+
+Method: "rebuild only the top-k chunks" (agihunt summary, key paragraph); values from
+the per-head predictor plus the stored residual corrections (cctest "How the method
+works": Amortised values, Residuals for difficult tokens).
+
+Tolerances, max |gpu - oracle| / RMS(oracle) over every rebuilt row of a layer call:
+- K~_rot 1e-3: bf16 coefficients times the bf16 basis, exact products summed in fp32
+  in Tensor Memory, then the fp32 rotation tables (each ~1e-6 relative);
+- the hidden activations and V~ 2e-2, the decode tolerance: the hidden layer takes K~ in
+  bf16 (2^-9 relative) and SiLU uses tanh.approx.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.lowram_oracle as O
+from long_context_decode_02_b200 import synth
+from tests import helpers as H
+from tests.test_gpu_decode import oracle_decode, prepared
+
+pytestmark = pytest.mark.gpu
+
+TOL_K = 1e-3
+TOL_HV = 2e-2
+
+
+@pytest.fixture(scope="module")
+def L(cuda_device):
+    from long_context_decode_02_b200 import lowram
+    return lowram
+
+
+def gpu_rows(L, sh, cache_dev, t_dev, q, sel):
+    dev = cache_dev["coef"].device
+    cfg = L.make_config(sh, decode_variant=L.DECODE_TCGEN05)
+    ctx = L.Context(cfg, dev.index or 0)
+    ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    k = sel.shape[-1]
+    rows = sh.batch * sh.n_kv_heads * k * sh.chunk
+    k_rot = torch.full((rows, sh.head_dim), float("nan"), device=dev)
+    h_act = torch.full((rows, sh.mlp_hidden), float("nan"), device=dev)
+    v_rec = torch.full((rows, sh.head_dim), float("nan"), device=dev)
+    out = torch.empty_like(q)
+    params = L.layer_params(*(t_dev[n] for n in ("basis", "w1", "b1", "w2", "b2")))
+    L.debug_reconstruct(ctx, cache_dev, params, q, sel, out, k_rot, h_act, v_rec, ws)
+    st = ctx.last_error()
+    ctx.close()
+    assert st == L.OK, L.lowram_status_string(st)
+    shape = (sh.batch, sh.n_kv_heads, k * sh.chunk)
+    return (H.f64(k_rot).reshape(*shape, -1), H.f64(h_act).reshape(*shape, -1),
+            H.f64(v_rec).reshape(*shape, -1), out)
+
+
+def oracle_rows(sh, t, co, sel_np):
+    p = H.oracle_params(t)
+    d = sh.head_dim
+    ks, hs, vs = [], [], []
+    for b in range(sh.batch):
+        for h in range(sh.n_kv_heads):
+            toks, k_rot, v_rec = O.reconstruct_chunks(
+                sel_np[b, h], co["coef"][b], p["basis"], h, d, sh.chunk,
+                co["res_idx"][b, h], co["res_val"][b, h], co["chunk_ptr"][b, h],
+                p["w1"][h], p["b1"][h], p["w2"][h], p["b2"][h], sh.act, sh.theta)
+            k_pre = O.rebuild_keys(co["coef"][b][toks], p["basis"], h, d)
+            hid = O.activation(k_pre @ p["w1"][h].T + p["b1"][h], sh.act)
+            ks.append(k_rot)
+            hs.append(hid)
+            vs.append(v_rec)
+    shape = (sh.batch, sh.n_kv_heads, -1)
+    return (np.stack(ks).reshape(*shape, d), np.stack(hs).reshape(*shape, sh.mlp_hidden),
+            np.stack(vs).reshape(*shape, d))
+
+
+def check_rows(L, sh, prep, step=0):
+    t, t_dev, cdev, co, _ = prep
+    q = synth.queries(sh, 0, step)
+    osel, _ = O.select_chunks(H.f64(q), co["landmark"], sh.top_k)
+    sel = torch.from_numpy(osel.astype(np.int32)).contiguous().to(cdev["coef"].device)
+    gk, gh, gv, out = gpu_rows(L, sh, cdev, t_dev, q.to(cdev["coef"].device), sel)
+    ok, oh, ov = oracle_rows(sh, t, co, osel)
+    ek, eh, ev = H.rel_err(gk, ok), H.rel_err(gh, oh), H.rel_err(gv, ov)
+    assert ek <= TOL_K, ("k_rot", ek)
+    assert eh <= TOL_HV, ("h_act", eh)
+    assert ev <= TOL_HV, ("v_rec", ev)
+    # rows that hold a residual: V~ = MLP + R, so a dropped or misplaced residual shows
+    # here even though it moves the attention output little
+    want, _ = oracle_decode(sh, co, t, q, sel=osel)
+    assert H.rel_err(H.f64(out), want) <= H.TOL[sh.dtype]
+    return ek, eh, ev
+
+
+@pytest.fixture(scope="module")
+def config1_layer0(cuda_device):
+    sh = synth.CONFIGS[1]
+    return sh, prepared(sh, 0, cuda_device)
+
+
+def test_rebuilt_rows_config1(L, config1_layer0):
+    sh, prep = config1_layer0
+    errs = [check_rows(L, sh, prep, step) for step in range(2)]
+    print("config1 rebuilt rows: max rel err k %.2e  h %.2e  v %.2e"
+          % tuple(max(e[i] for e in errs) for i in range(3)))
+
+
+SMALL = synth.CONFIGS[1].replace(name="rows-small", n_tokens=2048, batch=2, seed=78)
+
+
+@pytest.mark.parametrize("over", [
+    dict(top_k=10 ** 6),          # every chunk selected
+    dict(top_k=37),               # ragged last tile
+    dict(top_k=1),
+    dict(res_frac=0.0),           # no residuals
+    dict(res_frac=1.0),           # every token a residual
+    dict(rank=128, act=synth.ACT_GELU_ERF),
+], ids=["all", "ragged", "k1", "nores", "allres", "r128gelu"])
+def test_rebuilt_rows_edge_cases(L, cuda_device, over):
+    sh = SMALL.replace(**over)
+    check_rows(L, sh, prepared(sh, 0, cuda_device))
+
+
+def test_tensor_core_full_rank_full_budget_equals_dense_attention(L, cuda_device):
+    """One KV head, rank = D = 128 (a square orthogonal basis), every token a residual,
+    every chunk selected, bf16: GPU encode, then the tensor-core decode, equals exact
+    dense attention over the original keys and values within the bf16 tolerance (the
+    stored bf16 basis and coefficients, and V~ = V_hat + R with R stored in bf16, are
+    the only departures from exactness)."""
+    sh = SMALL.replace(name="tc-fullrank", n_kv_heads=1, n_q_heads=4, rank=128,
+                       res_frac=1.0, top_k=10 ** 6, n_tokens=1024, batch=2, seed=6)
+    dev = cuda_device
+    t = H.stored_layer(sh, 0)
+    td = {k: v.to(dev) for k, v in t.items()}
+    cfg = L.make_config(sh, decode_variant=L.DECODE_TCGEN05)
+    ctx = L.Context(cfg, dev.index or 0)
+    cache = L.alloc_cache(cfg, dev)
+    params = L.layer_params(*(td[n] for n in ("basis", "w1", "b1", "w2", "b2")))
+    ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=dev)
+    L.encode(ctx, td["k"], td["v"], params, cache, ws)
+    assert ctx.last_error() == L.OK
+    wsd = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    dense_errs = []
+    for step in range(2):
+        q = synth.queries(sh, 0, step)
+        out = torch.empty_like(q, device=dev)
+        L.decode_step(ctx, cache, params, q.to(dev), out, wsd)
+        assert ctx.last_error() == L.OK
+        dense = O.dense_attention(H.f64(q), H.f64(t["k"]), H.f64(t["v"]))
+        dense_errs.append(H.rel_err(H.f64(out), dense))
+    ctx.close()
+    print("tc full rank vs dense attention: max rel err %.2e" % max(dense_errs))
+    assert max(dense_errs) <= 2e-2
+
+
+def test_expired_wait_reports_timeout_and_context_recovers(L, cuda_device):
+    """The attend kernel waits on per-pair ready flags that no selection sets in this
+    call: its bounded wait gives up (about 2 s), it returns with LOWRAM_ERR_TIMEOUT, and
+    the same context then decodes correctly."""
+    sh = SMALL
+    dev = cuda_device
+    t, t_dev, cdev, co, _ = prepared(sh, 0, dev)
+    cfg = L.make_config(sh, decode_variant=L.DECODE_TCGEN05)
+    ctx = L.Context(cfg, dev.index or 0)
+    ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    params = L.layer_params(*(t_dev[n] for n in ("basis", "w1", "b1", "w2", "b2")))
+    q = synth.queries(sh, 0, 0)
+    qd = q.to(dev)
+    osel, scores = O.select_chunks(H.f64(q), co["landmark"], sh.top_k)
+    sel = torch.from_numpy(osel.astype(np.int32)).contiguous().to(dev)
+    out = torch.empty_like(qd)
+    t0 = time.time()
+    L.debug_attend_unpublished(ctx, cdev, params, qd, sel, out, ws)
+    st = ctx.last_error()
+    waited = time.time() - t0
+    assert st == L.ERR_TIMEOUT, L.lowram_status_string(st)
+    assert waited < 30.0
+    assert ctx.last_error() == L.OK          # the status word was cleared by the read
+    for step in range(2):                    # the same context decodes normally
+        q = synth.queries(sh, 0, step + 1)
+        qd = q.to(dev)
+        out = torch.empty_like(qd)
+        k = min(sh.top_k, sh.n_chunks)
+        sel = torch.full((sh.batch, sh.n_kv_heads, k), -1, dtype=torch.int32, device=dev)
+        L.decode_step(ctx, cdev, params, qd, out, ws, sel_out=sel)
+        assert ctx.last_error() == L.OK
+        sel_np = sel.cpu().numpy()
+        osel, scores = O.select_chunks(H.f64(q), co["landmark"], sh.top_k)
+        H.compare_selection(sel_np, osel, scores, k)
+        want, _ = oracle_decode(sh, co, t, q, sel=sel_np.astype(np.int64))
+        assert H.rel_err(H.f64(out), want) <= H.TOL[sh.dtype]
+    ctx.close()
+    print("expired wait returned after %.2f s" % waited)
