@@ -46,6 +46,11 @@ design notes of the repository):
   subspace of the group's stacked pre-RoPE key rows, found by a randomised range finder
   (subspace iteration, Cholesky-QR applied twice, a Rayleigh-Ritz step) whose random
   test matrix is an input.
+- Composition with quantisation (LowRAM-Q): residual rows stored as symmetric int4
+  codes with an fp16 scale per 32 elements, s = fp16(max|x| / 7), q = clamp(rne(x / s),
+  -8, 7). Composition with eviction (LowRAM-E/EQ): per batch element, the chunks with
+  the smallest all-head landmark norm are evicted before compression; the kept chunks
+  keep their original RoPE positions.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against something other
 than itself (closed forms, brute force, invariants, library routines); none is
@@ -238,6 +243,84 @@ def predictor(x: np.ndarray, w1, b1, w2, b2, act: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------------
+# composition with quantisation and eviction ([summary] composition paragraph: residuals
+# stored at low precision free memory for more residuals (LowRAM-Q); eviction shortens
+# the sequence (LowRAM-E, LowRAM-EQ))
+# ----------------------------------------------------------------------------------
+INT4_GROUP = 32
+
+
+def f64_to_f16(x: np.ndarray) -> np.ndarray:
+    """Value of ``x`` after rounding to IEEE half precision (nearest, ties to even), as
+    fp64."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def quantize_int4_g32(x: np.ndarray):
+    """Symmetric int4 codes of a residual row, one fp16 scale per 32 consecutive elements.
+
+    Reading: s = fp16(max|x| / 7) per group; q = clamp(round-half-even(x / s), -8, 7),
+    q = 0 where s = 0. x: [..., d] with d % 32 == 0. Returns (codes int8 [..., d],
+    scales [..., d/32] as fp64 values of fp16 numbers).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    g = x.reshape(*x.shape[:-1], d // INT4_GROUP, INT4_GROUP)
+    s = f64_to_f16(np.abs(g).max(axis=-1) / 7.0)
+    safe = np.where(s > 0, s, 1.0)[..., None]
+    q = np.where(s[..., None] > 0, np.clip(np.rint(g / safe), -8, 7), 0.0)
+    return q.astype(np.int8).reshape(x.shape), s
+
+
+def dequantize_int4_g32(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """x_hat = q * s, group by group. codes [..., d]; scales [..., d/32] -> [..., d]."""
+    codes = np.asarray(codes, dtype=np.float64)
+    d = codes.shape[-1]
+    g = codes.reshape(*codes.shape[:-1], d // INT4_GROUP, INT4_GROUP)
+    return (g * np.asarray(scales, dtype=np.float64)[..., None]).reshape(codes.shape)
+
+
+def eviction_keep(landmark_b: np.ndarray, n_keep: int) -> np.ndarray:
+    """Chunks of one batch element that survive eviction, ascending.
+
+    Reading: the n_keep chunks with the largest all-head landmark norm (the squared L2
+    norm over every KV head's landmark, sum_h |L_c,h|^2), ties to the lower chunk index;
+    the others are evicted with their coefficients, landmarks and residual rows.
+    landmark_b: [H, N_c, d] (the stored landmarks) -> [n_keep].
+    """
+    lm = np.asarray(landmark_b, dtype=np.float64)
+    return topk_ascending((lm * lm).sum(axis=(0, 2)), n_keep)
+
+
+def encode_evicted(k_cache, v, basis, w1, b1, w2, b2, *, chunk, keep_frac, res_frac, theta,
+                   act, store, res_format="store"):
+    """Eviction, then compression of what is kept (LowRAM-E / LowRAM-EQ).
+
+    Per batch element: landmarks of the whole prefix (stored rounded), the kept chunks
+    (eviction_keep with n_keep = floor(keep_frac * N_c)), then encode() of the kept
+    tokens at their original RoPE positions with n_res = floor(res_frac * kept tokens).
+    Returns encode()'s cache of the kept tokens plus chunk_pos [B, n_keep], the original
+    chunk index of every kept chunk (ascending).
+    """
+    k_cache = np.asarray(k_cache, np.float64)
+    v = np.asarray(v, np.float64)
+    B, T, H, d = k_cache.shape
+    n_chunks = T // chunk
+    n_keep = int(math.floor(keep_frac * n_chunks + 1e-9))
+    landmark = round_to_storage(chunk_landmarks(k_cache, chunk), store)
+    chunk_pos = np.stack([eviction_keep(landmark[b], n_keep) for b in range(B)])
+    rows = (chunk_pos[:, :, None] * chunk + np.arange(chunk)[None, None, :]).reshape(B, -1)
+    kk = np.stack([k_cache[b, rows[b]] for b in range(B)])
+    vv = np.stack([v[b, rows[b]] for b in range(B)])
+    n_res = int(math.floor(res_frac * n_keep * chunk + 1e-9))
+    out = encode(kk, vv, basis, w1, b1, w2, b2, chunk=chunk, n_res=n_res, theta=theta,
+                 act=act, store=store, positions=rows, res_format=res_format)
+    out["chunk_pos"] = chunk_pos
+    out["full_landmark"] = landmark
+    return out
+
+
+# ----------------------------------------------------------------------------------
 # encode [keys], [values], [how: Residuals for difficult tokens]
 # ----------------------------------------------------------------------------------
 def residual_errors(v_h: np.ndarray, coef_exact: np.ndarray, basis, h, w1, b1, w2, b2,
@@ -254,11 +337,16 @@ def residual_chunk_ptr(res_idx: np.ndarray, n_tokens: int, chunk: int) -> np.nda
     return np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
 
 
-def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store):
+def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store,
+           positions=None, res_format="store"):
     """Compress one layer's prefix.
 
     k_cache, v: [B, T, H, d] (post-RoPE keys, values); basis [D, r]; w1 [H, F, d];
-    b1 [H, F]; w2 [H, d, F]; b2 [H, d]. Steps, in the pages' order:
+    b1 [H, F]; w2 [H, d, F]; b2 [H, d]. ``positions`` [B, T] are the tokens' RoPE
+    positions (default 0 .. T-1; after eviction, the kept tokens' original positions).
+    ``res_format`` "store" keeps residual rows in the storage precision; "int4" keeps
+    them as int4 codes with an fp16 scale per 32 elements (res_q, res_scale), and
+    res_val holds their dequantized values. Steps, in the pages' order:
       1. invert RoPE on the keys;
       2. project every token's flattened key onto the shared basis (coefficients are
          stored rounded to ``store``);
@@ -272,8 +360,8 @@ def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store
     v = np.asarray(v, np.float64)
     B, T, H, d = k_cache.shape
     D = H * d
-    pos = np.arange(T)
-    k_pre = rope_rotate(k_cache, pos[None, :, None], theta, inverse=True)
+    pos = np.broadcast_to(np.arange(T), (B, T)) if positions is None else np.asarray(positions)
+    k_pre = rope_rotate(k_cache, pos[:, :, None], theta, inverse=True)
     coef_exact = project_keys(k_pre.reshape(B, T, D), basis)
     coef = round_to_storage(coef_exact, store)
     landmark = round_to_storage(chunk_landmarks(k_cache, chunk), store)
@@ -282,6 +370,9 @@ def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store
     res_idx = np.empty((B, H, n_res), np.int64)
     res_val = np.empty((B, H, n_res, d))
     chunk_ptr = np.empty((B, H, n_chunks + 1), np.int64)
+    if res_format == "int4":
+        res_q = np.empty((B, H, n_res, d), np.int8)
+        res_scale = np.empty((B, H, n_res, d // INT4_GROUP))
     for b in range(B):
         for h in range(H):
             err[b, h] = residual_errors(v[b, :, h], coef_exact[b], basis, h,
@@ -290,10 +381,18 @@ def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store
             vhat_stored = predictor(rebuild_keys(coef[b, idx], basis, h, d),
                                     w1[h], b1[h], w2[h], b2[h], act)
             res_idx[b, h] = idx
-            res_val[b, h] = round_to_storage(v[b, idx, h] - vhat_stored, store)
+            if res_format == "int4":
+                codes, scales = quantize_int4_g32(v[b, idx, h] - vhat_stored)
+                res_q[b, h], res_scale[b, h] = codes, scales
+                res_val[b, h] = dequantize_int4_g32(codes, scales)
+            else:
+                res_val[b, h] = round_to_storage(v[b, idx, h] - vhat_stored, store)
             chunk_ptr[b, h] = residual_chunk_ptr(idx, T, chunk)
-    return {"coef": coef, "coef_exact": coef_exact, "landmark": landmark,
-            "res_idx": res_idx, "res_val": res_val, "chunk_ptr": chunk_ptr, "err": err}
+    out = {"coef": coef, "coef_exact": coef_exact, "landmark": landmark,
+           "res_idx": res_idx, "res_val": res_val, "chunk_ptr": chunk_ptr, "err": err}
+    if res_format == "int4":
+        out["res_q"], out["res_scale"] = res_q, res_scale
+    return out
 
 
 # ----------------------------------------------------------------------------------
@@ -319,16 +418,20 @@ def select_chunks(q, landmark, top_k):
 
 
 def reconstruct_chunks(sel_bh, coef_b, basis, h, d, chunk, res_idx_bh, res_val_bh,
-                       chunk_ptr_bh, w1, b1, w2, b2, act, theta):
+                       chunk_ptr_bh, w1, b1, w2, b2, act, theta, chunk_pos_b=None):
     """Rebuild K (post-RoPE) and V for the selected chunks of one (batch, KV head).
 
-    Returns (tokens [n], k_rot [n, d], v_rec [n, d]) with tokens in selection order.
-    V = MLP_h(B_h coef_t), plus the stored residual R_t where t holds one.
+    Returns (tokens [n], k_rot [n, d], v_rec [n, d]) with tokens (rows of the cache) in
+    selection order. V = MLP_h(B_h coef_t), plus the stored residual R_t where t holds
+    one. ``chunk_pos_b`` maps a stored chunk to its original chunk index (eviction): RoPE
+    is re-applied at the original positions.
     """
     sel_bh = np.asarray(sel_bh, np.int64)
     tokens = (sel_bh[:, None] * chunk + np.arange(chunk)[None, :]).reshape(-1)
+    base = sel_bh if chunk_pos_b is None else np.asarray(chunk_pos_b, np.int64)[sel_bh]
+    positions = (base[:, None] * chunk + np.arange(chunk)[None, :]).reshape(-1)
     k_pre = rebuild_keys(np.asarray(coef_b, np.float64)[tokens], basis, h, d)
-    k_rot = rope_rotate(k_pre, tokens, theta)
+    k_rot = rope_rotate(k_pre, positions, theta)
     v_rec = predictor(k_pre, w1, b1, w2, b2, act)
     for slot, c in enumerate(sel_bh):
         for i in range(int(chunk_ptr_bh[c]), int(chunk_ptr_bh[c + 1])):
@@ -342,8 +445,9 @@ def decode_step(q, cache, basis, w1, b1, w2, b2, *, chunk, top_k, theta, act, se
     """One decode step of one layer over the compressed cache.
 
     q: [B, H_q, d] (post-RoPE). cache: dict with coef [B,T,r], landmark [B,H,N_c,d],
-    res_idx [B,H,n_res], res_val [B,H,n_res,d], chunk_ptr [B,H,N_c+1]. ``sel`` may
-    override the selection (used when a caller's selection differs only by ties).
+    res_idx [B,H,n_res], res_val [B,H,n_res,d], chunk_ptr [B,H,N_c+1], and after eviction
+    chunk_pos [B,N_c] (original chunk index of each stored chunk). ``sel`` may override
+    the selection (used when a caller's selection differs only by ties).
     Returns (out [B, H_q, d], sel [B, H, k]).
     """
     q = np.asarray(q, np.float64)
@@ -358,7 +462,8 @@ def decode_step(q, cache, basis, w1, b1, w2, b2, *, chunk, top_k, theta, act, se
             _, k_rot, v_rec = reconstruct_chunks(
                 sel[b, h], cache["coef"][b], basis, h, d, chunk,
                 cache["res_idx"][b, h], cache["res_val"][b, h], cache["chunk_ptr"][b, h],
-                w1[h], b1[h], w2[h], b2[h], act, theta)
+                w1[h], b1[h], w2[h], b2[h], act, theta,
+                None if cache.get("chunk_pos") is None else cache["chunk_pos"][b])
             for g in range(G):
                 z = k_rot @ q[b, h * G + g] / math.sqrt(d)
                 p = np.exp(z - z.max())

@@ -328,10 +328,109 @@ def check_fit_basis_recovers_generator(M):
     assert np.linalg.norm(B @ B.T - bg @ bg.T, 2) < 0.03
 
 
+def check_int4_quantize(M):
+    """int4 codes with an fp16 scale per 32 elements: exact on grids of fp16 multiples,
+    half a step at most elsewhere, ties to even, zero groups, and the fp16 rounding
+    itself against torch's conversion (a library routine)."""
+    rng = np.random.default_rng(31)
+    # rows whose groups are exact multiples of an fp16 step, with a +-7 step present
+    steps = np.float16(rng.uniform(0.01, 2.0, (5, 4))).astype(np.float64)
+    ints = rng.integers(-7, 8, (5, 4, 32))
+    ints[:, :, 0] = np.where(rng.random((5, 4)) < 0.5, 7, -7)
+    x = (ints * steps[..., None]).reshape(5, 128)
+    q, s = M.quantize_int4_g32(x)
+    assert np.array_equal(s, steps)
+    assert np.array_equal(q.reshape(5, 4, 32), ints)
+    assert np.array_equal(M.dequantize_int4_g32(q, s), x)
+    # arbitrary rows: within half a step, codes in range, the largest element at +-7
+    x = rng.standard_normal((50, 128)) * 10.0 ** rng.integers(-3, 3, (50, 1))
+    q, s = M.quantize_int4_g32(x)
+    err = np.abs(M.dequantize_int4_g32(q, s) - x).reshape(50, 4, 32)
+    assert np.all(err <= s[..., None] / 2 * (1 + 1e-12))
+    assert q.min() >= -8 and q.max() <= 7
+    g = np.abs(x).reshape(50, 4, 32)
+    top = np.take_along_axis(np.abs(q).reshape(50, 4, 32), g.argmax(-1)[..., None], -1)
+    assert np.all(top == 7)
+    # ties to even: x / s = 2.5 -> 2, 3.5 -> 4, -2.5 -> -2, -0.5 -> 0
+    row = np.zeros(32)
+    row[:5] = [7.0, 2.5, 3.5, -2.5, -0.5]
+    q, s = M.quantize_int4_g32(row)
+    assert s[0] == 1.0 and list(q[:5]) == [7, 2, 4, -2, 0]
+    # an all-zero group has scale 0 and codes 0
+    q, s = M.quantize_int4_g32(np.zeros(64))
+    assert np.all(s == 0) and np.all(q == 0)
+    # fp16 rounding of fp32 values (torch converts those with one rounding; from fp64 it
+    # rounds through fp32 first, which is not a reference for fp64 inputs)
+    y = (rng.standard_normal(4000) * 10.0 ** rng.integers(-6, 4, 4000)).astype(np.float32)
+    y[:3] = [1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2048.0 + 1.0]   # ties
+    ref = torch.from_numpy(y).to(torch.float16).to(torch.float64).numpy()
+    assert np.array_equal(M.f64_to_f16(y.astype(np.float64)), ref)
+    assert M.f64_to_f16(np.array([1.0 + 2.0 ** -11 + 2.0 ** -40]))[0] == 1.0 + 2.0 ** -10
+
+
+def check_eviction(M):
+    """The kept chunks are those with the largest all-head landmark norm, ties to the
+    lower chunk index (brute force: fsum of squares, Python sort), ascending."""
+    rng = np.random.default_rng(32)
+    H, n, d = 3, 40, 8
+    lm = rng.standard_normal((H, n, d))
+    lm[:, 7] = lm[:, 3]            # exact ties in norm
+    lm[:, 30] = -lm[:, 3]
+    for n_keep in (1, 13, 20, 40):
+        norm = [math.fsum(float(lm[h, c, j]) ** 2 for h in range(H) for j in range(d))
+                for c in range(n)]
+        brute = sorted(sorted(range(n), key=lambda c: (-norm[c], c))[:n_keep])
+        assert list(M.eviction_keep(lm, n_keep)) == brute, n_keep
+
+
+def check_evicted_full_rank_exactness(M):
+    """Eviction of half the chunks, then full rank, every kept token a residual and every
+    kept chunk selected (f64 storage): decode equals dense attention over the kept
+    tokens' original keys and values, at their original positions."""
+    sh = tiny_shape(rank=16, n_kv_heads=2, head_dim=8, res_frac=1.0, top_k=10 ** 6,
+                    n_tokens=64, chunk=4)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    cache = M.encode_evicted(L["k"], L["v"], L["basis"], *L["w"], keep_frac=0.5,
+                             res_frac=1.0, store=M.STORE_F64, **kw)
+    pos = cache["chunk_pos"]
+    assert pos.shape == (sh.batch, sh.n_chunks // 2)
+    rows = (pos[:, :, None] * sh.chunk + np.arange(sh.chunk)).reshape(sh.batch, -1)
+    kk = np.stack([L["k"][b, rows[b]] for b in range(sh.batch)])
+    vv = np.stack([L["v"][b, rows[b]] for b in range(sh.batch)])
+    out, _ = M.decode_step(L["q"], cache, L["basis"], *L["w"], top_k=sh.top_k, **kw)
+    assert np.allclose(out, M.dense_attention(L["q"], kk, vv), atol=1e-12)
+    # the eviction kept the largest all-head landmark norms of the stored landmarks
+    for b in range(sh.batch):
+        nrm = (cache["full_landmark"][b] ** 2).sum(axis=(0, 2))
+        assert nrm[pos[b]].min() >= np.delete(nrm, pos[b]).max()
+
+
+def check_int4_residual_encode(M):
+    """encode with int4 residual rows: res_val is the dequantized code, and the stored
+    prediction plus it restores V within half a quantisation step per element."""
+    sh = synth.CONFIGS[0].replace(n_layers=1, n_tokens=256)
+    L = make_layer(sh)
+    cache = M.encode(L["k"], L["v"], L["basis"], *L["w"], chunk=sh.chunk, n_res=sh.n_res,
+                     theta=sh.theta, act=sh.act, store=M.STORE_BF16, res_format="int4")
+    assert np.array_equal(cache["res_val"],
+                          M.dequantize_int4_g32(cache["res_q"], cache["res_scale"]))
+    w1, b1, w2, b2 = L["w"]
+    d = sh.head_dim
+    for h in range(sh.n_kv_heads):
+        idx = cache["res_idx"][0, h]
+        vhat = M.predictor(M.rebuild_keys(cache["coef"][0, idx], L["basis"], h, d),
+                           w1[h], b1[h], w2[h], b2[h], sh.act)
+        err = np.abs(vhat + cache["res_val"][0, h] - L["v"][0, idx, h]).reshape(len(idx), -1, 32)
+        assert np.all(err <= cache["res_scale"][0, h][..., None] / 2 * (1 + 1e-9) + 1e-12)
+
+
 ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
               check_landmarks_and_scores, check_encode_landmarks, check_topk, check_predictor,
               check_full_rank_exactness, check_residual_pick, check_selection_and_edges,
-              check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator]
+              check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator,
+              check_int4_quantize, check_eviction, check_evicted_full_rank_exactness,
+              check_int4_residual_encode]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -489,3 +588,31 @@ def test_mutation_cholesky_qr_wrong_factor(monkeypatch):
         r_up = np.linalg.cholesky(y.T @ y).T
         return np.linalg.solve(r_up, y.T).T
     _fails(check_cholesky_qr, monkeypatch, "cholesky_qr", bad)
+
+
+def test_mutation_int4_scale_over_eight(monkeypatch):
+    def bad(x):
+        x = np.asarray(x, np.float64)
+        g = x.reshape(*x.shape[:-1], -1, 32)
+        sc = O.f64_to_f16(np.abs(g).max(axis=-1) / 8.0)
+        safe = np.where(sc > 0, sc, 1.0)[..., None]
+        q = np.where(sc[..., None] > 0, np.clip(np.rint(g / safe), -8, 7), 0.0)
+        return q.astype(np.int8).reshape(x.shape), sc
+    _fails(check_int4_quantize, monkeypatch, "quantize_int4_g32", bad)
+
+
+def test_mutation_eviction_keeps_smallest(monkeypatch):
+    def bad(lm, n_keep):
+        lm = np.asarray(lm, np.float64)
+        return O.topk_ascending(-(lm * lm).sum(axis=(0, 2)), n_keep)
+    _fails(check_eviction, monkeypatch, "eviction_keep", bad)
+
+
+def test_mutation_evicted_positions_ignored(monkeypatch):
+    """Reconstruction re-applying RoPE at the stored slot instead of the original
+    position."""
+    orig = O.reconstruct_chunks
+
+    def bad(*args):
+        return orig(*args[:15], None)
+    _fails(check_evicted_full_rank_exactness, monkeypatch, "reconstruct_chunks", bad)
