@@ -36,6 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "decode tokens/s + achieved HBM GB/s (% of ~8 TB/s) at 128K context"
 NOMINAL_HBM_GBS = 8000.0
+MODEL_SHAPE = {2: "Llama-3-8B", 3: "Mistral-7B"}
 
 
 def parse_args(argv=None):
@@ -46,9 +47,18 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only the first L layers (profiling runs)")
+    ap.add_argument("--config", type=int, choices=[2, 3, 4], default=2,
+                    help="2: Llama-3-8B-shaped, batch 8, 128K (the headline line); "
+                         "3: Mistral-7B-shaped, batch 4, 262K, rank 128, 15%% residuals; "
+                         "4: LowRAM-EQ (half the chunks evicted, int4 residual rows for 40%% "
+                         "of the kept tokens) at 64K over a batch sweep")
+    ap.add_argument("--batches", default="1,4,8,16,28",
+                    help="batch sizes of the config-4 sweep")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip timing the uncompressed dense-decode baseline")
     return ap.parse_args(argv)
 
 
@@ -183,7 +193,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    base = synth.CONFIGS[2]
+    base = synth.CONFIGS[args.config]
     n_layers = args.layers or base.n_layers
     sh = rank_shape(base, rank)
     cfg = L.make_config(sh)
@@ -358,6 +368,49 @@ def run_ours(args):
                "path": "lowram_decode_step per layer (eager), pinned host queries/outputs"}
     clocks = sampler.stop()
 
+    # ---- the uncompressed baseline on the same box: exact dense GQA decode of one layer
+    # over the full bf16 cache (layer 0's keys and values), timed per layer call; the
+    # per-layer time does not depend on how many layers are resident, so tokens/s is
+    # B / (layers x time per layer)
+    dense = None
+    if not args.no_dense:
+        kd = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        vd = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        basis0 = synth.group_basis(sh, 0)
+        w0 = synth.layer_weights(sh, 0)
+        for b in range(B):
+            kb, vb = synth.layer_kv(sh, basis0, w0, 0, b, device=dev, compute_dtype=torch.float32)
+            kd[b], vd[b] = kb, vb
+            del kb, vb
+        ws_dense = torch.empty(L.workspace_size(cfg, L.OP_DENSE), dtype=torch.uint8, device=dev)
+        od = torch.empty(B, sh.n_q_heads, d, dtype=st, device=dev)
+        n_dense = 20
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                L.dense_decode(ctx, kd, vd, q_all[W + i, 0], od, ws_dense)
+            torch.cuda.synchronize()
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            for i in range(n_dense):
+                L.dense_decode(ctx, kd, vd, q_all[W + (i % K), 0], od, ws_dense)
+            d1.record(stream)
+        torch.cuda.synchronize()
+        ms_dense = max_over_ranks(d0.elapsed_time(d1) / n_dense, dev)
+        dense_bytes = 2 * B * T * Hk * d * 2 + 2 * B * sh.n_q_heads * d * 2
+        dense_tps = B * world / (n_layers * ms_dense / 1e3)
+        lay_bytes = sum(L.cache_layout(cfg))
+        dense = {"kernel": "dense_decode_kernel + dense_combine_kernel (exact GQA flash-decode "
+                           "over the uncompressed bf16 cache)",
+                 "us_per_layer": round(ms_dense * 1e3, 2), "tokens_per_s": round(dense_tps, 1),
+                 "achieved_gbs": round(dense_bytes / (ms_dense / 1e3) / 1e9, 1),
+                 "hbm_frac": round(dense_bytes / (ms_dense / 1e3) / 1e9 / hbm_peak_of(ROOT), 4),
+                 "bytes_per_layer": dense_bytes,
+                 "compressed_speedup": round(tokens_per_s_of(B, world, ms_step) / dense_tps, 3),
+                 "cache_bytes_per_layer": {"uncompressed_bf16": 2 * B * T * Hk * d * 2,
+                                           "compressed": int(lay_bytes)},
+                 "compression_ratio": round(2 * B * T * Hk * d * 2 / lay_bytes, 3)}
+        del kd, vd, ws_dense
+
     ms_step_max = max_over_ranks(ms_step, dev)
     ms_a_max = max_over_ranks(ms_a, dev)
     ms_b_max = max_over_ranks(ms_b, dev)
@@ -410,10 +463,12 @@ def run_ours(args):
         parity["residual_pick"] = residual_pick_vs_oracle(sh, layers[0], kv0)
 
     line = {
-        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s",
+        "metric": METRIC if args.config == 2 else METRIC.replace("128K", "262K"),
+        "value": round(tokens_per_s, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step_max, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, encoded on device",
+        "data": f"synthetic: seeded {MODEL_SHAPE[args.config]}-shaped GQA keys/values, "
+                "encoded on device",
         "config": {"workload": f"{base.name}" + ("" if n_layers == base.n_layers else f"-{n_layers}layers"),
                    "batch_per_gpu": B, "context": T, "layers": n_layers, "kv_heads": Hk,
                    "q_heads": sh.n_q_heads, "head_dim": d, "rank": sh.rank, "chunk": sh.chunk,
@@ -427,6 +482,7 @@ def run_ours(args):
         "roofline_reconstruct_attend": roof_b,
         "cpu_baseline": cpu,
         "parity_vs_oracle": parity,
+        "dense_baseline": dense,
         "e2e": e2e,
         "gpu_launches": 3 * n_layers * K,
         "clocks": clocks,
@@ -441,6 +497,17 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def hbm_peak_of(root: str) -> float:
+    try:
+        return float(json.load(open(os.path.join(root, "MEASURED_PEAKS.json")))["hbm_gbs"])
+    except Exception:
+        return 6650.0
+
+
+def tokens_per_s_of(B: int, world: int, ms_step: float) -> float:
+    return B * world / (ms_step / 1e3)
 
 
 def measured_traffic(kernel: str):
@@ -587,7 +654,7 @@ def run_reference(args):
     import oracle.lowram_oracle as O
     from long_context_decode_02_b200 import synth
 
-    base = synth.CONFIGS[2]
+    base = synth.CONFIGS[args.config]
     sh = base.replace(batch=1)
     n_layers = args.layers or base.n_layers
     # one batch element of layer 0, generated and encoded on the CPU by the oracle
@@ -628,11 +695,14 @@ def run_reference(args):
               f"cache, a fresh query per call) = {tokens_per_step:g} token(s) of one "
               f"sequence through {n_layers} layers")
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s",
+        "impl": "reference",
+        "metric": METRIC if args.config == 2 else METRIC.replace("128K", "262K"),
+        "value": round(value, 4), "unit": "tokens/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": K, "warmup": W,
         "ms_per_step": round(ms_step, 2), "tokens_per_step": tokens_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, encoded by the oracle",
+        "data": f"synthetic: seeded {MODEL_SHAPE[args.config]}-shaped GQA keys/values, "
+                "encoded by the oracle",
         "config": {"workload": base.name, "batch_per_gpu": base.batch, "context": base.n_tokens,
                    "layers": n_layers, "sampled": sample},
         "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": _threads(),
@@ -643,10 +713,162 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------------
+# LowRAM-Q/EQ batch sweep (config 4): eviction + int4 residual rows, footprint vs dense
+# ----------------------------------------------------------------------------------
+def encode_layers(L, sh, cfg, ctx, n_layers, dev):
+    """Seeded keys/values of every layer, evicted (when the shape evicts) and encoded on
+    the device; returns the layers' caches and parameters and the encode ms per layer."""
+    import torch
+
+    from long_context_decode_02_b200 import synth
+    st = sh.torch_dtype
+    B, T, Hk, d = sh.batch, sh.n_tokens, sh.n_kv_heads, sh.head_dim
+    enc_ws = torch.empty(L.workspace_size(cfg, L.OP_ENCODE), dtype=torch.uint8, device=dev)
+    ev_ws = (torch.empty(L.workspace_size(cfg, L.OP_EVICT), dtype=torch.uint8, device=dev)
+             if sh.evicted else None)
+    layers, enc_ms = [], []
+    basis64 = basis_dev = None
+    for layer in range(n_layers):
+        if layer % 2 == 0:
+            basis64 = synth.group_basis(sh, layer // 2)
+            basis_dev = basis64.to(st).to(dev)
+        w = synth.layer_weights(sh, layer)
+        wd = [x.to(st).to(dev) for x in w]
+        k = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        v = torch.empty(B, T, Hk, d, dtype=st, device=dev)
+        for b in range(B):
+            kb, vb = synth.layer_kv(sh, basis64, w, layer, b, device=dev,
+                                    compute_dtype=torch.float32)
+            k[b], v[b] = kb, vb
+            del kb, vb
+        cache = L.alloc_cache(cfg, dev)
+        params = L.layer_params(basis_dev, *wd)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if sh.evicted:
+            kk = torch.empty(B, sh.n_kept_tokens, Hk, d, dtype=st, device=dev)
+            vk = torch.empty_like(kk)
+            L.evict(ctx, k, v, kk, vk, cache["chunk_pos"], ev_ws)
+            del k, v
+            k, v = kk, vk
+        L.encode(ctx, k, v, params, cache, enc_ws)
+        e1.record()
+        torch.cuda.synchronize()
+        enc_ms.append(e0.elapsed_time(e1))
+        layers.append({"cache": cache, "params": params, "keep": (basis_dev, wd)})
+        del k, v
+    del enc_ws, ev_ws
+    torch.cuda.empty_cache()
+    assert ctx.last_error() == L.OK, "encode reported a device status"
+    return layers, enc_ms
+
+
+def time_decode_steps(L, sh, cfg, ctx, layers, n_layers, W, K, dev):
+    """ms per captured decode step of every layer (fresh queries each step)."""
+    import torch
+
+    from long_context_decode_02_b200 import synth
+    st = sh.torch_dtype
+    B, d = sh.batch, sh.head_dim
+    q_all = torch.empty(W + K, n_layers, B, sh.n_q_heads, d, dtype=st, device=dev)
+    for i in range(W + K):
+        for layer in range(n_layers):
+            q_all[i, layer] = synth.queries(sh, layer, i, device=dev)
+    q_buf = torch.empty(n_layers, B, sh.n_q_heads, d, dtype=st, device=dev)
+    out_buf = torch.empty_like(q_buf)
+    ws = torch.empty(L.workspace_size(cfg, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_calls():
+        for layer in range(n_layers):
+            Ld = layers[layer]
+            L.decode_step(ctx, Ld["cache"], Ld["params"], q_buf[layer], out_buf[layer], ws)
+
+    with torch.cuda.stream(stream):
+        q_buf.copy_(q_all[0])
+        step_calls()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        step_calls()
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            q_buf.copy_(q_all[i])
+            g.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for i in range(K):
+            q_buf.copy_(q_all[W + i])
+            g.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    assert ctx.last_error() == L.OK
+    g.reset()
+    return t0.elapsed_time(t1) / K
+
+
+def run_sweep(args):
+    """LowRAM-Q/EQ (config 4): decode tokens/s and HBM footprint over a batch sweep, with
+    the uncompressed bf16 cache's footprint beside it (it no longer fits the GPU at the
+    largest batches)."""
+    import torch
+
+    from long_context_decode_02_b200 import lowram as L
+    from long_context_decode_02_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = synth.CONFIGS[4]
+    n_layers = args.layers or base.n_layers
+    hbm_total = torch.cuda.get_device_properties(dev).total_memory
+    rows = []
+    for B in [int(x) for x in args.batches.split(",")]:
+        sh = base.replace(batch=B)
+        cfg = L.make_config(sh)
+        ctx = L.Context(cfg, 0)
+        layers, enc_ms = encode_layers(L, sh, cfg, ctx, n_layers, dev)
+        ms = time_decode_steps(L, sh, cfg, ctx, layers, n_layers, args.warmup, args.steps, dev)
+        cache_bytes = int(sum(L.cache_layout(cfg))) * n_layers
+        weight_bytes = sum(int(t.numel() * t.element_size())
+                           for Ld in layers for t in Ld["keep"][1]) + \
+            sum(int(layers[i]["keep"][0].numel() * 2) for i in range(0, n_layers, 2))
+        dense_bytes = 2 * B * sh.n_tokens * sh.n_kv_heads * sh.head_dim * 2 * n_layers
+        rows.append({"batch": B, "tokens_per_s": round(B / (ms / 1e3), 1),
+                     "ms_per_step": round(ms, 4),
+                     "compressed_cache_gb": round(cache_bytes / 1e9, 3),
+                     "weights_gb": round(weight_bytes / 1e9, 3),
+                     "uncompressed_bf16_cache_gb": round(dense_bytes / 1e9, 3),
+                     "compression_ratio": round(dense_bytes / cache_bytes, 3),
+                     "uncompressed_fits_in_hbm": dense_bytes < hbm_total,
+                     "encode_ms_per_layer": round(statistics.mean(enc_ms), 2)})
+        for Ld in layers:
+            Ld.clear()
+        del layers
+        ctx.close()
+        torch.cuda.empty_cache()
+    top = rows[-1]
+    line = {"metric": "LowRAM-EQ decode tokens/s and HBM footprint at 64K context, batch sweep",
+            "value": top["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": top["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded Llama-3-8B-shaped GQA keys/values, evicted and encoded "
+                    "on device",
+            "config": {"workload": base.name, "context": base.n_tokens, "layers": n_layers,
+                       "kept_chunks": base.keep_frac, "residual_frac_of_kept": base.res_frac,
+                       "residual_storage": "int4, fp16 scale per 32", "rank": base.rank,
+                       "top_k_chunks": base.top_k, "hbm_total_gb": round(hbm_total / 1e9, 1)},
+            "sweep": rows}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.config == 4:
+        run_sweep(args)
     else:
         run_ours(args)
 

@@ -62,7 +62,13 @@ enum { LOWRAM_ACT_SILU = 0, LOWRAM_ACT_GELU_ERF = 1 };
  * CUDA-core kernel otherwise (always for fp32, whose 1e-4 tolerance tensor cores cannot
  * meet). */
 enum { LOWRAM_DECODE_AUTO = 0, LOWRAM_DECODE_SIMT = 1, LOWRAM_DECODE_TCGEN05 = 2 };
-enum { LOWRAM_OP_ENCODE = 0, LOWRAM_OP_DECODE = 1 };
+enum { LOWRAM_OP_ENCODE = 0, LOWRAM_OP_DECODE = 1, LOWRAM_OP_DENSE = 2, LOWRAM_OP_EVICT = 3 };
+/* How residual rows are stored. STORE: in cfg->dtype. INT4_G32 (LowRAM-Q, the residuals
+ * stored at low precision of the agihunt summary's composition paragraph): symmetric
+ * int4 codes, two per byte (element 2i in the low nibble), with one fp16 scale per 32
+ * elements, s = fp16(max|x| / 7), q = clamp(round-half-even(x / s), -8, 7); the row's
+ * value is q * s. bf16 caches with the tensor-core encode's sizes only. */
+enum { LOWRAM_RES_STORE = 0, LOWRAM_RES_INT4_G32 = 1 };
 
 /* Sizes of one layer call. T % chunk == 0; n_q_heads % n_kv_heads == 0. */
 typedef struct lowram_config {
@@ -79,6 +85,12 @@ typedef struct lowram_config {
   int32_t act;            /* LOWRAM_ACT_*                                               */
   int32_t dtype;          /* LOWRAM_DTYPE_*                                             */
   int32_t decode_variant; /* LOWRAM_DECODE_*                                            */
+  int32_t res_format;     /* LOWRAM_RES_*                                               */
+  int32_t n_positions;    /* RoPE positions of the original prefix, 0 .. n_positions-1;
+                             0 means n_tokens. Larger than n_tokens only for a cache whose
+                             chunks were evicted (lowram_evict): the cache then holds
+                             n_tokens tokens of kept chunks and cache->chunk_pos gives each
+                             stored chunk's original index. A multiple of chunk.          */
   int32_t reserved;       /* must be 0                                                  */
   double rope_theta;      /* RoPE base; theta_i = rope_theta^(-2i/d)                    */
 } lowram_config;
@@ -109,9 +121,16 @@ typedef struct lowram_layer_params {
  *                                writes it; lowram_landmark_norms recomputes it for a
  *                                cache built elsewhere. A value below the true maximum
  *                                can change the selection.
+ *   chunk_pos [B][T/C]           int32 original chunk index of each stored chunk,
+ *                                ascending (eviction; RoPE is re-applied at position
+ *                                chunk_pos*C + j). NULL when n_positions == n_tokens.
+ *   res_scale [B][H_kv][n_res][d/32] fp16 scales of int4 residual rows (res_format
+ *                                INT4_G32; res_val then holds [B][H_kv][n_res][d/2] bytes
+ *                                of codes). NULL otherwise.
  * The layout is fixed by these shapes, so a cache can be saved and restored byte for
- * byte (lowram_cache_layout gives the six sizes). res_idx and res_val may be NULL when
- * n_res == 0. */
+ * byte (lowram_cache_layout gives the eight sizes). res_idx, res_val and res_scale may be
+ * NULL when n_res == 0. With eviction, decode selects among the stored chunks: sel_out
+ * holds stored-chunk indices (map them through chunk_pos). */
 typedef struct lowram_cache {
   void* coef;
   void* landmark;
@@ -119,6 +138,8 @@ typedef struct lowram_cache {
   void* res_val;
   int32_t* chunk_ptr;
   float* landmark_norm;
+  int32_t* chunk_pos;
+  void* res_scale;
 } lowram_cache;
 
 typedef struct lowram_ctx lowram_ctx;
@@ -138,9 +159,9 @@ lowram_status lowram_create(const lowram_config* cfg, int device, lowram_ctx** o
  * stream still using the context. NULL is accepted. */
 void lowram_destroy(lowram_ctx* ctx);
 
-/* Host only. bytes_out[0..5] = sizes of coef, landmark, res_idx, res_val, chunk_ptr,
- * landmark_norm. */
-lowram_status lowram_cache_layout(const lowram_config* cfg, size_t bytes_out[6]);
+/* Host only. bytes_out[0..7] = sizes of coef, landmark, res_idx, res_val, chunk_ptr,
+ * landmark_norm, chunk_pos (0 without eviction), res_scale (0 unless int4 residuals). */
+lowram_status lowram_cache_layout(const lowram_config* cfg, size_t bytes_out[8]);
 
 /* Host only. Workspace bytes needed by op (LOWRAM_OP_ENCODE or LOWRAM_OP_DECODE). The
  * workspace needs no initialisation and holds nothing between calls. */
@@ -158,6 +179,46 @@ lowram_status lowram_workspace_size(const lowram_config* cfg, int op, size_t* by
 lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
                             const lowram_layer_params* params, const lowram_cache* out,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Eviction before compression (LowRAM-E / LowRAM-EQ: eviction composes with the method,
+ * agihunt summary, composition paragraph). For every batch element, keeps the
+ * n_tokens / C chunks of the n_positions-token prefix with the largest all-head landmark
+ * norm (sum over KV heads of |landmark|^2, landmarks as lowram_encode stores them: the
+ * fp32 chunk mean rounded to the cache dtype; norms summed in fp64), ties to the lower
+ * chunk, and copies their keys and values out in ascending order.
+ *   k_full, v_full [B][n_positions][H_kv][d] (post-RoPE keys, values; inputs);
+ *   k_kept, v_kept [B][n_tokens][H_kv][d] (written);
+ *   chunk_pos [B][n_tokens / C] int32 (written): the kept chunks' original indices,
+ *   ascending; pass it as cache->chunk_pos to lowram_encode and to decode.
+ * Workspace: lowram_workspace_size(cfg, LOWRAM_OP_EVICT). Needs n_positions > n_tokens. */
+lowram_status lowram_evict(lowram_ctx* ctx, const void* k_full, const void* v_full,
+                           void* k_kept, void* v_kept, int32_t* chunk_pos, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* The xKV basis of one layer group from its keys, by a randomised range finder with
+ * Cholesky-QR in place of an exact SVD (agihunt summary, key paragraph: adjacent layers
+ * share one SVD basis, computed by a randomised Cholesky-QR instead of the exact SVD).
+ * With A the group's pre-RoPE key rows (every token of every layer and batch element,
+ * flattened over D = H_kv*d):
+ *   Y = A^T A omega;  Q = CholQR2(Y);  n_power times: Q = CholQR2(A^T A Q);
+ *   S = Q^T A^T A Q = U diag(lambda) U^T (Rayleigh-Ritz);  basis = Q U[:, :r]
+ * with the columns of U by decreasing lambda (ties to the lower index), CholQR2 = Q from
+ * Cholesky-QR applied twice (Y^T Y = R^T R, Q = Y R^-1). All in fp64 (A^T A formed once
+ * as a D x D Gram matrix; the eigenproblem by Jacobi rotations). Each column of the
+ * result is defined up to its sign.
+ *   k_layers  HOST array of n_layers (1..8) device pointers, each [B][T][H_kv][d] post-RoPE
+ *             keys of one layer of the group (the context's sizes; no eviction);
+ *   omega     [D][l] fp64 random test matrix (input), r <= l <= min(D, 256);
+ *   basis_out [D][r] in cfg->dtype (written): orthonormal columns.
+ * Workspace: lowram_fit_basis_workspace_size. Cholesky-QR needs Y of full column rank:
+ * keys of rank below l make a pivot non-positive, which lowram_last_error reports as
+ * LOWRAM_ERR_DEVICE_CHECK (the result is then not valid). */
+lowram_status lowram_fit_basis(lowram_ctx* ctx, const void* const* k_layers, int32_t n_layers,
+                               const double* omega, int32_t l, int32_t n_power,
+                               void* basis_out, void* workspace, size_t workspace_bytes,
+                               void* stream);
+lowram_status lowram_fit_basis_workspace_size(const lowram_config* cfg, int32_t l,
+                                              size_t* bytes);
 
 /* One decode step of one layer.
  *   q   [B][H_q][d]  post-RoPE queries (input)
@@ -221,6 +282,20 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
 lowram_status lowram_decode_step_static(lowram_ctx* ctx, const lowram_cache* cache,
                                         const lowram_layer_params* params, const void* q,
                                         void* out, int32_t* sel_out, void* stream);
+
+/* The uncompressed baseline the method is measured against (the pages compare decode
+ * throughput with the uncompressed model: "up to 5x higher peak decode throughput",
+ * agihunt summary, efficiency paragraph; abstract): exact GQA decode attention over the
+ * full bf16 cache, out_g = sum_t softmax_t(q_g . K_t / sqrt(d)) V_t over every position
+ * t < T, for each query head g.
+ *   k_cache [B][T][H_kv][d], v [B][T][H_kv][d] (post-RoPE keys and values, bf16, as
+ *   lowram_encode takes them); q [B][H_q][d]; out [B][H_q][d] (written).
+ * Uses the context's sizes and device only (rank, chunk, predictor and residual settings
+ * are ignored). Workspace: lowram_workspace_size(cfg, LOWRAM_OP_DENSE). bf16 with d = 128
+ * and G = 4 only (LOWRAM_ERR_UNSUPPORTED otherwise). */
+lowram_status lowram_dense_decode(lowram_ctx* ctx, const void* k_cache, const void* v,
+                                  const void* q, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* Synchronise the device, then return and clear the context's status word: LOWRAM_OK,
  * LOWRAM_ERR_DEVICE_CHECK (a kernel met a residual index outside its chunk or a CSR

@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(kSimtThreads) attend_simt_kernel(const AttendA
   float* qs = vv + kSimtTT * D;            // [G][D]
   float* pp = qs + G * D;                  // [G][TT]   logits, then probabilities
   __shared__ int s_cid[kSimtTT];
-  __shared__ int s_pos[kSimtTT];
+  __shared__ int s_pos[kSimtTT];    // row of the token in the cache (-1: none)
+  __shared__ int s_rpos[kSimtTT];   // its RoPE position (the original one after eviction)
   __shared__ float s_ml[kMaxG][2];
 
   if (tid < CPT) {
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(kSimtThreads) attend_simt_kernel(const AttendA
   if (tid < kSimtTT) {
     const int c = s_cid[tid / C];
     s_pos[tid] = c >= 0 ? c * C + tid % C : -1;
+    s_rpos[tid] = c >= 0 ? chunk_position(dm, a.chunk_pos, b, c, a.status) * C + tid % C : -1;
   }
   __syncthreads();
 
@@ -105,7 +107,7 @@ __global__ void __launch_bounds__(kSimtThreads) attend_simt_kernel(const AttendA
     for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
     if (pos >= 0) {
       for (int i = part; i < D / 2; i += 8) {
-        const float2 cs2 = rope_cs32(a.rope, i, pos);
+        const float2 cs2 = rope_cs32(a.rope, i, s_rpos[t]);
         const float x = kp[t * D + i], y = kp[t * D + i + D / 2];
         const float xr = x * cs2.x - y * cs2.y;
         const float yr = x * cs2.y + y * cs2.x;
@@ -189,7 +191,10 @@ __global__ void __launch_bounds__(kSimtThreads) attend_simt_kernel(const AttendA
           if (j == 0) raise_status(a.status, kStatusDeviceCheck);
           continue;
         }
-        vv[(slot * C + t) * D + j] += ldf(rval, (size_t)e * D + j);
+        vv[(slot * C + t) * D + j] +=
+            dm.res_int4 ? int4_residual((const uint8_t*)a.res_val, (const __half*)a.res_scale, dm,
+                                        (size_t)p * dm.n_res + e, j)
+                        : ldf(rval, (size_t)e * D + j);
       }
     }
   }

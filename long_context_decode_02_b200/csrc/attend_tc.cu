@@ -34,6 +34,7 @@
 // own outstanding copies and MMAs (again bounded), frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "device_common.cuh"
 #include "sm100_ptx.cuh"
@@ -461,9 +462,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         const uint32_t rfull = bar(BAR_ROT_FULL0 + rs);
         if (lane == 0) mbar_arrive_expect_tx(rfull, (uint32_t)(kChunksPerTile * (kD / 2) * 8));
         __syncwarp();
-        if (lane < kChunksPerTile)
+        if (lane < kChunksPerTile) {
+          // the chunk's original position (eviction), bounds-checked
+          const int cpos = cid < 0 ? 0 : chunk_position(dm, a.chunk_pos, b, cid, a.status);
           bulk_load(smem_u32(sRot + (rs * kChunksPerTile + lane) * kRotStride),
-                    a.rope.chunk32 + (size_t)(cid < 0 ? 0 : cid) * (kD / 2), (kD / 2) * 8, rfull);
+                    a.rope.chunk32 + (size_t)cpos * (kD / 2), (kD / 2) * 8, rfull);
+        }
         rot_issued = i;
       }
       // advance the pipeline
@@ -775,10 +779,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       for (int w = 0; w < kResPrefetch / 4; ++w) pre_row[w] = 0xFFFFFFFFu;
 #pragma unroll
       for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
+      const bool q4 = dm.res_int4 != 0;   // int4 rows: read in the loop after the sums
 #pragma unroll
       for (int v = 0; v < kResPrefetch; ++v) {
         const int ei = hf + 2 * v;
-        const uint32_t ent = ei < nres ? M->res[ei] : 255u;
+        const uint32_t ent = (ei < nres && !q4) ? M->res[ei] : 255u;
         const uint32_t row = ent & 255u;
         pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
         if (row != 255u) {
@@ -860,11 +865,13 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         racc[2] = fmaf(pv.z, r, racc[2]);
         racc[3] = fmaf(pv.w, r, racc[3]);
       }
-      for (int ei = hf + 2 * kResPrefetch; ei < nres; ei += 2) {   // rows beyond the prefetch
+      for (int ei = hf + (q4 ? 0 : 2 * kResPrefetch); ei < nres; ei += 2) {   // beyond the prefetch
         const uint32_t ent = M->res[ei];
         const int row = (int)(ent & 255u);
         if (row == 255) continue;
-        const float r = __bfloat162float(rbase[(size_t)(ent >> 8) * kD]);
+        const float r = q4 ? int4_residual((const uint8_t*)a.res_val, (const __half*)a.res_scale,
+                                           dm, (size_t)p * dm.n_res + (ent >> 8), j)
+                           : __bfloat162float(rbase[(size_t)(ent >> 8) * kD]);
         if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r;
         const float4 pv = P4[row];
         racc[0] = fmaf(pv.x, r, racc[0]);

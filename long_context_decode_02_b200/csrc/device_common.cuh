@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "lowram_internal.h"
@@ -62,6 +63,33 @@ template <> struct VecLoad<float, 2> {
 // ------------------------------------------------------------------ status word
 __device__ __forceinline__ void raise_status(int* status, int bit) {
   if (status) atomicOr(status, bit);
+}
+
+// ------------------------------------------------------------------ evicted caches
+// Original chunk index of stored chunk c of batch element b (c itself without eviction).
+// An entry outside [0, P / C) is reported and replaced by 0, so no table is read out of
+// bounds.
+__device__ __forceinline__ int chunk_position(const Dims& dm, const int32_t* chunk_pos, int b,
+                                              int c, int* status) {
+  if (!chunk_pos) return c;
+  const int v = chunk_pos[(size_t)b * dm.Nc + c];
+  if (v < 0 || v >= dm.P / dm.C) {
+    raise_status(status, kStatusDeviceCheck);
+    return 0;
+  }
+  return v;
+}
+__device__ __forceinline__ int token_position(const Dims& dm, const int32_t* chunk_pos, int b,
+                                              int t, int* status) {
+  return chunk_pos ? chunk_position(dm, chunk_pos, b, t / dm.C, status) * dm.C + t % dm.C : t;
+}
+
+// Value of element j of an int4 residual row e of pair p: code * scale (exact in fp32).
+__device__ __forceinline__ float int4_residual(const uint8_t* codes, const __half* scales,
+                                               const Dims& dm, size_t row, int j) {
+  const uint8_t byte = codes[row * (dm.d / 2) + (j >> 1)];
+  const int q = (j & 1) ? (int)(byte >> 4) : (int)(byte & 15);
+  return (float)(q >= 8 ? q - 16 : q) * __half2float(scales[row * (dm.d / kInt4Group) + j / kInt4Group]);
 }
 
 // ------------------------------------------------------------------ RoPE

@@ -122,10 +122,9 @@ __global__ void __launch_bounds__(kEncThreads) project_error_kernel(const Encode
     const int i = o % (D / 2);
     const int h = (o / (D / 2)) % H;
     const int t = o / ((D / 2) * H);
-    const int pos = t0 + t;
-    const size_t base = (((size_t)b * dm.T + pos) * H + h) * D;
+    const size_t base = (((size_t)b * dm.T + t0 + t) * H + h) * D;
     const float x = ldf(kc, base + i), y = ldf(kc, base + i + D / 2);
-    const float2 c2 = rope_cs32(a.rope, i, pos);
+    const float2 c2 = rope_cs32(a.rope, i, token_position(dm, a.chunk_pos, b, t0 + t, a.status));
     kp[t * Dt + h * D + i] = x * c2.x + y * c2.y;
     kp[t * Dt + h * D + i + D / 2] = y * c2.x - x * c2.y;
   }
@@ -236,7 +235,7 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
       const int i = o % (D / 2), hh = o / (D / 2);
       const size_t base = (((size_t)b * dm.T + t) * H + hh) * D;
       const double x = ldd(kc, base + i), y = ldd(kc, base + i + D / 2);
-      const double2 c2 = rope_cs64(a.rope, i, t);
+      const double2 c2 = rope_cs64(a.rope, i, token_position(dm, a.chunk_pos, b, t, a.status));
       kp[hh * D + i] = x * c2.x + y * c2.y;
       kp[hh * D + i + D / 2] = y * c2.x - x * c2.y;
     }
@@ -365,7 +364,11 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
     landmark_kernel<T><<<blocks, 256, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  {
+  const bool tc = a.c_ws != nullptr && encode_tc_supported(dm);
+  if (tc) {   // E1 + E2 and E4 on the tensor cores
+    if ((e = launch_encode_project_tc(a, a.basis_t, a.c_ws, a.num_sms, s)) != cudaSuccess) return e;
+    if ((e = launch_encode_predict_tc(a, a.c_ws, false, a.num_sms, s)) != cudaSuccess) return e;
+  } else {
     const size_t smem = sizeof(float) * ((size_t)kTE * dm.H * D + (size_t)kTE * dm.r +
                                          kTE * D + kTE * FH);
     auto kern = project_error_kernel<T, D, FH>;
@@ -386,7 +389,9 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
   }
   residual_finalize_kernel<<<dm.B * dm.H, kSelEncThreads, 0, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (dm.n_res > 0) {
+  if (dm.n_res > 0 && tc) {   // E6 on the tensor cores
+    if ((e = launch_encode_predict_tc(a, a.c_ws, true, a.num_sms, s)) != cudaSuccess) return e;
+  } else if (dm.n_res > 0) {
     const size_t smem = sizeof(float) * ((size_t)kTE * dm.r + kTE * D + kTE * FH);
     auto kern = residual_rows_kernel<T, D, FH>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

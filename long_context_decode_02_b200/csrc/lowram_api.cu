@@ -56,8 +56,12 @@ Dims dims_of(const lowram_config& c) {
   d.n_res = c.n_res;
   d.act = c.act;
   d.dtype = c.dtype;
+  d.P = c.n_positions > 0 ? c.n_positions : c.n_tokens;
+  d.res_int4 = c.res_format == LOWRAM_RES_INT4_G32 ? 1 : 0;
   return d;
 }
+
+bool evicted(const lowram_config& c) { return c.n_positions > 0 && c.n_positions > c.n_tokens; }
 
 bool use_tc(const lowram_config& c) {
   if (c.decode_variant == LOWRAM_DECODE_SIMT) return false;
@@ -110,13 +114,17 @@ DecodeWs decode_ws(const lowram_config& c) {
 }
 
 struct EncodeWs {
-  size_t err, cand_e64, cand_idx, flags, cand_count, in_count, total;
+  size_t err, cand_e64, cand_idx, flags, cand_count, in_count, c_ws, basis_t, total;
 };
 EncodeWs encode_ws(const lowram_config& c) {
   const size_t pairs = (size_t)c.batch * c.n_kv_heads;
   const size_t T = (size_t)c.n_tokens;
   EncodeWs w{};
   size_t o = 0;
+  if (encode_tc_supported(dims_of(c))) {   // the tensor-core encode's own arrays
+    w.c_ws = o;     o = align_up(o + (size_t)c.batch * T * c.rank * sizeof(float));
+    w.basis_t = o;  o = align_up(o + (size_t)c.rank * c.n_kv_heads * c.head_dim * 2);
+  }
   w.err = o;        o = align_up(o + pairs * T * sizeof(float));
   w.cand_e64 = o;   o = align_up(o + pairs * T * sizeof(double));
   w.cand_idx = o;   o = align_up(o + pairs * T * sizeof(int));
@@ -148,15 +156,29 @@ lowram_status check_layer_params(const lowram_layer_params* p) {
   return LOWRAM_OK;
 }
 
-// res_idx / res_val may be NULL when the configuration keeps no residual rows.
-lowram_status check_cache(const lowram_cache* c, int n_res) {
+// res_idx / res_val (/ res_scale) may be NULL when the configuration keeps no residual
+// rows; chunk_pos is required exactly when chunks were evicted.
+lowram_status check_cache(const lowram_cache* c, const lowram_config& cfg) {
+  const int n_res = cfg.n_res;
   if (!c || !c->coef || !c->landmark || !c->chunk_ptr || !c->landmark_norm)
     return LOWRAM_ERR_INVALID_ARG;
   if (n_res > 0 && (!c->res_idx || !c->res_val)) return LOWRAM_ERR_INVALID_ARG;
+  if (n_res > 0 && cfg.res_format == LOWRAM_RES_INT4_G32 && !c->res_scale)
+    return LOWRAM_ERR_INVALID_ARG;
+  if (evicted(cfg) && !c->chunk_pos) return LOWRAM_ERR_INVALID_ARG;
   if (!aligned16(c->coef) || !aligned16(c->landmark) || !aligned16(c->res_idx) ||
-      !aligned16(c->res_val) || !aligned16(c->chunk_ptr) || !aligned16(c->landmark_norm))
+      !aligned16(c->res_val) || !aligned16(c->chunk_ptr) || !aligned16(c->landmark_norm) ||
+      !aligned16(c->chunk_pos) || !aligned16(c->res_scale))
     return LOWRAM_ERR_ALIGN;
   return LOWRAM_OK;
+}
+
+// the pointers the kernels see: chunk_pos only with eviction, res_scale only for int4
+const int32_t* chunk_pos_of(const lowram_cache* c, const lowram_config& cfg) {
+  return evicted(cfg) ? c->chunk_pos : nullptr;
+}
+const void* res_scale_of(const lowram_cache* c, const lowram_config& cfg) {
+  return cfg.res_format == LOWRAM_RES_INT4_G32 ? c->res_scale : nullptr;
 }
 
 }  // namespace
@@ -170,6 +192,13 @@ lowram_status lowram_check_config(const lowram_config* c) {
   if (c->decode_variant < LOWRAM_DECODE_AUTO || c->decode_variant > LOWRAM_DECODE_TCGEN05)
     return LOWRAM_ERR_INVALID_ARG;
   if (c->reserved != 0) return LOWRAM_ERR_INVALID_ARG;
+  if (c->res_format != LOWRAM_RES_STORE && c->res_format != LOWRAM_RES_INT4_G32)
+    return LOWRAM_ERR_INVALID_ARG;
+  if (c->n_positions < 0) return LOWRAM_ERR_SHAPE;
+  if (c->n_positions > 0 && (c->n_positions < c->n_tokens || c->chunk < 1 ||
+                             c->n_positions % c->chunk != 0))
+    return LOWRAM_ERR_SHAPE;
+  if (c->n_positions > (1 << 24)) return LOWRAM_ERR_UNSUPPORTED;
   if (!(c->rope_theta > 0.0) || !std::isfinite(c->rope_theta)) return LOWRAM_ERR_INVALID_ARG;
   if (c->batch < 1 || c->n_tokens < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 ||
       c->head_dim < 1 || c->rank < 1 || c->chunk < 1 || c->mlp_hidden < 1)
@@ -190,21 +219,27 @@ lowram_status lowram_check_config(const lowram_config* c) {
     return LOWRAM_ERR_UNSUPPORTED;   // landmark rows of one call, indexed in 32 bits
   if (c->decode_variant == LOWRAM_DECODE_TCGEN05 && !attend_tc_supported(dims_of(*c)))
     return LOWRAM_ERR_UNSUPPORTED;
+  // int4 residual rows are written by the tensor-core encode
+  if (c->res_format == LOWRAM_RES_INT4_G32 && !encode_tc_supported(dims_of(*c)))
+    return LOWRAM_ERR_UNSUPPORTED;
   return LOWRAM_OK;
 }
 
-lowram_status lowram_cache_layout(const lowram_config* c, size_t bytes_out[6]) {
+lowram_status lowram_cache_layout(const lowram_config* c, size_t bytes_out[8]) {
   if (!bytes_out) return LOWRAM_ERR_INVALID_ARG;
   const lowram_status st = lowram_check_config(c);
   if (st != LOWRAM_OK) return st;
   const size_t es = elem_size(*c);
   const size_t B = c->batch, T = c->n_tokens, H = c->n_kv_heads, d = c->head_dim;
+  const bool q4 = c->res_format == LOWRAM_RES_INT4_G32;
   bytes_out[0] = B * T * c->rank * es;
   bytes_out[1] = B * H * (T / c->chunk) * d * es;
   bytes_out[2] = B * H * (size_t)c->n_res * sizeof(int32_t);
-  bytes_out[3] = B * H * (size_t)c->n_res * d * es;
+  bytes_out[3] = B * H * (size_t)c->n_res * (q4 ? d / 2 : d * es);
   bytes_out[4] = B * H * (T / c->chunk + 1) * sizeof(int32_t);
   bytes_out[5] = B * H * sizeof(float);
+  bytes_out[6] = evicted(*c) ? B * (T / c->chunk) * sizeof(int32_t) : 0;
+  bytes_out[7] = q4 ? B * H * (size_t)c->n_res * (d / kInt4Group) * 2 : 0;
   return LOWRAM_OK;
 }
 
@@ -214,6 +249,16 @@ lowram_status lowram_workspace_size(const lowram_config* c, int op, size_t* byte
   if (st != LOWRAM_OK) return st;
   if (op == LOWRAM_OP_ENCODE) { *bytes = encode_ws(*c).total; return LOWRAM_OK; }
   if (op == LOWRAM_OP_DECODE) { *bytes = decode_ws(*c).total; return LOWRAM_OK; }
+  if (op == LOWRAM_OP_EVICT) {
+    if (!evicted(*c)) return LOWRAM_ERR_SHAPE;
+    *bytes = evict_workspace_bytes(dims_of(*c));
+    return LOWRAM_OK;
+  }
+  if (op == LOWRAM_OP_DENSE) {
+    if (!dense_supported(dims_of(*c))) return LOWRAM_ERR_UNSUPPORTED;
+    *bytes = dense_workspace_bytes(dims_of(*c));
+    return LOWRAM_OK;
+  }
   return LOWRAM_ERR_INVALID_ARG;
 }
 
@@ -234,12 +279,13 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
   ctx->device = device;
   cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, device);
   const int half = c->head_dim / 2;
-  ctx->n_hi = (c->n_tokens + kRopeLo - 1) / kRopeLo;
+  const int n_pos = dims_of(*c).P;   // RoPE positions (the original prefix)
+  ctx->n_hi = (n_pos + kRopeLo - 1) / kRopeLo;
   // two-level tables, fp64 on the host: theta_i = theta^(-2i/d)
   std::vector<float2> lo32((size_t)half * kRopeLo), hi32((size_t)half * ctx->n_hi);
   std::vector<double2> lo64((size_t)half * kRopeLo), hi64((size_t)half * ctx->n_hi);
   std::vector<double> th64((size_t)half);
-  const size_t n_chunks = (size_t)(c->n_tokens / c->chunk);
+  const size_t n_chunks = (size_t)(n_pos / c->chunk);
   std::vector<float2> chunk32(n_chunks * half);
   for (int i = 0; i < half; ++i) {
     const double th = std::pow(c->rope_theta, -2.0 * i / c->head_dim);
@@ -315,7 +361,7 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
   if (!ctx || !k_cache || !v || !workspace) return LOWRAM_ERR_INVALID_ARG;
   lowram_status st = check_layer_params(params);
   if (st != LOWRAM_OK) return st;
-  if ((st = check_cache(out, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if ((st = check_cache(out, ctx->cfg)) != LOWRAM_OK) return st;
   if (!aligned16(k_cache) || !aligned16(v) || !aligned16(workspace)) return LOWRAM_ERR_ALIGN;
   const lowram_config& c = ctx->cfg;
   const EncodeWs w = encode_ws(c);
@@ -330,6 +376,8 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
   a.basis = params->basis; a.w1 = params->w1; a.b1 = params->b1; a.w2 = params->w2; a.b2 = params->b2;
   a.coef = out->coef; a.landmark = out->landmark; a.res_idx = out->res_idx;
   a.res_val = out->res_val; a.chunk_ptr = out->chunk_ptr;
+  a.chunk_pos = chunk_pos_of(out, c);
+  a.res_scale = const_cast<void*>(res_scale_of(out, c));
   a.err = reinterpret_cast<float*>(ws + w.err);
   a.cand_e64 = reinterpret_cast<double*>(ws + w.cand_e64);
   a.cand_idx = reinterpret_cast<int*>(ws + w.cand_idx);
@@ -338,6 +386,11 @@ lowram_status lowram_encode(lowram_ctx* ctx, const void* k_cache, const void* v,
   a.in_count = reinterpret_cast<int*>(ws + w.in_count);
   a.rope = rope_of(ctx);
   a.status = ctx->status;
+  if (encode_tc_supported(a.dm)) {
+    a.c_ws = reinterpret_cast<float*>(ws + w.c_ws);
+    a.basis_t = ws + w.basis_t;
+  }
+  a.num_sms = ctx->num_sms;
   cudaError_t e = launch_encode(a, static_cast<cudaStream_t>(stream));
   if (e == cudaSuccess)
     e = launch_landmark_norms(dims_of(c), out->landmark, out->landmark_norm,
@@ -384,6 +437,8 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   aa.res_idx = cache->res_idx;
   aa.res_val = cache->res_val;
   aa.chunk_ptr = cache->chunk_ptr;
+  aa.chunk_pos = chunk_pos_of(cache, c);
+  aa.res_scale = res_scale_of(cache, c);
   aa.basis = params->basis; aa.w1 = params->w1; aa.b1 = params->b1; aa.w2 = params->w2; aa.b2 = params->b2;
   aa.q = q;
   aa.out = out;
@@ -452,7 +507,7 @@ lowram_status lowram_attend_selected(lowram_ctx* ctx, const lowram_cache* cache,
   if (!ctx || !q || !sel || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
   lowram_status st = check_layer_params(params);
   if (st != LOWRAM_OK) return st;
-  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg)) != LOWRAM_OK) return st;
   if (!aligned16(q) || !aligned16(sel) || !aligned16(out) || !aligned16(workspace))
     return LOWRAM_ERR_ALIGN;
   const DecodeWs w = decode_ws(ctx->cfg);
@@ -472,7 +527,7 @@ lowram_status lowram_debug_reconstruct(lowram_ctx* ctx, const lowram_cache* cach
     return LOWRAM_ERR_INVALID_ARG;
   lowram_status st = check_layer_params(params);
   if (st != LOWRAM_OK) return st;
-  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg)) != LOWRAM_OK) return st;
   if (!aligned16(q) || !aligned16(sel) || !aligned16(out) || !aligned16(workspace) ||
       !aligned16(k_rot) || !aligned16(h_act) || !aligned16(v_rec))
     return LOWRAM_ERR_ALIGN;
@@ -502,7 +557,7 @@ lowram_status lowram_debug_attend_unpublished(lowram_ctx* ctx, const lowram_cach
   if (!ctx || !q || !sel || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
   lowram_status st = check_layer_params(params);
   if (st != LOWRAM_OK) return st;
-  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg)) != LOWRAM_OK) return st;
   if (!aligned16(q) || !aligned16(sel) || !aligned16(out) || !aligned16(workspace))
     return LOWRAM_ERR_ALIGN;
   if (!use_tc(ctx->cfg)) return LOWRAM_ERR_UNSUPPORTED;
@@ -522,7 +577,7 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
   if (!ctx || !q || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
   lowram_status st = check_layer_params(params);
   if (st != LOWRAM_OK) return st;
-  if ((st = check_cache(cache, ctx->cfg.n_res)) != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg)) != LOWRAM_OK) return st;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) ||
       (sel_out && !aligned16(sel_out)))
     return LOWRAM_ERR_ALIGN;
@@ -538,6 +593,85 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
       LOWRAM_OK)
     return st;
   return attend_impl(ctx, cache, params, q, sel, out, ws, w, s, tc);
+}
+
+lowram_status lowram_evict(lowram_ctx* ctx, const void* k_full, const void* v_full,
+                           void* k_kept, void* v_kept, int32_t* chunk_pos, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (!ctx || !k_full || !v_full || !k_kept || !v_kept || !chunk_pos || !workspace)
+    return LOWRAM_ERR_INVALID_ARG;
+  if (!aligned16(k_full) || !aligned16(v_full) || !aligned16(k_kept) || !aligned16(v_kept) ||
+      !aligned16(chunk_pos) || !aligned16(workspace))
+    return LOWRAM_ERR_ALIGN;
+  if (!evicted(ctx->cfg)) return LOWRAM_ERR_SHAPE;
+  const Dims dm = dims_of(ctx->cfg);
+  if (workspace_bytes < evict_workspace_bytes(dm)) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  if (launch_evict(dm, k_full, v_full, k_kept, v_kept, chunk_pos, workspace,
+                   static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_fit_basis_workspace_size(const lowram_config* c, int32_t l, size_t* bytes) {
+  if (!bytes) return LOWRAM_ERR_INVALID_ARG;
+  const lowram_status st = lowram_check_config(c);
+  if (st != LOWRAM_OK) return st;
+  const int D = c->n_kv_heads * c->head_dim;
+  if (l < c->rank || l > D || l > 256) return LOWRAM_ERR_SHAPE;
+  if (D % 64 != 0) return LOWRAM_ERR_UNSUPPORTED;
+  *bytes = fit_basis_workspace_bytes(dims_of(*c), l);
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_fit_basis(lowram_ctx* ctx, const void* const* k_layers, int32_t n_layers,
+                               const double* omega, int32_t l, int32_t n_power,
+                               void* basis_out, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!ctx || !k_layers || !omega || !basis_out || !workspace) return LOWRAM_ERR_INVALID_ARG;
+  if (n_layers < 1 || n_layers > 8 || n_power < 0 || n_power > 16) return LOWRAM_ERR_INVALID_ARG;
+  for (int i = 0; i < n_layers; ++i) {
+    if (!k_layers[i]) return LOWRAM_ERR_INVALID_ARG;
+    if (!aligned16(k_layers[i])) return LOWRAM_ERR_ALIGN;
+  }
+  if (!aligned16(omega) || !aligned16(basis_out) || !aligned16(workspace)) return LOWRAM_ERR_ALIGN;
+  if (evicted(ctx->cfg)) return LOWRAM_ERR_UNSUPPORTED;
+  size_t need = 0;
+  lowram_status st = lowram_fit_basis_workspace_size(&ctx->cfg, l, &need);
+  if (st != LOWRAM_OK) return st;
+  if (workspace_bytes < need) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  if (launch_fit_basis(dims_of(ctx->cfg), k_layers, n_layers, omega, l, n_power, basis_out,
+                       rope_of(ctx), ctx->status, workspace,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_dense_decode(lowram_ctx* ctx, const void* k_cache, const void* v,
+                                  const void* q, void* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!ctx || !k_cache || !v || !q || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v) || !aligned16(q) || !aligned16(out) ||
+      !aligned16(workspace))
+    return LOWRAM_ERR_ALIGN;
+  const Dims dm = dims_of(ctx->cfg);
+  if (!dense_supported(dm)) return LOWRAM_ERR_UNSUPPORTED;
+  if (workspace_bytes < dense_workspace_bytes(dm)) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  if (launch_dense_decode(dm, k_cache, v, q, out, workspace, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
 }
 
 lowram_status lowram_last_error(lowram_ctx* ctx) {

@@ -39,7 +39,10 @@ struct RopeTables {
 
 struct Dims {
   int B, T, H, Hq, G, d, r, C, F, Nc, k, n_res, act, dtype;
+  int P;          // RoPE positions of the original prefix (T unless chunks were evicted)
+  int res_int4;   // residual rows stored as int4 codes + fp16 scales per 32 elements
 };
+constexpr int kInt4Group = 32;
 
 // ---------------- decode: landmark scoring + top-k selection ----------------
 struct SelectArgs {
@@ -76,6 +79,8 @@ struct AttendArgs {
   const int32_t* res_idx; // [B][H][n_res]
   const void* res_val;    // [B][H][n_res][d]
   const int32_t* chunk_ptr; // [B][H][Nc+1]
+  const int32_t* chunk_pos; // [B][Nc] original chunk index of each stored chunk, or null
+  const void* res_scale;  // [B][H][n_res][d/32] fp16 (int4 residual rows), or null
   const void* basis;      // [H*d][r]
   const void* w1; const void* b1; const void* w2; const void* b2;
   const void* q;          // [B][Hq][d]
@@ -113,6 +118,25 @@ cudaError_t launch_combine(const AttendArgs& a, bool reorder_form, cudaStream_t 
 // test only: dbg_v[row] += W2_h dbg_h[row] + b2_h for every row of a.dbg_h
 cudaError_t launch_debug_values(const AttendArgs& a, cudaStream_t s);
 
+// ---------------- eviction ----------------
+// keep the T / C chunks (of P / C) with the largest all-head landmark norm per batch
+// element; gather their keys and values; chunk_pos ascending
+size_t evict_workspace_bytes(const Dims& dm);
+cudaError_t launch_evict(const Dims& dm, const void* k_full, const void* v_full, void* k_kept,
+                         void* v_kept, int32_t* chunk_pos, void* ws, cudaStream_t s);
+
+// ---------------- basis fit (randomised range finder, Cholesky-QR) ----------------
+size_t fit_basis_workspace_bytes(const Dims& dm, int l);
+cudaError_t launch_fit_basis(const Dims& dm, const void* const* k_layers, int n_layers,
+                             const double* omega, int l, int n_power, void* basis_out,
+                             const RopeTables& rope, int* status, void* ws, cudaStream_t s);
+
+// ---------------- uncompressed baseline ----------------
+bool dense_supported(const Dims& dm);
+size_t dense_workspace_bytes(const Dims& dm);
+cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, const void* q,
+                                void* out, void* ws, cudaStream_t s);
+
 // ---------------- encode ----------------
 struct EncodeArgs {
   Dims dm;
@@ -120,6 +144,8 @@ struct EncodeArgs {
   const void* v;          // [B][T][H][d]
   const void* basis; const void* w1; const void* b1; const void* w2; const void* b2;
   void* coef; void* landmark; int32_t* res_idx; void* res_val; int32_t* chunk_ptr;
+  const int32_t* chunk_pos; // cache [B][Nc] original chunk of each stored chunk, or null
+  void* res_scale;        // cache [B][H][n_res][d/32] fp16 (int4 residual rows), or null
   float* err;             // ws [B*H][T]
   double* cand_e64;       // ws [B*H][T]
   int* cand_idx;          // ws [B*H][T]
@@ -128,8 +154,17 @@ struct EncodeArgs {
   int* in_count;          // ws [B*H]
   RopeTables rope;
   int* status;
+  // tensor-core path (encode_tc_supported), else null
+  float* c_ws;            // ws [B*T][r] fp32: the unrounded coefficients
+  void* basis_t;          // ws [r][H*d] bf16: the basis transposed
+  int num_sms;
 };
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t s);
+bool encode_tc_supported(const Dims& dm);
+cudaError_t launch_encode_project_tc(const EncodeArgs& a, void* basis_t, float* c_ws,
+                                     int num_sms, cudaStream_t s);
+cudaError_t launch_encode_predict_tc(const EncodeArgs& a, const float* c_ws, bool residual_rows,
+                                     int num_sms, cudaStream_t s);
 
 // 2D tiled TMA map over a row-major [rows][cols] array of dtype (LOWRAM_DTYPE_*), box
 // box_rows x box_cols, swizzle 0/32/64/128 bytes. False if the driver refuses it.

@@ -41,6 +41,10 @@ DECODE_SIMT = 1
 DECODE_TCGEN05 = 2
 OP_ENCODE = 0
 OP_DECODE = 1
+OP_DENSE = 2
+OP_EVICT = 3
+RES_STORE = 0
+RES_INT4_G32 = 1
 
 
 class lowram_config(ctypes.Structure):
@@ -50,7 +54,8 @@ class lowram_config(ctypes.Structure):
                 ("chunk", ctypes.c_int32), ("mlp_hidden", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("n_res", ctypes.c_int32),
                 ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("decode_variant", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("decode_variant", ctypes.c_int32), ("res_format", ctypes.c_int32),
+                ("n_positions", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("rope_theta", ctypes.c_double)]
 
 
@@ -62,7 +67,8 @@ class lowram_layer_params(ctypes.Structure):
 class lowram_cache(ctypes.Structure):
     _fields_ = [("coef", ctypes.c_void_p), ("landmark", ctypes.c_void_p),
                 ("res_idx", ctypes.c_void_p), ("res_val", ctypes.c_void_p),
-                ("chunk_ptr", ctypes.c_void_p), ("landmark_norm", ctypes.c_void_p)]
+                ("chunk_ptr", ctypes.c_void_p), ("landmark_norm", ctypes.c_void_p),
+                ("chunk_pos", ctypes.c_void_p), ("res_scale", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -89,6 +95,12 @@ _sig = {
     "lowram_last_error": (_S, [_P]),
     "lowram_status_string": (ctypes.c_char_p, [_S]),
     "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
+    "lowram_dense_decode": (_S, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_evict": (_S, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_fit_basis": (_S, [_P, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, _P,
+                              ctypes.c_int32, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_fit_basis_workspace_size": (_S, [ctypes.POINTER(lowram_config), ctypes.c_int32,
+                                             ctypes.POINTER(ctypes.c_size_t)]),
     "lowram_debug_reconstruct": (_S, [_P, ctypes.POINTER(lowram_cache),
                                       ctypes.POINTER(lowram_layer_params), _P, _P, _P, _P, _P,
                                       _P, _P, ctypes.c_size_t, _P]),
@@ -119,12 +131,16 @@ def check(status: int, where: str) -> None:
 # ------------------------------------------------------------------ torch helpers
 def make_config(shape, decode_variant: int = DECODE_AUTO, **over) -> lowram_config:
     """lowram_config from a workload shape (long_context_decode_02_b200.synth.Shape)."""
-    c = lowram_config(batch=shape.batch, n_tokens=shape.n_tokens, n_kv_heads=shape.n_kv_heads,
+    kept = getattr(shape, "n_kept_tokens", shape.n_tokens)
+    c = lowram_config(batch=shape.batch, n_tokens=kept, n_kv_heads=shape.n_kv_heads,
                       n_q_heads=shape.n_q_heads, head_dim=shape.head_dim, rank=shape.rank,
                       chunk=shape.chunk, mlp_hidden=shape.mlp_hidden, top_k=shape.top_k,
                       n_res=shape.n_res, act=shape.act,
                       dtype=DTYPE_BF16 if shape.dtype == "bf16" else DTYPE_F32,
-                      decode_variant=decode_variant, reserved=0, rope_theta=shape.theta)
+                      decode_variant=decode_variant,
+                      res_format=RES_INT4_G32 if getattr(shape, "res_int4", False) else RES_STORE,
+                      n_positions=shape.n_tokens if kept < shape.n_tokens else 0,
+                      reserved=0, rope_theta=shape.theta)
     for k, v in over.items():
         setattr(c, k, v)
     return c
@@ -147,7 +163,7 @@ def _stream(stream):
 
 
 def cache_layout(cfg: lowram_config):
-    out = (ctypes.c_size_t * 6)()
+    out = (ctypes.c_size_t * 8)()
     check(lowram_cache_layout(ctypes.byref(cfg), out), "lowram_cache_layout")
     return list(out)
 
@@ -193,9 +209,10 @@ def layer_params(basis, w1, b1, w2, b2) -> lowram_layer_params:
     return p
 
 
-def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr, landmark_norm) -> lowram_cache:
+def cache_struct(coef, landmark, res_idx, res_val, chunk_ptr, landmark_norm, chunk_pos=None,
+                 res_scale=None) -> lowram_cache:
     return lowram_cache(_ptr(coef), _ptr(landmark), _ptr(res_idx), _ptr(res_val),
-                        _ptr(chunk_ptr), _ptr(landmark_norm))
+                        _ptr(chunk_ptr), _ptr(landmark_norm), _ptr(chunk_pos), _ptr(res_scale))
 
 
 def alloc_cache(cfg: lowram_config, device):
@@ -204,14 +221,21 @@ def alloc_cache(cfg: lowram_config, device):
     dt = torch.bfloat16 if cfg.dtype == DTYPE_BF16 else torch.float32
     B, T, H, d = cfg.batch, cfg.n_tokens, cfg.n_kv_heads, cfg.head_dim
     nc = T // cfg.chunk
-    return {
+    q4 = cfg.res_format == RES_INT4_G32
+    out = {
         "coef": torch.empty(B, T, cfg.rank, dtype=dt, device=device),
         "landmark": torch.empty(B, H, nc, d, dtype=dt, device=device),
         "res_idx": torch.empty(B, H, cfg.n_res, dtype=torch.int32, device=device),
-        "res_val": torch.empty(B, H, cfg.n_res, d, dtype=dt, device=device),
+        "res_val": (torch.empty(B, H, cfg.n_res, d // 2, dtype=torch.uint8, device=device) if q4
+                    else torch.empty(B, H, cfg.n_res, d, dtype=dt, device=device)),
         "chunk_ptr": torch.empty(B, H, nc + 1, dtype=torch.int32, device=device),
         "landmark_norm": torch.empty(B, H, dtype=torch.float32, device=device),
     }
+    if cfg.n_positions > cfg.n_tokens:
+        out["chunk_pos"] = torch.empty(B, nc, dtype=torch.int32, device=device)
+    if q4:
+        out["res_scale"] = torch.empty(B, H, cfg.n_res, d // 32, dtype=torch.float16, device=device)
+    return out
 
 
 def encode(ctx: Context, k_cache, v, params: lowram_layer_params, cache: dict, workspace,
@@ -289,3 +313,39 @@ def debug_attend_unpublished(ctx: Context, cache: dict, params: lowram_layer_par
                                           workspace.numel() * workspace.element_size(),
                                           _stream(stream)),
           "lowram_debug_attend_unpublished")
+
+
+def dense_decode(ctx: Context, k_cache, v, q, out, workspace, stream=None) -> None:
+    """lowram_dense_decode: exact GQA decode attention over the uncompressed bf16 cache."""
+    check(lowram_dense_decode(ctx.handle, _ptr(k_cache), _ptr(v), _ptr(q), _ptr(out),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream)),
+          "lowram_dense_decode")
+
+
+def evict(ctx: Context, k_full, v_full, k_kept, v_kept, chunk_pos, workspace, stream=None) -> None:
+    """lowram_evict: keep the chunks with the largest all-head landmark norm (LowRAM-E)."""
+    check(lowram_evict(ctx.handle, _ptr(k_full), _ptr(v_full), _ptr(k_kept), _ptr(v_kept),
+                       _ptr(chunk_pos), _ptr(workspace),
+                       workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_evict")
+
+
+def fit_basis_workspace_size(cfg: lowram_config, l: int) -> int:
+    n = ctypes.c_size_t()
+    check(lowram_fit_basis_workspace_size(ctypes.byref(cfg), l, ctypes.byref(n)),
+          "lowram_fit_basis_workspace_size")
+    return n.value
+
+
+def fit_basis(ctx: Context, k_layers, omega, n_power: int, basis_out, workspace,
+              stream=None) -> None:
+    """lowram_fit_basis: the group's xKV basis by a randomised range finder with
+    Cholesky-QR. k_layers: list of device tensors [B][T][H][d]; omega [D][l] fp64."""
+    arr = (ctypes.c_void_p * len(k_layers))(*[t.data_ptr() for t in k_layers])
+    for t in k_layers:
+        _ptr(t)   # contiguity check
+    check(lowram_fit_basis(ctx.handle, arr, len(k_layers), _ptr(omega), omega.shape[1],
+                           n_power, _ptr(basis_out), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_fit_basis")

@@ -53,14 +53,30 @@ class Shape:
     noise: float = 0.05
     outlier_std: float = 3.0
     seed: int = 0
+    keep_frac: float = 1.0      # fraction of chunks kept by eviction (1: no eviction)
+    res_int4: bool = False      # residual rows stored as int4 codes + fp16 scales
 
     @property
     def n_res(self) -> int:
-        return int(math.floor(self.res_frac * self.n_tokens + 1e-9))
+        """Residual rows per (batch, KV head): a fraction of the tokens the cache holds."""
+        return int(math.floor(self.res_frac * self.n_kept_tokens + 1e-9))
 
     @property
     def n_chunks(self) -> int:
-        return self.n_tokens // self.chunk
+        """Chunks the cache holds (after eviction)."""
+        return self.n_kept_chunks
+
+    @property
+    def n_kept_chunks(self) -> int:
+        return int(math.floor(self.keep_frac * (self.n_tokens // self.chunk) + 1e-9))
+
+    @property
+    def n_kept_tokens(self) -> int:
+        return self.n_kept_chunks * self.chunk
+
+    @property
+    def evicted(self) -> bool:
+        return self.n_kept_tokens < self.n_tokens
 
     @property
     def group(self) -> int:
@@ -97,6 +113,12 @@ CONFIGS = {
              n_kv_heads=8, n_q_heads=32, head_dim=128, rank=128, chunk=8, top_k=256,
              res_frac=0.15, mlp_hidden=256, act=ACT_SILU, dtype="bf16", theta=1e6,
              outlier_frac=0.03, steps=16, seed=3000),
+    # LowRAM-Q/EQ composition: config 2's shapes at 64K, int4 residual rows for the worst
+    # 40% of the kept tokens, half the chunks evicted; batch swept 1, 4, 8, 16, 28
+    4: Shape("llama8b-32layer-64k-eq", batch=8, n_tokens=65536, n_layers=32, n_kv_heads=8,
+             n_q_heads=32, head_dim=128, rank=160, chunk=8, top_k=256, res_frac=0.4,
+             mlp_hidden=256, act=ACT_SILU, dtype="bf16", theta=5e5, outlier_frac=0.03,
+             steps=16, seed=4000, keep_frac=0.5, res_int4=True),
 }
 
 

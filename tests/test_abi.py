@@ -56,6 +56,12 @@ def test_check_config(L):
         (dict(rope_theta=-1.0), L.ERR_INVALID_ARG),
         (dict(dtype=L.DTYPE_F32, decode_variant=L.DECODE_TCGEN05), L.ERR_UNSUPPORTED),
         (dict(rank=192, decode_variant=L.DECODE_TCGEN05), L.ERR_UNSUPPORTED),
+        (dict(res_format=2), L.ERR_INVALID_ARG),
+        (dict(n_positions=-8), L.ERR_SHAPE),
+        (dict(n_positions=16384), L.ERR_SHAPE),      # fewer positions than stored tokens
+        (dict(n_positions=65540), L.ERR_SHAPE),      # not a multiple of the chunk
+        (dict(res_format=1, rank=192), L.ERR_UNSUPPORTED),   # int4 needs the tc encode
+        (dict(res_format=1, dtype=L.DTYPE_F32), L.ERR_UNSUPPORTED),
     ]
     for over, want in bad:
         c = _cfg(L, **over)
@@ -69,9 +75,24 @@ def test_cache_layout_and_workspace(L):
     B, T, H, d, r = 1, 32768, 8, 128, 160
     n_res = int(0.2 * T)
     assert sizes == [B * T * r * 2, B * H * (T // 8) * d * 2, B * H * n_res * 4,
-                     B * H * n_res * d * 2, B * H * (T // 8 + 1) * 4, B * H * 4]
-    for op in (L.OP_ENCODE, L.OP_DECODE):
+                     B * H * n_res * d * 2, B * H * (T // 8 + 1) * 4, B * H * 4, 0, 0]
+    for op in (L.OP_ENCODE, L.OP_DECODE, L.OP_DENSE):
         assert L.workspace_size(c, op) > 0
+    with pytest.raises(L.LowRAMError):          # eviction needs n_positions > n_tokens
+        L.workspace_size(c, L.OP_EVICT)
+    # LowRAM-EQ: half the chunks kept, int4 residual rows with fp16 scales per 32
+    from long_context_decode_02_b200 import synth
+    sh = synth.CONFIGS[4]
+    ce = L.make_config(sh)
+    assert ce.n_tokens == sh.n_tokens // 2 and ce.n_positions == sh.n_tokens
+    assert ce.res_format == L.RES_INT4_G32
+    Be, Te, nre = sh.batch, ce.n_tokens, ce.n_res
+    assert nre == int(0.4 * Te)
+    se = L.cache_layout(ce)
+    assert se[3] == Be * H * nre * d // 2                 # two codes per byte
+    assert se[6] == Be * (Te // 8) * 4                    # chunk_pos
+    assert se[7] == Be * H * nre * (d // 32) * 2          # fp16 scales
+    assert L.workspace_size(ce, L.OP_EVICT) >= Be * (sh.n_tokens // 8) * 9
     n = ctypes.c_size_t()
     assert L.lowram_workspace_size(ctypes.byref(c), 9, ctypes.byref(n)) == L.ERR_INVALID_ARG
 

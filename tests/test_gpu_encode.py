@@ -123,3 +123,21 @@ def test_encode_edge_budgets(L, cuda_device):
     for over in (dict(res_frac=0.0), dict(res_frac=1.0), dict(res_frac=1.0 / 1024)):
         sh = synth.CONFIGS[0].replace(n_tokens=1024, **over)
         check_encode(L, sh, cuda_device)
+
+
+@pytest.mark.parametrize("over", [
+    dict(res_frac=0.0),                       # no residual rows: no residual-row pass
+    dict(res_frac=1.0),                       # every token picked
+    dict(res_frac=1.0 / 1024),                # two rows per (b, h)
+    dict(res_frac=0.3),                       # 614 rows: a ragged last tile of 128
+    dict(rank=128, act=synth.ACT_GELU_ERF),   # the other activation and rank
+    dict(rank=32, batch=3),
+], ids=["nores", "allres", "tworows", "ragged", "r128gelu", "r32b3"])
+def test_tensor_core_encode_edges(L, cuda_device, over):
+    """bf16, d 128, F 256: the tensor-core encode (projection and predictor on tcgen05)
+    against the oracle, with the same bars as above."""
+    kw = dict(name="enc-tc", n_tokens=2048, batch=2, seed=55)
+    kw.update(over)
+    sh = synth.CONFIGS[1].replace(**kw)
+    ties, *_ = check_encode(L, sh, cuda_device)
+    H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, f"tc encode {over}")
