@@ -236,6 +236,26 @@ lowram_status lowram_decode_step(lowram_ctx* ctx, const lowram_cache* cache,
                                  void* out, int32_t* sel_out, void* workspace,
                                  size_t workspace_bytes, void* stream);
 
+/* One decode step over the compressed prefix plus an uncompressed suffix of generated
+ * tokens (long generation keeps recent tokens uncompressed until they are compressed in
+ * turn; agihunt summary, limitations paragraph). One softmax spans the selected chunks'
+ * rebuilt tokens and every suffix token:
+ *   k_suffix, v_suffix [B][s_max][H_kv][d] (post-RoPE keys, values; bf16), rows
+ *   0 .. n_suffix-1 valid (0 <= n_suffix <= s_max; NULL allowed when n_suffix == 0);
+ *   q, out, sel_out as in lowram_decode_step.
+ * The compressed part runs as in lowram_decode_step with its output kept in fp32; the
+ * suffix is attended by the dense flash-decode kernel and the two merged by their
+ * softmax statistics. Workspace: lowram_suffix_workspace_size(cfg, s_max). bf16 with
+ * d = 128 and G = 4 only (LOWRAM_ERR_UNSUPPORTED otherwise). */
+lowram_status lowram_decode_step_suffix(lowram_ctx* ctx, const lowram_cache* cache,
+                                        const lowram_layer_params* params, const void* q,
+                                        const void* k_suffix, const void* v_suffix,
+                                        int32_t s_max, int32_t n_suffix, void* out,
+                                        int32_t* sel_out, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+lowram_status lowram_suffix_workspace_size(const lowram_config* cfg, int32_t s_max,
+                                           size_t* bytes);
+
 /* Decode sub-step 1 (kernel (a) alone): score every chunk by max over the GQA group of
  * q . landmark and write the top-k chunks per (batch, KV head), ascending, ties to the
  * lower chunk (agihunt summary, key paragraph; cctest "Selective reconstruction").

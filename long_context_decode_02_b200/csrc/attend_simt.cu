@@ -249,7 +249,16 @@ __global__ void __launch_bounds__(256) combine_plain_kernel(const AttendArgs a) 
       L = fmaf(w, pt[1], L);
       O = fmaf(w, pt[2 + j], O);
     }
-    ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] = from_f<T>(O / L);
+    const size_t oi = ((size_t)b * dm.Hq + (size_t)h * G + g) * D + j;
+    if (a.out_f32) {   // decode with a suffix: the merge kernel finishes the output
+      a.out_f32[oi] = O / L;
+      if (j == 0) {
+        a.out_ml[2 * (oi / D)] = M;
+        a.out_ml[2 * (oi / D) + 1] = L;
+      }
+    } else {
+      ((T*)a.out)[oi] = from_f<T>(O / L);
+    }
   }
 }
 
@@ -337,9 +346,19 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
     for (int e = 0; e < 8; ++e) acc = fmaf(w[e], hh[8 * i + e], acc);
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-  if (half == 0)
-    ((T*)a.out)[((size_t)b * dm.Hq + (size_t)h * G + g) * D + j] =
-        from_f<T>((acc + rs[0][j] + rs[1][j]) / s_L + b2);
+  if (half == 0) {
+    const size_t oi = ((size_t)b * dm.Hq + (size_t)h * G + g) * D + j;
+    const float o = (acc + rs[0][j] + rs[1][j]) / s_L + b2;
+    if (a.out_f32) {   // decode with a suffix: max in natural-log units, and the sum
+      a.out_f32[oi] = o;
+      if (j == 0) {
+        a.out_ml[2 * (oi / D)] = M * 0.69314718055994531f;
+        a.out_ml[2 * (oi / D) + 1] = s_L;
+      }
+    } else {
+      ((T*)a.out)[oi] = from_f<T>(o);
+    }
+  }
 }
 
 template <typename T, int D, int FH>

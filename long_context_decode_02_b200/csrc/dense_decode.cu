@@ -33,6 +33,7 @@ struct DenseArgs {
   __nv_bfloat16* out;       // [B][Hq][d]
   float* part;              // [B*H][n_split][G][2 + d]
   int n_split;
+  int t_valid;              // positions 0 .. t_valid-1 of each row block are attended
 };
 
 __global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const DenseArgs a) {
@@ -41,7 +42,7 @@ __global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const De
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 4, gl = lane & 15;
   const int t_begin = split * kDenseSplit;
-  const int t_end = min(a.T, t_begin + kDenseSplit);
+  const int t_end = min(a.t_valid, t_begin + kDenseSplit);
   // this lane's 8 dimensions of the group's queries, scaled to log2 units
   const float zs = 1.4426950408889634f * rsqrtf((float)kDD);
   float qv[kDG][8];
@@ -227,7 +228,61 @@ __global__ void __launch_bounds__(kDD) dense_combine_kernel(const DenseArgs a) {
   a.out[(size_t)bq * kDD + j] = __float2bfloat16_rn(O / L);
 }
 
+// Prefix (normalised fp32 output O_c, softmax max M_c in natural-log units and sum L_c)
+// merged with the suffix's splits (max in log2 units, sum, unnormalised O):
+//   out = (O_c L_c e^(M_c - M) + sum_s O_s e^(M_s - M)) / (L_c e^(M_c - M) + sum_s L_s e^(M_s - M))
+__global__ void __launch_bounds__(kDD) suffix_merge_kernel(const DenseArgs a, const float* pre_out,
+                                                           const float* pre_ml) {
+  const int bq = blockIdx.x;
+  const int b = bq / a.Hq, hq = bq % a.Hq, h = hq / kDG, g = hq % kDG;
+  const int j = threadIdx.x;
+  constexpr float kLn2 = 0.69314718055994531f;
+  const float Mc = pre_ml[2 * bq], Lc = pre_ml[2 * bq + 1];
+  const float* part = a.part + (size_t)(b * a.H + h) * a.n_split * kPartStride + g * (2 + kDD);
+  const int ns = a.t_valid > 0 ? a.n_split : 0;
+  float M = Mc;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, part[(size_t)s * kPartStride] * kLn2);
+  const float wc = expf(Mc - M);
+  float L = Lc * wc, O = pre_out[(size_t)bq * kDD + j] * Lc * wc;
+  for (int s = 0; s < ns; ++s) {
+    const float* ps = part + (size_t)s * kPartStride;
+    const float c = ps[0] == -INFINITY ? 0.f : expf(ps[0] * kLn2 - M);
+    L = fmaf(c, ps[1], L);
+    O = fmaf(c, ps[2 + j], O);
+  }
+  a.out[(size_t)bq * kDD + j] = __float2bfloat16_rn(O / L);
+}
+
 }  // namespace
+
+size_t suffix_workspace_bytes(const Dims& dm, int s_max) {
+  const size_t n_split = (size_t)(s_max + kDenseSplit - 1) / kDenseSplit;
+  return (size_t)dm.B * dm.H * (n_split > 0 ? n_split : 1) * kPartStride * sizeof(float);
+}
+
+cudaError_t launch_suffix_merge(const Dims& dm, const void* k_suffix, const void* v_suffix,
+                                int s_max, int n_suffix, const void* q, const float* pre_out,
+                                const float* pre_ml, void* out, void* ws, cudaStream_t s) {
+  DenseArgs a{};
+  a.B = dm.B;
+  a.T = s_max;
+  a.H = dm.H;
+  a.Hq = dm.Hq;
+  a.k = (const __nv_bfloat16*)k_suffix;
+  a.v = (const __nv_bfloat16*)v_suffix;
+  a.q = (const __nv_bfloat16*)q;
+  a.out = (__nv_bfloat16*)out;
+  a.part = (float*)ws;
+  a.t_valid = n_suffix;
+  a.n_split = (n_suffix + kDenseSplit - 1) / kDenseSplit;
+  if (a.n_split > 0) {
+    dense_decode_kernel<<<dim3(a.n_split, dm.B * dm.H), kDenseThreads, 0, s>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  suffix_merge_kernel<<<dm.B * dm.Hq, kDD, 0, s>>>(a, pre_out, pre_ml);
+  return cudaGetLastError();
+}
 
 bool dense_supported(const Dims& dm) {
   return dm.dtype == LOWRAM_DTYPE_BF16 && dm.d == kDD && dm.G == kDG;
@@ -251,6 +306,7 @@ cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, co
   a.out = (__nv_bfloat16*)out;
   a.part = (float*)ws;
   a.n_split = (dm.T + kDenseSplit - 1) / kDenseSplit;
+  a.t_valid = dm.T;
   dense_decode_kernel<<<dim3(a.n_split, dm.B * dm.H), kDenseThreads, 0, s>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

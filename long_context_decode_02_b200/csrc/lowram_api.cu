@@ -27,6 +27,8 @@ struct lowram_ctx {
   float* scores;   // device [B*H][Nc], all bits set between launches
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   int* item_ctr;  // device [H]: tile counters of the tcgen05 attend kernel, 0 between calls
+  int* tc_sync;   // device [B*H + 2]: the tcgen05 kernel's tile-done counters, merge and
+                  // exit counters, 0 between calls
   double* theta64;  // device [d/2]
   float2* chunk32;  // device [T/C][d/2]: (cos, sin)(c C theta_i)
 };
@@ -314,6 +316,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->item_ctr, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
+            cudaMalloc(&ctx->tc_sync, (pairs + 2) * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess &&
             cudaMalloc(&ctx->chunk32, chunk32.size() * sizeof(float2)) == cudaSuccess;
@@ -326,6 +329,7 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->item_ctr, 0, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
+       cudaMemset(ctx->tc_sync, 0, (pairs + 2) * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->chunk32, chunk32.data(), chunk32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess;
@@ -350,6 +354,7 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->scores);
   cudaFree(ctx->ready);
   cudaFree(ctx->item_ctr);
+  cudaFree(ctx->tc_sync);
   cudaFree(ctx->theta64);
   cudaFree(ctx->chunk32);
   delete ctx;
@@ -428,7 +433,8 @@ lowram_status select_impl(lowram_ctx* ctx, const void* landmark, const float* la
 lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
                           const lowram_layer_params* params, const void* q, const int32_t* sel,
                           void* out, uint8_t* ws, const DecodeWs& w, cudaStream_t s,
-                          bool after_select, float* const* dbg = nullptr) {
+                          bool after_select, float* const* dbg = nullptr,
+                          float* const* f32 = nullptr) {
   const lowram_config& c = ctx->cfg;
   const Dims dm = dims_of(c);
   AttendArgs aa{};
@@ -453,13 +459,23 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   aa.ready = tc && after_select ? ctx->ready : nullptr;
   aa.wait_ready = aa.ready ? 1 : 0;
   aa.item_ctr = tc ? ctx->item_ctr : nullptr;
+  if (tc) {
+    const size_t pairs = (size_t)dm.B * dm.H;
+    aa.tiles_done = ctx->tc_sync;
+    aa.merge_ctr = ctx->tc_sync + pairs;
+    aa.exit_ctr = ctx->tc_sync + pairs + 1;
+  }
+  if (f32) {   // decode with a suffix: fp32 output and softmax statistics
+    aa.out_f32 = f32[0];
+    aa.out_ml = f32[1];
+  }
   if (dbg) {
     aa.dbg_k = dbg[0];
     aa.dbg_h = dbg[1];
     aa.dbg_v = dbg[2];
   }
   cudaError_t e = tc ? launch_attend_tc(aa, ctx->num_sms, s) : launch_attend_simt(aa, s);
-  if (e == cudaSuccess) e = launch_combine(aa, tc, s);
+  if (e == cudaSuccess && !tc) e = launch_combine(aa, false, s);   // tcgen05 merges itself
   if (e == cudaSuccess && dbg) e = launch_debug_values(aa, s);
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;
@@ -668,6 +684,75 @@ lowram_status lowram_dense_decode(lowram_ctx* ctx, const void* k_cache, const vo
   if (!g.ok) return LOWRAM_ERR_CUDA;
   if (launch_dense_decode(dm, k_cache, v, q, out, workspace, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
+}
+
+namespace {
+struct SuffixWs {
+  size_t out_f32, ml, part, total;
+};
+SuffixWs suffix_ws(const lowram_config& c, int s_max) {
+  const Dims dm = dims_of(c);
+  SuffixWs w{};
+  size_t o = align_up(decode_ws(c).total);
+  w.out_f32 = o; o = align_up(o + (size_t)dm.B * dm.Hq * dm.d * sizeof(float));
+  w.ml = o;      o = align_up(o + (size_t)dm.B * dm.Hq * 2 * sizeof(float));
+  w.part = o;    o = align_up(o + suffix_workspace_bytes(dm, s_max));
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+lowram_status lowram_suffix_workspace_size(const lowram_config* c, int32_t s_max, size_t* bytes) {
+  if (!bytes) return LOWRAM_ERR_INVALID_ARG;
+  const lowram_status st = lowram_check_config(c);
+  if (st != LOWRAM_OK) return st;
+  if (s_max < 0) return LOWRAM_ERR_SHAPE;
+  if (!dense_supported(dims_of(*c))) return LOWRAM_ERR_UNSUPPORTED;
+  *bytes = suffix_ws(*c, s_max).total;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_decode_step_suffix(lowram_ctx* ctx, const lowram_cache* cache,
+                                        const lowram_layer_params* params, const void* q,
+                                        const void* k_suffix, const void* v_suffix,
+                                        int32_t s_max, int32_t n_suffix, void* out,
+                                        int32_t* sel_out, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (!ctx || !q || !out || !workspace) return LOWRAM_ERR_INVALID_ARG;
+  if (s_max < 0 || n_suffix < 0 || n_suffix > s_max) return LOWRAM_ERR_SHAPE;
+  if (n_suffix > 0 && (!k_suffix || !v_suffix)) return LOWRAM_ERR_INVALID_ARG;
+  lowram_status st = check_layer_params(params);
+  if (st != LOWRAM_OK) return st;
+  if ((st = check_cache(cache, ctx->cfg)) != LOWRAM_OK) return st;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) ||
+      (sel_out && !aligned16(sel_out)) || !aligned16(k_suffix) || !aligned16(v_suffix))
+    return LOWRAM_ERR_ALIGN;
+  const Dims dm = dims_of(ctx->cfg);
+  if (!dense_supported(dm)) return LOWRAM_ERR_UNSUPPORTED;
+  const DecodeWs w = decode_ws(ctx->cfg);
+  const SuffixWs sw = suffix_ws(ctx->cfg, s_max);
+  if (workspace_bytes < sw.total) return LOWRAM_ERR_WORKSPACE;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + w.sel);
+  const bool tc = use_tc(ctx->cfg);
+  if ((st = select_impl(ctx, cache->landmark, cache->landmark_norm, q, sel, ws, w, s, tc)) !=
+      LOWRAM_OK)
+    return st;
+  float* pre_out = reinterpret_cast<float*>(ws + sw.out_f32);
+  float* pre_ml = reinterpret_cast<float*>(ws + sw.ml);
+  float* const f32[2] = {pre_out, pre_ml};
+  if ((st = attend_impl(ctx, cache, params, q, sel, out, ws, w, s, tc, nullptr, f32)) !=
+      LOWRAM_OK)
+    return st;
+  if (launch_suffix_merge(dm, k_suffix, v_suffix, s_max, n_suffix, q, pre_out, pre_ml, out,
+                          ws + sw.part, s) != cudaSuccess) {
     cudaGetLastError();
     return LOWRAM_ERR_CUDA;
   }

@@ -94,8 +94,18 @@ struct AttendArgs {
   int* ready;             // ctx [B*H] or null: per-pair selection flags; combine clears them
   int wait_ready;         // 1: launched as a programmatic dependent of the selection
                           // kernel; wait for ready[pair] before reading its selection
-  int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); combine
-                          // clears them
+  int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); cleared
+                          // by the kernel's last CTA
+  // tcgen05 kernel, which merges the tiles itself (no combine launch); all zero between
+  // calls, cleared by the kernel's last CTA:
+  int* tiles_done;        // ctx [B*H]: part-B warps done with the pair's tiles
+  int* merge_ctr;         // ctx [1]: next (pair, query head) merge task
+  int* exit_ctr;          // ctx [1]: CTAs finished
+  // decode with a suffix: the combine writes the normalised output in fp32 and the
+  // softmax (max in natural-log units, sum) of each query head instead of out; null
+  // otherwise
+  float* out_f32;         // [B][Hq][d]
+  float* out_ml;          // [B][Hq][2]
   // test only (lowram_debug_reconstruct), null otherwise: rebuilt rows of the selected
   // chunks in selection order, row = (b*H + h)*k*C + slot*C + j (j = token in chunk):
   float* dbg_k;           // [rows][d]  K~_rot, as epilogue part A holds it
@@ -136,6 +146,12 @@ bool dense_supported(const Dims& dm);
 size_t dense_workspace_bytes(const Dims& dm);
 cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, const void* q,
                                 void* out, void* ws, cudaStream_t s);
+// attention over an uncompressed suffix ([B][s_max][H][d], first n_suffix rows valid),
+// merged with the compressed prefix's normalised fp32 output and its softmax (max, sum)
+size_t suffix_workspace_bytes(const Dims& dm, int s_max);
+cudaError_t launch_suffix_merge(const Dims& dm, const void* k_suffix, const void* v_suffix,
+                                int s_max, int n_suffix, const void* q, const float* pre_out,
+                                const float* pre_ml, void* out, void* ws, cudaStream_t s);
 
 // ---------------- encode ----------------
 struct EncodeArgs {

@@ -97,6 +97,12 @@ _sig = {
     "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
     "lowram_dense_decode": (_S, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "lowram_evict": (_S, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_decode_step_suffix": (_S, [_P, ctypes.POINTER(lowram_cache),
+                                       ctypes.POINTER(lowram_layer_params), _P, _P, _P,
+                                       ctypes.c_int32, ctypes.c_int32, _P, _P, _P,
+                                       ctypes.c_size_t, _P]),
+    "lowram_suffix_workspace_size": (_S, [ctypes.POINTER(lowram_config), ctypes.c_int32,
+                                          ctypes.POINTER(ctypes.c_size_t)]),
     "lowram_fit_basis": (_S, [_P, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, _P,
                               ctypes.c_int32, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
     "lowram_fit_basis_workspace_size": (_S, [ctypes.POINTER(lowram_config), ctypes.c_int32,
@@ -349,3 +355,23 @@ def fit_basis(ctx: Context, k_layers, omega, n_power: int, basis_out, workspace,
                            n_power, _ptr(basis_out), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)),
           "lowram_fit_basis")
+
+
+def suffix_workspace_size(cfg: lowram_config, s_max: int) -> int:
+    n = ctypes.c_size_t()
+    check(lowram_suffix_workspace_size(ctypes.byref(cfg), s_max, ctypes.byref(n)),
+          "lowram_suffix_workspace_size")
+    return n.value
+
+
+def decode_step_suffix(ctx: Context, cache: dict, params: lowram_layer_params, q, k_suffix,
+                       v_suffix, n_suffix: int, out, workspace, sel_out=None,
+                       stream=None) -> None:
+    """lowram_decode_step_suffix: decode over the compressed prefix plus the first n_suffix
+    rows of an uncompressed suffix buffer [B][s_max][H][d]."""
+    cs = cache_struct(**cache)
+    check(lowram_decode_step_suffix(ctx.handle, ctypes.byref(cs), ctypes.byref(params), _ptr(q),
+                                    _ptr(k_suffix), _ptr(v_suffix), k_suffix.shape[1], n_suffix,
+                                    _ptr(out), _ptr(sel_out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+          "lowram_decode_step_suffix")

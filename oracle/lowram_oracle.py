@@ -472,6 +472,41 @@ def decode_step(q, cache, basis, w1, b1, w2, b2, *, chunk, top_k, theta, act, se
     return out, np.asarray(sel)
 
 
+def decode_step_with_suffix(q, cache, basis, w1, b1, w2, b2, k_suffix, v_suffix, *, chunk,
+                            top_k, theta, act, sel=None):
+    """One decode step over the compressed prefix plus an uncompressed suffix of
+    generated tokens (the pages leave long generation to a suffix that is compressed
+    periodically, agihunt summary, limitations paragraph).
+
+    Reading: one softmax over the union of the selected chunks' rebuilt tokens and every
+    suffix token; the suffix keys arrive post-RoPE like the cache's original keys.
+    k_suffix, v_suffix: [B, S, H, d] (S may be 0). Returns (out [B, H_q, d], sel).
+    """
+    q = np.asarray(q, np.float64)
+    ks, vs = np.asarray(k_suffix, np.float64), np.asarray(v_suffix, np.float64)
+    B, Hq, d = q.shape
+    H = cache["landmark"].shape[1]
+    G = Hq // H
+    if sel is None:
+        sel, _ = select_chunks(q, cache["landmark"], top_k)
+    out = np.empty((B, Hq, d))
+    for b in range(B):
+        for h in range(H):
+            _, k_rot, v_rec = reconstruct_chunks(
+                sel[b, h], cache["coef"][b], basis, h, d, chunk,
+                cache["res_idx"][b, h], cache["res_val"][b, h], cache["chunk_ptr"][b, h],
+                w1[h], b1[h], w2[h], b2[h], act, theta,
+                None if cache.get("chunk_pos") is None else cache["chunk_pos"][b])
+            keys = np.concatenate([k_rot, ks[b, :, h]])
+            vals = np.concatenate([v_rec, vs[b, :, h]])
+            for g in range(G):
+                z = keys @ q[b, h * G + g] / math.sqrt(d)
+                p = np.exp(z - z.max())
+                p /= p.sum()
+                out[b, h * G + g] = p @ vals
+    return out, np.asarray(sel)
+
+
 def dense_attention(q, k_cache, v):
     """Textbook GQA decode attention over the full uncompressed cache.
 

@@ -425,12 +425,43 @@ def check_int4_residual_encode(M):
         assert np.all(err <= cache["res_scale"][0, h][..., None] / 2 * (1 + 1e-9) + 1e-12)
 
 
+def check_suffix_decode(M):
+    """Compressed prefix + uncompressed suffix, one softmax: at full rank, every token a
+    residual and every chunk selected, it equals dense attention over the prefix's and
+    the suffix's keys and values together; an empty suffix leaves decode unchanged."""
+    sh = tiny_shape(rank=16, n_kv_heads=2, head_dim=8, res_frac=1.0, top_k=10 ** 6)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    cache = M.encode(L["k"], L["v"], L["basis"], *L["w"], n_res=sh.n_res,
+                     store=M.STORE_F64, **kw)
+    rng = np.random.default_rng(33)
+    S = 11
+    ks = rng.standard_normal((sh.batch, S, sh.n_kv_heads, sh.head_dim))
+    vs = rng.standard_normal((sh.batch, S, sh.n_kv_heads, sh.head_dim))
+    out, _ = M.decode_step_with_suffix(L["q"], cache, L["basis"], *L["w"], ks, vs,
+                                       top_k=sh.top_k, **kw)
+    dense = M.dense_attention(L["q"], np.concatenate([L["k"], ks], axis=1),
+                              np.concatenate([L["v"], vs], axis=1))
+    assert np.allclose(out, dense, atol=1e-12)
+    sh2 = tiny_shape(res_frac=0.25, top_k=5, rank=6)
+    L2 = make_layer(sh2)
+    c2 = M.encode(L2["k"], L2["v"], L2["basis"], *L2["w"], n_res=sh2.n_res,
+                  store=M.STORE_F32, chunk=sh2.chunk, theta=sh2.theta, act=sh2.act)
+    empty = np.zeros((sh2.batch, 0, sh2.n_kv_heads, sh2.head_dim))
+    a, _ = M.decode_step_with_suffix(L2["q"], c2, L2["basis"], *L2["w"], empty, empty,
+                                     chunk=sh2.chunk, top_k=sh2.top_k, theta=sh2.theta,
+                                     act=sh2.act)
+    b_, _ = M.decode_step(L2["q"], c2, L2["basis"], *L2["w"], chunk=sh2.chunk,
+                          top_k=sh2.top_k, theta=sh2.theta, act=sh2.act)
+    assert np.allclose(a, b_, atol=1e-14)
+
+
 ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
               check_landmarks_and_scores, check_encode_landmarks, check_topk, check_predictor,
               check_full_rank_exactness, check_residual_pick, check_selection_and_edges,
               check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator,
               check_int4_quantize, check_eviction, check_evicted_full_rank_exactness,
-              check_int4_residual_encode]
+              check_int4_residual_encode, check_suffix_decode]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -616,3 +647,14 @@ def test_mutation_evicted_positions_ignored(monkeypatch):
     def bad(*args):
         return orig(*args[:15], None)
     _fails(check_evicted_full_rank_exactness, monkeypatch, "reconstruct_chunks", bad)
+
+
+def test_mutation_suffix_softmax_separate(monkeypatch):
+    """Prefix and suffix attended with separate softmaxes, then averaged."""
+    def bad(q, cache, basis, w1, b1, w2, b2, ks, vs, *, chunk, top_k, theta, act, sel=None):
+        a, sel = O.decode_step(q, cache, basis, w1, b1, w2, b2, chunk=chunk, top_k=top_k,
+                               theta=theta, act=act, sel=sel)
+        if np.asarray(ks).shape[1] == 0:
+            return a, sel
+        return 0.5 * (a + O.dense_attention(q, ks, vs)), sel
+    _fails(check_suffix_decode, monkeypatch, "decode_step_with_suffix", bad)
