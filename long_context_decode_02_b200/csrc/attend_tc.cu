@@ -163,15 +163,29 @@ __device__ int wait_count_acquire(const int* p, int target, volatile int* abort)
   return 0;
 }
 
+// What the merge needs, passed by value: taking the address of the kernel's parameter
+// block (to pass it by reference to a function that is not inlined) would move the
+// whole block to local memory for every access in the tile loops.
+struct MergeArgs {
+  const float* part;
+  const __nv_bfloat16* w2;
+  const __nv_bfloat16* b2;
+  __nv_bfloat16* out;
+  float* out_f32;
+  float* out_ml;
+  int* tiles_done;
+  int* merge_ctr;
+  int n_tiles, H, Hq, total;
+};
+
 // Merge of one (pair, query head) by a group of 256 threads (named barrier bar_id): the
 // tiles' partials, weighted by 2^(m_t - M), and W2 applied once to the head-weighted
 // hidden sums (the exact reorder in the file comment):
 //   out_g = (W2 Hs_g + Rs_g) / L_g + b2.
 // scratch: 256 + 256 + 4 floats of shared memory.
-__device__ __noinline__ void merge_head(const AttendArgs& a, int p, int g, int t, int bar_id,
+__device__ __noinline__ void merge_head(const MergeArgs a, int p, int g, int t, int bar_id,
                                         float* scratch) {
-  const Dims& dm = a.dm;
-  const int b = p / dm.H, h = p % dm.H;
+  const int b = p / a.H, h = p % a.H;
   const int n = a.n_tiles, lane = t & 31;
   const float* part = a.part + (size_t)p * n * kPartFloats;
   float* hs = scratch;                 // [256]
@@ -181,11 +195,11 @@ __device__ __noinline__ void merge_head(const AttendArgs& a, int p, int g, int t
   uint4 w2v[kF / 2 / 8];
   {
     const uint4* wrow = reinterpret_cast<const uint4*>(
-        (const __nv_bfloat16*)a.w2 + ((size_t)h * kD + j) * kF + half * (kF / 2));
+        a.w2 + ((size_t)h * kD + j) * kF + half * (kF / 2));
 #pragma unroll
     for (int i = 0; i < kF / 2 / 8; ++i) w2v[i] = __ldg(wrow + i);
   }
-  const float b2 = __bfloat162float(((const __nv_bfloat16*)a.b2)[(size_t)h * kD + j]);
+  const float b2 = __bfloat162float(a.b2[(size_t)h * kD + j]);
   // partials are written by other CTAs in this launch: read them through L2
   const float m0 = lane < n ? __ldcg(part + (size_t)lane * kPartFloats + 2 * g) : -INFINITY;
   const float m1 = lane + 32 < n ? __ldcg(part + (size_t)(lane + 32) * kPartFloats + 2 * g) : -INFINITY;
@@ -240,7 +254,7 @@ __device__ __noinline__ void merge_head(const AttendArgs& a, int p, int g, int t
   }
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (half == 0) {
-    const size_t oi = ((size_t)b * dm.Hq + (size_t)h * kG + g) * kD + j;
+    const size_t oi = ((size_t)b * a.Hq + (size_t)h * kG + g) * kD + j;
     const float o = (acc + rs[j] + rs[128 + j]) / *sL + b2;
     if (a.out_f32) {   // decode with a suffix: max in natural-log units, and the sum
       a.out_f32[oi] = o;
@@ -249,7 +263,7 @@ __device__ __noinline__ void merge_head(const AttendArgs& a, int p, int g, int t
         a.out_ml[2 * (oi / kD) + 1] = *sL;
       }
     } else {
-      ((__nv_bfloat16*)a.out)[oi] = __float2bfloat16_rn(o);
+      a.out[oi] = __float2bfloat16_rn(o);
     }
   }
   named_bar_sync(bar_id, 256);   // the scratch is free again
@@ -258,10 +272,9 @@ __device__ __noinline__ void merge_head(const AttendArgs& a, int p, int g, int t
 // The merge phase of one group of 256 epilogue threads (named barrier bar_id): takes
 // (pair, query head) tasks from the launch's counter until none is left, waits (acquire,
 // bounded) until every part-B warp has finished the pair's tiles, and merges them.
-__device__ __noinline__ void merge_phase(const AttendArgs& a, int t, int bar_id, float* scratch,
+__device__ __noinline__ void merge_phase(const MergeArgs a, int t, int bar_id, float* scratch,
                                          volatile int* abort_flag) {
-  const Dims& dm = a.dm;
-  const int total = dm.B * dm.H * kG;
+  const int total = a.total;
   volatile int* slot = reinterpret_cast<volatile int*>(scratch + 516);
   for (;;) {
     if (t == 0) {
@@ -375,6 +388,19 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int32_t* sel_all = a.sel;
+  MergeArgs ma;
+  ma.part = a.part;
+  ma.w2 = (const __nv_bfloat16*)a.w2;
+  ma.b2 = (const __nv_bfloat16*)a.b2;
+  ma.out = (__nv_bfloat16*)a.out;
+  ma.out_f32 = a.out_f32;
+  ma.out_ml = a.out_ml;
+  ma.tiles_done = a.tiles_done;
+  ma.merge_ctr = a.merge_ctr;
+  ma.n_tiles = a.n_tiles;
+  ma.H = dm.H;
+  ma.Hq = dm.Hq;
+  ma.total = dm.B * dm.H * kG;
   // W1_h into Tensor Memory as the hidden-layer GEMM's A operand: row f = 128 hf + lane
   // of half hf in lane `lane`, columns 128 + 64 hf + (0..63) holding bf16 pairs along d.
   // Each epilogue warp (quadrant of trow, half hf, d-half dh) writes 32 columns from one
@@ -875,7 +901,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     for (int i = 0; part_a(i); ++i) {
     }
     // the coefficient buffers are idle once the last tile's K MMA has been consumed
-    merge_phase(a, et, 4, reinterpret_cast<float*>(gbase + L.coef), abort_flag);
+    merge_phase(ma, et, 4, reinterpret_cast<float*>(gbase + L.coef), abort_flag);
   } else {
     // ------------------------------------------------------------ epilogue, part B
     // 8 warps, two per TMEM lane quadrant: hidden half hf of H^T (lane = hidden unit f,
@@ -1034,7 +1060,7 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     };
     for (int i = 0; part_b(i); ++i) {
     }
-    merge_phase(a, etb, 5, reinterpret_cast<float*>(gbase + L.coef + 4096), abort_flag);
+    merge_phase(ma, etb, 5, reinterpret_cast<float*>(gbase + L.coef + 4096), abort_flag);
   }
 
   tc_fence_before();

@@ -74,10 +74,17 @@ def test_encode_properties_and_sampled_errors(full_layer):
         vt = H.f64(v[b, toks, h])
         kp = O.rope_rotate(kt, toks[:, None], sh.theta, inverse=True).reshape(len(toks), -1)
         c = O.project_keys(kp, basis)
-        # stored coefficients: the fp64 projection rounds to them (one bf16 step at most)
+        # stored coefficients: the fp64 projection rounds to them, or to a neighbour when
+        # the fp32 sum lies within its own error of a rounding midpoint; that error (2048
+        # exact products summed in fp32) is ~1e-6 of the row's largest coefficient, which
+        # matters only for coefficients near zero
         cg = H.f64(cache["coef"][b, toks])
         cst = O.round_to_storage(c, O.STORE_BF16)
-        assert np.all(np.abs(cg - cst) <= 2.0 ** (np.floor(np.log2(np.abs(cst) + 1e-30)) - 7) + 1e-6)
+        bound = 2.0 ** (np.floor(np.log2(np.abs(cst) + 1e-30)) - 7) + \
+            1e-5 * np.abs(c).max(axis=1, keepdims=True)
+        excess = np.abs(cg - cst) - bound
+        assert np.all(excess <= 0), (b, h, float(excess.max()),
+                                     float(np.abs(c).flat[np.argmax(excess)]))
         e = ((vt - O.predictor(O.rebuild_keys(c, basis, h, d), w1[h], b1[h], w2[h], b2[h],
                                sh.act)) ** 2).sum(-1)
         picked = np.isin(toks, ridx[b, h])
