@@ -141,157 +141,6 @@ __device__ __forceinline__ float warp_reduce4_scatter(const float (&v)[4], int l
   return w;
 }
 
-// Adds v to *p with release semantics at GPU scope (the caller's earlier writes, and those
-// ordered before it by a warp or CTA barrier, are visible to whoever acquires the value).
-__device__ __forceinline__ void red_release_add(int* p, int v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Polls *p until it reaches target, with acquire semantics (bounded: 2 s, or *abort set;
-// on giving up sets *abort and returns 0).
-__device__ int wait_count_acquire(const int* p, int target, volatile int* abort) {
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    if (v >= target) return 1;
-    if (*abort) return 0;
-    if (global_timer_ns() - t0 > 2000000000ull) break;
-    __nanosleep(128);
-  }
-  *abort = 1;
-  return 0;
-}
-
-// What the merge needs, passed by value: taking the address of the kernel's parameter
-// block (to pass it by reference to a function that is not inlined) would move the
-// whole block to local memory for every access in the tile loops.
-struct MergeArgs {
-  const float* part;
-  const __nv_bfloat16* w2;
-  const __nv_bfloat16* b2;
-  __nv_bfloat16* out;
-  float* out_f32;
-  float* out_ml;
-  int* tiles_done;
-  int* merge_ctr;
-  int n_tiles, H, Hq, total;
-};
-
-// Merge of one (pair, query head) by a group of 256 threads (named barrier bar_id): the
-// tiles' partials, weighted by 2^(m_t - M), and W2 applied once to the head-weighted
-// hidden sums (the exact reorder in the file comment):
-//   out_g = (W2 Hs_g + Rs_g) / L_g + b2.
-// scratch: 256 + 256 + 4 floats of shared memory.
-__device__ __noinline__ void merge_head(const MergeArgs a, int p, int g, int t, int bar_id,
-                                        float* scratch) {
-  const int b = p / a.H, h = p % a.H;
-  const int n = a.n_tiles, lane = t & 31;
-  const float* part = a.part + (size_t)p * n * kPartFloats;
-  float* hs = scratch;                 // [256]
-  float* rs = scratch + 256;           // [2][128]
-  float* sL = scratch + 512;
-  const int j = t >> 1, half = t & 1;
-  uint4 w2v[kF / 2 / 8];
-  {
-    const uint4* wrow = reinterpret_cast<const uint4*>(
-        a.w2 + ((size_t)h * kD + j) * kF + half * (kF / 2));
-#pragma unroll
-    for (int i = 0; i < kF / 2 / 8; ++i) w2v[i] = __ldg(wrow + i);
-  }
-  const float b2 = __bfloat162float(a.b2[(size_t)h * kD + j]);
-  // partials are written by other CTAs in this launch: read them through L2
-  const float m0 = lane < n ? __ldcg(part + (size_t)lane * kPartFloats + 2 * g) : -INFINITY;
-  const float m1 = lane + 32 < n ? __ldcg(part + (size_t)(lane + 32) * kPartFloats + 2 * g) : -INFINITY;
-  const float l0 = lane < n ? __ldcg(part + (size_t)lane * kPartFloats + 2 * g + 1) : 0.f;
-  const float l1 = lane + 32 < n ? __ldcg(part + (size_t)(lane + 32) * kPartFloats + 2 * g + 1) : 0.f;
-  float M = fmaxf(m0, m1);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
-  const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
-  const float* hsrc = part + 2 * kG + (size_t)g * kF + t;
-  const float* rsrc = part + 2 * kG + (size_t)kG * kF + (size_t)(t >> 7) * kG * kD +
-                      (size_t)g * kD + (t & 127);
-  float hacc = 0.f, racc = 0.f;
-  for (int t0 = 0; t0 < n; t0 += 8) {
-    float hv[8], rv[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int tt = t0 + u;
-      hv[u] = tt < n ? __ldcg(hsrc + (size_t)tt * kPartFloats) : 0.f;
-      rv[u] = tt < n ? __ldcg(rsrc + (size_t)tt * kPartFloats) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int tt = t0 + u;
-      const float wt = __shfl_sync(0xffffffffu, tt < 32 ? w0 : w1, tt & 31);
-      hacc = fmaf(wt, hv[u], hacc);
-      racc = fmaf(wt, rv[u], racc);
-    }
-  }
-  float L = w0 * l0 + w1 * l1;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-  hs[t] = hacc;
-  rs[(t >> 7) * 128 + (t & 127)] = racc;
-  if (t == 0) *sL = L;
-  named_bar_sync(bar_id, 256);
-  float acc = 0.f;
-  const float* hh = hs + half * (kF / 2);
-#pragma unroll
-  for (int i = 0; i < kF / 2 / 8; ++i) {
-    const uint4 v = w2v[i];
-    const float2 a0 = bf2_to_f2(v.x), a1 = bf2_to_f2(v.y), a2 = bf2_to_f2(v.z), a3 = bf2_to_f2(v.w);
-    acc = fmaf(a0.x, hh[8 * i + 0], acc);
-    acc = fmaf(a0.y, hh[8 * i + 1], acc);
-    acc = fmaf(a1.x, hh[8 * i + 2], acc);
-    acc = fmaf(a1.y, hh[8 * i + 3], acc);
-    acc = fmaf(a2.x, hh[8 * i + 4], acc);
-    acc = fmaf(a2.y, hh[8 * i + 5], acc);
-    acc = fmaf(a3.x, hh[8 * i + 6], acc);
-    acc = fmaf(a3.y, hh[8 * i + 7], acc);
-  }
-  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-  if (half == 0) {
-    const size_t oi = ((size_t)b * a.Hq + (size_t)h * kG + g) * kD + j;
-    const float o = (acc + rs[j] + rs[128 + j]) / *sL + b2;
-    if (a.out_f32) {   // decode with a suffix: max in natural-log units, and the sum
-      a.out_f32[oi] = o;
-      if (j == 0) {
-        a.out_ml[2 * (oi / kD)] = M * 0.69314718055994531f;
-        a.out_ml[2 * (oi / kD) + 1] = *sL;
-      }
-    } else {
-      a.out[oi] = __float2bfloat16_rn(o);
-    }
-  }
-  named_bar_sync(bar_id, 256);   // the scratch is free again
-}
-
-// The merge phase of one group of 256 epilogue threads (named barrier bar_id): takes
-// (pair, query head) tasks from the launch's counter until none is left, waits (acquire,
-// bounded) until every part-B warp has finished the pair's tiles, and merges them.
-__device__ __noinline__ void merge_phase(const MergeArgs a, int t, int bar_id, float* scratch,
-                                         volatile int* abort_flag) {
-  const int total = a.total;
-  volatile int* slot = reinterpret_cast<volatile int*>(scratch + 516);
-  for (;;) {
-    if (t == 0) {
-      int task = *abort_flag ? total : atomicAdd(a.merge_ctr, 1);
-      if (task < total &&
-          !wait_count_acquire(a.tiles_done + task / kG, a.n_tiles * kEpiWarpsB, abort_flag))
-        task = total;
-      *slot = task;
-    }
-    named_bar_sync(bar_id, 256);
-    const int task = *slot;
-    named_bar_sync(bar_id, 256);
-    if (task >= total) break;
-    merge_head(a, task / kG, task % kG, t, bar_id, scratch);
-  }
-}
-
 __device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
@@ -388,19 +237,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int32_t* sel_all = a.sel;
-  MergeArgs ma;
-  ma.part = a.part;
-  ma.w2 = (const __nv_bfloat16*)a.w2;
-  ma.b2 = (const __nv_bfloat16*)a.b2;
-  ma.out = (__nv_bfloat16*)a.out;
-  ma.out_f32 = a.out_f32;
-  ma.out_ml = a.out_ml;
-  ma.tiles_done = a.tiles_done;
-  ma.merge_ctr = a.merge_ctr;
-  ma.n_tiles = a.n_tiles;
-  ma.H = dm.H;
-  ma.Hq = dm.Hq;
-  ma.total = dm.B * dm.H * kG;
   // W1_h into Tensor Memory as the hidden-layer GEMM's A operand: row f = 128 hf + lane
   // of half hf in lane `lane`, columns 128 + 64 hf + (0..63) holding bf16 pairs along d.
   // Each epilogue warp (quadrant of trow, half hf, d-half dh) writes 32 columns from one
@@ -900,8 +736,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     // after a failed wait every later wait returns at once and the vote ends the loop
     for (int i = 0; part_a(i); ++i) {
     }
-    // the coefficient buffers are idle once the last tile's K MMA has been consumed
-    merge_phase(ma, et, 4, reinterpret_cast<float*>(gbase + L.coef), abort_flag);
   } else {
     // ------------------------------------------------------------ epilogue, part B
     // 8 warps, two per TMEM lane quadrant: hidden half hf of H^T (lane = hidden unit f,
@@ -1053,35 +887,17 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       if (lane == 0) {
         mbar_arrive(bar(BAR_P_EMPTY0 + u));
         mbar_arrive(bar(BAR_META_EMPTY0 + slot));
-        red_release_add(a.tiles_done + p, 1);   // this warp's share of the partial is out
       }
       if (!good) *abort_flag = 1;
       return true;
     };
     for (int i = 0; part_b(i); ++i) {
     }
-    merge_phase(ma, etb, 5, reinterpret_cast<float*>(gbase + L.coef + 4096), abort_flag);
   }
 
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) raise_status(a.status, kStatusTimeout);
-  if (threadIdx.x == 0) {
-    // the last CTA to finish clears the counters and ready flags for the next call: every
-    // other CTA has finished using them by then
-    __threadfence();
-    if (atomicAdd(a.exit_ctr, 1) == (int)gridDim.x - 1) {
-      __threadfence();
-      for (int i = 0; i < dm.B * dm.H; ++i) {
-        a.tiles_done[i] = 0;
-        if (a.ready) a.ready[i] = 0;
-      }
-      for (int i = 0; i < dm.H; ++i) a.item_ctr[i] = 0;
-      *a.merge_ctr = 0;
-      *a.exit_ctr = 0;
-      __threadfence();
-    }
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -215,66 +215,196 @@ __global__ void __launch_bounds__(kSelEncThreads) residual_threshold_kernel(cons
 }
 
 // E5b: fp64 error of every candidate: the whole chain recomputed in fp64 from the
-// stored inputs (inputs widen exactly; fp64 RoPE tables; fp64 exp / erf).
+// stored inputs (inputs widen exactly; fp64 RoPE tables; fp64 exp / erf), for a batch of
+// kNB candidates of one (b, h) per pass, so that every basis and weight element staged in
+// shared memory serves all kNB of them:
+//   c = B^T RoPE^-1(K)     (over the D = H d columns, one head's block at a time)
+//   K~ = B_h c;  hid = act(W1_h K~ + b1);  V_hat = W2_h hid + b2;  e = |V - V_hat|^2
+// Each product is a small GEMM with a 4 (candidates) x m (columns) register tile per
+// thread; the weights are staged transposed where that keeps the lanes' reads in
+// consecutive banks.
+constexpr int kNB = 32;   // candidates per pass
+
+template <typename T>
+__device__ __forceinline__ double ld64(const T* p, size_t i) { return (double)to_f(p[i]); }
+
 template <typename T, int D, int FH>
 __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const EncodeArgs a) {
   const Dims& dm = a.dm;
   const int p = blockIdx.y, b = p / dm.H, h = p % dm.H, tid = threadIdx.x;
-  const int H = dm.H, r = dm.r, Dt = H * D;
-  extern __shared__ double smd[];
-  double* kp = smd;            // [Dt]
-  double* c64 = kp + Dt;       // [r]
-  double* kt = c64 + r;        // [D]
-  double* hid = kt + D;        // [FH]
-  double* red = hid + FH;      // [kEncThreads / 32]
+  const int H = dm.H, r = dm.r;
   const int n = a.cand_count[p];
+  extern __shared__ double smd[];
+  // region A: [kNB][D] fp64 (pre-RoPE keys of one head, later K~)
+  // region B: 64 KB of staged operands (basis block, transposed basis_h, W1^T, W2^T)
+  // region C: [kNB][max(r, FH)] fp64 (c, later hid)
+  double* sA = smd;
+  T* sB = reinterpret_cast<T*>(smd + kNB * D);
+  double* sC = smd + kNB * D + 65536 / 8;
+  __shared__ int s_tok[kNB];
+  __shared__ double s_e[kNB];
+  const int cg = tid >> 5, lane = tid & 31;     // candidate group (4 each), column lane
   const T* kc = (const T*)a.k_cache;
-  for (int j = blockIdx.x; j < n; j += gridDim.x) {
-    const int t = a.cand_idx[(size_t)p * dm.T + j];
-    for (int o = tid; o < H * (D / 2); o += blockDim.x) {
-      const int i = o % (D / 2), hh = o / (D / 2);
-      const size_t base = (((size_t)b * dm.T + t) * H + hh) * D;
-      const double x = ldd(kc, base + i), y = ldd(kc, base + i + D / 2);
-      const double2 c2 = rope_cs64(a.rope, i, token_position(dm, a.chunk_pos, b, t, a.status));
-      kp[hh * D + i] = x * c2.x + y * c2.y;
-      kp[hh * D + i + D / 2] = y * c2.x - x * c2.y;
-    }
+  const T* basis = (const T*)a.basis;
+  for (int j0 = blockIdx.x * kNB; j0 < n; j0 += gridDim.x * kNB) {
+    const int nb = min(kNB, n - j0);
+    if (tid < kNB) s_tok[tid] = tid < nb ? a.cand_idx[(size_t)p * dm.T + j0 + tid] : -1;
     __syncthreads();
-    for (int kk = tid; kk < r; kk += blockDim.x) {
-      double acc = 0.0;
-      for (int i = 0; i < Dt; ++i) acc += ldd((const T*)a.basis, (size_t)i * r + kk) * kp[i];
-      c64[kk] = acc;
-    }
-    __syncthreads();
-    for (int jj = tid; jj < D; jj += blockDim.x) {
-      double acc = 0.0;
-      for (int kk = 0; kk < r; ++kk)
-        acc += ldd((const T*)a.basis, ((size_t)h * D + jj) * r + kk) * c64[kk];
-      kt[jj] = acc;
-    }
-    __syncthreads();
-    for (int f = tid; f < FH; f += blockDim.x) {
-      double acc = ldd((const T*)a.b1, (size_t)h * FH + f);
-      for (int jj = 0; jj < D; ++jj) acc += ldd((const T*)a.w1, ((size_t)h * FH + f) * D + jj) * kt[jj];
-      hid[f] = act_d(acc, dm.act);
-    }
-    __syncthreads();
-    double sq = 0.0;
-    for (int jj = tid; jj < D; jj += blockDim.x) {
-      double acc = ldd((const T*)a.b2, (size_t)h * D + jj);
-      for (int f = 0; f < FH; ++f) acc += ldd((const T*)a.w2, ((size_t)h * D + jj) * FH + f) * hid[f];
-      const double dv = ldd((const T*)a.v, (((size_t)b * dm.T + t) * H + h) * D + jj) - acc;
-      sq += dv * dv;
-    }
+    // ---- c[cand][kk] = sum over heads hh, dims i of kpre[cand][hh d + i] basis[hh d + i][kk]
+    constexpr int kMaxC = 8;   // columns per lane: r <= 256
+    double acc[4][kMaxC];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if ((tid & 31) == 0) red[tid >> 5] = sq;
-    __syncthreads();
-    if (tid == 0) {
-      double s = 0.0;
-      for (int w = 0; w < kEncThreads / 32; ++w) s += red[w];
-      a.cand_e64[(size_t)p * dm.T + j] = s;
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int m = 0; m < kMaxC; ++m) acc[x][m] = 0.0;
+    for (int hh = 0; hh < H; ++hh) {
+      __syncthreads();   // the previous head's operands are consumed
+      for (int o = tid; o < kNB * (D / 2); o += blockDim.x) {
+        const int c = o / (D / 2), i = o % (D / 2);
+        const int t = s_tok[c];
+        double x = 0.0, y = 0.0, cs = 1.0, sn = 0.0;
+        if (t >= 0) {
+          const size_t base = (((size_t)b * dm.T + t) * H + hh) * D;
+          x = ld64(kc, base + i);
+          y = ld64(kc, base + i + D / 2);
+          const double2 c2 = rope_cs64(a.rope, i, token_position(dm, a.chunk_pos, b, t, a.status));
+          cs = c2.x;
+          sn = c2.y;
+        }
+        sA[c * D + i] = x * cs + y * sn;
+        sA[c * D + i + D / 2] = y * cs - x * sn;
+      }
+      for (int o = tid; o < D * r; o += blockDim.x) sB[o] = basis[(size_t)hh * D * r + o];
+      __syncthreads();
+      for (int i = 0; i < D; ++i) {
+        double kv[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) kv[x] = sA[(4 * cg + x) * D + i];
+#pragma unroll
+        for (int m = 0; m < kMaxC; ++m) {
+          const int kk = lane + 32 * m;
+          if (kk < r) {
+            const double bv = (double)to_f(sB[i * r + kk]);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) acc[x][m] = fma(kv[x], bv, acc[x][m]);
+          }
+        }
+      }
     }
+    __syncthreads();
+    // c to region C; the head's basis block transposed into region B: sB[kk][j] = B_h[j][kk]
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int m = 0; m < kMaxC; ++m) {
+        const int kk = lane + 32 * m;
+        if (kk < r) sC[(4 * cg + x) * r + kk] = acc[x][m];
+      }
+    for (int o = tid; o < D * r; o += blockDim.x) {
+      const int j = o / r, kk = o % r;
+      sB[kk * D + j] = basis[((size_t)h * D + j) * r + kk];
+    }
+    __syncthreads();
+    // ---- K~[cand][j] = sum_kk c[cand][kk] B_h[j][kk]  (into region A)
+    {
+      constexpr int M = D / 32;
+      double kt[4][M];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int m = 0; m < M; ++m) kt[x][m] = 0.0;
+      for (int kk = 0; kk < r; ++kk) {
+        double cv[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) cv[x] = sC[(4 * cg + x) * r + kk];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const double bv = (double)to_f(sB[kk * D + lane + 32 * m]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) kt[x][m] = fma(cv[x], bv, kt[x][m]);
+        }
+      }
+      __syncthreads();   // region B (basis_h) and C (c) consumed; A is overwritten now
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int m = 0; m < M; ++m) sA[(4 * cg + x) * D + lane + 32 * m] = kt[x][m];
+    }
+    // W1_h transposed into region B: sB[j][f] = W1[h][f][j]
+    for (int o = tid; o < FH * D; o += blockDim.x) {
+      const int f = o / D, j = o % D;
+      sB[j * FH + f] = ((const T*)a.w1)[((size_t)h * FH + f) * D + j];
+    }
+    __syncthreads();
+    // ---- hid[cand][f] = act(sum_j K~[cand][j] W1[f][j] + b1[f])  (into region C)
+    {
+      constexpr int M = FH / 32;
+      double hv[4][M];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int m = 0; m < M; ++m) hv[x][m] = ld64((const T*)a.b1, (size_t)h * FH + lane + 32 * m);
+      for (int j = 0; j < D; ++j) {
+        double kv[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) kv[x] = sA[(4 * cg + x) * D + j];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const double wv = (double)to_f(sB[j * FH + lane + 32 * m]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) hv[x][m] = fma(kv[x], wv, hv[x][m]);
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int m = 0; m < M; ++m) sC[(4 * cg + x) * FH + lane + 32 * m] = act_d(hv[x][m], dm.act);
+    }
+    __syncthreads();   // region B (W1) consumed
+    // W2_h transposed into region B: sB[f][j] = W2[h][j][f]
+    for (int o = tid; o < D * FH; o += blockDim.x) {
+      const int j = o / FH, f = o % FH;
+      sB[f * D + j] = ((const T*)a.w2)[((size_t)h * D + j) * FH + f];
+    }
+    __syncthreads();
+    // ---- V_hat[cand][j] = sum_f hid[cand][f] W2[j][f] + b2[j];  e = sum_j (V - V_hat)^2
+    {
+      constexpr int M = D / 32;
+      double ov[4][M];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int m = 0; m < M; ++m) ov[x][m] = ld64((const T*)a.b2, (size_t)h * D + lane + 32 * m);
+      for (int f = 0; f < FH; ++f) {
+        double hvv[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) hvv[x] = sC[(4 * cg + x) * FH + f];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const double wv = (double)to_f(sB[f * D + lane + 32 * m]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) ov[x][m] = fma(hvv[x], wv, ov[x][m]);
+        }
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int c = 4 * cg + x;
+        const int t = s_tok[c];
+        double sq = 0.0;
+        if (t >= 0) {
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            const double dv = ld64((const T*)a.v, (((size_t)b * dm.T + t) * H + h) * D + lane + 32 * m) - ov[x][m];
+            sq = fma(dv, dv, sq);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        if (lane == 0) s_e[c] = sq;
+      }
+    }
+    __syncthreads();
+    if (tid < nb) a.cand_e64[(size_t)p * dm.T + j0 + tid] = s_e[tid];
     __syncthreads();
   }
 }
@@ -380,7 +510,8 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
   residual_threshold_kernel<<<dm.B * dm.H, kSelEncThreads, 0, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
-    const size_t smem = sizeof(double) * ((size_t)dm.H * D + dm.r + D + FH + kEncThreads / 32);
+    const int wc = dm.r > FH ? dm.r : FH;
+    const size_t smem = sizeof(double) * ((size_t)kNB * D + (size_t)kNB * wc) + 65536;
     auto kern = residual_rescore_kernel<T, D, FH>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess) return e;

@@ -68,7 +68,13 @@ __device__ __forceinline__ uint64_t desc_k(uint32_t base, int s, uint32_t blk) {
                           kSwizzle64B);
 }
 
-__device__ __forceinline__ float act_acc(float x, int act) { return act_f(x, act); }
+// The activation between the hidden and the output MMA: SiLU as x / (1 + e^-x) with the
+// fast exponential and division (relative error ~1e-6, far inside what the errors' fp64
+// re-scoring window allows); erf-GELU with erff.
+__device__ __forceinline__ float act_acc(float x, int act) {
+  if (act == LOWRAM_ACT_SILU) return __fdividef(x, 1.0f + __expf(-x));
+  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
 
 // ---------------------------------------------------------------- project kernel
 struct ProjMaps {
@@ -121,6 +127,18 @@ encode_project_tc_kernel(const EncodeArgs a, const __grid_constant__ ProjMaps ma
     const int b = tile / tiles_per_b, t0 = (tile % tiles_per_b) * kM;
     const int t = t0 + row;
     const int pos = token_position(dm, a.chunk_pos, b, t, a.status);   // RoPE position
+    // the token's rotations (cos, sin)(pos theta_i) of this thread's 32 pairs, shared by
+    // all heads; and head 0's key rows
+    float2 rc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rc[i] = rope_cs32(a.rope, 32 * hf + i, pos);
+    const __nv_bfloat16* src0 = kc + ((size_t)b * dm.T + t) * H * kD + 32 * hf;
+    uint4 xr[4], yr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      xr[q] = *reinterpret_cast<const uint4*>(src0 + 8 * q);
+      yr[q] = *reinterpret_cast<const uint4*>(src0 + kD / 2 + 8 * q);
+    }
     for (int h = 0; h < H; ++h) {
       const int n = it * H + h, u = n & 1, j = n >> 1;
       // buffer u is free once the MMAs of pass n - 2 have completed
@@ -131,13 +149,16 @@ encode_project_tc_kernel(const EncodeArgs a, const __grid_constant__ ProjMaps ma
           tma_load_2d(sB + (uint32_t)u * bt_bytes + (uint32_t)kb * (uint32_t)r * 64u,
                       &maps.basis_t, h * kD + kb * 32, 0, bar(u));
       }
-      // E1: K_pre = R(t)^T K of head h for pairs i = 32 hf .. 32 hf + 31 of this token
-      const __nv_bfloat16* src = kc + (((size_t)b * dm.T + t) * H + h) * kD + 32 * hf;
-      uint4 xr[4], yr[4];
+      // E1: K_pre = R(t)^T K of head h for pairs i = 32 hf .. 32 hf + 31 of this token;
+      // the next head's rows are loaded first, so their latency hides behind this head
+      uint4 xn[4], yn[4];
+      if (h + 1 < H) {
+        const __nv_bfloat16* src = src0 + (size_t)(h + 1) * kD;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xr[q] = *reinterpret_cast<const uint4*>(src + 8 * q);
-        yr[q] = *reinterpret_cast<const uint4*>(src + kD / 2 + 8 * q);
+        for (int q = 0; q < 4; ++q) {
+          xn[q] = *reinterpret_cast<const uint4*>(src + 8 * q);
+          yn[q] = *reinterpret_cast<const uint4*>(src + kD / 2 + 8 * q);
+        }
       }
       const uint32_t a_hi = sA + (uint32_t)u * 65536u, a_lo = a_hi + 32768u;
 #pragma unroll
@@ -148,8 +169,7 @@ encode_project_tc_kernel(const EncodeArgs a, const __grid_constant__ ProjMaps ma
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 x2 = bf2_to_f2(xw[e]), y2 = bf2_to_f2(yw[e]);
-          const int i0 = 32 * hf + 8 * q + 2 * e;
-          const float2 c0 = rope_cs32(a.rope, i0, pos), c1 = rope_cs32(a.rope, i0 + 1, pos);
+          const float2 c0 = rc[8 * q + 2 * e], c1 = rc[8 * q + 2 * e + 1];
           kx[2 * e] = x2.x * c0.x + y2.x * c0.y;
           ky[2 * e] = y2.x * c0.x - x2.x * c0.y;
           kx[2 * e + 1] = x2.y * c1.x + y2.y * c1.y;
@@ -158,6 +178,13 @@ encode_project_tc_kernel(const EncodeArgs a, const __grid_constant__ ProjMaps ma
         // columns 32 hf + 8 q .. (block hf) and 64 + 32 hf + 8 q .. (block 2 + hf)
         store_split8(a_hi, a_lo, row, 4 * hf + q, kx);
         store_split8(a_hi, a_lo, row, 8 + 4 * hf + q, ky);
+      }
+      if (h + 1 < H) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          xr[q] = xn[q];
+          yr[q] = yn[q];
+        }
       }
       fence_proxy_async_smem();
       __syncthreads();

@@ -27,8 +27,6 @@ struct lowram_ctx {
   float* scores;   // device [B*H][Nc], all bits set between launches
   int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
   int* item_ctr;  // device [H]: tile counters of the tcgen05 attend kernel, 0 between calls
-  int* tc_sync;   // device [B*H + 2]: the tcgen05 kernel's tile-done counters, merge and
-                  // exit counters, 0 between calls
   double* theta64;  // device [d/2]
   float2* chunk32;  // device [T/C][d/2]: (cos, sin)(c C theta_i)
 };
@@ -316,7 +314,6 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
             cudaMalloc(&ctx->counters, 4 * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->ready, pairs * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->item_ctr, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
-            cudaMalloc(&ctx->tc_sync, (pairs + 2) * sizeof(int)) == cudaSuccess &&
             cudaMalloc(&ctx->scores, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
             cudaMalloc(&ctx->theta64, th64.size() * sizeof(double)) == cudaSuccess &&
             cudaMalloc(&ctx->chunk32, chunk32.size() * sizeof(float2)) == cudaSuccess;
@@ -329,7 +326,6 @@ lowram_status lowram_create(const lowram_config* c, int device, lowram_ctx** out
        cudaMemset(ctx->counters, 0, 4 * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->ready, 0, pairs * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->item_ctr, 0, (size_t)c->n_kv_heads * sizeof(int)) == cudaSuccess &&
-       cudaMemset(ctx->tc_sync, 0, (pairs + 2) * sizeof(int)) == cudaSuccess &&
        cudaMemset(ctx->scores, 0xff, pairs * (size_t)(c->n_tokens / c->chunk) * sizeof(float)) == cudaSuccess &&
        cudaMemcpy(ctx->theta64, th64.data(), th64.size() * sizeof(double), cudaMemcpyHostToDevice) == cudaSuccess &&
        cudaMemcpy(ctx->chunk32, chunk32.data(), chunk32.size() * sizeof(float2), cudaMemcpyHostToDevice) == cudaSuccess;
@@ -354,7 +350,6 @@ void lowram_destroy(lowram_ctx* ctx) {
   cudaFree(ctx->scores);
   cudaFree(ctx->ready);
   cudaFree(ctx->item_ctr);
-  cudaFree(ctx->tc_sync);
   cudaFree(ctx->theta64);
   cudaFree(ctx->chunk32);
   delete ctx;
@@ -459,12 +454,6 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
   aa.ready = tc && after_select ? ctx->ready : nullptr;
   aa.wait_ready = aa.ready ? 1 : 0;
   aa.item_ctr = tc ? ctx->item_ctr : nullptr;
-  if (tc) {
-    const size_t pairs = (size_t)dm.B * dm.H;
-    aa.tiles_done = ctx->tc_sync;
-    aa.merge_ctr = ctx->tc_sync + pairs;
-    aa.exit_ctr = ctx->tc_sync + pairs + 1;
-  }
   if (f32) {   // decode with a suffix: fp32 output and softmax statistics
     aa.out_f32 = f32[0];
     aa.out_ml = f32[1];
@@ -475,7 +464,7 @@ lowram_status attend_impl(lowram_ctx* ctx, const lowram_cache* cache,
     aa.dbg_v = dbg[2];
   }
   cudaError_t e = tc ? launch_attend_tc(aa, ctx->num_sms, s) : launch_attend_simt(aa, s);
-  if (e == cudaSuccess && !tc) e = launch_combine(aa, false, s);   // tcgen05 merges itself
+  if (e == cudaSuccess) e = launch_combine(aa, tc, s);
   if (e == cudaSuccess && dbg) e = launch_debug_values(aa, s);
   if (e != cudaSuccess) { cudaGetLastError(); return LOWRAM_ERR_CUDA; }
   return LOWRAM_OK;

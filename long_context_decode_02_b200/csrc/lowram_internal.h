@@ -94,13 +94,8 @@ struct AttendArgs {
   int* ready;             // ctx [B*H] or null: per-pair selection flags; combine clears them
   int wait_ready;         // 1: launched as a programmatic dependent of the selection
                           // kernel; wait for ready[pair] before reading its selection
-  int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); cleared
-                          // by the kernel's last CTA
-  // tcgen05 kernel, which merges the tiles itself (no combine launch); all zero between
-  // calls, cleared by the kernel's last CTA:
-  int* tiles_done;        // ctx [B*H]: part-B warps done with the pair's tiles
-  int* merge_ctr;         // ctx [1]: next (pair, query head) merge task
-  int* exit_ctr;          // ctx [1]: CTAs finished
+  int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); combine
+                          // clears them
   // decode with a suffix: the combine writes the normalised output in fp32 and the
   // softmax (max in natural-log units, sum) of each query head instead of out; null
   // otherwise
