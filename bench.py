@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=None,
                     help="decode only the first L layers (profiling runs)")
+    ap.add_argument("--context", type=int, default=None,
+                    help="prefix length override (profiling runs on a smaller case)")
     ap.add_argument("--config", type=int, choices=[2, 3, 4], default=2,
                     help="2: Llama-3-8B-shaped, batch 8, 128K (the headline line); "
                          "3: Mistral-7B-shaped, batch 4, 262K, rank 128, 15%% residuals; "
@@ -194,6 +196,8 @@ def run_ours(args):
     dev = torch.device("cuda", local)
 
     base = synth.CONFIGS[args.config]
+    if args.context:
+        base = base.replace(name=f"{base.name}-ctx{args.context}", n_tokens=args.context)
     n_layers = args.layers or base.n_layers
     sh = rank_shape(base, rank)
     cfg = L.make_config(sh)
