@@ -391,7 +391,7 @@ def run_ours(args):
         n_dense = 20
         with torch.cuda.stream(stream):
             for i in range(3):
-                L.dense_decode(ctx, kd, vd, q_all[W + i, 0], od, ws_dense)
+                L.dense_decode(ctx, kd, vd, q_all[W + (i % K), 0], od, ws_dense)
             torch.cuda.synchronize()
             d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             d0.record(stream)
