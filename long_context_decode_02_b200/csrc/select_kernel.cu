@@ -12,13 +12,14 @@
 //    itself and the (b, h) pairs are completed one after another while the stream runs.
 //    A producer warp TMA-loads each stage into a 3-stage shared-memory ring (128-byte
 //    swizzle) and stages the pair's queries in fp32 beside it; 256 consumer threads
-//    score one row each (packed fp32x2 FMAs) and write the fp32 score.
+//    score the rows (packed fp32x2 FMAs; bf16 rows by lane pairs, each lane one half of
+//    the dims of two rows, so each query load serves two rows) and write fp32 scores.
 //  * Scores live in a context-owned buffer that holds a sentinel bit pattern between
 //    launches (0xFFFFFFFF, a NaN that fp32 arithmetic never produces), so a written score
 //    is its own completion flag: no counters or memory fences on the streaming path.
 //    Three selection warps per CTA take (b, h) pairs in order from a global counter,
 //    wait until the work counter has handed out all of the pair's stages and every score
-//    has landed, select, and put the sentinel back. Selections are spread over the CTAs
+//    has landed, select, set the pair's ready flag and put the sentinel back. Selections are spread over the CTAs
 //    and overlap the stream; a selection group only waits for stages held by running
 //    CTAs, and every wait is bounded.
 //  * Selection: the 16-bit key prefix of the j-th largest of 1024 evenly spaced scores
@@ -680,10 +681,10 @@ __device__ bool select_pair(const Grp& g, const SelectArgs& a, int p, float* cke
 }
 
 // ---------------------------------------------------------------- scoring
-// Score of landmark row r of a swizzled stage.
-template <typename T, int D, int G>
-__device__ __forceinline__ float score_row(const uint8_t* stage, int r, const float* sQ) {
-  using Gm = Geom<T, D>;
+// Score of landmark row r of a swizzled fp32 stage (one row per lane).
+template <int D, int G>
+__device__ __forceinline__ float score_row_f32(const uint8_t* stage, int r, const float* sQ) {
+  using Gm = Geom<float, D>;
   float2 acc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = make_float2(0.f, 0.f);
@@ -692,34 +693,81 @@ __device__ __forceinline__ float score_row(const uint8_t* stage, int r, const fl
     const int box = c >> 3, cc = c & 7;
     const uint4 w = *reinterpret_cast<const uint4*>(
         stage + box * Gm::kLps * 128 + r * 128 + ((cc ^ (r & 7)) << 4));
-    if constexpr (sizeof(T) == 2) {
-      // 8 bf16: chunk c holds dims 8c .. 8c+7
-      const float2 v0 = bf2_to_f2(w.x), v1 = bf2_to_f2(w.y), v2 = bf2_to_f2(w.z), v3 = bf2_to_f2(w.w);
+    // 4 fp32: chunk c holds dims 4c .. 4c+3
+    const float2 v0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+    const float2 v1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c);
-        const float4 q1 = *reinterpret_cast<const float4*>(sQ + g * D + 8 * c + 4);
-        acc[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, acc[g]);
-        acc[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, acc[g]);
-        acc[g] = __ffma2_rn(make_float2(q1.x, q1.y), v2, acc[g]);
-        acc[g] = __ffma2_rn(make_float2(q1.z, q1.w), v3, acc[g]);
-      }
-    } else {
-      // 4 fp32: chunk c holds dims 4c .. 4c+3
-      const float2 v0 = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
-      const float2 v1 = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 4 * c);
-        acc[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, acc[g]);
-        acc[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, acc[g]);
-      }
+    for (int g = 0; g < G; ++g) {
+      const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + 4 * c);
+      acc[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, acc[g]);
+      acc[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, acc[g]);
     }
   }
   float best = acc[0].x + acc[0].y;
 #pragma unroll
   for (int g = 1; g < G; ++g) best = fmaxf(best, acc[g].x + acc[g].y);
   return best;
+}
+
+// Position in a stage's query block of dim d of a head (bf16 landmarks): the upper half
+// of the dims has its 16-byte units XOR 4, so the two lanes of a pair in score_rows_pair,
+// which read the lower and the upper half at the same step, hit different banks.
+template <int D>
+__device__ __forceinline__ int q_pos(int d) {
+  return d < D / 2 ? d : ((((d >> 2) ^ 4) << 2) | (d & 3));
+}
+
+// Scores of rows r0 and r1 of a bf16 stage by a pair of lanes (lane half hh = lane & 1):
+// each lane sums its half of the dims for both rows, so every query load feeds two rows
+// (half the query traffic of one row per lane), and one shuffle per head and row adds the
+// partner's half. The upper half walks its 16-byte chunks in XOR-4 order so the pair's
+// landmark loads fall in different banks as well. Returns (score r0, score r1), the same
+// in both lanes (fp32 addition commutes).
+template <int D, int G>
+__device__ __forceinline__ float2 score_rows_pair(const uint8_t* stage, int r0, int r1, int hh,
+                                                  const float* sQ) {
+  using Gm = Geom<__nv_bfloat16, D>;
+  constexpr int H = Gm::kChunks / 2;   // 16-byte chunks per half row: 8 (D 128), 4 (D 64)
+  float2 a0[G], a1[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    a0[g] = make_float2(0.f, 0.f);
+    a1[g] = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int st = 0; st < H; ++st) {
+    const int c = hh * H + ((H == 8 && hh) ? (st ^ 4) : st);   // chunk: dims 8c .. 8c + 7
+    const int box = c >> 3, cc = c & 7;
+    const uint8_t* bp = stage + box * Gm::kLps * 128;
+    const uint4 w0 = *reinterpret_cast<const uint4*>(bp + r0 * 128 + ((cc ^ (r0 & 7)) << 4));
+    const uint4 w1 = *reinterpret_cast<const uint4*>(bp + r1 * 128 + ((cc ^ (r1 & 7)) << 4));
+    const float2 v0 = bf2_to_f2(w0.x), v1 = bf2_to_f2(w0.y), v2 = bf2_to_f2(w0.z), v3 = bf2_to_f2(w0.w);
+    const float2 u0 = bf2_to_f2(w1.x), u1 = bf2_to_f2(w1.y), u2 = bf2_to_f2(w1.z), u3 = bf2_to_f2(w1.w);
+    const int qa = q_pos<D>(8 * c), qb = q_pos<D>(8 * c + 4);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4 q0 = *reinterpret_cast<const float4*>(sQ + g * D + qa);
+      const float4 q1 = *reinterpret_cast<const float4*>(sQ + g * D + qb);
+      a0[g] = __ffma2_rn(make_float2(q0.x, q0.y), v0, a0[g]);
+      a1[g] = __ffma2_rn(make_float2(q0.x, q0.y), u0, a1[g]);
+      a0[g] = __ffma2_rn(make_float2(q0.z, q0.w), v1, a0[g]);
+      a1[g] = __ffma2_rn(make_float2(q0.z, q0.w), u1, a1[g]);
+      a0[g] = __ffma2_rn(make_float2(q1.x, q1.y), v2, a0[g]);
+      a1[g] = __ffma2_rn(make_float2(q1.x, q1.y), u2, a1[g]);
+      a0[g] = __ffma2_rn(make_float2(q1.z, q1.w), v3, a0[g]);
+      a1[g] = __ffma2_rn(make_float2(q1.z, q1.w), u3, a1[g]);
+    }
+  }
+  float best0 = -INFINITY, best1 = -INFINITY;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float z0 = a0[g].x + a0[g].y, z1 = a1[g].x + a1[g].y;
+    z0 += __shfl_xor_sync(0xffffffffu, z0, 1);
+    z1 += __shfl_xor_sync(0xffffffffu, z1, 1);
+    best0 = fmaxf(best0, z0);
+    best1 = fmaxf(best1, z1);
+  }
+  return make_float2(best0, best1);
 }
 
 template <typename T, int D, int G>
@@ -806,7 +854,13 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (u >= U) return 1;   // slot s is free for the closing fill
       float* q_s = sQ + s * kQ;
 #pragma unroll
-      for (int j = 0; j < kQL; ++j) q_s[lane + 32 * j] = qc[j];
+      for (int j = 0; j < kQL; ++j) {
+        const int f = lane + 32 * j;   // head f / D, dim f % D
+        if constexpr (sizeof(T) == 2)
+          q_s[(f / D) * D + q_pos<D>(f % D)] = qc[j];
+        else
+          q_s[f] = qc[j];
+      }
       if (lane == 0) {
         stage_unit[s] = u;
         const int pair = u / upp, st = u % upp;
@@ -860,10 +914,20 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       const int u = stage_unit[s];
       if (u < 0) break;
       const int pair = u / upp, st = u % upp;
-      const int c = st * Gm::kLps + tid;
-      if (tid < Gm::kLps && c < Nc)
-        a.scores[(size_t)pair * Nc + c] =
-            score_row<T, D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
+      if constexpr (sizeof(T) == 2) {
+        // lanes 2i, 2i + 1 score rows i and i + kLps/2 of the stage (kLps == 256 threads)
+        static_assert(Gm::kLps == kConsumers, "one lane pair per two rows");
+        const int hh = tid & 1, r0 = tid >> 1, r1 = r0 + Gm::kLps / 2;
+        const float2 sc = score_rows_pair<D, G>(gbase + L.stages + s * kStageBytes, r0, r1, hh,
+                                                sQ + s * kQ);
+        const int c = st * Gm::kLps + (hh ? r1 : r0);
+        if (c < Nc) a.scores[(size_t)pair * Nc + c] = hh ? sc.y : sc.x;
+      } else {
+        const int c = st * Gm::kLps + tid;
+        if (tid < Gm::kLps && c < Nc)
+          a.scores[(size_t)pair * Nc + c] =
+              score_row_f32<D, G>(gbase + L.stages + s * kStageBytes, tid, sQ + s * kQ);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
     }
@@ -911,11 +975,12 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (pair < 0) break;
       // a failed wait has raised the abort flag: the next step ends the loop
       if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) continue;
-      clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
       if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
         __threadfence();
         st_release(a.ready + pair, 1);
       }
+      // the sentinel goes back after the flag: only the next launch reads these scores
+      clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
     }
   }
   __syncthreads();
