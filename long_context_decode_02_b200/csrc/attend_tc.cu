@@ -318,9 +318,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     // up to kMetaSlots (kRotSlots for rotations) tiles ahead of the epilogue.
     // The four dependent global reads of a tile (its item from the head's counter, its
     // chunk ids, their CSR spans, the residual rows) are software-pipelined over four
-    // tiles: one pass of the loop issues the counter take of tile j + 3, the chunk ids of
-    // j + 2, the spans of j + 1 and the residual rows of j, so a tile costs about one
-    // memory round trip instead of four.
+    // tiles: one pass of the loop issues the counter take of tile j + 3, the spans of
+    // j + 1 and the residual rows of j, posts tile j, then issues the chunk ids of j + 2,
+    // so a tile costs about one memory round trip instead of four.
     const int32_t* ptr_all = a.chunk_ptr;
     const int32_t* ridx_all = a.res_idx;
     // tiles come from this head's counter (lane 0 takes, the warp learns it later)
@@ -337,14 +337,20 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       return cid;
     };
     // when the selection kernel may still be running: wait until item it's pair is
-    // published (acquire); false after a timeout (the abort flag is then set)
+    // published (acquire); false after a timeout (the abort flag is then set). A flag
+    // once seen set stays set for the launch, so the pairs (b, h) already seen (b < 64)
+    // are remembered and not read again.
+    uint64_t seen_ready = 0;
     auto pair_ready = [&](int it) -> bool {
       if (!a.wait_ready) return true;
       int b, tile;
       item_of(it, b, tile);
+      if (b < 64 && ((seen_ready >> b) & 1ull)) return true;
       int ok = 1;
       if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
-      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok && b < 64) seen_ready |= 1ull << b;
+      return ok != 0;
     };
     // an id outside [-1, Nc) is reported and dropped (the chunk is skipped)
     auto sanitize = [&](int cid) -> int {
@@ -416,8 +422,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
       cid1 = sanitize(cid1);
       load_span(it1, cid1, e0r, e1r);
-      int cid2 = -1;
-      if (it2 < n_items && pair_ready(it2)) cid2 = load_cid(it2);
 
       int got = 0;
       if (lane == 0)
@@ -470,6 +474,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         }
         rot_issued = i;
       }
+      // the chunk ids of tile i + 2, once tile i is posted (its pair may need a wait)
+      int cid2 = -1;
+      if (it2 < n_items && pair_ready(it2)) cid2 = load_cid(it2);
       // advance the pipeline
       it0 = it1;
       it1 = it2;
