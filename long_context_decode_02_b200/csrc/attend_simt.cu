@@ -293,7 +293,8 @@ __global__ void __launch_bounds__(256) combine_reorder_kernel(const AttendArgs a
   // launched as a programmatic dependent of the attend kernel: W2 above is independent
   // of it; the partials, flags and counters below are not
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (a.ready && g == 0 && threadIdx.x == 0) a.ready[p] = 0;   // the next step's flags
+  if (a.ready && g == 0 && threadIdx.x == 0 && (b & 31) == 0)   // the next step's words
+    a.ready[ready_word(dm, b, h)] = 0;
   if (a.item_ctr && p < dm.H && g == 0 && threadIdx.x == 0) a.item_ctr[p] = 0;   // tile counters
   const float b2 = ldf((const T*)a.b2, (size_t)h * D + j);
   // tile weights, computed by every warp: lane t holds tile t (and t + 32)

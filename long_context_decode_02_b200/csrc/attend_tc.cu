@@ -141,12 +141,14 @@ __device__ __forceinline__ float warp_reduce4_scatter(const float (&v)[4], int l
   return w;
 }
 
-__device__ int wait_flag_acquire(const int* flag, volatile int* abort) {
+// Polls *word (acquire) until it has bit `bit`; returns the word (0 after giving up: 2 s,
+// or the abort flag, which is then set).
+__device__ uint32_t wait_bit_acquire(const int* word, int bit, volatile int* abort) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    if (v != 0) return 1;
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
+    if ((v >> bit) & 1u) return v;
     if (*abort) return 0;
     if (global_timer_ns() - t0 > 2000000000ull) break;
     __nanosleep(256);
@@ -337,20 +339,21 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       return cid;
     };
     // when the selection kernel may still be running: wait until item it's pair is
-    // published (acquire); false after a timeout (the abort flag is then set). A flag
-    // once seen set stays set for the launch, so the pairs (b, h) already seen (b < 64)
-    // are remembered and not read again.
+    // published (acquire on the head's readiness word); false after a timeout (the abort
+    // flag is then set). Bits once seen stay set for the launch, so every pair (b < 64)
+    // a read has shown published is remembered and not read again.
     uint64_t seen_ready = 0;
     auto pair_ready = [&](int it) -> bool {
       if (!a.wait_ready) return true;
       int b, tile;
       item_of(it, b, tile);
       if (b < 64 && ((seen_ready >> b) & 1ull)) return true;
-      int ok = 1;
-      if (lane == 0) ok = wait_flag_acquire(a.ready + b * dm.H + h, abort_flag);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok && b < 64) seen_ready |= 1ull << b;
-      return ok != 0;
+      uint32_t w = 1;
+      if (lane == 0) w = wait_bit_acquire(a.ready + ready_word(dm, b, h), b & 31, abort_flag);
+      w = __shfl_sync(0xffffffffu, w, 0);
+      if (w == 0) return false;
+      if (b < 64) seen_ready |= (uint64_t)w << (b & 32);
+      return true;
     };
     // an id outside [-1, Nc) is reported and dropped (the chunk is skipped)
     auto sanitize = [&](int cid) -> int {

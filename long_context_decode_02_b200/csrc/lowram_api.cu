@@ -25,7 +25,7 @@ struct lowram_ctx {
   int* status;    // device word
   int* counters;  // device [4]: the selection kernel's work, exit and pair counters
   float* scores;   // device [B*H][Nc], all bits set between launches
-  int* ready;     // device [B*H]: per-pair selection flags of a decode step, 0 between steps
+  int* ready;     // device [B*H] ints (H * ceil(B/32) used): readiness words, 0 between steps
   int* item_ctr;  // device [H]: tile counters of the tcgen05 attend kernel, 0 between calls
   double* theta64;  // device [d/2]
   float2* chunk32;  // device [T/C][d/2]: (cos, sin)(c C theta_i)

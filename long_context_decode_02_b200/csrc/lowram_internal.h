@@ -42,6 +42,15 @@ struct Dims {
   int P;          // RoPE positions of the original prefix (T unless chunks were evicted)
   int res_int4;   // residual rows stored as int4 codes + fp16 scales per 32 elements
 };
+
+// Pair (b, h)'s selection is published by bit b % 32 of word ready_word(dm, b, h) of the
+// context's readiness array: H * ceil(B / 32) words, one run per KV head, so one read
+// tells the reader of a head every batch element published so far.
+__host__ __device__ inline int ready_words_per_head(const Dims& dm) { return (dm.B + 31) / 32; }
+__host__ __device__ inline int ready_word(const Dims& dm, int b, int h) {
+  return h * ready_words_per_head(dm) + (b >> 5);
+}
+
 constexpr int kInt4Group = 32;
 
 // ---------------- decode: landmark scoring + top-k selection ----------------
@@ -56,7 +65,7 @@ struct SelectArgs {
   uint8_t* flags;         // ws [B*H][Nc]
   int* counters;          // ctx [4]: work, exit and pair counters, zero between launches
   int32_t* sel;           // [B*H][k]
-  int* ready;             // ctx [B*H] or null: set to 1 once a pair's selection is written
+  int* ready;             // ctx or null: readiness words, see ready_word()
   int* status;
 };
 cudaError_t launch_select(const SelectArgs& a, int num_sms, cudaStream_t s);
@@ -91,7 +100,7 @@ struct AttendArgs {
   int* status;
   int n_tiles;            // tiles per (b, h)
   int tile_tokens;
-  int* ready;             // ctx [B*H] or null: per-pair selection flags; combine clears them
+  int* ready;             // ctx or null: readiness words (ready_word()); combine clears them
   int wait_ready;         // 1: launched as a programmatic dependent of the selection
                           // kernel; wait for ready[pair] before reading its selection
   int* item_ctr;          // ctx [H]: next tile of each KV head (tcgen05 kernel); combine

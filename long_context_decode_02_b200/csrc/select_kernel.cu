@@ -105,8 +105,8 @@ static_assert(kStages * 4 <= 64 && 2 * kStages * 8 + 4 <= 64, "stage units and b
 
 constexpr uint32_t kScoreEmpty = 0xFFFFFFFFu;   // sentinel of an unwritten score
 
-__device__ __forceinline__ void st_release(int* p, int v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ void or_release(int* p, uint32_t bits) {
+  asm volatile("red.release.gpu.global.or.b32 [%0], %1;" ::"l"(p), "r"(bits) : "memory");
 }
 
 __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
@@ -977,7 +977,8 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
       if (!select_pair<T, D, G>(g, a, pair, ckey, cidv, bits, ms, abort_flag)) continue;
       if (a.ready && g.tid == 0) {   // select_pair ended on a group barrier
         __threadfence();
-        st_release(a.ready + pair, 1);
+        const int b = pair / dm.H, hh = pair % dm.H;
+        or_release(a.ready + ready_word(dm, b, hh), 1u << (b & 31));
       }
       // the sentinel goes back after the flag: only the next launch reads these scores
       clear_scores(g, reinterpret_cast<uint32_t*>(a.scores + (size_t)pair * Nc), Nc);
