@@ -66,21 +66,28 @@ struct TileMeta {
   int cid[kChunksPerTile];  // chunk id of each slot of the tile; -1 past the selection
   int nres;                 // residual rows of the tile
   int item;                 // b * n_tiles + tile; -1: this CTA has no more tiles
-  int pad[2];
+  int nstaged;              // residual entries 0 .. nstaged-1 are in the tile's row buffer
+  int pad;
   uint32_t res[kTile];      // (row of res_val) << 8 | token row in the tile (255 = skip)
   uint4 q[64];              // the tile's G = 4 query rows, bf16 [4][128]
 };
 static_assert(sizeof(TileMeta) == 1616, "TileMeta layout");
 constexpr int kMetaSlots = 4;
-constexpr int kResPrefetch = 16;   // residual rows per thread loaded before the hidden layer
+// bf16 residual rows of a tile are copied into one of two row buffers by the metadata
+// warp (bulk copies of each chunk's contiguous span); entries past kResCap (a tile with
+// more than 48 of its 128 tokens residual) are read from global memory
+constexpr int kResCap = 48;
+constexpr int kResBufs = 2;
 
 constexpr int kRotSlots = 2;   // chunk-base rotations, one slot per tile in flight
 // float2 stride of a chunk's 64 rotations: padded by 2 so the four chunks one warp reads
 // fall in different shared-memory banks
 constexpr int kRotStride = kD / 2 + 2;
 
+constexpr uint32_t kBarBytes = 320;   // mbarriers, the TMEM address and the abort word
+
 struct Layout {
-  uint32_t basis, coef, kbf, p, p2, q, b1, zx, red, rot, roff, meta, bar, total;
+  uint32_t basis, coef, kbf, p, p2, q, b1, zx, red, rot, roff, meta, rbuf, bar, total;
 };
 __host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) {
   return (x + a - 1) / a * a;
@@ -100,8 +107,9 @@ __host__ __device__ inline Layout make_layout(int r) {
   L.rot = L.red + 512;          // [kRotSlots][16 chunks][kRotStride] float2 (cos, sin)
   L.roff = L.rot + kRotSlots * kChunksPerTile * kRotStride * 8;  // [64 pairs][8] float2
   L.meta = L.roff + (kD / 2) * kChunk * 8;  // kMetaSlots x TileMeta
-  L.bar = L.meta + kMetaSlots * (uint32_t)sizeof(TileMeta);  // barriers + TMEM holder
-  L.total = L.bar + 256 + 1024; // + alignment slack of the dynamic base
+  L.rbuf = align_up(L.meta + kMetaSlots * (uint32_t)sizeof(TileMeta), 128);  // residual rows
+  L.bar = L.rbuf + kResBufs * kResCap * kD * 2;   // barriers + TMEM holder
+  L.total = L.bar + kBarBytes + 1024;  // + alignment slack of the dynamic base
   return L;
 }
 
@@ -112,9 +120,11 @@ enum {
   BAR_P_FULL0, BAR_P_FULL1, BAR_P_EMPTY0, BAR_P_EMPTY1,
   BAR_ROT_FULL0, BAR_ROT_EMPTY0 = BAR_ROT_FULL0 + kRotSlots,
   BAR_META_FULL0 = BAR_ROT_EMPTY0 + kRotSlots, BAR_META_EMPTY0 = BAR_META_FULL0 + kMetaSlots,
-  BAR_COUNT = BAR_META_EMPTY0 + kMetaSlots
+  BAR_RES_FULL0 = BAR_META_EMPTY0 + kMetaSlots,   // a slot's residual list (and rows) landed
+  BAR_RBUF_EMPTY0 = BAR_RES_FULL0 + kMetaSlots,   // part B is done with a residual row buffer
+  BAR_COUNT = BAR_RBUF_EMPTY0 + kResBufs
 };
-static_assert(BAR_COUNT * 8 + 8 <= 256, "barrier area");
+static_assert(BAR_COUNT * 8 + 8 <= kBarBytes, "barrier area");
 
 template <int ACT>
 __device__ __forceinline__ float act_fast(float x) {
@@ -223,7 +233,9 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     for (int i = 0; i < kMetaSlots; ++i) {
       mbar_init(bar(BAR_META_FULL0 + i), 1);
       mbar_init(bar(BAR_META_EMPTY0 + i), kEpiWarpsB);
+      mbar_init(bar(BAR_RES_FULL0 + i), 1);
     }
+    for (int i = 0; i < kResBufs; ++i) mbar_init(bar(BAR_RBUF_EMPTY0 + i), kEpiWarpsB);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -325,8 +337,12 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     // so a tile costs about one memory round trip instead of four.
     const int32_t* ptr_all = a.chunk_ptr;
     const int32_t* ridx_all = a.res_idx;
-    // tiles come from this head's counter (lane 0 takes, the warp learns it later)
-    auto take_raw = [&]() -> int { return lane == 0 ? atomicAdd(a.item_ctr + h, 1) : 0; };
+    // tiles come from this head's counter (lane 0 takes, the warp learns it later); the
+    // first tile of the c-th CTA of the head is tile c, so the counter starts after them
+    const int ctas_h = ((int)gridDim.x - h + dm.H - 1) / dm.H;   // CTAs serving head h
+    auto take_raw = [&]() -> int {
+      return lane == 0 ? ctas_h + atomicAdd(a.item_ctr + h, 1) : 0;
+    };
     // chunk ids of item `it` (issued, not waited for); -1 past the selection
     auto load_cid = [&](int it) -> int {
       int b, tile;
@@ -376,13 +392,30 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       }
     };
     int rot_issued = -1;   // last tile whose rotations were requested (for the drain)
-    // prologue: items of tiles 0..2, chunk ids of 0 and 1, spans of 0
-    int tk0 = take_raw(), tk1 = take_raw(), tk2 = take_raw();
-    int it0 = __shfl_sync(0xffffffffu, tk0, 0);
-    int it1 = __shfl_sync(0xffffffffu, tk1, 0);
-    int it2 = __shfl_sync(0xffffffffu, tk2, 0);
+    int res_issued = -1;   // last tile whose residual rows were requested (for the drain)
+    // the queries of item it (issued, written into the slot when it is posted)
+    auto load_q = [&](int it, uint4& qa, uint4& qb) {
+      qa = make_uint4(0u, 0u, 0u, 0u);
+      qb = qa;
+      if (it < n_items) {
+        int b, tile;
+        item_of(it, b, tile);
+        const uint4* qsrc = reinterpret_cast<const uint4*>(
+            (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
+        qa = qsrc[lane];
+        qb = qsrc[lane + 32];
+      }
+    };
+    // prologue: the CTA's own first tile and two tiles from the counter; chunk ids and
+    // queries of tile 0, chunk ids of tile 1, spans of tile 0
+    int tk1 = take_raw(), tk2 = take_raw();
+    int it0 = (int)blockIdx.x / dm.H;
     int cid0 = -1, cid1 = -1;
     if (it0 < n_items && pair_ready(it0)) cid0 = load_cid(it0);
+    uint4 qa0, qb0;
+    load_q(it0, qa0, qb0);
+    int it1 = __shfl_sync(0xffffffffu, tk1, 0);
+    int it2 = __shfl_sync(0xffffffffu, tk2, 0);
     if (it1 < n_items && pair_ready(it1)) cid1 = load_cid(it1);
     cid0 = sanitize(cid0);
     int e0r, e1r;
@@ -390,71 +423,28 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
     for (int i = 0;; ++i) {
       const int it = it0;
       const int slot = i % kMetaSlots;
-      if (it >= n_items) {   // no more tiles: post the end marker
-        int got = 0;
-        if (lane == 0)
-          got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
-        if (__shfl_sync(0xffffffffu, got, 0) && lane == 0) {
-          meta[slot].item = -1;
-          mbar_arrive(bar(BAR_META_FULL0 + slot));
-        }
-        break;
-      }
-      // issue: the take of tile i + 3, the queries and residual rows of tile i, the spans
-      // of tile i + 1, the chunk ids of tile i + 2
-      const int tk3 = take_raw();
-      int b, tile;
-      item_of(it, b, tile);
-      const int p = b * dm.H + h;
-      const uint4* qsrc = reinterpret_cast<const uint4*>(
-          (const __nv_bfloat16*)a.q + ((size_t)b * dm.Hq + (size_t)h * kG) * kD);
-      const uint4 q0 = qsrc[lane], q1 = qsrc[lane + 32];
-      const int cid = cid0;
-      int e0 = 0, n = 0;
-      if (lane < kChunksPerTile && cid >= 0) {
-        if (e0r < 0 || e1r < e0r || e1r > dm.n_res || e1r - e0r > kChunk) {
-          raise_status(a.status, kStatusDeviceCheck);
-        } else {
-          e0 = e0r;
-          n = e1r - e0r;
-        }
-      }
-      const int32_t* ridx = ridx_all + (size_t)p * dm.n_res + e0;
-      int t[kChunk];
-#pragma unroll
-      for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
-      cid1 = sanitize(cid1);
-      load_span(it1, cid1, e0r, e1r);
-
       int got = 0;
       if (lane == 0)
         got = mbar_wait_bounded(bar(BAR_META_EMPTY0 + slot), ((i / kMetaSlots) & 1) ^ 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       TileMeta* M = meta + slot;
-      if (lane < kChunksPerTile) M->cid[lane] = cid;
-      int incl = n;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int off = incl - n;
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-      for (int j = 0; j < kChunk; ++j) {
-        if (j < n) {
-          const int tt = t[j] - cid * kChunk;
-          const bool good = tt >= 0 && tt < kChunk;
-          if (!good) raise_status(a.status, kStatusDeviceCheck);
-          M->res[off + j] = ((uint32_t)(e0 + j) << 8) | (good ? (uint32_t)(lane * kChunk + tt) : 255u);
+      if (it >= n_items) {   // no more tiles: post the end marker
+        if (lane == 0) {
+          M->item = -1;
+          mbar_arrive(bar(BAR_META_FULL0 + slot));
         }
+        break;
       }
-      if (lane == 0) {
-        M->nres = total;
-        M->item = it;
-      }
-      M->q[lane] = q0;
-      M->q[lane + 32] = q1;
+      int b, tile;
+      item_of(it, b, tile);
+      const int p = b * dm.H + h;
+      const int cid = cid0;
+      // first half of the slot: chunk ids, queries, item. The coefficient gather, the K~
+      // GEMM and part A need nothing else, so they start before the residual reads below.
+      if (lane < kChunksPerTile) M->cid[lane] = cid;
+      M->q[lane] = qa0;
+      M->q[lane + 32] = qb0;
+      if (lane == 0) M->item = it;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_META_FULL0 + slot));
       // chunk-base rotations (cos, sin)(C cid theta_i) of the tile's chunks: one 512-byte
@@ -477,9 +467,70 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         }
         rot_issued = i;
       }
-      // the chunk ids of tile i + 2, once tile i is posted (its pair may need a wait)
+      // issue: the take of tile i + 3, the residual rows of tile i (its spans arrived in
+      // the previous pass), the queries and spans of tile i + 1, the chunk ids of tile i + 2
+      const int tk3 = take_raw();
+      int e0 = 0, n = 0;
+      if (lane < kChunksPerTile && cid >= 0) {
+        if (e0r < 0 || e1r < e0r || e1r > dm.n_res || e1r - e0r > kChunk) {
+          raise_status(a.status, kStatusDeviceCheck);
+        } else {
+          e0 = e0r;
+          n = e1r - e0r;
+        }
+      }
+      const int32_t* ridx = ridx_all + (size_t)p * dm.n_res + e0;
+      int t[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) t[j] = j < n ? ridx[j] : 0;
+      load_q(it1, qa0, qb0);
+      cid1 = sanitize(cid1);
+      load_span(it1, cid1, e0r, e1r);
       int cid2 = -1;
       if (it2 < n_items && pair_ready(it2)) cid2 = load_cid(it2);
+      // second half of the slot: the tile's residual list for part B and, for bf16 rows,
+      // the rows themselves: each chunk's span (contiguous in res_val) is bulk-copied into
+      // the tile's row buffer once part B is done with that buffer's previous tile
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int off = incl - n;
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      const bool stage = dm.res_int4 == 0;
+      const int rb = i % kResBufs;
+      if (stage) {
+        int eg = 0;
+        if (lane == 0)
+          eg = mbar_wait_bounded(bar(BAR_RBUF_EMPTY0 + rb), ((i / kResBufs) & 1) ^ 1, abort_flag);
+        if (!__shfl_sync(0xffffffffu, eg, 0)) break;
+      }
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) {
+        if (j < n) {
+          const int tt = t[j] - cid * kChunk;
+          const bool good = tt >= 0 && tt < kChunk;
+          if (!good) raise_status(a.status, kStatusDeviceCheck);
+          M->res[off + j] = ((uint32_t)(e0 + j) << 8) | (good ? (uint32_t)(lane * kChunk + tt) : 255u);
+        }
+      }
+      const int nst = stage ? min(total, kResCap) : 0;
+      if (lane == 0) {
+        M->nres = total;
+        M->nstaged = nst;
+      }
+      __syncwarp();
+      const uint32_t rfull = bar(BAR_RES_FULL0 + slot);
+      if (lane == 0) mbar_arrive_expect_tx(rfull, (uint32_t)(nst * kD * 2));
+      __syncwarp();
+      const int ncp = stage ? max(0, min(n, kResCap - off)) : 0;   // this chunk's staged rows
+      if (ncp > 0)
+        bulk_load(smem_u32(gbase + L.rbuf) + (uint32_t)((rb * kResCap + off) * kD * 2),
+                  (const __nv_bfloat16*)a.res_val + ((size_t)p * dm.n_res + e0) * kD,
+                  (uint32_t)(ncp * kD * 2), rfull);
+      res_issued = i;
       // advance the pipeline
       it0 = it1;
       it1 = it2;
@@ -487,12 +538,19 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       cid0 = cid1;
       cid1 = cid2;
     }
-    // drain: rotation copies still in flight (only possible after an abort) land first
+    // drain: rotation and residual-row copies still in flight (only possible after an
+    // abort) land first
     if (lane == 0 && *abort_flag) {
       for (int t = rot_issued - kRotSlots + 1; t <= rot_issued; ++t) {
         if (t < 0) continue;
         int dummy = 0;
         mbar_wait_bounded(bar(BAR_ROT_FULL0 + t % kRotSlots), (uint32_t)((t / kRotSlots) & 1),
+                          (volatile int*)&dummy);
+      }
+      for (int t = res_issued - kResBufs + 1; t <= res_issued; ++t) {
+        if (t < 0) continue;
+        int dummy = 0;
+        mbar_wait_bounded(bar(BAR_RES_FULL0 + t % kMetaSlots), (uint32_t)((t / kMetaSlots) & 1),
                           (volatile int*)&dummy);
       }
     }
@@ -778,30 +836,10 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       float* part = a.part + ((size_t)p * a.n_tiles + tile) * kPartFloats;
       // first debug row of this tile (DBG only); a row is stored only if its chunk exists
       const size_t dbg_row0 = ((size_t)p * dm.k * kChunk + (size_t)tile * kTile);
-      // residual rows of the tile: thread = column j; rows split between the two halves.
-      // The first kResPrefetch of this thread's rows are loaded now, as raw bf16 bits:
-      // nothing waits for them until the residual sum after the hidden layer.
+      // residual rows of the tile: thread = column j, rows split between the two halves
       const int j = trow;
-      const int nres = M->nres;
       const __nv_bfloat16* rbase = rval_all + (size_t)p * dm.n_res * kD + j;
-      uint32_t pre_row[kResPrefetch / 4], pre_val[kResPrefetch / 2];
-#pragma unroll
-      for (int w = 0; w < kResPrefetch / 4; ++w) pre_row[w] = 0xFFFFFFFFu;
-#pragma unroll
-      for (int w = 0; w < kResPrefetch / 2; ++w) pre_val[w] = 0u;
-      const bool q4 = dm.res_int4 != 0;   // int4 rows: read in the loop after the sums
-#pragma unroll
-      for (int v = 0; v < kResPrefetch; ++v) {
-        const int ei = hf + 2 * v;
-        const uint32_t ent = (ei < nres && !q4) ? M->res[ei] : 255u;
-        const uint32_t row = ent & 255u;
-        pre_row[v >> 2] = (pre_row[v >> 2] & ~(255u << (8 * (v & 3)))) | (row << (8 * (v & 3)));
-        if (row != 255u) {
-          const uint32_t raw =
-              __ldg(reinterpret_cast<const unsigned short*>(rbase + (size_t)(ent >> 8) * kD));
-          pre_val[v >> 1] |= raw << (16 * (v & 1));
-        }
-      }
+      const bool q4 = dm.res_int4 != 0;   // int4 rows are read from global memory
       good = mbar_wait_bounded(bar(BAR_P_FULL0 + u), (i >> 1) & 1, abort_flag) && good;
       good = mbar_wait_bounded(bar(BAR_H_FULL), i & 1, abort_flag) && good;
       tc_fence_after();
@@ -818,6 +856,11 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
         float hv[32];
         tmem_ld_x32(tmem + lane_addr + 256u + (uint32_t)(hf * 128 + 32 * c), hv);
         tmem_wait_ld();
+        if (c == 3) {   // all of H^T is in registers: the next tile's hidden-layer GEMM may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
+        }
         if (ACT == LOWRAM_ACT_SILU) {
           // two tokens per step: hx = (h + b1)/2, silu = hx + hx tanh(hx)
           const float2 half2 = make_float2(0.5f, 0.5f);
@@ -850,9 +893,6 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_H_EMPTY));
       if (ACT == LOWRAM_ACT_SILU) {
         hacc01 = make_float2(acc2[0].x + acc2[0].y, acc2[1].x + acc2[1].y);
         hacc23 = make_float2(acc2[2].x + acc2[2].y, acc2[3].x + acc2[3].y);
@@ -862,32 +902,50 @@ attend_tc_kernel(const AttendArgs a, const __grid_constant__ TcMaps maps) {
       part[2 * kG + 2 * kF + f] = hacc23.x;
       part[2 * kG + 3 * kF + f] = hacc23.y;
 
+      // V~ = MLP + R on the residual rows: the list and (bf16) the rows, copied into the
+      // tile's row buffer by the metadata warp, are waited for only now
+      good = mbar_wait_bounded(bar(BAR_RES_FULL0 + slot), (i / kMetaSlots) & 1, abort_flag) && good;
+      const int nres = good ? M->nres : 0;
+      const int nst = good ? M->nstaged : 0;
+      const __nv_bfloat16* rstage = reinterpret_cast<const __nv_bfloat16*>(gbase + L.rbuf) +
+                                    (size_t)(i % kResBufs) * kResCap * kD + j;
       float racc[kG] = {0.f, 0.f, 0.f, 0.f};
+      // this half's entries ei = hf, hf + 2, ... in batches of four, whose loads are all
+      // issued before the sums (accumulated in entry order)
+      for (int e4 = hf; e4 < nres; e4 += 8) {
+        uint32_t ent[4];
 #pragma unroll
-      for (int v = 0; v < kResPrefetch; ++v) {
-        const uint32_t row = (pre_row[v >> 2] >> (8 * (v & 3))) & 255u;
-        if (row == 255u) continue;
-        const float4 pv = P4[row];
-        const float r = __uint_as_float(((pre_val[v >> 1] >> (16 * (v & 1))) & 0xFFFFu) << 16);
-        if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r;
-        racc[0] = fmaf(pv.x, r, racc[0]);
-        racc[1] = fmaf(pv.y, r, racc[1]);
-        racc[2] = fmaf(pv.z, r, racc[2]);
-        racc[3] = fmaf(pv.w, r, racc[3]);
+        for (int k2 = 0; k2 < 4; ++k2) ent[k2] = e4 + 2 * k2 < nres ? M->res[e4 + 2 * k2] : 255u;
+        float r[4];
+        float4 pv[4];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const int ei = e4 + 2 * k2;
+          const uint32_t row = ent[k2] & 255u;
+          r[k2] = 0.f;
+          pv[k2] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (row != 255u) {
+            r[k2] = q4 ? int4_residual((const uint8_t*)a.res_val, (const __half*)a.res_scale, dm,
+                                       (size_t)p * dm.n_res + (ent[k2] >> 8), j)
+                       : __bfloat162float(ei < nst ? rstage[(size_t)ei * kD]
+                                                   : rbase[(size_t)(ent[k2] >> 8) * kD]);
+            pv[k2] = P4[row];
+          }
+        }
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          const uint32_t row = ent[k2] & 255u;
+          if (row == 255u) continue;
+          if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r[k2];
+          racc[0] = fmaf(pv[k2].x, r[k2], racc[0]);
+          racc[1] = fmaf(pv[k2].y, r[k2], racc[1]);
+          racc[2] = fmaf(pv[k2].z, r[k2], racc[2]);
+          racc[3] = fmaf(pv[k2].w, r[k2], racc[3]);
+        }
       }
-      for (int ei = hf + (q4 ? 0 : 2 * kResPrefetch); ei < nres; ei += 2) {   // beyond the prefetch
-        const uint32_t ent = M->res[ei];
-        const int row = (int)(ent & 255u);
-        if (row == 255) continue;
-        const float r = q4 ? int4_residual((const uint8_t*)a.res_val, (const __half*)a.res_scale,
-                                           dm, (size_t)p * dm.n_res + (ent >> 8), j)
-                           : __bfloat162float(rbase[(size_t)(ent >> 8) * kD]);
-        if constexpr (DBG) a.dbg_v[(dbg_row0 + row) * kD + j] = r;
-        const float4 pv = P4[row];
-        racc[0] = fmaf(pv.x, r, racc[0]);
-        racc[1] = fmaf(pv.y, r, racc[1]);
-        racc[2] = fmaf(pv.z, r, racc[2]);
-        racc[3] = fmaf(pv.w, r, racc[3]);
+      if (!q4) {   // the row buffer may take tile i + kResBufs
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_RBUF_EMPTY0 + i % kResBufs));
       }
       float* pr = part + 2 * kG + kG * kF + (size_t)hf * kG * kD;
 #pragma unroll

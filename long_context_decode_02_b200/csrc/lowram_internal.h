@@ -187,9 +187,11 @@ cudaError_t launch_encode_predict_tc(const EncodeArgs& a, const float* c_ws, boo
                                      int num_sms, cudaStream_t s);
 
 // 2D tiled TMA map over a row-major [rows][cols] array of dtype (LOWRAM_DTYPE_*), box
-// box_rows x box_cols, swizzle 0/32/64/128 bytes. False if the driver refuses it.
+// box_rows x box_cols, swizzle 0/32/64/128 bytes; L2 fetches promoted to l2_promo bytes
+// (128 or 256). False if the driver refuses it.
 bool make_tensor_map_2d(CUtensorMap* m, const void* ptr, int dtype, uint64_t cols,
-                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
+                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes,
+                        int l2_promo = 128);
 
 // Read-only access to a context's configuration and device.
 const lowram_config* ctx_config(const lowram_ctx* ctx);

@@ -1012,7 +1012,8 @@ cudaError_t launch_typed(const SelectArgs& a, int num_sms, cudaStream_t s) {
   using Gm = Geom<T, D>;
   CUtensorMap map;
   if (!make_tensor_map_2d(&map, a.landmark, a.dm.dtype, (uint64_t)D,
-                          (uint64_t)a.dm.B * a.dm.H * a.dm.Nc, Gm::kBoxCols, Gm::kLps, 128))
+                          (uint64_t)a.dm.B * a.dm.H * a.dm.Nc, Gm::kBoxCols, Gm::kLps, 128,
+                          256))
     return cudaErrorInvalidValue;
   const SelSmem L = sel_smem(G, D);
   if (L.total > (uint32_t)kSmemLimit) return cudaErrorInvalidValue;

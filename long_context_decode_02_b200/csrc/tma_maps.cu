@@ -28,7 +28,8 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 bool make_tensor_map_2d(CUtensorMap* m, const void* ptr, int dtype, uint64_t cols,
-                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
+                        uint64_t rows, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes,
+                        int l2_promo) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const size_t es = dtype == LOWRAM_DTYPE_BF16 ? 2 : 4;
@@ -43,7 +44,8 @@ bool make_tensor_map_2d(CUtensorMap* m, const void* ptr, int dtype, uint64_t col
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            l2_promo == 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
