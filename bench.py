@@ -435,7 +435,8 @@ def run_ours(args):
     hbm_gbs = step_bytes / (ms_step_max / 1e3) / 1e9
 
     traffic = measured_traffic("score_select_kernel")
-    traffic_b = measured_traffic("attend_tc_kernel")
+    t_att, t_comb = measured_traffic("attend_tc_kernel"), measured_traffic("combine_reorder_kernel")
+    traffic_b = t_att + t_comb if t_att is not None and t_comb is not None else None
 
     ach_a = bytes_a / (ms_a_max / 1e3) / 1e9
     ach_b = bytes_b / (ms_b_max / 1e3) / 1e9
