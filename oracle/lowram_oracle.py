@@ -27,6 +27,9 @@ the plainest reading of the prose):
            predictor fitted at test time, residuals only for the tokens it
            reconstructs worst, reconstruction of a selected subset of KV pairs at each
            decoding step.
+[summary]  the agihunt.info summary, its composition paragraph (quantised residuals,
+           eviction) and its limitations paragraph (long generation: the generated
+           suffix kept dense and compressed periodically).
 
 Readings taken where the pages are silent (each is listed, with its reason, in the
 design notes of the repository):
@@ -51,6 +54,10 @@ design notes of the repository):
   -8, 7). Composition with eviction (LowRAM-E/EQ): per batch element, the chunks with
   the smallest all-head landmark norm are evicted before compression; the kept chunks
   keep their original RoPE positions.
+- Periodic re-compression of the generated suffix: a block of whole chunks is
+  compressed like a prefix (same basis and predictor, RoPE inverted at its true
+  positions, its own residual budget chosen within the block) and appended after the
+  compressed prefix, whose arrays are left as they are.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against something other
 than itself (closed forms, brute force, invariants, library routines); none is
@@ -392,6 +399,60 @@ def encode(k_cache, v, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act, store
            "res_idx": res_idx, "res_val": res_val, "chunk_ptr": chunk_ptr, "err": err}
     if res_format == "int4":
         out["res_q"], out["res_scale"] = res_q, res_scale
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# periodic re-compression of the generated suffix [summary, limitations paragraph]
+# ----------------------------------------------------------------------------------
+def encode_block(k_block, v_block, basis, w1, b1, w2, b2, *, chunk, n_res, theta, act,
+                 store, first_position, res_format="store"):
+    """Compression of a block of whole chunks of generated tokens that sits after the
+    compressed prefix: encode() of the block with the same basis and predictor, RoPE
+    inverted at the tokens' true positions first_position .. first_position + T_b - 1.
+
+    Reading: the pages name the periodic compression of the generated suffix and leave
+    its steps open; the plainest reading keeps every step of encode() and its residual
+    budget, applied within the block (n_res of its own largest-error tokens), and leaves
+    the compressed prefix as it is (no re-selection of its residuals).
+    """
+    k_block = np.asarray(k_block, np.float64)
+    B, Tb = k_block.shape[:2]
+    pos = np.broadcast_to(first_position + np.arange(Tb), (B, Tb))
+    return encode(k_block, v_block, basis, w1, b1, w2, b2, chunk=chunk, n_res=n_res,
+                  theta=theta, act=act, store=store, positions=pos, res_format=res_format)
+
+
+def append_block(prefix, block, *, prefix_tokens, chunk, block_first_chunk):
+    """The compressed cache of prefix + block: every per-token and per-chunk array of the
+    block follows the prefix's (coefficients, landmarks, errors), the block's residual
+    rows follow the prefix's rows of each (batch, head) with their token indices moved by
+    prefix_tokens, and the block's CSR offsets by the prefix's row count. When either
+    part holds chunk positions (eviction), the result holds them for every chunk (the
+    prefix's own, or 0 .. N_c-1; the block's chunks at block_first_chunk + i).
+    """
+    Np = prefix["landmark"].shape[2]
+    Nb = block["landmark"].shape[2]
+    B = prefix["coef"].shape[0]
+    n_res_p = prefix["res_idx"].shape[2]
+    out = {
+        "coef": np.concatenate([prefix["coef"], block["coef"]], axis=1),
+        "coef_exact": np.concatenate([prefix["coef_exact"], block["coef_exact"]], axis=1),
+        "landmark": np.concatenate([prefix["landmark"], block["landmark"]], axis=2),
+        "err": np.concatenate([prefix["err"], block["err"]], axis=2),
+        "res_idx": np.concatenate([prefix["res_idx"], block["res_idx"] + prefix_tokens], axis=2),
+        "res_val": np.concatenate([prefix["res_val"], block["res_val"]], axis=2),
+        "chunk_ptr": np.concatenate([prefix["chunk_ptr"][:, :, :Np],
+                                     block["chunk_ptr"] + n_res_p], axis=2),
+    }
+    for key in ("res_q", "res_scale"):
+        if key in prefix:
+            out[key] = np.concatenate([prefix[key], block[key]], axis=2)
+    if prefix.get("chunk_pos") is not None or block_first_chunk != Np:
+        pp = prefix.get("chunk_pos")
+        pp = np.broadcast_to(np.arange(Np), (B, Np)) if pp is None else np.asarray(pp)
+        out["chunk_pos"] = np.concatenate(
+            [pp, np.broadcast_to(block_first_chunk + np.arange(Nb), (B, Nb))], axis=1)
     return out
 
 

@@ -456,12 +456,92 @@ def check_suffix_decode(M):
     assert np.allclose(a, b_, atol=1e-14)
 
 
+def _block_errors_brute(k_block, v_block, basis, w, first, theta, act, h):
+    """Squared predictor errors of a block's tokens for head h, written out per token
+    with RoPE undone through complex numbers (pairs (i, i + d/2) as x + iy)."""
+    w1, b1, w2, b2 = w
+    B, Tb, H, d = k_block.shape
+    half = d // 2
+    inv = theta ** (-2.0 * np.arange(half) / d)
+    out = np.empty((B, Tb))
+    for b in range(B):
+        for t in range(Tb):
+            rows = []
+            for hh in range(H):
+                z = (k_block[b, t, hh, :half] + 1j * k_block[b, t, hh, half:]) * np.exp(
+                    -1j * (first + t) * inv)
+                rows.append(np.concatenate([z.real, z.imag]))
+            c = basis.T @ np.concatenate(rows)
+            x = basis[h * d:(h + 1) * d] @ c
+            pre = w1[h] @ x + b1[h]
+            a = pre / (1.0 + np.exp(-pre)) if act == O.ACT_SILU else 0.5 * pre * (
+                1.0 + np.vectorize(math.erf)(pre / math.sqrt(2.0)))
+            vh = w2[h] @ a + b2[h]
+            out[b, t] = float(((v_block[b, t, h] - vh) ** 2).sum())
+    return out
+
+
+def check_block_append(M):
+    """Periodic re-compression: a block of whole chunks compressed at its true positions
+    and appended after the compressed prefix. (1) Full rank, every token a residual and
+    every chunk selected: decode equals dense attention over prefix and block together,
+    also after eviction of half the prefix's chunks. (2) The block's residual rows are
+    its own largest-error tokens (errors written out per token), moved past the prefix's
+    rows; the CSR counts each chunk's rows."""
+    sh = tiny_shape(rank=16, n_kv_heads=2, head_dim=8, res_frac=1.0, top_k=10 ** 6)
+    L = make_layer(sh)
+    kw = dict(chunk=sh.chunk, theta=sh.theta, act=sh.act)
+    T0 = 48
+    pre = M.encode(L["k"][:, :T0], L["v"][:, :T0], L["basis"], *L["w"], n_res=T0,
+                   store=M.STORE_F64, **kw)
+    blk = M.encode_block(L["k"][:, T0:], L["v"][:, T0:], L["basis"], *L["w"],
+                         n_res=sh.n_tokens - T0, store=M.STORE_F64, first_position=T0, **kw)
+    cat = M.append_block(pre, blk, prefix_tokens=T0, chunk=sh.chunk,
+                         block_first_chunk=T0 // sh.chunk)
+    assert cat.get("chunk_pos") is None
+    out, _ = M.decode_step(L["q"], cat, L["basis"], *L["w"], top_k=sh.top_k, **kw)
+    assert np.allclose(out, M.dense_attention(L["q"], L["k"], L["v"]), atol=1e-12)
+    # an evicted prefix (half its chunks kept) followed by the block
+    ev = M.encode_evicted(L["k"][:, :T0], L["v"][:, :T0], L["basis"], *L["w"], keep_frac=0.5,
+                          res_frac=1.0, store=M.STORE_F64, **kw)
+    cat2 = M.append_block(ev, blk, prefix_tokens=T0 // 2, chunk=sh.chunk,
+                          block_first_chunk=T0 // sh.chunk)
+    rows = (ev["chunk_pos"][:, :, None] * sh.chunk + np.arange(sh.chunk)).reshape(sh.batch, -1)
+    kk = np.stack([np.concatenate([L["k"][b, rows[b]], L["k"][b, T0:]]) for b in range(sh.batch)])
+    vv = np.stack([np.concatenate([L["v"][b, rows[b]], L["v"][b, T0:]]) for b in range(sh.batch)])
+    out2, _ = M.decode_step(L["q"], cat2, L["basis"], *L["w"], top_k=sh.top_k, **kw)
+    assert np.allclose(out2, M.dense_attention(L["q"], kk, vv), atol=1e-12)
+    # (2) a quarter of each part's tokens residual
+    sh2 = tiny_shape(res_frac=0.25, rank=6, top_k=5)
+    L2 = make_layer(sh2)
+    kw2 = dict(chunk=sh2.chunk, theta=sh2.theta, act=sh2.act)
+    nb = (sh2.n_tokens - T0) // 4
+    pre2 = M.encode(L2["k"][:, :T0], L2["v"][:, :T0], L2["basis"], *L2["w"], n_res=T0 // 4,
+                    store=M.STORE_F32, **kw2)
+    blk2 = M.encode_block(L2["k"][:, T0:], L2["v"][:, T0:], L2["basis"], *L2["w"], n_res=nb,
+                          store=M.STORE_F32, first_position=T0, **kw2)
+    cat3 = M.append_block(pre2, blk2, prefix_tokens=T0, chunk=sh2.chunk,
+                          block_first_chunk=T0 // sh2.chunk)
+    for h in range(sh2.n_kv_heads):
+        e = _block_errors_brute(L2["k"][:, T0:], L2["v"][:, T0:], L2["basis"], L2["w"], T0,
+                                sh2.theta, sh2.act, h)
+        for b in range(sh2.batch):
+            want = np.sort(np.argsort(-e[b], kind="stable")[:nb]) + T0
+            assert np.array_equal(cat3["res_idx"][b, h, T0 // 4:], want)
+            assert np.array_equal(cat3["res_idx"][b, h, :T0 // 4], pre2["res_idx"][b, h])
+            counts = np.bincount(cat3["res_idx"][b, h] // sh2.chunk,
+                                 minlength=sh2.n_tokens // sh2.chunk)
+            assert np.array_equal(np.diff(cat3["chunk_ptr"][b, h]), counts)
+            assert cat3["chunk_ptr"][b, h, 0] == 0
+    assert np.array_equal(cat3["res_val"][:, :, T0 // 4:], blk2["res_val"])
+
+
 ALL_CHECKS = [check_rope_closed_form, check_rope_group_properties, check_projection,
               check_landmarks_and_scores, check_encode_landmarks, check_topk, check_predictor,
               check_full_rank_exactness, check_residual_pick, check_selection_and_edges,
               check_cholesky_qr, check_fit_basis, check_fit_basis_recovers_generator,
               check_int4_quantize, check_eviction, check_evicted_full_rank_exactness,
-              check_int4_residual_encode, check_suffix_decode]
+              check_int4_residual_encode, check_suffix_decode, check_block_append]
 
 
 @pytest.mark.parametrize("check", ALL_CHECKS, ids=lambda f: f.__name__)
@@ -658,3 +738,35 @@ def test_mutation_suffix_softmax_separate(monkeypatch):
             return a, sel
         return 0.5 * (a + O.dense_attention(q, ks, vs)), sel
     _fails(check_suffix_decode, monkeypatch, "decode_step_with_suffix", bad)
+
+
+def test_mutation_block_indices_not_moved(monkeypatch):
+    """The block's residual token indices appended without moving them past the prefix."""
+    orig = O.append_block
+
+    def bad(prefix, block, *, prefix_tokens, chunk, block_first_chunk):
+        return orig(prefix, block, prefix_tokens=0, chunk=chunk,
+                    block_first_chunk=block_first_chunk)
+    _fails(check_block_append, monkeypatch, "append_block", bad)
+
+
+def test_mutation_block_positions_from_zero(monkeypatch):
+    """The block compressed as if it started at position 0."""
+    orig = O.encode_block
+
+    def bad(*args, first_position, **kw):
+        return orig(*args, first_position=0, **kw)
+    _fails(check_block_append, monkeypatch, "encode_block", bad)
+
+
+def test_mutation_block_csr_not_moved(monkeypatch):
+    """The block's CSR offsets appended without the prefix's row count."""
+    orig = O.append_block
+
+    def bad(prefix, block, **kw):
+        out = orig(prefix, block, **kw)
+        Np = prefix["landmark"].shape[2]
+        out["chunk_ptr"] = np.concatenate([prefix["chunk_ptr"][:, :, :Np], block["chunk_ptr"]],
+                                          axis=2)
+        return out
+    _fails(check_block_append, monkeypatch, "append_block", bad)
