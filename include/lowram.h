@@ -256,6 +256,34 @@ lowram_status lowram_decode_step_suffix(lowram_ctx* ctx, const lowram_cache* cac
 lowram_status lowram_suffix_workspace_size(const lowram_config* cfg, int32_t s_max,
                                            size_t* bytes);
 
+/* Periodic re-compression of the generated suffix (agihunt summary, limitations
+ * paragraph: long generation keeps the generated suffix dense and compresses it
+ * periodically). A block of whole chunks of generated tokens is compressed with
+ * lowram_encode under its own context (same basis and predictor; configuration
+ * n_tokens = the block's tokens, n_positions > n_tokens, and cache->chunk_pos = the
+ * block's chunk positions, so RoPE is inverted at the tokens' true positions; its own
+ * n_res residual rows chosen within the block). lowram_append then writes into `dst` the
+ * cache of the prefix followed by the block:
+ *   coef, landmark: the prefix's tokens / chunks, then the block's;
+ *   res_idx, res_val, res_scale: per (b, h) the prefix's n_res_p rows, then the block's
+ *   (token indices moved by the prefix's n_tokens);
+ *   chunk_ptr: the prefix's offsets, then the block's moved by n_res_p;
+ *   landmark_norm: the larger of the two bounds;
+ *   chunk_pos (written when dst's configuration has n_positions > n_tokens): the
+ *   prefix's (0, 1, ... when it has none), then the block's.
+ * When dst has no chunk_pos, the block's chunk_pos must be N_p, N_p + 1, ... (N_p the
+ * prefix's chunk count): checked on the device, LOWRAM_ERR_DEVICE_CHECK through
+ * lowram_last_error(dst_ctx) otherwise, the copies still made.
+ * The three configurations must agree in batch, heads, head_dim, rank, chunk,
+ * mlp_hidden, act, dtype and res_format, with dst n_tokens = prefix n_tokens + block
+ * n_tokens and dst n_res = prefix n_res + block n_res (LOWRAM_ERR_SHAPE otherwise).
+ * dst must not overlap the sources. coef, landmark and res_val of all three 16-byte
+ * aligned. Asynchronous on `stream`; no workspace. */
+lowram_status lowram_append(lowram_ctx* dst_ctx, const lowram_cache* dst,
+                            const lowram_ctx* prefix_ctx, const lowram_cache* prefix,
+                            const lowram_ctx* block_ctx, const lowram_cache* block,
+                            void* stream);
+
 /* Decode sub-step 1 (kernel (a) alone): score every chunk by max over the GQA group of
  * q . landmark and write the top-k chunks per (batch, KV head), ascending, ties to the
  * lower chunk (agihunt summary, key paragraph; cctest "Selective reconstruction").

@@ -621,6 +621,52 @@ lowram_status lowram_evict(lowram_ctx* ctx, const void* k_full, const void* v_fu
   return LOWRAM_OK;
 }
 
+lowram_status lowram_append(lowram_ctx* dst_ctx, const lowram_cache* dst,
+                            const lowram_ctx* prefix_ctx, const lowram_cache* prefix,
+                            const lowram_ctx* block_ctx, const lowram_cache* block,
+                            void* stream) {
+  if (!dst_ctx || !dst || !prefix_ctx || !prefix || !block_ctx || !block)
+    return LOWRAM_ERR_INVALID_ARG;
+  const lowram_config &cd = dst_ctx->cfg, &cp = prefix_ctx->cfg, &cb = block_ctx->cfg;
+  auto same = [](const lowram_config& x, const lowram_config& y) {
+    return x.batch == y.batch && x.n_kv_heads == y.n_kv_heads && x.n_q_heads == y.n_q_heads &&
+           x.head_dim == y.head_dim && x.rank == y.rank && x.chunk == y.chunk &&
+           x.mlp_hidden == y.mlp_hidden && x.act == y.act && x.dtype == y.dtype &&
+           x.res_format == y.res_format;
+  };
+  if (!same(cd, cp) || !same(cd, cb)) return LOWRAM_ERR_SHAPE;
+  if (cd.n_tokens != cp.n_tokens + cb.n_tokens || cd.n_res != cp.n_res + cb.n_res)
+    return LOWRAM_ERR_SHAPE;
+  // the block carries its chunks' positions; a result that keeps positions must cover them
+  if (!evicted(cb)) return LOWRAM_ERR_SHAPE;
+  if (evicted(cd) && cd.n_positions < cb.n_positions) return LOWRAM_ERR_SHAPE;
+  lowram_status st;
+  if ((st = check_cache(dst, cd)) != LOWRAM_OK) return st;
+  if ((st = check_cache(prefix, cp)) != LOWRAM_OK) return st;
+  if ((st = check_cache(block, cb)) != LOWRAM_OK) return st;
+  if (prefix_ctx->device != dst_ctx->device || block_ctx->device != dst_ctx->device)
+    return LOWRAM_ERR_INVALID_ARG;
+  auto view = [](const lowram_cache* c, const lowram_config& cfg) {
+    return CacheView{c->coef, c->landmark, c->res_idx, c->res_val, c->chunk_ptr,
+                     c->landmark_norm, const_cast<int32_t*>(chunk_pos_of(c, cfg)),
+                     const_cast<void*>(res_scale_of(c, cfg))};
+  };
+  AppendArgs a{};
+  a.pre = dims_of(cp);
+  a.blk = dims_of(cb);
+  a.prefix = view(prefix, cp);
+  a.block = view(block, cb);
+  a.dst = view(dst, cd);
+  a.status = dst_ctx->status;
+  DeviceGuard g(dst_ctx->device);
+  if (!g.ok) return LOWRAM_ERR_CUDA;
+  if (launch_append(a, dst_ctx->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return LOWRAM_ERR_CUDA;
+  }
+  return LOWRAM_OK;
+}
+
 lowram_status lowram_fit_basis_workspace_size(const lowram_config* c, int32_t l, size_t* bytes) {
   if (!bytes) return LOWRAM_ERR_INVALID_ARG;
   const lowram_status st = lowram_check_config(c);

@@ -186,6 +186,24 @@ cudaError_t launch_encode_project_tc(const EncodeArgs& a, void* basis_t, float* 
 cudaError_t launch_encode_predict_tc(const EncodeArgs& a, const float* c_ws, bool residual_rows,
                                      int num_sms, cudaStream_t s);
 
+// ---------------- periodic re-compression: a compressed block appended ----------------
+struct CacheView {   // one cache's arrays (chunk_pos / res_scale null when absent)
+  void* coef;
+  void* landmark;
+  int32_t* res_idx;
+  void* res_val;
+  int32_t* chunk_ptr;
+  float* landmark_norm;
+  int32_t* chunk_pos;
+  void* res_scale;
+};
+struct AppendArgs {
+  Dims pre, blk;     // the prefix's and the block's dimensions
+  CacheView prefix, block, dst;
+  int* status;
+};
+cudaError_t launch_append(const AppendArgs& a, int num_sms, cudaStream_t s);
+
 // 2D tiled TMA map over a row-major [rows][cols] array of dtype (LOWRAM_DTYPE_*), box
 // box_rows x box_cols, swizzle 0/32/64/128 bytes; L2 fetches promoted to l2_promo bytes
 // (128 or 256). False if the driver refuses it.

@@ -97,6 +97,8 @@ _sig = {
     "lowram_debug_tc_tile": (_S, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P]),
     "lowram_dense_decode": (_S, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "lowram_evict": (_S, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "lowram_append": (_S, [_P, ctypes.POINTER(lowram_cache), _P, ctypes.POINTER(lowram_cache),
+                           _P, ctypes.POINTER(lowram_cache), _P]),
     "lowram_decode_step_suffix": (_S, [_P, ctypes.POINTER(lowram_cache),
                                        ctypes.POINTER(lowram_layer_params), _P, _P, _P,
                                        ctypes.c_int32, ctypes.c_int32, _P, _P, _P,
@@ -335,6 +337,15 @@ def evict(ctx: Context, k_full, v_full, k_kept, v_kept, chunk_pos, workspace, st
                        _ptr(chunk_pos), _ptr(workspace),
                        workspace.numel() * workspace.element_size(), _stream(stream)),
           "lowram_evict")
+
+
+def append(dst_ctx: Context, dst: dict, prefix_ctx: Context, prefix: dict, block_ctx: Context,
+           block: dict, stream=None) -> None:
+    """lowram_append: the cache of a compressed prefix followed by a compressed block of
+    generated tokens (periodic re-compression of the suffix)."""
+    cd, cp, cb = cache_struct(**dst), cache_struct(**prefix), cache_struct(**block)
+    check(lowram_append(dst_ctx.handle, ctypes.byref(cd), prefix_ctx.handle, ctypes.byref(cp),
+                        block_ctx.handle, ctypes.byref(cb), _stream(stream)), "lowram_append")
 
 
 def fit_basis_workspace_size(cfg: lowram_config, l: int) -> int:
