@@ -12,24 +12,26 @@
 // with h_t = act(W1 K~_pre,t + b1): W2 is applied once per query head in the combine
 // kernel instead of once per token, removing a third of the tensor work.
 //
-// Per persistent CTA (one KV head h; weights B_h and W1_h stay in shared memory), per
-// tile of 128 selected tokens (16 chunks of 8):
-//   producer warp : TMA-gathers the 16 chunks' coefficient rows (each chunk is a
-//                   contiguous 8 x r block) into a 64B-swizzled K-major tile.
-//   MMA warp      : K~_pre^T... as D[tok][d] = coef[tok][r] . B_h[d][r]^T   -> TMEM
-//                   H^T  as D[f][tok] = W1[f][d] . K~bf16[tok][d]^T (2 x M=128) -> TMEM
-//   8 epilogue warps (two per TMEM lane quadrant):
-//     A: K~_pre rows from TMEM -> bf16 into shared memory (operand of the H GEMM);
-//        RoPE from host-fp64 tables; logits for the 4 query heads; tile max and
-//        p = 2^(z - m) in fp32 -> shared memory.
-//     B: H^T rows from TMEM (lane = hidden unit f, columns = tokens): act(h + b1) and
-//        Hacc_g[f] += p_g(t) act  (a reduction along each thread's own row);
-//        residual rows of the tile's chunks (CSR spans): Racc_g[j] += p_g(t) R_t[j].
-//     The tile's (m, l, Hacc, Racc) go to a split-K partial; the combine kernel merges
-//     the tiles and applies W2 and b2.
-// The epilogue interleaves A(i+1) before B(i) so the H GEMM of tile i runs under the
-// CUDA-core work of tile i+1; TMEM holds two K~ buffers (2 x 128 columns) and H^T
-// (256 columns). Rebuilt keys and values never leave the SM.
+// Per persistent CTA (one KV head h), per tile of 128 selected tokens (16 chunks of 8),
+// 20 warps:
+//   warp 0 (TMA)      : B_h once; each tile's 16 chunks' coefficient rows into one of
+//                       two coefficient buffers (the next tile's gather under this one).
+//   warp 1 (MMA)      : K~_pre as D[tok][d] = coef[tok][r] . B_h[d][r]^T -> TMEM.
+//   warp 2 (metadata) : the tile's chunk ids and queries, then its residual list, and
+//                       the bulk copies of its chunk-base rotations and bf16 residual rows.
+//   warps 3-10 (A)    : K~_pre from TMEM -> bf16 shared memory (the hidden GEMM's
+//                       operand); RoPE; logits of the 4 query heads; tile max and
+//                       p = 2^(z - m).
+//   warp 19 (MMA)     : H^T as D[f][tok] = W1_h[f][d] . K~bf16[tok][d]^T (2 x M = 128),
+//                       W1_h held in TMEM.
+//   warps 11-18 (B)   : H^T from TMEM (lane = hidden unit f, columns = tokens):
+//                       act(h + b1) and Hacc_g[f] += p_g(t) act, a reduction along each
+//                       thread's own row; then the tile's residual rows from the staged
+//                       row buffer: Racc_g[j] += p_g(t) R_t[j].
+//   The tile's (m, l, Hacc, Racc) go to a split-K partial; the combine kernel merges the
+//   tiles and applies W2 and b2. Parts A and B run on their own warps at the same time,
+//   A one tile ahead; TMEM holds K~ (128 columns), W1_h (128) and H^T (256). Rebuilt keys
+//   and values never leave the SM.
 // Every wait is bounded (~2 s); on expiry the kernel raises a timeout status, drains its
 // own outstanding copies and MMAs (again bounded), frees TMEM and returns.
 #include <cuda.h>
