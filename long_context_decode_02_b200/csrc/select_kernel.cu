@@ -19,9 +19,11 @@
 //    is its own completion flag: no counters or memory fences on the streaming path.
 //    Three selection warps per CTA take (b, h) pairs in order from a global counter,
 //    wait until the work counter has handed out all of the pair's stages and every score
-//    has landed, select, set the pair's ready flag and put the sentinel back. Selections are spread over the CTAs
-//    and overlap the stream; a selection group only waits for stages held by running
-//    CTAs, and every wait is bounded.
+//    has landed, select, set the pair's readiness bit and put the sentinel back.
+//    Selections are spread over the CTAs and overlap the stream; a selection group only
+//    waits for stages held by running CTAs, and every wait is bounded. Pairs whose
+//    scoring ends in the last wave of stages are selected by the whole CTA once its
+//    stream is done.
 //  * Selection: the 16-bit key prefix of the j-th largest of 1024 evenly spaced scores
 //    gives a threshold t0; every score >= t0 is a candidate; three radix passes find the
 //    24-bit prefix bucket [tau_lo, tau_hi] holding the k-th largest candidate.
@@ -31,8 +33,8 @@
 //    D terms accumulated with fused multiply-adds is within gamma_D * sum|q_i L_i| <=
 //    gamma_D * |q|_2 |L|_2 of the exact value (gamma_n = n u / (1 - n u), u = 2^-24), with
 //    |L|_2 bounded by the cache's per-pair landmark norm. So the result equals the
-//    selection made in fp64, and the window usually holds exactly the
-//    rows still needed, which then need no re-scoring. When the candidate set cannot be proven to
+//    selection made in fp64, and the window usually holds exactly the rows still
+//    needed, which then need no re-scoring. When the candidate set cannot be proven to
 //    hold the answer, a radix select over all scores decides instead. The chunk ids are
 //    written in ascending order.
 #include <cuda_bf16.h>
@@ -47,7 +49,11 @@ using namespace sm100;
 
 constexpr int kConsumers = 256;               // consumer threads (warps 0..7)
 constexpr int kSelectors = 96;                // selection threads (warps 9..11)
-constexpr int kLateWaves = 10;                // stages per CTA that count as the last wave
+// stages per CTA that count as the last wave: more for long pairs, whose selections
+// beside the stream are slow (measured: 10 best at N_c 16384, 16 at N_c 32768)
+constexpr int kLateWaves = 10;
+constexpr int kLateWavesLong = 16;
+constexpr int kLongPair = 16384;              // N_c above which kLateWavesLong applies
 constexpr int kJoinBar = 3;                   // named barrier of the joint selection group
 constexpr int kSelThreads = kConsumers + 32 + kSelectors;  // + producer warp 8
 constexpr int kStages = 3;
@@ -937,14 +943,15 @@ score_select_kernel(const SelectArgs a, const __grid_constant__ CUtensorMap lmap
     // The selection warps take the next (b, h), wait until all of its stages are handed
     // out and all of its scores have landed, select, and restore the sentinel; one
     // verdict per step for the whole group keeps its barrier sequence uniform. A pair
-    // whose scoring ends in the last wave of stages (about the last kLateWaves stages of
+    // whose scoring ends in the last wave of stages (about the last `waves` stages of
     // every CTA) is not selected by these three warps: it is handed over, claimed, to the
     // consumers and the selection warps together (all but the producer), who meet once
     // the consumers have no stages left and select it several times faster right when
     // its last scores land, then any pairs still in the queue. The selection warps also
     // hand over (with no pair) when the queue is empty, so the meeting always happens.
     const bool sel_warp = warp > kConsumers / 32;
-    const long long late_from = (long long)U - (long long)kLateWaves * gridDim.x;
+    const int waves = Nc > kLongPair ? kLateWavesLong : kLateWaves;
+    const long long late_from = (long long)U - (long long)waves * gridDim.x;
     bool joined = !sel_warp;
     if (!sel_warp) named_bar_sync(kJoinBar, kConsumers + kSelectors);
     for (;;) {
