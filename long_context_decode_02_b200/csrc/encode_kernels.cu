@@ -228,7 +228,9 @@ constexpr int kNB = 32;   // candidates per pass
 template <typename T>
 __device__ __forceinline__ double ld64(const T* p, size_t i) { return (double)to_f(p[i]); }
 
-template <typename T, int D, int FH>
+// MC: 32-column blocks of c per lane, ceil(r / 32) when it is known at compile time (the
+// projection loop then runs no predicated-off blocks), 8 for any r <= 256 otherwise.
+template <typename T, int D, int FH, int MC>
 __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const EncodeArgs a) {
   const Dims& dm = a.dm;
   const int p = blockIdx.y, b = p / dm.H, h = p % dm.H, tid = threadIdx.x;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
     if (tid < kNB) s_tok[tid] = tid < nb ? a.cand_idx[(size_t)p * dm.T + j0 + tid] : -1;
     __syncthreads();
     // ---- c[cand][kk] = sum over heads hh, dims i of kpre[cand][hh d + i] basis[hh d + i][kk]
-    constexpr int kMaxC = 8;   // columns per lane: r <= 256
+    constexpr int kMaxC = MC;   // columns per lane
     double acc[4][kMaxC];
 #pragma unroll
     for (int x = 0; x < 4; ++x)
@@ -512,7 +514,9 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
   {
     const int wc = dm.r > FH ? dm.r : FH;
     const size_t smem = sizeof(double) * ((size_t)kNB * D + (size_t)kNB * wc) + 65536;
-    auto kern = residual_rescore_kernel<T, D, FH>;
+    auto kern = dm.r == 160   ? residual_rescore_kernel<T, D, FH, 5>
+                : dm.r == 128 ? residual_rescore_kernel<T, D, FH, 4>
+                              : residual_rescore_kernel<T, D, FH, 8>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)smem)) != cudaSuccess) return e;
     kern<<<dim3(kRescoreCtas, dm.B * dm.H), kEncThreads, smem, s>>>(a);
