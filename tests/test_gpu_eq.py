@@ -225,3 +225,63 @@ def test_end_to_end_eq_against_oracle_pipeline(L, eq_cache):
         want, _ = O.decode_step(H.f64(q), enc, p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
                                 chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta, act=sh.act)
         assert H.rel_err(H.f64(out), want) <= H.TOL["bf16"]
+
+
+def test_append_block_to_evicted_int4_cache(L, eq_cache):
+    """Periodic re-compression on the LowRAM-EQ cache: a block of generated tokens after
+    the full prefix, compressed with int4 rows at its true positions, appended to the
+    evicted prefix (lowram_append). The result keeps chunk positions (the prefix's kept
+    chunks, then the block's), its arrays are the two caches concatenated bit for bit
+    (int4 codes and fp16 scales included), and decode over it matches the oracle."""
+    sh, ctx, cfg, cache, params, t, td, kk, vk = eq_cache
+    dev = kk.device
+    P, Tb = sh.n_tokens, 512
+    nb = int(sh.res_frac * Tb)
+    longer = SHAPE.replace(name="eq-block", n_tokens=P + Tb)
+    tl = H.stored_layer(longer, 0)
+    kb = tl["k"][:, P:].contiguous().to(dev)
+    vb = tl["v"][:, P:].contiguous().to(dev)
+    cfg_b = L.make_config(sh, n_tokens=Tb, n_positions=P + Tb, n_res=nb)
+    ctx_b = L.Context(cfg_b, dev.index or 0)
+    blk = L.alloc_cache(cfg_b, dev)
+    blk["chunk_pos"].copy_(torch.arange(P // sh.chunk, (P + Tb) // sh.chunk, dtype=torch.int32,
+                                        device=dev).expand(sh.batch, -1))
+    ws = torch.empty(L.workspace_size(cfg_b, L.OP_ENCODE), dtype=torch.uint8, device=dev)
+    L.encode(ctx_b, kb, vb, params, blk, ws)
+    torch.cuda.synchronize()
+    assert ctx_b.last_error() == L.OK
+    T0 = sh.n_kept_tokens
+    cfg_d = L.make_config(sh, n_tokens=T0 + Tb, n_positions=P + Tb, n_res=sh.n_res + nb)
+    ctx_d = L.Context(cfg_d, dev.index or 0)
+    dst = L.alloc_cache(cfg_d, dev)
+    L.append(ctx_d, dst, ctx, cache, ctx_b, blk)
+    torch.cuda.synchronize()
+    assert ctx_d.last_error() == L.OK
+    for name, dim in (("coef", 1), ("landmark", 2), ("res_val", 2), ("res_scale", 2),
+                      ("chunk_pos", 1)):
+        assert torch.equal(dst[name], torch.cat([cache[name], blk[name]], dim=dim)), name
+    assert torch.equal(dst["res_idx"], torch.cat([cache["res_idx"], blk["res_idx"] + T0], dim=2))
+    n_p = cache["chunk_ptr"].shape[2] - 1
+    assert torch.equal(dst["chunk_ptr"], torch.cat([cache["chunk_ptr"][:, :, :n_p],
+                                                    blk["chunk_ptr"] + sh.n_res], dim=2))
+    assert torch.equal(dst["landmark_norm"], torch.maximum(cache["landmark_norm"],
+                                                           blk["landmark_norm"]))
+    # decode over the appended cache against the oracle on the same arrays
+    wsd = torch.empty(L.workspace_size(cfg_d, L.OP_DECODE), dtype=torch.uint8, device=dev)
+    co = gpu_cache_to_oracle(dst)
+    p = H.oracle_params(t)
+    k = min(sh.top_k, (T0 + Tb) // sh.chunk)
+    q = synth.queries(sh, 0, 5)
+    out = torch.empty_like(q, device=dev)
+    sel = torch.empty(sh.batch, sh.n_kv_heads, k, dtype=torch.int32, device=dev)
+    L.decode_step(ctx_d, dst, params, q.to(dev), out, wsd, sel_out=sel)
+    torch.cuda.synchronize()
+    assert ctx_d.last_error() == L.OK
+    sel_np = sel.cpu().numpy()
+    osel, scores = O.select_chunks(H.f64(q), co["landmark"], sh.top_k)
+    ties = H.compare_selection(sel_np, osel, scores, k)
+    H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, "EQ appended-cache decode")
+    want, _ = O.decode_step(H.f64(q), co, p["basis"], p["w1"], p["b1"], p["w2"], p["b2"],
+                            chunk=sh.chunk, top_k=sh.top_k, theta=sh.theta, act=sh.act,
+                            sel=sel_np.astype(np.int64))
+    assert H.rel_err(H.f64(out), want) <= H.TOL["bf16"]
