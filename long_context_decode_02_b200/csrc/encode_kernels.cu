@@ -228,6 +228,19 @@ constexpr int kNB = 32;   // candidates per pass
 template <typename T>
 __device__ __forceinline__ double ld64(const T* p, size_t i) { return (double)to_f(p[i]); }
 
+// Eight consecutive elements at p (16-byte aligned), read through the read-only path so
+// that the loads of a staging loop are issued together rather than one round trip each.
+__device__ __forceinline__ void ld8_raw(const __nv_bfloat16* p, __nv_bfloat16 (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  *reinterpret_cast<uint4*>(v) = u;
+}
+__device__ __forceinline__ void ld8_raw(const float* p, float (&v)[8]) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
 // MC: 32-column blocks of c per lane, ceil(r / 32) when it is known at compile time (the
 // projection loop then runs no predicated-off blocks), 8 for any r <= 256 otherwise.
 template <typename T, int D, int FH, int MC>
@@ -259,24 +272,48 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
     for (int x = 0; x < 4; ++x)
 #pragma unroll
       for (int m = 0; m < kMaxC; ++m) acc[x][m] = 0.0;
+    // this thread's RoPE^-1 work in every head: candidate kc_c, rotary pairs kc_i0 ..
+    // kc_i0 + 7 (the same positions in every head, so their rotations are read once)
+    constexpr int kBlk = D / 16;   // blocks of 8 rotary pairs per candidate
+    const bool kc_act = tid < kNB * kBlk;
+    const int kc_c = kc_act ? tid / kBlk : 0, kc_i0 = (tid % kBlk) * 8;
+    const int kc_t = kc_act ? s_tok[kc_c] : -1;
+    double cs8[8], sn8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { cs8[e] = 1.0; sn8[e] = 0.0; }
+    if (kc_t >= 0) {
+      const int pos = token_position(dm, a.chunk_pos, b, kc_t, a.status);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const double2 c2 = rope_cs64(a.rope, kc_i0 + e, pos);
+        cs8[e] = c2.x;
+        sn8[e] = c2.y;
+      }
+    }
     for (int hh = 0; hh < H; ++hh) {
       __syncthreads();   // the previous head's operands are consumed
-      for (int o = tid; o < kNB * (D / 2); o += blockDim.x) {
-        const int c = o / (D / 2), i = o % (D / 2);
-        const int t = s_tok[c];
-        double x = 0.0, y = 0.0, cs = 1.0, sn = 0.0;
-        if (t >= 0) {
-          const size_t base = (((size_t)b * dm.T + t) * H + hh) * D;
-          x = ld64(kc, base + i);
-          y = ld64(kc, base + i + D / 2);
-          const double2 c2 = rope_cs64(a.rope, i, token_position(dm, a.chunk_pos, b, t, a.status));
-          cs = c2.x;
-          sn = c2.y;
+      if (kc_act) {
+        T xr[8], yr[8];
+        if (kc_t >= 0) {
+          const T* krow = kc + (((size_t)b * dm.T + kc_t) * H + hh) * D;
+          ld8_raw(krow + kc_i0, xr);
+          ld8_raw(krow + kc_i0 + D / 2, yr);
         }
-        sA[c * D + i] = x * cs + y * sn;
-        sA[c * D + i + D / 2] = y * cs - x * sn;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const double x = kc_t >= 0 ? (double)to_f(xr[e]) : 0.0;
+          const double y = kc_t >= 0 ? (double)to_f(yr[e]) : 0.0;
+          sA[kc_c * D + kc_i0 + e] = x * cs8[e] + y * sn8[e];
+          sA[kc_c * D + kc_i0 + e + D / 2] = y * cs8[e] - x * sn8[e];
+        }
       }
-      for (int o = tid; o < D * r; o += blockDim.x) sB[o] = basis[(size_t)hh * D * r + o];
+      {   // the head's basis block [D][r], contiguous: 16-byte units
+        const uint4* src = reinterpret_cast<const uint4*>(basis + (size_t)hh * D * r);
+        uint4* dst = reinterpret_cast<uint4*>(sB);
+        const int n16 = (int)((size_t)D * r * sizeof(T) / 16);
+#pragma unroll 4
+        for (int o = tid; o < n16; o += blockDim.x) dst[o] = __ldg(src + o);
+      }
       __syncthreads();
       for (int i = 0; i < D; ++i) {
         double kv[4];
@@ -302,9 +339,13 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
         const int kk = lane + 32 * m;
         if (kk < r) sC[(4 * cg + x) * r + kk] = acc[x][m];
       }
-    for (int o = tid; o < D * r; o += blockDim.x) {
-      const int j = o / r, kk = o % r;
-      sB[kk * D + j] = basis[((size_t)h * D + j) * r + kk];
+#pragma unroll 2
+    for (int o = tid; o < D * r / 8; o += blockDim.x) {   // 8 consecutive kk of row j
+      const int j = o / (r / 8), kk0 = (o % (r / 8)) * 8;
+      T v[8];
+      ld8_raw(basis + ((size_t)h * D + j) * r + kk0, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sB[(kk0 + e) * D + j] = v[e];
     }
     __syncthreads();
     // ---- K~[cand][j] = sum_kk c[cand][kk] B_h[j][kk]  (into region A)
@@ -333,9 +374,13 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
         for (int m = 0; m < M; ++m) sA[(4 * cg + x) * D + lane + 32 * m] = kt[x][m];
     }
     // W1_h transposed into region B: sB[j][f] = W1[h][f][j]
-    for (int o = tid; o < FH * D; o += blockDim.x) {
-      const int f = o / D, j = o % D;
-      sB[j * FH + f] = ((const T*)a.w1)[((size_t)h * FH + f) * D + j];
+#pragma unroll 2
+    for (int o = tid; o < FH * D / 8; o += blockDim.x) {   // 8 consecutive j of row f
+      const int f = o / (D / 8), j0 = (o % (D / 8)) * 8;
+      T v[8];
+      ld8_raw((const T*)a.w1 + ((size_t)h * FH + f) * D + j0, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sB[(j0 + e) * FH + f] = v[e];
     }
     __syncthreads();
     // ---- hid[cand][f] = act(sum_j K~[cand][j] W1[f][j] + b1[f])  (into region C)
@@ -364,9 +409,13 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
     }
     __syncthreads();   // region B (W1) consumed
     // W2_h transposed into region B: sB[f][j] = W2[h][j][f]
-    for (int o = tid; o < D * FH; o += blockDim.x) {
-      const int j = o / FH, f = o % FH;
-      sB[f * D + j] = ((const T*)a.w2)[((size_t)h * D + j) * FH + f];
+#pragma unroll 2
+    for (int o = tid; o < D * FH / 8; o += blockDim.x) {   // 8 consecutive f of row j
+      const int j = o / (FH / 8), f0 = (o % (FH / 8)) * 8;
+      T v[8];
+      ld8_raw((const T*)a.w2 + ((size_t)h * D + j) * FH + f0, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sB[(f0 + e) * D + j] = v[e];
     }
     __syncthreads();
     // ---- V_hat[cand][j] = sum_f hid[cand][f] W2[j][f] + b2[j];  e = sum_j (V - V_hat)^2
