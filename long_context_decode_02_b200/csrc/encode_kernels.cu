@@ -225,6 +225,13 @@ __global__ void __launch_bounds__(kSelEncThreads) residual_threshold_kernel(cons
 // consecutive banks.
 constexpr int kNB = 32;   // candidates per pass
 
+// Bytes of the re-score's staging region B: the largest operand staged there, a head's
+// basis block [D][r] (or its transpose), W1_h^T [D][FH] or W2_h^T [FH][D], in T.
+template <typename T>
+__host__ __device__ constexpr size_t rescore_stage_bytes(int D, int r, int FH) {
+  return (size_t)D * (size_t)(r > FH ? r : FH) * sizeof(T);   // a multiple of 16 bytes
+}
+
 template <typename T>
 __device__ __forceinline__ double ld64(const T* p, size_t i) { return (double)to_f(p[i]); }
 
@@ -251,11 +258,12 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
   const int n = a.cand_count[p];
   extern __shared__ double smd[];
   // region A: [kNB][D] fp64 (pre-RoPE keys of one head, later K~)
-  // region B: 64 KB of staged operands (basis block, transposed basis_h, W1^T, W2^T)
+  // region B: staged operands (basis block, transposed basis_h, W1^T, W2^T), sized for
+  //           the largest of them
   // region C: [kNB][max(r, FH)] fp64 (c, later hid)
   double* sA = smd;
   T* sB = reinterpret_cast<T*>(smd + kNB * D);
-  double* sC = smd + kNB * D + 65536 / 8;
+  double* sC = smd + kNB * D + rescore_stage_bytes<T>(D, r, FH) / 8;
   __shared__ int s_tok[kNB];
   __shared__ double s_e[kNB];
   const int cg = tid >> 5, lane = tid & 31;     // candidate group (4 each), column lane
@@ -562,7 +570,8 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     const int wc = dm.r > FH ? dm.r : FH;
-    const size_t smem = sizeof(double) * ((size_t)kNB * D + (size_t)kNB * wc) + 65536;
+    const size_t smem = sizeof(double) * ((size_t)kNB * D + (size_t)kNB * wc) +
+                        rescore_stage_bytes<T>(D, dm.r, FH);   // <= 224 KB (d <= 128, r, F <= 256)
     auto kern = dm.r == 160   ? residual_rescore_kernel<T, D, FH, 5>
                 : dm.r == 128 ? residual_rescore_kernel<T, D, FH, 4>
                               : residual_rescore_kernel<T, D, FH, 8>;

@@ -60,6 +60,16 @@ def check_encode(L, shape, device):
     for name in ("coef", "landmark"):
         g, w = H.f64(cache[name]), enc[name]
         bound = ulp_bound(w, shape.dtype) * 1.01 + 1e-6 * np.abs(w).max()
+        if name == "coef" and shape.dtype == "f32":
+            # fp32 storage is no coarser than the fp32 arithmetic, so one storage rounding
+            # does not cover it: add the bound of an fp32 dot product of n = H d terms
+            # (RoPE inversion included as a few more), gamma_n sum_i |k_i B_i|
+            kpre = O.rope_rotate(H.f64(t["k"]), np.arange(shape.n_tokens)[None, :, None],
+                                 shape.theta, inverse=True)
+            kpre = kpre.reshape(shape.batch, shape.n_tokens, -1)
+            n = kpre.shape[-1] + 8
+            u = 2.0 ** -24
+            bound = bound + (n * u / (1 - n * u)) * (np.abs(kpre) @ np.abs(H.f64(t["basis"])))
         assert np.all(np.abs(g - w) <= bound), (name, float(np.max(np.abs(g - w) - bound)))
     # landmark_norm: an upper bound of max_c |L_c|_2 of the stored landmarks, within two
     # fp32 steps of the definition written out on the host
@@ -141,3 +151,14 @@ def test_tensor_core_encode_edges(L, cuda_device, over):
     sh = synth.CONFIGS[1].replace(**kw)
     ties, *_ = check_encode(L, sh, cuda_device)
     H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, f"tc encode {over}")
+
+
+@pytest.mark.parametrize("rank", [160, 256], ids=["r160", "r256"])
+def test_f32_d128_encode(L, cuda_device, rank):
+    """fp32 storage at d 128, F 256: the CUDA-core projection and the fp64 re-score with
+    its largest staged operands (W1_h^T in fp32 is 128 KB; at r 256 so is a head's basis
+    block) against the oracle, with the same bars as above."""
+    sh = synth.CONFIGS[1].replace(name="enc-f32-d128", dtype="f32", n_tokens=2048, batch=1,
+                                  rank=rank, seed=77)
+    ties, *_ = check_encode(L, sh, cuda_device)
+    H.assert_ties_bounded(ties, sh.batch * sh.n_kv_heads, f"f32 d128 encode r{rank}")
