@@ -298,15 +298,31 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
         sn8[e] = c2.y;
       }
     }
-    for (int hh = 0; hh < H; ++hh) {
-      __syncthreads();   // the previous head's operands are consumed
+    // A head's operands: this thread's key slices and its share of the basis block
+    // [D][r] (contiguous, 16-byte units). When the share fits in registers, the next
+    // head's are loaded while this head's products run.
+    constexpr int kBV = (int)(((size_t)D * 32 * MC * sizeof(T) / 16 + kEncThreads - 1) / kEncThreads);
+    constexpr bool kPrefetch = kBV <= 16;
+    const int n16 = (int)((size_t)D * r * sizeof(T) / 16);
+    T xr[8], yr[8];
+    uint4 bv16[kPrefetch ? kBV : 1];
+    auto load_keys = [&](int hh) {
+      if (kc_act && kc_t >= 0) {
+        const T* krow = kc + (((size_t)b * dm.T + kc_t) * H + hh) * D;
+        ld8_raw(krow + kc_i0, xr);
+        ld8_raw(krow + kc_i0 + D / 2, yr);
+      }
+    };
+    auto load_basis = [&](int hh) {
+      const uint4* src = reinterpret_cast<const uint4*>(basis + (size_t)hh * D * r);
+#pragma unroll
+      for (int q = 0; q < (kPrefetch ? kBV : 1); ++q) {
+        const int o = tid + q * kEncThreads;
+        if (o < n16) bv16[q] = __ldg(src + o);
+      }
+    };
+    auto store_operands = [&](int hh) {
       if (kc_act) {
-        T xr[8], yr[8];
-        if (kc_t >= 0) {
-          const T* krow = kc + (((size_t)b * dm.T + kc_t) * H + hh) * D;
-          ld8_raw(krow + kc_i0, xr);
-          ld8_raw(krow + kc_i0 + D / 2, yr);
-        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const double x = kc_t >= 0 ? (double)to_f(xr[e]) : 0.0;
@@ -315,14 +331,30 @@ __global__ void __launch_bounds__(kEncThreads) residual_rescore_kernel(const Enc
           sA[kc_c * D + kc_i0 + e + D / 2] = y * cs8[e] - x * sn8[e];
         }
       }
-      {   // the head's basis block [D][r], contiguous: 16-byte units
+      uint4* dst = reinterpret_cast<uint4*>(sB);
+      if constexpr (kPrefetch) {
+#pragma unroll
+        for (int q = 0; q < kBV; ++q) {
+          const int o = tid + q * kEncThreads;
+          if (o < n16) dst[o] = bv16[q];
+        }
+      } else {
         const uint4* src = reinterpret_cast<const uint4*>(basis + (size_t)hh * D * r);
-        uint4* dst = reinterpret_cast<uint4*>(sB);
-        const int n16 = (int)((size_t)D * r * sizeof(T) / 16);
 #pragma unroll 4
-        for (int o = tid; o < n16; o += blockDim.x) dst[o] = __ldg(src + o);
+        for (int o = tid; o < n16; o += kEncThreads) dst[o] = __ldg(src + o);
       }
+    };
+    load_keys(0);
+    if constexpr (kPrefetch) load_basis(0);
+    for (int hh = 0; hh < H; ++hh) {
+      __syncthreads();   // the previous head's operands are consumed
+      if (!kPrefetch) load_keys(hh);
+      store_operands(hh);
       __syncthreads();
+      if (kPrefetch && hh + 1 < H) {   // in flight under this head's products
+        load_keys(hh + 1);
+        load_basis(hh + 1);
+      }
       for (int i = 0; i < D; ++i) {
         double kv[4];
 #pragma unroll
