@@ -4,9 +4,9 @@ epilogue holds them: K~_rot in part A, act(W1 K~_pre + b1) and the residual row 
 part B); the tensor-core kernel at full rank against exact dense attention; and a
 bounded wait that runs out on purpose.
 
-Method: "rebuild only the top-k chunks" (agihunt summary, key paragraph); values from
-the per-head predictor plus the stored residual corrections (cctest "How the method
-works": Amortised values, Residuals for difficult tokens).
+Method: only the top-k chunks are rebuilt at each step (agihunt summary, key
+paragraph); values from the per-head predictor plus the stored residual corrections
+(cctest "How the method works": Amortised values, Residuals for difficult tokens).
 
 Tolerances, max |gpu - oracle| / RMS(oracle) over every rebuilt row of a layer call:
 - K~_rot 1e-3: bf16 coefficients times the bf16 basis, exact products summed in fp32
