@@ -357,7 +357,7 @@ const char* lowram_status_string(lowram_status status);
 /* Test only: lowram_attend_selected on the tensor-core kernel (LOWRAM_ERR_UNSUPPORTED
  * where it does not apply) that also stores the rows it rebuilds, at the points where its
  * epilogue holds them, so they can be compared element by element with the method's
- * rebuilt keys and values ("rebuild only the top-k chunks", agihunt summary, key
+ * rebuilt keys and values (only the top-k chunks are rebuilt: agihunt summary, key
  * paragraph; cctest "Residuals for difficult tokens"). Rows are in selection order:
  * row = (b*H_kv + h)*k*C + s*C + j for token j of the chunk sel[b][h][s]; rows = B*H_kv*k*C
  * with k = min(top_k, T/C). All three outputs are device fp32 arrays, zeroed first:
