@@ -7,23 +7,44 @@
 //   query head g of the KV head's GQA group (the oracle's dense_attention).
 //
 // HBM-bound (every K and V byte is read once, ~4 FLOP per byte): CUDA cores, no tensor
-// cores. Split-K: a CTA takes 1024 positions of one (b, h); 16 lanes hold one position's
-// row (8 dimensions each, so a warp loads two 256-byte rows per instruction); every lane
-// group takes four positions per iteration, reduces their 16 logits with one
-// reduce-scatter (15 shuffles), updates the online softmax once per four positions, and
-// accumulates V. The CTA's partial (m, l, O) goes to the workspace; a combine kernel
-// merges the splits of each query head.
+// cores. Split-K: a CTA takes 1024 positions of one (b, h). Its K and V rows arrive by
+// TMA in tiles of 64 positions (one 64 x 128 box of each, 32 KB) into a 3-stage ring,
+// so the loads stay in flight while the warps compute; one elected thread refills a
+// stage once all eight warps have released it. In a tile, warp w takes positions
+// 8w .. 8w + 7; 16 lanes hold one position's row (8 dimensions each, one 16-byte
+// shared-memory load); every lane group takes four positions, reduces their 16 logits
+// with one reduce-scatter (15 shuffles), updates the online softmax once, and accumulates
+// V. The CTA's partial (m, l, O) goes to the workspace; a combine kernel merges the
+// splits of each query head. Every wait is bounded; on expiry the kernel raises a
+// timeout status, lets its copies in flight land and returns.
+#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace lowram {
 namespace {
+
+using namespace sm100;
 
 constexpr int kDD = 128, kDG = 4;
 constexpr int kDenseThreads = 256;
 constexpr int kDenseSplit = 1024;   // positions per CTA
 constexpr int kPartStride = kDG * (2 + kDD);
+constexpr int kTilePos = 64;                             // positions per TMA tile
+constexpr int kDStages = 3;                              // ring depth
+constexpr uint32_t kRowBytes = kDD * 2;                  // one head's row, bf16
+constexpr uint32_t kHalfBytes = kTilePos * kRowBytes;    // K (or V) of one tile: 16 KB
+constexpr uint32_t kStageBytes = 2 * kHalfBytes;
+constexpr size_t kDenseSmem = (size_t)kDStages * kStageBytes + 128 + 128;   // + barriers + align
+static_assert(kDenseSplit % kTilePos == 0 && kTilePos == 8 * (kDenseThreads / 32),
+              "a tile gives each warp 8 positions");
+
+struct DenseMaps {
+  CUtensorMap k;   // [B*T rows][H*d cols] bf16, box 128 x 64
+  CUtensorMap v;
+};
 
 struct DenseArgs {
   int B, T, H, Hq;
@@ -34,15 +55,47 @@ struct DenseArgs {
   float* part;              // [B*H][n_split][G][2 + d]
   int n_split;
   int t_valid;              // positions 0 .. t_valid-1 of each row block are attended
+  int* status;              // device status word (timeout)
 };
 
-__global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const DenseArgs a) {
+__global__ void __launch_bounds__(kDenseThreads, 2)
+dense_decode_kernel(const DenseArgs a, const __grid_constant__ DenseMaps maps) {
   const int p = blockIdx.y, b = p / a.H, h = p % a.H;
   const int split = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane >> 4, gl = lane & 15;
   const int t_begin = split * kDenseSplit;
   const int t_end = min(a.t_valid, t_begin + kDenseSplit);
+  const int n_tiles = (t_end - t_begin + kTilePos - 1) / kTilePos;
+  extern __shared__ uint8_t dsm_raw[];
+  const uint32_t raw = smem_u32(dsm_raw);
+  const uint32_t ring = (raw + 127u) & ~127u;
+  uint8_t* gring = dsm_raw + (ring - raw);
+  const uint32_t bars = ring + kDStages * kStageBytes;   // full[kDStages], empty[kDStages]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gring + kDStages * kStageBytes + 64);
+  auto full = [&](int st) { return bars + 8u * (uint32_t)st; };
+  auto empty = [&](int st) { return bars + 8u * (uint32_t)(kDStages + st); };
+  // tile j: positions t_begin + 64 j .., rows b T + t of the [B*T][H*d] view, columns h d ..
+  auto issue = [&](int j) {
+    const int st = j % kDStages;
+    const uint32_t dst = ring + (uint32_t)st * kStageBytes;
+    mbar_arrive_expect_tx(full(st), kStageBytes);
+    const int y = b * a.T + t_begin + kTilePos * j;
+    tma_load_2d(dst, &maps.k, h * kDD, y, full(st));
+    tma_load_2d(dst + kHalfBytes, &maps.v, h * kDD, y, full(st));
+  };
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int st = 0; st < kDStages; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), kDenseThreads / 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  int issued = 0, landed = 0;   // thread 0: tiles requested / seen complete (for the drain)
+  if (tid == 0)
+    for (; issued < kDStages && issued < n_tiles; ++issued) issue(issued);
   // this lane's 8 dimensions of the group's queries, scaled to log2 units
   const float zs = 1.4426950408889634f * rsqrtf((float)kDD);
   float qv[kDG][8];
@@ -65,29 +118,29 @@ __global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const De
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
   }
-  // positions of this warp: [w0, w0 + 128); lane group grp takes w0 + 8 i + 4 grp + u
-  const int w0 = t_begin + warp * (kDenseSplit / (kDenseThreads / 32));
-  const size_t row_stride = (size_t)a.H * kDD;
-  const __nv_bfloat16* kbase = a.k + ((size_t)b * a.T * a.H + h) * kDD + 8 * gl;
-  const __nv_bfloat16* vbase = a.v + ((size_t)b * a.T * a.H + h) * kDD + 8 * gl;
-  constexpr int kIters = kDenseSplit / (kDenseThreads / 32) / 8;
-  auto load = [&](int i, uint4 (&kk)[4], uint4 (&vv)[4]) {
+  // in tile j, lane group grp of warp w takes positions 8 w + 4 grp + u (u < 4)
+  bool good = true;
+#pragma unroll 1
+  for (int i = 0; i < n_tiles; ++i) {
+    const int st = i % kDStages;
+    good = good && mbar_wait_bounded(full(st), (uint32_t)((i / kDStages) & 1), abort_flag);
+    if (tid == 0 && good) landed = i + 1;
+    const int pl0 = 8 * warp + 4 * grp;                  // first position of the lane group
+    const int w0 = t_begin + kTilePos * i + pl0;
+    const uint8_t* kst = gring + st * kStageBytes + (size_t)pl0 * kRowBytes + 16 * gl;
+    uint4 kr[4], vr[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int t = w0 + 8 * i + 4 * grp + u;
-      if (t < t_end) {
-        kk[u] = __ldcs(reinterpret_cast<const uint4*>(kbase + (size_t)t * row_stride));
-        vv[u] = __ldcs(reinterpret_cast<const uint4*>(vbase + (size_t)t * row_stride));
-      } else {
-        kk[u] = make_uint4(0u, 0u, 0u, 0u);
-        vv[u] = kk[u];
-      }
+      kr[u] = *reinterpret_cast<const uint4*>(kst + u * kRowBytes);
+      vr[u] = *reinterpret_cast<const uint4*>(kst + kHalfBytes + u * kRowBytes);
     }
-  };
-#pragma unroll 1
-  for (int i = 0; i < kIters; ++i) {
-    uint4 kr[4], vr[4];
-    load(i, kr, vr);
+    // the stage may be refilled once every warp has its rows in registers
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(st));
+    if (tid == 0 && i + kDStages < n_tiles) {
+      good = good && mbar_wait_bounded(empty(st), (uint32_t)((i / kDStages) & 1), abort_flag);
+      if (good) issue(issued++);
+    }
     // partial logits: z[u][g] over this lane's 8 dimensions
     float z[16];
 #pragma unroll
@@ -121,7 +174,7 @@ __global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const De
       }
     }
     const int my_u = gl >> 2, my_g = gl & 3;
-    const bool valid = w0 + 8 * i + 4 * grp + my_u < t_end;
+    const bool valid = good && w0 + my_u < t_end;
     float zz = valid ? z[0] : -INFINITY;
     // block max per head: over the four lanes holding that head's positions
     float bm = fmaxf(zz, __shfl_xor_sync(0xffffffffu, zz, 4));
@@ -161,6 +214,13 @@ __global__ void __launch_bounds__(kDenseThreads, 2) dense_decode_kernel(const De
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pg, vf[e], acc[g][e]);
       }
+    }
+  }
+  if (tid == 0 && *abort_flag) {   // a wait gave up: the copies still in flight land first
+    raise_status(a.status, kStatusTimeout);
+    for (int j = landed; j < issued; ++j) {
+      int dummy = 0;
+      mbar_wait_bounded(full(j % kDStages), (uint32_t)((j / kDStages) & 1), (volatile int*)&dummy);
     }
   }
   // the two lane groups of the warp, then the warps of the CTA
@@ -253,6 +313,21 @@ __global__ void __launch_bounds__(kDD) suffix_merge_kernel(const DenseArgs a, co
   a.out[(size_t)bq * kDD + j] = __float2bfloat16_rn(O / L);
 }
 
+// The split kernel over a.n_split x (B*H) CTAs: tensor maps over the [B*T][H*d] views of
+// K and V (one head's 64 x 128 box per tile), then the launch.
+cudaError_t launch_splits(const DenseArgs& a, cudaStream_t s) {
+  DenseMaps maps;
+  const uint64_t rows = (uint64_t)a.B * a.T, cols = (uint64_t)a.H * kDD;
+  if (!make_tensor_map_2d(&maps.k, a.k, LOWRAM_DTYPE_BF16, cols, rows, kDD, kTilePos, 0, 256) ||
+      !make_tensor_map_2d(&maps.v, a.v, LOWRAM_DTYPE_BF16, cols, rows, kDD, kTilePos, 0, 256))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(dense_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kDenseSmem);
+  if (e != cudaSuccess) return e;
+  dense_decode_kernel<<<dim3(a.n_split, a.B * a.H), kDenseThreads, kDenseSmem, s>>>(a, maps);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t suffix_workspace_bytes(const Dims& dm, int s_max) {
@@ -262,7 +337,8 @@ size_t suffix_workspace_bytes(const Dims& dm, int s_max) {
 
 cudaError_t launch_suffix_merge(const Dims& dm, const void* k_suffix, const void* v_suffix,
                                 int s_max, int n_suffix, const void* q, const float* pre_out,
-                                const float* pre_ml, void* out, void* ws, cudaStream_t s) {
+                                const float* pre_ml, void* out, void* ws, int* status,
+                                cudaStream_t s) {
   DenseArgs a{};
   a.B = dm.B;
   a.T = s_max;
@@ -274,10 +350,10 @@ cudaError_t launch_suffix_merge(const Dims& dm, const void* k_suffix, const void
   a.out = (__nv_bfloat16*)out;
   a.part = (float*)ws;
   a.t_valid = n_suffix;
+  a.status = status;
   a.n_split = (n_suffix + kDenseSplit - 1) / kDenseSplit;
   if (a.n_split > 0) {
-    dense_decode_kernel<<<dim3(a.n_split, dm.B * dm.H), kDenseThreads, 0, s>>>(a);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_splits(a, s);
     if (e != cudaSuccess) return e;
   }
   suffix_merge_kernel<<<dm.B * dm.Hq, kDD, 0, s>>>(a, pre_out, pre_ml);
@@ -294,7 +370,7 @@ size_t dense_workspace_bytes(const Dims& dm) {
 }
 
 cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, const void* q,
-                                void* out, void* ws, cudaStream_t s) {
+                                void* out, void* ws, int* status, cudaStream_t s) {
   DenseArgs a{};
   a.B = dm.B;
   a.T = dm.T;
@@ -307,8 +383,8 @@ cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, co
   a.part = (float*)ws;
   a.n_split = (dm.T + kDenseSplit - 1) / kDenseSplit;
   a.t_valid = dm.T;
-  dense_decode_kernel<<<dim3(a.n_split, dm.B * dm.H), kDenseThreads, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
+  a.status = status;
+  cudaError_t e = launch_splits(a, s);
   if (e != cudaSuccess) return e;
   dense_combine_kernel<<<dm.B * dm.Hq, kDD, 0, s>>>(a);
   return cudaGetLastError();

@@ -717,8 +717,8 @@ lowram_status lowram_dense_decode(lowram_ctx* ctx, const void* k_cache, const vo
   if (workspace_bytes < dense_workspace_bytes(dm)) return LOWRAM_ERR_WORKSPACE;
   DeviceGuard g(ctx->device);
   if (!g.ok) return LOWRAM_ERR_CUDA;
-  if (launch_dense_decode(dm, k_cache, v, q, out, workspace, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess) {
+  if (launch_dense_decode(dm, k_cache, v, q, out, workspace, ctx->status,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return LOWRAM_ERR_CUDA;
   }
@@ -787,7 +787,7 @@ lowram_status lowram_decode_step_suffix(lowram_ctx* ctx, const lowram_cache* cac
       LOWRAM_OK)
     return st;
   if (launch_suffix_merge(dm, k_suffix, v_suffix, s_max, n_suffix, q, pre_out, pre_ml, out,
-                          ws + sw.part, s) != cudaSuccess) {
+                          ws + sw.part, ctx->status, s) != cudaSuccess) {
     cudaGetLastError();
     return LOWRAM_ERR_CUDA;
   }

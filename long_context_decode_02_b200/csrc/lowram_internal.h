@@ -149,13 +149,14 @@ cudaError_t launch_fit_basis(const Dims& dm, const void* const* k_layers, int n_
 bool dense_supported(const Dims& dm);
 size_t dense_workspace_bytes(const Dims& dm);
 cudaError_t launch_dense_decode(const Dims& dm, const void* k, const void* v, const void* q,
-                                void* out, void* ws, cudaStream_t s);
+                                void* out, void* ws, int* status, cudaStream_t s);
 // attention over an uncompressed suffix ([B][s_max][H][d], first n_suffix rows valid),
 // merged with the compressed prefix's normalised fp32 output and its softmax (max, sum)
 size_t suffix_workspace_bytes(const Dims& dm, int s_max);
 cudaError_t launch_suffix_merge(const Dims& dm, const void* k_suffix, const void* v_suffix,
                                 int s_max, int n_suffix, const void* q, const float* pre_out,
-                                const float* pre_ml, void* out, void* ws, cudaStream_t s);
+                                const float* pre_ml, void* out, void* ws, int* status,
+                                cudaStream_t s);
 
 // ---------------- encode ----------------
 struct EncodeArgs {
