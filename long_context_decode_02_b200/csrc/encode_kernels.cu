@@ -25,24 +25,53 @@ constexpr int kEncThreads = 256;
 constexpr int kTE = 16;          // tokens per CTA in the projection / residual kernels
 constexpr int kSelEncThreads = 1024;
 constexpr int kRescoreCtas = 96; // CTAs per (b, h) looping over the fp64 candidates
+constexpr int kNormRows = 256;   // landmark rows per CTA of the norm bound
 
-// E3: landmarks, one thread per output element.
+// Eight consecutive elements at p (16-byte aligned), read through the read-only path so
+// that the loads of a staging loop are issued together rather than one round trip each.
+__device__ __forceinline__ void ld8_raw(const __nv_bfloat16* p, __nv_bfloat16 (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  *reinterpret_cast<uint4*>(v) = u;
+}
+__device__ __forceinline__ void ld8_raw(const float* p, float (&v)[8]) {
+  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+}
+
+// E3: landmarks, one thread per 8 consecutive output elements (16- or 32-byte loads of
+// each of the chunk's C keys, summed in fp32 in token order, then divided by C).
 template <typename T>
 __global__ void landmark_kernel(const EncodeArgs a) {
   const Dims& dm = a.dm;
-  const size_t n = (size_t)dm.B * dm.H * dm.Nc * dm.d;
-  for (size_t o = (size_t)blockIdx.x * blockDim.x + threadIdx.x; o < n;
+  const size_t n8 = (size_t)dm.B * dm.H * dm.Nc * dm.d / 8;
+  const T* kc = (const T*)a.k_cache;
+  for (size_t o = (size_t)blockIdx.x * blockDim.x + threadIdx.x; o < n8;
        o += (size_t)gridDim.x * blockDim.x) {
-    const int j = (int)(o % dm.d);
-    size_t rest = o / dm.d;
+    const int j0 = (int)(o % (dm.d / 8)) * 8;
+    size_t rest = o / (dm.d / 8);
     const int c = (int)(rest % dm.Nc);
     rest /= dm.Nc;
     const int h = (int)(rest % dm.H);
     const int b = (int)(rest / dm.H);
-    float acc = 0.f;
-    for (int i = 0; i < dm.C; ++i)
-      acc += ldf((const T*)a.k_cache, (((size_t)b * dm.T + (size_t)c * dm.C + i) * dm.H + h) * dm.d + j);
-    ((T*)a.landmark)[o] = from_f<T>(acc / (float)dm.C);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < dm.C; ++i) {
+      T v[8];
+      ld8_raw(kc + (((size_t)b * dm.T + (size_t)c * dm.C + i) * dm.H + h) * dm.d + j0, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += to_f(v[e]);
+    }
+    T out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = from_f<T>(acc[e] / (float)dm.C);
+    T* dst = (T*)a.landmark + o * 8;
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(out);
+    } else {
+      reinterpret_cast<float4*>(dst)[0] = *reinterpret_cast<const float4*>(out);
+      reinterpret_cast<float4*>(dst)[1] = *reinterpret_cast<const float4*>(out + 4);
+    }
   }
 }
 
@@ -235,18 +264,6 @@ __host__ __device__ constexpr size_t rescore_stage_bytes(int D, int r, int FH) {
 template <typename T>
 __device__ __forceinline__ double ld64(const T* p, size_t i) { return (double)to_f(p[i]); }
 
-// Eight consecutive elements at p (16-byte aligned), read through the read-only path so
-// that the loads of a staging loop are issued together rather than one round trip each.
-__device__ __forceinline__ void ld8_raw(const __nv_bfloat16* p, __nv_bfloat16 (&v)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  *reinterpret_cast<uint4*>(v) = u;
-}
-__device__ __forceinline__ void ld8_raw(const float* p, float (&v)[8]) {
-  const float4 x = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-  v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
-}
 
 // MC: 32-column blocks of c per lane, ceil(r / 32) when it is known at compile time (the
 // projection loop then runs no predicated-off blocks), 8 for any r <= 256 otherwise.
@@ -580,8 +597,8 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
   const Dims& dm = a.dm;
   cudaError_t e;
   {
-    const size_t n = (size_t)dm.B * dm.H * dm.Nc * dm.d;
-    const int blocks = (int)((n + 255) / 256 < 65535 * 8 ? (n + 255) / 256 : 65535 * 8);
+    const size_t n8 = (size_t)dm.B * dm.H * dm.Nc * dm.d / 8;
+    const int blocks = (int)((n8 + 255) / 256 < 65535 * 8 ? (n8 + 255) / 256 : 65535 * 8);
     landmark_kernel<T><<<blocks, 256, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -629,41 +646,59 @@ cudaError_t launch_encode_typed(const EncodeArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-// landmark_norm[p] = max over chunks of |L_pc|_2, one warp per row (exact squares, fp64
-// sums), rounded up to fp32 with a margin for the fp64 rounding.
+// landmark_norm[p] = max over chunks of |L_pc|_2 (exact squares, fp64 sums), rounded up
+// to fp32 with a margin for the fp64 rounding.
 template <typename T>
 __global__ void __launch_bounds__(256) landmark_norm_kernel(const Dims dm, const T* landmark,
                                                             float* norm) {
-  const int p = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA (x, p): landmark rows [kNormRows x, kNormRows (x + 1)) of (b, h) pair p; d / 8
+  // lanes per row (8 elements each), squares summed in fp64. Each CTA raises norm[p] to its own
+  // rounded-up bound with an integer max on the (non-negative) fp32 bits, so the result
+  // is the bound of the largest row: rounding up and the square root are monotonic.
+  const int p = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const T* Lp = landmark + (size_t)p * dm.Nc * dm.d;
+  const int c_end = min(dm.Nc, (int)(blockIdx.x + 1) * kNormRows);
+  const int per_row = dm.d / 8;   // lanes per row (16 at d = 128, 8 at d = 64)
+  const int rows_per_warp = 32 / per_row;
   double best = 0.0;
-  for (int c = warp; c < dm.Nc; c += blockDim.x >> 5) {
-    const T* row = Lp + (size_t)c * dm.d;
+  for (int c0 = blockIdx.x * kNormRows + warp * rows_per_warp; c0 < c_end;
+       c0 += (blockDim.x >> 5) * rows_per_warp) {
+    const int c = c0 + lane / per_row;
     double ss = 0.0;
-    for (int j = lane; j < dm.d; j += 32) {
-      const double x = ldd(row, j);
-      ss = fma(x, x, ss);
-    }
+    if (c < c_end) {
+      T v[8];
+      ld8_raw(Lp + (size_t)c * dm.d + 8 * (lane % per_row), v);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      for (int e = 0; e < 8; ++e) {
+        const double x = (double)to_f(v[e]);
+        ss = fma(x, x, ss);
+      }
+    }
+    for (int o = per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     best = fmax(best, ss);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
   __shared__ double wmax[8];
   if (lane == 0) wmax[warp] = best;
   __syncthreads();
   if (threadIdx.x == 0) {
     for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = fmax(best, wmax[w]);
-    norm[p] = __double2float_ru(sqrt(best) * (1.0 + 1e-12));
+    const float bound = __double2float_ru(sqrt(best) * (1.0 + 1e-12));
+    atomicMax(reinterpret_cast<unsigned int*>(norm + p), __float_as_uint(bound));
   }
 }
 
 cudaError_t launch_landmark_norms(const Dims& dm, const void* landmark, float* norm,
                                   cudaStream_t s) {
   const int pairs = dm.B * dm.H;
+  cudaError_t e = cudaMemsetAsync(norm, 0, (size_t)pairs * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((dm.Nc + kNormRows - 1) / kNormRows), (unsigned)pairs);
   if (dm.dtype == LOWRAM_DTYPE_BF16)
-    landmark_norm_kernel<__nv_bfloat16><<<pairs, 256, 0, s>>>(dm, (const __nv_bfloat16*)landmark, norm);
+    landmark_norm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(dm, (const __nv_bfloat16*)landmark, norm);
   else
-    landmark_norm_kernel<float><<<pairs, 256, 0, s>>>(dm, (const float*)landmark, norm);
+    landmark_norm_kernel<float><<<grid, 256, 0, s>>>(dm, (const float*)landmark, norm);
   return cudaGetLastError();
 }
 
