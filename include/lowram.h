@@ -332,8 +332,9 @@ lowram_status lowram_decode_step_static(lowram_ctx* ctx, const lowram_cache* cac
                                         void* out, int32_t* sel_out, void* stream);
 
 /* The uncompressed baseline the method is measured against (the pages compare decode
- * throughput with the uncompressed model: "up to 5x higher peak decode throughput",
- * agihunt summary, efficiency paragraph; abstract): exact GQA decode attention over the
+ * throughput with the uncompressed model and report about five times its peak decode
+ * throughput at 262K tokens: agihunt summary, efficiency paragraph; cctest "How the
+ * method works", Selective reconstruction; abstract): exact GQA decode attention over the
  * full bf16 cache, out_g = sum_t softmax_t(q_g . K_t / sqrt(d)) V_t over every position
  * t < T, for each query head g.
  *   k_cache [B][T][H_kv][d], v [B][T][H_kv][d] (post-RoPE keys and values, bf16, as

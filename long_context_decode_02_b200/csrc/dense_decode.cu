@@ -1,7 +1,8 @@
 // Uncompressed GQA flash-decode over a bf16 KV cache: the baseline that LowRAM's
 // compressed decode is compared against (the pages compare decode throughput with the
-// uncompressed model: "up to 5x higher peak decode throughput", agihunt summary,
-// efficiency paragraph, and the abstract).
+// uncompressed model and report about five times its peak decode throughput at 262K
+// tokens: agihunt summary, efficiency paragraph; cctest "How the method works",
+// Selective reconstruction; the abstract).
 //
 //   out_g = sum_t softmax_t(q_g . K_t / sqrt(d)) V_t over every position t < T, for each
 //   query head g of the KV head's GQA group (the oracle's dense_attention).
