@@ -130,8 +130,27 @@ encode_project_tc_kernel(const EncodeArgs a, const __grid_constant__ ProjMaps ma
     // the token's rotations (cos, sin)(pos theta_i) of this thread's 32 pairs, shared by
     // all heads; and head 0's key rows
     float2 rc[32];
+    {   // 16-byte loads of both tables' rows (pairs 32 hf .. 32 hf + 31 are contiguous)
+      const float4* lo4 = reinterpret_cast<const float4*>(
+          a.rope.lo32 + (size_t)(pos & (kRopeLo - 1)) * a.rope.half + 32 * hf);
+      const float4* hi4 = reinterpret_cast<const float4*>(
+          a.rope.hi32 + (size_t)(pos >> kRopeLoBits) * a.rope.half + 32 * hf);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) rc[i] = rope_cs32(a.rope, 32 * hf + i, pos);
+      for (int m8 = 0; m8 < 16; m8 += 8) {
+        float4 lv[8], hv[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          lv[m] = __ldg(lo4 + m8 + m);
+          hv[m] = __ldg(hi4 + m8 + m);
+        }
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          rc[2 * (m8 + m)] = rope_combine(make_float2(hv[m].x, hv[m].y), make_float2(lv[m].x, lv[m].y));
+          rc[2 * (m8 + m) + 1] =
+              rope_combine(make_float2(hv[m].z, hv[m].w), make_float2(lv[m].z, lv[m].w));
+        }
+      }
+    }
     const __nv_bfloat16* src0 = kc + ((size_t)b * dm.T + t) * H * kD + 32 * hf;
     uint4 xr[4], yr[4];
 #pragma unroll
